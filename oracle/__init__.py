@@ -1,0 +1,112 @@
+"""CPU oracle for the key-only GLA token mixer -- TEST INFRASTRUCTURE ONLY.
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and the ``cpu_baseline`` /
+``--impl reference`` legs of ``bench.py`` may import this package.  The
+product path (``recurrent_vision_backbone_only_b200``) never imports it and
+shares no code with it.
+
+The arithmetic lives in ``gla_oracle.c`` (plain sequential fp64 recurrence,
+OpenMP over independent (batch, head) pairs); this module only compiles it
+with gcc and marshals numpy arrays.  Source: "GTR: Gated Token Recurrence for
+Efficient Dense Prediction" (arXiv 2609.26590), method section (GLA
+recurrence, retention gate, output gate, scan directions).
+
+Parity status: the recurrence, gate, scale, epilogue and direction map are
+pinned by tests/test_oracle_pins.py against closed forms, the brute-force
+quadratic form, library routines and direction invariants.  Parity with the
+authors' own (unpublished) outputs is unpinned: the pages print no numbers
+for the operator.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "gla_oracle.c")
+_LIB = os.path.join(_HERE, "liboracle.so")
+_lib = None
+
+TAU = 16.0
+EPS = 1e-6
+DIR_L2R, DIR_R2L, DIR_T2B, DIR_B2T, DIR_CYCLE = 0, 1, 2, 3, 4
+
+
+def build(force: bool = False) -> str:
+    """Compile gla_oracle.c into liboracle.so (gcc, OpenMP) when stale."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + ".tmp%d" % os.getpid()
+        subprocess.check_call(["gcc", "-O2", "-fopenmp", "-shared", "-fPIC",
+                               "-o", tmp, _SRC, "-lm"])
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+def load_library(path: str):
+    """Open a compiled oracle library and declare its signatures."""
+    lib = ctypes.CDLL(path)
+    dp = ctypes.POINTER(ctypes.c_double)
+    lib.gla_oracle_fwd.restype = ctypes.c_int
+    lib.gla_oracle_fwd.argtypes = [dp] * 8 + [ctypes.c_int] * 7 + [
+        ctypes.c_double, ctypes.c_double, ctypes.c_int]
+    lib.gla_oracle_spatial_index.restype = ctypes.c_long
+    lib.gla_oracle_spatial_index.argtypes = [ctypes.c_int, ctypes.c_long,
+                                             ctypes.c_long, ctypes.c_long]
+    return lib
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        _lib = load_library(build())
+    return _lib
+
+
+def _f64(x):
+    return np.ascontiguousarray(np.asarray(x, dtype=np.float64))
+
+
+def _ptr(x):
+    return x.ctypes.data_as(ctypes.POINTER(ctypes.c_double))
+
+
+def spatial_index(direction: int, p: int, grid_h: int, grid_w: int) -> int:
+    """Scan position p -> row-major spatial index (the oracle's own map)."""
+    return int(_load().gla_oracle_spatial_index(direction, p, grid_h, grid_w))
+
+
+def gla_forward(q, k, v, a, g, w, grid_h: int, grid_w: int, direction: int,
+                eps: float = EPS, tau: float = TAU, threads: int = 0,
+                return_o: bool = False, lib=None):
+    """Run the fp64 recurrence.
+
+    q, k, a: [B, L, H, d_k]; v, g: [B, L, H, d_v]; w: [d_v]; L = grid_h*grid_w.
+    Inputs of any float dtype are widened to fp64 (exactly, for fp16/fp32).
+    Returns u (fp64, same shape as v), and o (pre-epilogue readout) when
+    ``return_o``.  ``lib`` selects another compiled copy (used by the
+    mutation tests, which compile deliberately broken variants).
+    """
+    q, k, v, a, g, w = (_f64(t) for t in (q, k, v, a, g, w))
+    if q.ndim != 4:
+        raise ValueError("q must be [B, L, H, d_k]")
+    B, L, H, d_k = q.shape
+    d_v = v.shape[-1]
+    if L != grid_h * grid_w:
+        raise ValueError("L must equal grid_h * grid_w")
+    for t, d in ((k, d_k), (a, d_k), (v, d_v), (g, d_v)):
+        if t.shape != (B, L, H, d):
+            raise ValueError("inconsistent input shapes")
+    if w.shape != (d_v,):
+        raise ValueError("w must be [d_v]")
+    out = np.empty((B, L, H, d_v), dtype=np.float64)
+    o = np.empty_like(out) if return_o else None
+    rc = (lib or _load()).gla_oracle_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(a), _ptr(g), _ptr(w),
+                                _ptr(out), _ptr(o) if o is not None else None,
+                                B, H, grid_h, grid_w, d_k, d_v, direction,
+                                float(eps), float(tau), int(threads))
+    if rc != 0:
+        raise RuntimeError("gla_oracle_fwd failed with code %d" % rc)
+    return (out, o) if return_o else out
