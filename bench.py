@@ -1,0 +1,403 @@
+"""Throughput bench for the GLA token mixer (libgla.so) on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+One step = the whole hot path over one batch of the 640-px workload (40x40
+patch grid, B=1, H=6, d_k=d_v=64, fp16): four gla_fwd launches, one per
+scan direction (L->R, R->L, T->B, B->T), each on its own input set taken
+from a rotating pool larger than the 126 MB L2, so every launch reads cold
+inputs from HBM.  The K timed steps run as CUDA-graph replays; timing uses
+CUDA events on the launching stream with a barrier and synchronize on both
+sides, and the max over ranks.  With N > 1 (torchrun) every rank runs an
+independent replica (the operator has no cross-GPU exchange) and `value` is
+the total over ranks.
+
+--impl reference times the fp64 CPU oracle (test infrastructure, the only
+reference implementation that exists) on the machine's host cores on a bounded
+sample of the same workload; under torchrun only rank 0 runs it.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "GLA fwd Mtokens/s (B·H·L) at 40×40 grid fp16; % of HBM/tensor roofline"
+WORKLOAD = "gtr640"
+DIRECTIONS = (0, 1, 2, 3)
+L2_BYTES = 126 * 1024 * 1024
+FALLBACK_HBM_GBS = 6650.0
+PROFILE_TRAFFIC = os.path.join(ROOT, "profiles", "traffic.json")
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--e2e-steps", type=int, default=50)
+    ap.add_argument("--cpu-seconds", type=float, default=10.0,
+                    help="CPU-oracle sample budget for cpu_baseline / --impl reference")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+def dist_env():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def profile_traffic():
+    """dram bytes per launch from the committed ncu summary, if it matches this kernel build."""
+    try:
+        with open(PROFILE_TRAFFIC) as f:
+            d = json.load(f)
+        from recurrent_vision_backbone_only_b200 import build as _b
+        if d.get("workload") != WORKLOAD or d.get("lib_sources_digest") != _b.sources_digest():
+            return None
+        return d.get("dram_bytes_per_launch")
+    except Exception:
+        return None
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle sampling during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "--query-gpu=" + self.FIELDS, "--format=csv,noheader,nounits",
+                 "-lms", "50", "-i", str(self.gpu)],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            time.sleep(0.3)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        self.out = ""
+        if self.proc is not None:
+            time.sleep(0.1)
+            self.proc.terminate()
+            try:
+                self.out, _ = self.proc.communicate(timeout=5)
+            except Exception:
+                self.proc.kill()
+                self.out = ""
+
+    def summary(self):
+        rows = []
+        for line in (self.out or "").splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                rows.append(dict(sm=float(parts[1]), max=float(parts[2]), reasons=parts[5:9]))
+            except ValueError:
+                continue
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"], "samples": 0}
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        seen = sorted({names[i] for r in rows for i, v in enumerate(r["reasons"])
+                       if v.lower() == "active"})
+        return {"sm_mhz": statistics.median(r["sm"] for r in rows),
+                "sm_max_mhz": max(r["max"] for r in rows), "reasons": seen,
+                "samples": len(rows)}
+
+
+def cpu_oracle_sample(wl, x, budget_s: float):
+    """Time the fp64 oracle on whole (direction) passes of the workload until the budget."""
+    import numpy as np
+    import oracle
+    xs = {n: np.asarray(x[n], dtype=np.float64) for n in ("q", "k", "v", "a", "g", "w")}
+    threads = os.cpu_count() or 1
+    oracle.gla_forward(xs["q"][:, :16], xs["k"][:, :16], xs["v"][:, :16], xs["a"][:, :16],
+                       xs["g"][:, :16], xs["w"], 4, 4, 0, threads=threads)   # warm
+    passes, tokens = 0, 0
+    t0 = time.perf_counter()
+    while True:
+        d = DIRECTIONS[passes % len(DIRECTIONS)]
+        oracle.gla_forward(xs["q"], xs["k"], xs["v"], xs["a"], xs["g"], xs["w"],
+                           wl.grid_h, wl.grid_w, d, threads=threads)
+        passes += 1
+        tokens += wl.tokens
+        el = time.perf_counter() - t0
+        if el >= budget_s or passes >= 4000:
+            break
+    return {"value": tokens / el / 1e6, "unit": "Mtokens/s", "cores": threads, "kind": "oracle",
+            "sample": "%d full passes (directions cycling L2R,R2L,T2B,B2T) of the %s workload, "
+                      "%.1f s, fp64, OpenMP over (b,h)" % (passes, wl.name, el)}
+
+
+def run_reference(args, ws, rank):
+    """The reference arm: the fp64 CPU oracle on this arm's workload and step definition.
+
+    One step = the four scan directions over H' of the workload's heads, H'
+    chosen (from a timed probe) so that K steps take about two minutes;
+    H' = H is the full workload.  Tokens are counted as processed.
+    """
+    from recurrent_vision_backbone_only_b200 import synth
+    if rank != 0:
+        return
+    import numpy as np
+    import oracle
+    wl = synth.WORKLOADS[WORKLOAD]
+    x = synth.make_inputs(wl)
+    xs = {n: np.asarray(x[n], dtype=np.float64) for n in ("q", "k", "v", "a", "g", "w")}
+    threads = os.cpu_count() or 1
+    K = max(1, args.steps)
+
+    sliced = {}
+
+    def one_step(heads):
+        if heads not in sliced:
+            sliced[heads] = [np.ascontiguousarray(xs[n][:, :, :heads])
+                             for n in ("q", "k", "v", "a", "g")]
+        for d in DIRECTIONS:
+            oracle.gla_forward(*sliced[heads], xs["w"], wl.grid_h, wl.grid_w, d, threads=threads)
+
+    t0 = time.perf_counter()
+    one_step(wl.H)
+    full_s = time.perf_counter() - t0
+    heads = wl.H
+    while heads > 1 and K * full_s * heads / wl.H > 120.0:
+        heads -= 1
+    for _ in range(args.warmup):
+        one_step(heads)
+    t0 = time.perf_counter()
+    done = 0
+    for _ in range(K):
+        one_step(heads)
+        done += 1
+        if time.perf_counter() - t0 > 240.0:
+            break
+    el = time.perf_counter() - t0
+    tokens_per_step = wl.B * heads * wl.L * len(DIRECTIONS)
+    value = done * tokens_per_step / el / 1e6
+    sample = ("%d steps x 4 directions over %d of %d heads of the %s workload, fp64, %d host "
+              "threads" % (done, heads, wl.H, wl.name, threads))
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "Mtokens/s",
+        "n_gpus": args.gpus, "steps": done, "warmup": args.warmup,
+        "ms_per_step": el / done * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": "%s: %dx%d patch grid (L=%d), B=%d, H=%d, d_k=d_v=%d, fp16-rounded "
+                               "inputs; one step = 4 directions" % (wl.name, wl.grid_h, wl.grid_w,
+                                                                   wl.L, wl.B, wl.H, wl.d_k),
+                   "sample_heads": heads},
+        "cpu_baseline": {"value": value, "unit": "Mtokens/s", "cores": threads, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": "Mtokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def run_ours(args, ws, rank, local):
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+    from recurrent_vision_backbone_only_b200 import build as _b, gla, synth
+
+    _b.build()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    wl = synth.WORKLOADS[WORKLOAD]
+    x = synth.make_inputs(wl)
+    gh, gw = wl.grid_h, wl.grid_w
+
+    # rotating pool of input sets, total larger than L2
+    set_bytes = wl.tokens * wl.bytes_per_token
+    n_sets = max(8, math.ceil(2 * L2_BYTES / set_bytes))
+    base = {n: torch.from_numpy(x[n]).to(dev) for n in ("q", "k", "v", "a", "g")}
+    w = torch.from_numpy(x["w"]).to(dev)
+    sets = []
+    for _ in range(n_sets):
+        s = {n: base[n].clone() for n in base}
+        s["out"] = torch.empty_like(base["v"])
+        sets.append(s)
+    launches_per_step = len(DIRECTIONS)
+
+    def step(i):
+        for j, d in enumerate(DIRECTIONS):
+            s = sets[(i * launches_per_step + j) % n_sets]
+            gla.gla_fwd(s["q"], s["k"], s["v"], s["a"], s["g"], w, s["out"], gh, gw, d)
+
+    stream = torch.cuda.Stream(device=dev)
+    torch.cuda.synchronize()
+    with torch.cuda.stream(stream):
+        for i in range(args.warmup):
+            step(i)
+    torch.cuda.synchronize()
+    if gla.get_status(stream) != 0:
+        raise RuntimeError("device status set during warm-up")
+
+    # capture the K timed steps as replays of a graph of G steps (+ a remainder graph)
+    K = args.steps
+    G = min(K, 100)
+    graphs = []
+    with torch.cuda.stream(stream):
+        g_main = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g_main, stream=stream):
+            for i in range(G):
+                step(i)
+        rem = K % G
+        g_rem = None
+        if rem:
+            g_rem = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g_rem, stream=stream):
+                for i in range(rem):
+                    step(i)
+    plan = [g_main] * (K // G) + ([g_rem] if g_rem is not None else [])
+    with torch.cuda.stream(stream):
+        g_main.replay()                     # untimed: graph upload
+        if g_rem is not None:
+            g_rem.replay()
+    torch.cuda.synchronize()
+
+    ev0 = torch.cuda.Event(enable_timing=True)
+    ev1 = torch.cuda.Event(enable_timing=True)
+    if ws > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        with torch.cuda.stream(stream):
+            ev0.record(stream)
+            for gr in plan:
+                gr.replay()
+            ev1.record(stream)
+        torch.cuda.synchronize()
+    if ws > 1:
+        dist.barrier()
+    elapsed_ms = ev0.elapsed_time(ev1)
+    if gla.get_status(stream) != 0:
+        raise RuntimeError("device status set during the timed region")
+    t = torch.tensor([elapsed_ms], dtype=torch.float64, device=dev)
+    if ws > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    max_ms = float(t.item())
+
+    tokens_per_step = wl.tokens * launches_per_step
+    value = tokens_per_step * ws * K / (max_ms / 1e3) / 1e6
+    launch_s = (elapsed_ms / 1e3) / (K * launches_per_step)
+    bytes_per_launch = wl.tokens * wl.bytes_per_token
+    peak, peak_kind = measured_peaks()
+    achieved = bytes_per_launch / launch_s / 1e9
+
+    # ---- e2e through the public host-buffer entry point (H2D + kernel + D2H) ----
+    e2e_steps = max(1, min(args.e2e_steps, K))
+    hx = {n: torch.from_numpy(np.ascontiguousarray(x[n])).pin_memory()
+          for n in ("q", "k", "v", "a", "g", "w")}
+    hout = torch.empty(tuple(x["v"].shape), dtype=torch.float16).pin_memory()
+    with torch.cuda.stream(stream):
+        for d in DIRECTIONS:  # warm the staging buffers
+            gla.gla_fwd_host(hx["q"], hx["k"], hx["v"], hx["a"], hx["g"], hx["w"], hout, gh, gw,
+                             d, stream=stream)
+        if ws > 1:
+            dist.barrier()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for i in range(e2e_steps):
+            for d in DIRECTIONS:
+                gla.gla_fwd_host(hx["q"], hx["k"], hx["v"], hx["a"], hx["g"], hx["w"], hout, gh,
+                                 gw, d, stream=stream)
+        e1.record(stream)
+    torch.cuda.synchronize()
+    te = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=dev)
+    if ws > 1:
+        dist.all_reduce(te, op=dist.ReduceOp.MAX)
+    e2e_ms = float(te.item())
+    h2d = launches_per_step * sum(hx[n].numel() * hx[n].element_size()
+                                  for n in ("q", "k", "v", "a", "g", "w"))
+    d2h = launches_per_step * hout.numel() * hout.element_size()
+    e2e = {"value": tokens_per_step * ws * e2e_steps / (e2e_ms / 1e3) / 1e6, "unit": "Mtokens/s",
+           "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+           "steps": e2e_steps, "ms_per_step": e2e_ms / e2e_steps}
+
+    if rank != 0:
+        return
+    clocks = clk.summary()
+    line = {
+        "metric": METRIC, "value": value, "unit": "Mtokens/s", "n_gpus": ws, "steps": K,
+        "warmup": args.warmup, "ms_per_step": max_ms / K, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f16", "data": "synthetic",
+        "config": {
+            "workload": "%s: %dx%d patch grid (L=%d), B=%d, H=%d, d_k=d_v=%d, fp16 I/O, fp32 "
+                        "accumulation; one step = 4 launches (L2R, R2L, T2B, B2T)"
+                        % (wl.name, gh, gw, wl.L, wl.B, wl.H, wl.d_k),
+            "tokens_per_step": tokens_per_step,
+            "l2": "rotating pool of %d input sets (%.0f MB > 126 MB L2); no flush kernel"
+                  % (n_sets, n_sets * set_bytes / 1e6),
+            "timing": "CUDA-graph replays (graphs of %d steps), CUDA events on the launch "
+                      "stream; warm-up = %d eager steps + one untimed replay" % (G, args.warmup),
+            "parallelism": "replicas" if ws > 1 else "single GPU",
+        },
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                     "frac": achieved / peak, "traffic": profile_traffic(),
+                     "peak_source": "%s (MEASURED_PEAKS.json hbm_gbs)" % peak_kind
+                     if peak_kind == "measured" else "fallback 6.65 TB/s",
+                     "bytes_per_launch": bytes_per_launch,
+                     "launch_us": launch_s * 1e6},
+        "e2e": e2e,
+        "gpu_launches": K * launches_per_step,
+        "clocks": clocks,
+    }
+    if ws == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_oracle_sample(wl, x, args.cpu_seconds)
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse()
+    ws, rank, local = dist_env()
+    if args.impl == "reference":
+        run_reference(args, ws, rank)
+        return
+    if ws > 1:
+        import datetime
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    try:
+        run_ours(args, ws, rank, local)
+    finally:
+        if ws > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

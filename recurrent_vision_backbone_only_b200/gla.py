@@ -1,0 +1,170 @@
+"""ctypes binding of libgla.so -- argument marshalling only.
+
+Every step of the GLA token mixer runs in libgla.so's CUDA kernels; this
+module checks tensor shapes/dtypes, passes raw device pointers and the
+current CUDA stream, and turns status codes into exceptions.  There is no
+fallback: if the library is missing or the device is not an sm_100 GPU the
+call raises.
+
+Tensor layout (token-major, head interleaved): q, k, a: [B, L, H, d_k];
+v, g, out: [B, L, H, d_v]; w: [d_v] float32; L = grid_h * grid_w row-major.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+from typing import Optional
+
+PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(PKG, "libgla.so")
+HEADER = os.path.join(os.path.dirname(PKG), "include", "gla.h")
+
+GLA_OK = 0
+STATUS_NAMES = {0: "GLA_OK", 1: "GLA_ERR_NULL", 2: "GLA_ERR_SHAPE", 3: "GLA_ERR_UNSUPPORTED",
+                4: "GLA_ERR_DIRECTION", 5: "GLA_ERR_ALIAS", 6: "GLA_ERR_CUDA",
+                7: "GLA_ERR_TIMEOUT", 8: "GLA_ERR_RANGE", 9: "GLA_ERR_NO_DEVICE"}
+DIR_L2R, DIR_R2L, DIR_T2B, DIR_B2T, DIR_CYCLE = 0, 1, 2, 3, 4
+
+_lib = None
+
+
+class GLAError(RuntimeError):
+    def __init__(self, code: int, where: str):
+        self.code = code
+        super().__init__("%s failed: %s" % (where, status_string(code)))
+
+
+def load() -> ctypes.CDLL:
+    """Open libgla.so (built in-tree by build.py); raise if it is missing."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError("libgla.so is not built (run recurrent_vision_backbone_only_b200"
+                               ".build or __graft_entry__.build()); there is no fallback path")
+        lib = ctypes.CDLL(LIB_PATH)
+        vp, i, f = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
+        common = [vp] * 7 + [i] * 7
+        lib.gla_fwd.argtypes = common + [vp]
+        lib.gla_fwd_f32.argtypes = common + [vp]
+        lib.gla_fwd_host.argtypes = common + [i, vp]
+        lib.gla_fwd_ex.argtypes = common + [i, i, i, f, vp]
+        lib.gla_get_status.argtypes = [vp, ctypes.POINTER(ctypes.c_int)]
+        lib.gla_status_string.argtypes = [i]
+        lib.gla_status_string.restype = ctypes.c_char_p
+        lib.gla_version.argtypes = []
+        for fn in (lib.gla_fwd, lib.gla_fwd_f32, lib.gla_fwd_host, lib.gla_fwd_ex,
+                   lib.gla_get_status, lib.gla_version):
+            fn.restype = ctypes.c_int
+        _lib = lib
+    return _lib
+
+
+def header_functions() -> list:
+    """Names of the functions declared in include/gla.h."""
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(gla_[a-z0-9_]+)\s*\(", text)))
+
+
+def status_string(code: int) -> str:
+    try:
+        return load().gla_status_string(int(code)).decode()
+    except Exception:  # library missing: still give a readable message
+        return STATUS_NAMES.get(code, "status %d" % code)
+
+
+def _check(rc: int, where: str):
+    if rc != GLA_OK:
+        raise GLAError(rc, where)
+
+
+def _stream_ptr(stream):
+    import torch
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _dims(q, v, grid_h, grid_w):
+    if q.dim() != 4 or v.dim() != 4:
+        raise ValueError("q and v must be [B, L, H, d]")
+    B, L, H, dk = q.shape
+    dv = v.shape[-1]
+    if L != grid_h * grid_w:
+        raise ValueError("L = %d does not equal grid_h*grid_w = %d" % (L, grid_h * grid_w))
+    return int(B), int(H), int(dk), int(dv)
+
+
+def _check_tensors(q, k, v, a, g, w, out, dtype):
+    import torch
+    B, L, H, dk = q.shape
+    dv = v.shape[-1]
+    for name, t, d in (("q", q, dk), ("k", k, dk), ("a", a, dk), ("v", v, dv),
+                       ("g", g, dv), ("out", out, dv)):
+        if tuple(t.shape) != (B, L, H, d):
+            raise ValueError("%s has shape %s, expected %s" % (name, tuple(t.shape), (B, L, H, d)))
+        if t.dtype != dtype or not t.is_cuda or not t.is_contiguous():
+            raise ValueError("%s must be a contiguous CUDA %s tensor" % (name, dtype))
+    if tuple(w.shape) != (dv,) or w.dtype != torch.float32 or not w.is_cuda or not w.is_contiguous():
+        raise ValueError("w must be a contiguous CUDA float32 tensor of shape [d_v]")
+
+
+def gla_fwd(q, k, v, a, g, w, out, grid_h: int, grid_w: int, direction: int, stream=None):
+    """u = GLA(q, k, v; gate a) with SiLU(g) * RMSNorm epilogue, into `out` (fp16 or fp32)."""
+    import torch
+    B, H, dk, dv = _dims(q, v, grid_h, grid_w)
+    _check_tensors(q, k, v, a, g, w, out, q.dtype)
+    args = [ctypes.c_void_p(t.data_ptr()) for t in (q, k, v, a, g, w, out)]
+    args += [B, H, grid_h, grid_w, dk, dv, direction, _stream_ptr(stream)]
+    if q.dtype == torch.float16:
+        _check(load().gla_fwd(*args), "gla_fwd")
+    elif q.dtype == torch.float32:
+        _check(load().gla_fwd_f32(*args), "gla_fwd_f32")
+    else:
+        raise ValueError("q must be float16 or float32")
+    return out
+
+
+def gla_fwd_ex(q, k, v, a, g, w, out, grid_h: int, grid_w: int, direction: int,
+               chunk: int = 0, segments: int = 0, eps: float = 1e-6, stream=None):
+    """gla_fwd with the chunk length, segments per pair and epsilon exposed (tests)."""
+    import torch
+    B, H, dk, dv = _dims(q, v, grid_h, grid_w)
+    _check_tensors(q, k, v, a, g, w, out, q.dtype)
+    dtype = {torch.float16: 0, torch.float32: 1}[q.dtype]
+    args = [ctypes.c_void_p(t.data_ptr()) for t in (q, k, v, a, g, w, out)]
+    args += [B, H, grid_h, grid_w, dk, dv, direction, dtype, chunk, segments,
+             ctypes.c_float(eps), _stream_ptr(stream)]
+    _check(load().gla_fwd_ex(*args), "gla_fwd_ex")
+    return out
+
+
+def gla_fwd_host(q, k, v, a, g, w, out, grid_h: int, grid_w: int, direction: int, stream=None):
+    """The same operation on HOST tensors (CPU, ideally pinned); synchronous."""
+    import torch
+    B, L, H, dk = q.shape
+    dv = v.shape[-1]
+    if L != grid_h * grid_w:
+        raise ValueError("L must equal grid_h*grid_w")
+    for t in (q, k, v, a, g, w, out):
+        if t.is_cuda or not t.is_contiguous():
+            raise ValueError("gla_fwd_host takes contiguous host tensors")
+    dtype = {torch.float16: 0, torch.float32: 1}[q.dtype]
+    args = [ctypes.c_void_p(t.data_ptr()) for t in (q, k, v, a, g, w, out)]
+    args += [int(B), int(H), grid_h, grid_w, int(dk), int(dv), direction, dtype,
+             _stream_ptr(stream)]
+    _check(load().gla_fwd_host(*args), "gla_fwd_host")
+    return out
+
+
+def get_status(stream=None) -> int:
+    """Synchronise `stream` and return (and clear) the latched device status."""
+    val = ctypes.c_int(0)
+    _check(load().gla_get_status(_stream_ptr(stream), ctypes.byref(val)), "gla_get_status")
+    return val.value
+
+
+def raw_call(name: str, *args) -> int:
+    """Call an entry point with raw ctypes-compatible arguments (host-side error tests)."""
+    return getattr(load(), name)(*args)

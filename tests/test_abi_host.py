@@ -1,0 +1,100 @@
+"""Host-side checks of the C ABI (no GPU needed).
+
+The library must load on a machine without a GPU, export every function
+declared in include/gla.h, and reject bad arguments synchronously with the
+documented status codes before touching CUDA.
+"""
+import ctypes
+import os
+
+import pytest
+
+from recurrent_vision_backbone_only_b200 import build, gla
+
+ALIGNED = [0x10000 * (i + 1) for i in range(7)]   # fake, never dereferenced
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return gla.load()
+
+
+def test_exports_every_declared_symbol(lib):
+    names = gla.header_functions()
+    assert {"gla_fwd", "gla_fwd_f32", "gla_fwd_ex", "gla_fwd_host", "gla_get_status",
+            "gla_status_string", "gla_version"} <= set(names)
+    for n in names:
+        assert hasattr(lib, n), n
+
+
+def test_exports_via_nm():
+    import subprocess
+    build.build()
+    out = subprocess.run(["nm", "-D", "--defined-only", gla.LIB_PATH], capture_output=True,
+                         text=True, check=True).stdout
+    exported = {line.split()[-1] for line in out.splitlines() if line.strip()}
+    for n in gla.header_functions():
+        assert n in exported, n
+
+
+def test_version_and_strings(lib):
+    assert lib.gla_version() >= 100
+    for code in range(10):
+        s = gla.status_string(code)
+        assert s.startswith(gla.STATUS_NAMES[code])
+    assert "unknown" in gla.status_string(99)
+
+
+def call(fn, ptrs=None, B=1, H=2, gh=4, gw=5, dk=64, dv=64, direction=0, extra=()):
+    ptrs = ALIGNED if ptrs is None else ptrs
+    args = [ctypes.c_void_p(p) if p is not None else None for p in ptrs]
+    args += [B, H, gh, gw, dk, dv, direction, *extra, None]
+    return gla.raw_call(fn, *args)
+
+
+@pytest.mark.parametrize("fn,extra", [("gla_fwd", ()), ("gla_fwd_f32", ()),
+                                      ("gla_fwd_host", (0,)),
+                                      ("gla_fwd_ex", (0, 0, 0, ctypes.c_float(1e-6)))])
+def test_argument_errors(lib, fn, extra):
+    for i in range(7):
+        ptrs = list(ALIGNED)
+        ptrs[i] = None
+        assert call(fn, ptrs, extra=extra) == 1            # GLA_ERR_NULL
+    for kw in (dict(B=0), dict(H=-1), dict(gh=0), dict(gw=0)):
+        assert call(fn, extra=extra, **kw) == 2            # GLA_ERR_SHAPE
+    assert call(fn, extra=extra, gh=1 << 16, gw=1 << 15) == 2
+    for d in (16, 48, 96, 256):
+        assert call(fn, extra=extra, dk=d) == 3            # GLA_ERR_UNSUPPORTED
+        assert call(fn, extra=extra, dv=d) == 3
+    for d in (-1, 5, 100):
+        assert call(fn, extra=extra, direction=d) == 4     # GLA_ERR_DIRECTION
+    if fn != "gla_fwd_host":
+        mis = list(ALIGNED)
+        mis[2] += 8
+        assert call(fn, mis, extra=extra) == 3             # misaligned
+        alias = list(ALIGNED)
+        alias[6] = alias[0]                                # out == q
+        assert call(fn, alias, extra=extra) == 5           # GLA_ERR_ALIAS
+
+
+def test_ex_rejects_bad_schedule(lib):
+    bad = [(5, 0, 0), (0, 0, 17), (0, -1, 0), (1, 0, -2)]   # dtype, chunk, segments
+    for dtype, chunk, segs in bad:
+        rc = call("gla_fwd_ex", extra=(dtype, chunk, segs, ctypes.c_float(1e-6)))
+        assert rc == 3 or (rc == 9 and dtype in (0, 1)), (dtype, chunk, segs, rc)
+
+
+def test_no_device_is_reported_not_faked(lib):
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present")
+    assert call("gla_fwd") == 9                            # GLA_ERR_NO_DEVICE
+    assert call("gla_fwd_f32") == 9
+
+
+def test_binding_raises_when_library_missing(monkeypatch, tmp_path):
+    monkeypatch.setattr(gla, "_lib", None)
+    monkeypatch.setattr(gla, "LIB_PATH", os.path.join(str(tmp_path), "missing.so"))
+    with pytest.raises(RuntimeError, match="no fallback"):
+        gla.load()

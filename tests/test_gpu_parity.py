@@ -1,0 +1,174 @@
+"""GPU parity: libgla.so (through the C ABI) against the fp64 CPU oracle.
+
+Tolerances (on u, the kernel's final output): fp16 I/O with fp32
+accumulation -- max-abs <= 1e-2 and relative L2 <= 2e-3; fp32 I/O -- max-abs
+<= 1e-5.  Every workload runs at its full size in the launch configuration
+the bench uses; the stress workload (L = 16384, d = 128) is compared on
+sampled (b, h) pairs, each of which the oracle recomputes from scratch.
+"""
+import numpy as np
+import pytest
+
+import oracle
+from recurrent_vision_backbone_only_b200 import gla, synth
+
+pytestmark = pytest.mark.gpu
+
+TOL = {"f16": dict(max_abs=1e-2, rel_l2=2e-3), "f32": dict(max_abs=1e-5, rel_l2=1e-5)}
+
+
+def torch_dev(x):
+    import torch
+    return torch.from_numpy(np.ascontiguousarray(x)).cuda()
+
+
+def run_gpu(x, gh, gw, direction, chunk=0, segments=0, eps=1e-6):
+    import torch
+    t = {n: torch_dev(x[n]) for n in ("q", "k", "v", "a", "g", "w")}
+    out = torch.empty_like(t["v"])
+    if chunk or segments or eps != 1e-6:
+        gla.gla_fwd_ex(t["q"], t["k"], t["v"], t["a"], t["g"], t["w"], out, gh, gw, direction,
+                       chunk=chunk, segments=segments, eps=eps)
+    else:
+        gla.gla_fwd(t["q"], t["k"], t["v"], t["a"], t["g"], t["w"], out, gh, gw, direction)
+    torch.cuda.synchronize()
+    assert gla.get_status() == 0
+    return out.cpu().numpy()
+
+
+def errors(u, ref):
+    u = u.astype(np.float64)
+    d = u - ref
+    return float(np.max(np.abs(d))), float(np.linalg.norm(d) / max(np.linalg.norm(ref), 1e-30))
+
+
+def assert_close(u, ref, dtype):
+    assert np.all(np.isfinite(u))
+    max_abs, rel = errors(u, ref)
+    tol = TOL[dtype]
+    assert max_abs <= tol["max_abs"] and rel <= tol["rel_l2"], (max_abs, rel)
+
+
+def oracle_ref(x, gh, gw, direction):
+    return oracle.gla_forward(x["q"], x["k"], x["v"], x["a"], x["g"], x["w"], gh, gw, direction)
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib(cuda_ok):
+    from recurrent_vision_backbone_only_b200 import build
+    build.build()
+    gla.load()
+
+
+@pytest.mark.parametrize("direction", [0, 1, 2, 3])
+def test_tiny_fp32(direction):
+    wl = synth.WORKLOADS["tiny"]
+    x = synth.make_inputs(wl)
+    u = run_gpu(x, wl.grid_h, wl.grid_w, direction, chunk=wl.chunk)
+    assert_close(u, oracle_ref(x, wl.grid_h, wl.grid_w, direction), "f32")
+    u2 = run_gpu(x, wl.grid_h, wl.grid_w, direction)
+    assert_close(u2, oracle_ref(x, wl.grid_h, wl.grid_w, direction), "f32")
+
+
+@pytest.mark.parametrize("name", ["gtr640", "highres"])
+def test_full_workloads_all_directions(name):
+    wl = synth.WORKLOADS[name]
+    x = synth.make_inputs(wl)
+    for d in wl.directions:
+        assert_close(run_gpu(x, wl.grid_h, wl.grid_w, d), oracle_ref(x, wl.grid_h, wl.grid_w, d),
+                     wl.dtype)
+
+
+def test_batched_cycle():
+    wl = synth.WORKLOADS["batched"]
+    x = synth.make_inputs(wl)
+    u = run_gpu(x, wl.grid_h, wl.grid_w, 4)
+    assert_close(u, oracle_ref(x, wl.grid_h, wl.grid_w, 4), wl.dtype)
+
+
+@pytest.mark.parametrize("direction", [2, 3])
+def test_stress_sampled_pairs(direction):
+    wl = synth.WORKLOADS["stress"]
+    x = synth.make_inputs(wl)
+    u = run_gpu(x, wl.grid_h, wl.grid_w, direction)
+    assert np.all(np.isfinite(u.astype(np.float32)))
+    for b, h in [(0, 0), (1, 5)]:
+        xs = {n: x[n][b:b + 1, :, h:h + 1] for n in ("q", "k", "v", "a", "g")}
+        xs["w"] = x["w"]
+        ref = oracle_ref(xs, wl.grid_h, wl.grid_w, direction)
+        assert_close(u[b:b + 1, :, h:h + 1], ref, wl.dtype)
+
+
+@pytest.mark.parametrize("dtype", ["f16", "f32"])
+def test_chunk_and_segment_invariance(dtype):
+    wl = synth.WORKLOADS["gtr640"].with_(H=2, dtype=dtype, grid_h=24, grid_w=37)
+    x = synth.make_inputs(wl)
+    gh, gw = wl.grid_h, wl.grid_w
+    ref = oracle_ref(x, gh, gw, 1)
+    outs = []
+    for chunk in (16, 32, 64):
+        for segs in (1, 3, 16):
+            u = run_gpu(x, gh, gw, 1, chunk=chunk, segments=segs)
+            assert_close(u, ref, dtype)
+            outs.append(u.astype(np.float64))
+    for u in outs[1:]:
+        assert_close(u, outs[0], dtype)
+
+
+@pytest.mark.parametrize("gh,gw,dk,dv", [(1, 1, 64, 64), (7, 9, 64, 64), (1, 33, 32, 128),
+                                         (17, 3, 128, 32), (5, 5, 128, 128)])
+@pytest.mark.parametrize("dtype", ["f16", "f32"])
+def test_ragged_and_mixed_dims(gh, gw, dk, dv, dtype):
+    wl = synth.WORKLOADS["gtr640"].with_(grid_h=gh, grid_w=gw, d_k=dk, d_v=dv, B=2, H=3,
+                                         dtype=dtype, a_std=3.0, a_mean=0.0)
+    x = synth.make_inputs(wl, seed=gh * 100 + gw)
+    for d in (0, 3, 4):
+        assert_close(run_gpu(x, gh, gw, d), oracle_ref(x, gh, gw, d), dtype)
+
+
+@pytest.mark.parametrize("dtype", ["f16", "f32"])
+def test_extreme_gates(dtype):
+    # gamma ~ 0 (a = -30) and gamma ~ 1 (a = +30) mixed per channel and token
+    wl = synth.WORKLOADS["gtr640"].with_(grid_h=12, grid_w=12, H=2, dtype=dtype)
+    x = synth.make_inputs(wl, seed=3)
+    rng = np.random.default_rng(3)
+    x["a"] = np.where(rng.random(x["a"].shape) < 0.5, -30.0, 30.0).astype(x["a"].dtype)
+    for d in (0, 2):
+        assert_close(run_gpu(x, 12, 12, d), oracle_ref(x, 12, 12, d), dtype)
+
+
+def test_zero_keys_exact_zero():
+    wl = synth.WORKLOADS["gtr640"].with_(grid_h=10, grid_w=13, H=2)
+    x = synth.make_inputs(wl, seed=4)
+    x["k"][:] = 0
+    u = run_gpu(x, 10, 13, 1)
+    assert np.all(u == 0)
+
+
+def test_many_pairs_small_grid():
+    wl = synth.WORKLOADS["gtr640"].with_(grid_h=4, grid_w=4, B=64, H=4)
+    x = synth.make_inputs(wl, seed=5)
+    assert_close(run_gpu(x, 4, 4, 4), oracle_ref(x, 4, 4, 4), "f16")
+
+
+def test_host_entry_matches_device_entry():
+    import torch
+    wl = synth.WORKLOADS["gtr640"].with_(grid_h=16, grid_w=20, H=3)
+    x = synth.make_inputs(wl, seed=6)
+    dev = run_gpu(x, 16, 20, 2)
+    h = {n: torch.from_numpy(np.ascontiguousarray(x[n])).pin_memory()
+         for n in ("q", "k", "v", "a", "g", "w")}
+    out = torch.empty_like(h["v"]).pin_memory()
+    gla.gla_fwd_host(h["q"], h["k"], h["v"], h["a"], h["g"], h["w"], out, 16, 20, 2)
+    np.testing.assert_array_equal(out.numpy(), dev)
+
+
+def test_eps_is_honoured():
+    # tiny inputs: |o|^2 is comparable to eps, so eps changes the answer
+    wl = synth.WORKLOADS["tiny"].with_(qkv_std=0.02)
+    x = synth.make_inputs(wl)
+    for eps in (1e-6, 1e-3):
+        u = run_gpu(x, 8, 8, 0, eps=eps)
+        ref = oracle.gla_forward(x["q"], x["k"], x["v"], x["a"], x["g"], x["w"], 8, 8, 0,
+                                 eps=eps)
+        assert_close(u, ref, "f32")
