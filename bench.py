@@ -362,6 +362,7 @@ def run_ours(args, ws, rank, local):
             "timing": "CUDA-graph replays (graphs of %d steps), CUDA events on the launch "
                       "stream; warm-up = %d eager steps + one untimed replay" % (G, args.warmup),
             "parallelism": "replicas" if ws > 1 else "single GPU",
+            "schedule": gla.plan(wl.B, wl.H, gh, gw, wl.d_k, wl.d_v, 0),
         },
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": achieved / peak, "traffic": profile_traffic(),

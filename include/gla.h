@@ -133,6 +133,32 @@ const char *gla_status_string(int code);
 /* gla_version -- library version, major*10000 + minor*100 + patch. */
 int gla_version(void);
 
+/*
+ * gla_plan -- the schedule gla_fwd (dtype 0) / gla_fwd_f32 (dtype 1) would
+ * use for these shapes on the current device, without launching anything:
+ * *kernel = 1 (tensor-core kernel) or 2 (CUDA-core kernel), *segments = CTAs
+ * (one thread-block cluster) per (b, h) pair, *seg_len = scan positions per
+ * segment, *ctas = total CTAs, *max_active_clusters = clusters of that shape
+ * the device can hold at once.  Same argument errors as gla_fwd.
+ */
+int gla_plan(int B, int H, int grid_h, int grid_w, int d_k, int d_v, int dtype, int *kernel,
+             int *segments, int *seg_len, int *ctas, int *max_active_clusters);
+
+/*
+ * gla_selftest_mma -- diagnostic: runs ONE of the tensor-core kernel's four
+ * matrix products on a single CTA, with the kernel's own shared-memory
+ * layouts and descriptors, on row-major float32 DEVICE arrays:
+ *   kind 0  D[128][128] = A[128][64] * B[128][64]^T   (split tf32: each operand is
+ *           held as tf32 high + low parts, three products; ~fp32 accuracy)
+ *   kind 1  D[64][64]   = A[128][64]^T * B[128][64]   (fp16 operands, the state product)
+ *   kind 2  D[128][64]  = A[128][128] * B[128][64]    (fp16 operands, P * V)
+ *   kind 3  D[128][64]  = A[128][64] * B[64][64]^T    (tf32, the inter-chunk product)
+ * Inputs are rounded to the operand type (tf32 or fp16; kind 0 splits them)
+ * on the way in; accumulation is fp32.  Asynchronous on `stream`.  Returns GLA_ERR_UNSUPPORTED
+ * for another kind.  Not part of the operation itself.
+ */
+int gla_selftest_mma(int kind, const float *A, const float *B, float *D, void *stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -14,6 +14,7 @@
 #include "gla.h"
 #include "gla_common.cuh"
 #include "gla_simt.cuh"
+#include "gla_tc.cuh"
 
 #define GLA_VERSION_CODE 100  // 0.1.0
 
@@ -95,76 +96,98 @@ int current_device_info(DeviceInfo *info) {
 
 int ceil_div(long long a, long long b) { return (int)((a + b - 1) / b); }
 
-// True when at least one cluster of this launch shape can be resident.
+// Launch schedule: `segs` CTAs (one thread-block cluster) per (b, h) pair,
+// each owning `seg_len` consecutive scan positions.
+struct Plan {
+    int kernel = 0;            // 1 = tensor-core kernel, 2 = CUDA-core kernel
+    int segs = 1;
+    int seg_len = 0;
+    int chunk = 0;             // tokens per chunk (CUDA-core) / largest chunk (tensor-core)
+    size_t smem = 0;
+    int max_active_clusters = 0;
+    cudaLaunchConfig_t cfg{};
+    cudaLaunchAttribute attr[1];
+};
+
+void configure_launch(Plan &pl, int n_pairs, int threads, cudaStream_t st) {
+    pl.cfg = cudaLaunchConfig_t{};
+    pl.cfg.gridDim = dim3((unsigned)(n_pairs * pl.segs), 1, 1);
+    pl.cfg.blockDim = dim3((unsigned)threads, 1, 1);
+    pl.cfg.dynamicSmemBytes = pl.smem;
+    pl.cfg.stream = st;
+    pl.attr[0].id = cudaLaunchAttributeClusterDimension;
+    pl.attr[0].val.clusterDim.x = (unsigned)pl.segs;
+    pl.attr[0].val.clusterDim.y = 1;
+    pl.attr[0].val.clusterDim.z = 1;
+    pl.cfg.attrs = pl.attr;
+    pl.cfg.numAttrs = 1;
+}
+
+// Pick the segment count (auto when segs <= 0), shrinking it until a cluster
+// fits on the device.  `unit` is the granularity of a segment's length.
 template <typename K>
-bool cluster_fits(K kern, const cudaLaunchConfig_t &cfg) {
-    int n = 0;
-    if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess) {
+int make_plan(K kern, Plan &pl, int L, int n_pairs, int segs, int unit, int threads,
+              cudaStream_t st, const DeviceInfo &di) {
+    if (pl.smem > (size_t)di.max_smem_optin) return GLA_ERR_UNSUPPORTED;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)pl.smem) !=
+            cudaSuccess ||
+        cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) != cudaSuccess) {
         cudaGetLastError();
-        return false;
+        return GLA_ERR_CUDA;
     }
-    return n > 0;
+    const bool auto_segs = segs <= 0;
+    if (auto_segs) {
+        segs = di.sms / n_pairs;
+        segs = segs < 1 ? 1 : (segs > 16 ? 16 : segs);
+    }
+    if (segs > 16) return GLA_ERR_UNSUPPORTED;
+    const int n_units = ceil_div(L, unit);
+    auto plan_segs = [&](int s) {  // whole units per segment, none empty
+        if (s > n_units) s = n_units;
+        pl.seg_len = ceil_div(n_units, s) * unit;
+        pl.segs = ceil_div(L, pl.seg_len);
+    };
+    plan_segs(segs);
+    configure_launch(pl, n_pairs, threads, st);
+    for (;;) {
+        int n = 0;
+        if (cudaOccupancyMaxActiveClusters(&n, kern, &pl.cfg) != cudaSuccess) {
+            cudaGetLastError();
+            n = 0;
+        }
+        pl.max_active_clusters = n;
+        if (n > 0) return GLA_OK;
+        if (!auto_segs || pl.segs == 1) return GLA_ERR_UNSUPPORTED;
+        plan_segs((pl.segs + 1) / 2);
+        configure_launch(pl, n_pairs, threads, st);
+    }
 }
 
 // ---------------------------------------------------------------- SIMT path
 template <typename T, int DK, int DV>
-int launch_simt_t(const Args &x, int chunk, int segs, float eps, cudaStream_t st,
-                  const DeviceInfo &di) {
+int run_simt_t(const Args &x, int chunk, int segs, float eps, cudaStream_t st,
+               const DeviceInfo &di, Plan *query) {
     auto kern = gla_simt_kernel<T, DK, DV>;
     const int L = x.gh * x.gw;
     const int n_pairs = x.B * x.H;
     if (chunk <= 0) chunk = 16;
     if (chunk % 16 != 0 || chunk > 64) return GLA_ERR_UNSUPPORTED;
-    const size_t smem = simt_smem_floats(DK, DV, chunk) * sizeof(float);
-    if (smem > (size_t)di.max_smem_optin) return GLA_ERR_UNSUPPORTED;
-    const bool auto_segs = segs <= 0;
-    if (auto_segs) {
-        segs = ceil_div(di.sms, n_pairs);
-        segs = segs < 1 ? 1 : (segs > 16 ? 16 : segs);
-    }
-    if (segs > 16) return GLA_ERR_UNSUPPORTED;
-    const int n_chunks = ceil_div(L, chunk);
-    int seg_len = 0;
-    auto plan = [&](int s) {  // whole chunks per segment, no empty segment
-        if (s > n_chunks) s = n_chunks;
-        seg_len = ceil_div(n_chunks, s) * chunk;
-        return ceil_div(L, seg_len);
-    };
-    segs = plan(segs);
-
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess ||
-        cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) != cudaSuccess) {
-        cudaGetLastError();
-        return GLA_ERR_CUDA;
-    }
-
-    cudaLaunchConfig_t cfg = {};
-    cudaLaunchAttribute attr[1];
-    auto configure = [&](int s) {
-        cfg = cudaLaunchConfig_t{};
-        cfg.gridDim = dim3((unsigned)(n_pairs * s), 1, 1);
-        cfg.blockDim = dim3(kSimtThreads, 1, 1);
-        cfg.dynamicSmemBytes = smem;
-        cfg.stream = st;
-        attr[0].id = cudaLaunchAttributeClusterDimension;
-        attr[0].val.clusterDim.x = (unsigned)s;
-        attr[0].val.clusterDim.y = 1;
-        attr[0].val.clusterDim.z = 1;
-        cfg.attrs = attr;
-        cfg.numAttrs = 1;
-    };
-    configure(segs);
-    while (!cluster_fits(kern, cfg)) {
-        if (!auto_segs || segs == 1) return GLA_ERR_UNSUPPORTED;
-        segs = plan((segs + 1) / 2);
-        configure(segs);
+    Plan pl;
+    pl.kernel = 2;
+    pl.chunk = chunk;
+    pl.smem = simt_smem_floats(DK, DV, chunk) * sizeof(float);
+    int rc = make_plan(kern, pl, L, n_pairs, segs, chunk, kSimtThreads, st, di);
+    if (rc != GLA_OK) return rc;
+    if (query) {
+        *query = pl;
+        return GLA_OK;
     }
     SimtParams p;
     p.q = x.q; p.k = x.k; p.v = x.v; p.a = x.a; p.g = x.g; p.w = x.w; p.out = x.out;
     p.B = x.B; p.H = x.H; p.gh = x.gh; p.gw = x.gw; p.L = L;
-    p.dir = x.dir; p.chunk = chunk; p.segs = segs; p.seg_len = seg_len;
+    p.dir = x.dir; p.chunk = chunk; p.segs = pl.segs; p.seg_len = pl.seg_len;
     p.eps = eps; p.scale = 1.0f / sqrtf((float)DK);
-    if (cudaLaunchKernelEx(&cfg, kern, p) != cudaSuccess) {
+    if (cudaLaunchKernelEx(&pl.cfg, kern, p) != cudaSuccess) {
         cudaGetLastError();
         return GLA_ERR_CUDA;
     }
@@ -172,35 +195,73 @@ int launch_simt_t(const Args &x, int chunk, int segs, float eps, cudaStream_t st
 }
 
 template <typename T, int DK>
-int launch_simt_dv(const Args &x, int chunk, int segs, float eps, cudaStream_t st, const DeviceInfo &di) {
+int run_simt_dv(const Args &x, int chunk, int segs, float eps, cudaStream_t st, const DeviceInfo &di,
+                Plan *query) {
     switch (x.dv) {
-    case 32: return launch_simt_t<T, DK, 32>(x, chunk, segs, eps, st, di);
-    case 64: return launch_simt_t<T, DK, 64>(x, chunk, segs, eps, st, di);
-    default: return launch_simt_t<T, DK, 128>(x, chunk, segs, eps, st, di);
+    case 32: return run_simt_t<T, DK, 32>(x, chunk, segs, eps, st, di, query);
+    case 64: return run_simt_t<T, DK, 64>(x, chunk, segs, eps, st, di, query);
+    default: return run_simt_t<T, DK, 128>(x, chunk, segs, eps, st, di, query);
     }
 }
 
 template <typename T>
-int launch_simt(const Args &x, int chunk, int segs, float eps, cudaStream_t st, const DeviceInfo &di) {
+int run_simt(const Args &x, int chunk, int segs, float eps, cudaStream_t st, const DeviceInfo &di,
+             Plan *query) {
     switch (x.dk) {
-    case 32: return launch_simt_dv<T, 32>(x, chunk, segs, eps, st, di);
-    case 64: return launch_simt_dv<T, 64>(x, chunk, segs, eps, st, di);
-    default: return launch_simt_dv<T, 128>(x, chunk, segs, eps, st, di);
+    case 32: return run_simt_dv<T, 32>(x, chunk, segs, eps, st, di, query);
+    case 64: return run_simt_dv<T, 64>(x, chunk, segs, eps, st, di, query);
+    default: return run_simt_dv<T, 128>(x, chunk, segs, eps, st, di, query);
     }
+}
+
+// ---------------------------------------------------------- tensor-core path
+// fp16 I/O with d_k = d_v = 64.  One cluster of `segs` CTAs per (b, h) pair.
+int run_tc(const Args &x, int chunk, int segs, float eps, cudaStream_t st, const DeviceInfo &di,
+           Plan *query) {
+    auto kern = tc::gla_tc_kernel<64>;
+    const int L = x.gh * x.gw;
+    const int n_pairs = x.B * x.H;
+    if (chunk <= 0) chunk = tc::kC;
+    if (chunk % 16 != 0 || chunk > tc::kC) return GLA_ERR_UNSUPPORTED;
+    Plan pl;
+    pl.kernel = 1;
+    pl.chunk = chunk;
+    pl.smem = tc::kSmemBytes;
+    int rc = make_plan(kern, pl, L, n_pairs, segs, 1, tc::kThreads, st, di);
+    if (rc != GLA_OK) return rc;
+    if (query) {
+        *query = pl;
+        return GLA_OK;
+    }
+    tc::Params p;
+    p.q = static_cast<const __half *>(x.q); p.k = static_cast<const __half *>(x.k);
+    p.v = static_cast<const __half *>(x.v); p.a = static_cast<const __half *>(x.a);
+    p.g = static_cast<const __half *>(x.g); p.w = x.w; p.out = static_cast<__half *>(x.out);
+    p.B = x.B; p.H = x.H; p.gh = x.gh; p.gw = x.gw; p.L = L; p.dir = x.dir;
+    p.segs = pl.segs; p.seg_len = pl.seg_len; p.chunk_max = chunk;
+    p.eps = eps; p.scale = 0.125f;  // 64^{-1/2}
+    if (cudaLaunchKernelEx(&pl.cfg, kern, p) != cudaSuccess) {
+        cudaGetLastError();
+        return GLA_ERR_CUDA;
+    }
+    return GLA_OK;
 }
 
 // ------------------------------------------------------------- dispatch
 constexpr float kEps = 1e-6f;
 
-int run(const Args &x, int dtype, int chunk, int segs, float eps, cudaStream_t st) {
+// Validate, then launch (query == nullptr) or only report the schedule.
+int run(const Args &x, int dtype, int chunk, int segs, float eps, cudaStream_t st,
+        Plan *query = nullptr) {
     int rc = validate(x);
     if (rc != GLA_OK) return rc;
     if (segs < 0 || segs > 16 || chunk < 0 || !(eps >= 0.0f)) return GLA_ERR_UNSUPPORTED;
     DeviceInfo di;
     rc = current_device_info(&di);
     if (rc != GLA_OK) return rc;
-    if (dtype == 1) return launch_simt<float>(x, chunk, segs, eps, st, di);
-    return launch_simt<__half>(x, chunk, segs, eps, st, di);
+    if (dtype == 1) return run_simt<float>(x, chunk, segs, eps, st, di, query);
+    if (x.dk == 64 && x.dv == 64) return run_tc(x, chunk, segs, eps, st, di, query);
+    return run_simt<__half>(x, chunk, segs, eps, st, di, query);
 }
 
 Args make_args(const void *q, const void *k, const void *v, const void *a, const void *g,
@@ -342,5 +403,48 @@ const char *gla_status_string(int code) {
 }
 
 int gla_version(void) { return GLA_VERSION_CODE; }
+
+int gla_plan(int B, int H, int grid_h, int grid_w, int d_k, int d_v, int dtype, int *kernel,
+             int *segments, int *seg_len, int *ctas, int *max_active_clusters) {
+    if (!kernel || !segments || !seg_len || !ctas || !max_active_clusters) return GLA_ERR_NULL;
+    if (dtype != 0 && dtype != 1) return GLA_ERR_UNSUPPORTED;
+    // placeholder, 16-byte aligned, non-overlapping addresses: only shapes are used
+    static const uintptr_t kFake = 1u << 20;
+    const size_t span = (size_t)B * grid_h * grid_w * H * 128 * 4 + 4096;
+    const uintptr_t base = kFake;
+    const Args x = make_args(reinterpret_cast<const void *>(base), reinterpret_cast<const void *>(base + span),
+                             reinterpret_cast<const void *>(base + 2 * span),
+                             reinterpret_cast<const void *>(base + 3 * span),
+                             reinterpret_cast<const void *>(base + 4 * span),
+                             reinterpret_cast<const float *>(base + 5 * span),
+                             reinterpret_cast<void *>(base + 6 * span), B, H, grid_h, grid_w, d_k, d_v,
+                             0, dtype == 0 ? 2 : 4);
+    Plan pl;
+    const int rc = run(x, dtype, 0, 0, kEps, nullptr, &pl);
+    if (rc != GLA_OK) return rc;
+    *kernel = pl.kernel;
+    *segments = pl.segs;
+    *seg_len = pl.seg_len;
+    *ctas = B * H * pl.segs;
+    *max_active_clusters = pl.max_active_clusters;
+    return GLA_OK;
+}
+
+int gla_selftest_mma(int kind, const float *A, const float *B, float *D, void *stream) {
+    if (!A || !B || !D) return GLA_ERR_NULL;
+    if (kind < 0 || kind > 3) return GLA_ERR_UNSUPPORTED;
+    DeviceInfo di;
+    int rc = current_device_info(&di);
+    if (rc != GLA_OK) return rc;
+    auto kern = tc::gla_tc_selftest_kernel;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tc::kSmemBytes) !=
+        cudaSuccess) {
+        cudaGetLastError();
+        return GLA_ERR_CUDA;
+    }
+    kern<<<1, tc::kThreads, tc::kSmemBytes, static_cast<cudaStream_t>(stream)>>>(kind, A, B, D);
+    if (cudaGetLastError() != cudaSuccess) return GLA_ERR_CUDA;
+    return GLA_OK;
+}
 
 }  // extern "C"

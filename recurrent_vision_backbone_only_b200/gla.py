@@ -53,8 +53,12 @@ def load() -> ctypes.CDLL:
         lib.gla_status_string.argtypes = [i]
         lib.gla_status_string.restype = ctypes.c_char_p
         lib.gla_version.argtypes = []
+        lib.gla_selftest_mma.argtypes = [i, vp, vp, vp, vp]
+        ip = ctypes.POINTER(ctypes.c_int)
+        lib.gla_plan.argtypes = [i] * 7 + [ip] * 5
+        lib.gla_plan.restype = ctypes.c_int
         for fn in (lib.gla_fwd, lib.gla_fwd_f32, lib.gla_fwd_host, lib.gla_fwd_ex,
-                   lib.gla_get_status, lib.gla_version):
+                   lib.gla_get_status, lib.gla_version, lib.gla_selftest_mma):
             fn.restype = ctypes.c_int
         _lib = lib
     return _lib
@@ -156,6 +160,17 @@ def gla_fwd_host(q, k, v, a, g, w, out, grid_h: int, grid_w: int, direction: int
              _stream_ptr(stream)]
     _check(load().gla_fwd_host(*args), "gla_fwd_host")
     return out
+
+
+def plan(B: int, H: int, grid_h: int, grid_w: int, d_k: int = 64, d_v: int = 64,
+         dtype: int = 0) -> dict:
+    """The launch schedule the library picks for these shapes on the current device."""
+    vals = [ctypes.c_int(0) for _ in range(5)]
+    _check(load().gla_plan(B, H, grid_h, grid_w, d_k, d_v, dtype, *[ctypes.byref(v) for v in vals]),
+           "gla_plan")
+    kernel, segs, seg_len, ctas, mac = (v.value for v in vals)
+    return {"kernel": {1: "tensor-core", 2: "cuda-core"}.get(kernel, kernel), "segments": segs,
+            "seg_len": seg_len, "ctas": ctas, "max_active_clusters": mac}
 
 
 def get_status(stream=None) -> int:

@@ -23,7 +23,7 @@ def lib():
 def test_exports_every_declared_symbol(lib):
     names = gla.header_functions()
     assert {"gla_fwd", "gla_fwd_f32", "gla_fwd_ex", "gla_fwd_host", "gla_get_status",
-            "gla_status_string", "gla_version"} <= set(names)
+            "gla_status_string", "gla_version", "gla_selftest_mma"} <= set(names)
     for n in names:
         assert hasattr(lib, n), n
 
@@ -76,6 +76,14 @@ def test_argument_errors(lib, fn, extra):
         alias = list(ALIGNED)
         alias[6] = alias[0]                                # out == q
         assert call(fn, alias, extra=extra) == 5           # GLA_ERR_ALIAS
+
+
+def test_selftest_rejects_bad_arguments(lib):
+    f = lib.gla_selftest_mma
+    f.argtypes = [ctypes.c_int] + [ctypes.c_void_p] * 4
+    assert f(0, None, 16, 16, None) == 1
+    assert f(4, 16, 16, 16, None) == 3
+    assert f(-1, 16, 16, 16, None) == 3
 
 
 def test_ex_rejects_bad_schedule(lib):

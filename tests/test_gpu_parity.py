@@ -6,6 +6,8 @@ accumulation -- max-abs <= 1e-2 and relative L2 <= 2e-3; fp32 I/O -- max-abs
 the bench uses; the stress workload (L = 16384, d = 128) is compared on
 sampled (b, h) pairs, each of which the oracle recomputes from scratch.
 """
+import os
+
 import numpy as np
 import pytest
 
@@ -42,9 +44,20 @@ def errors(u, ref):
     return float(np.max(np.abs(d))), float(np.linalg.norm(d) / max(np.linalg.norm(ref), 1e-30))
 
 
+def _report(max_abs, rel, dtype):
+    """Append the error to $GLA_PARITY_REPORT (one JSON line per comparison)."""
+    path = os.environ.get("GLA_PARITY_REPORT")
+    if path:
+        import json
+        with open(path, "a") as f:
+            f.write(json.dumps({"test": os.environ.get("PYTEST_CURRENT_TEST", "?").split(" ")[0],
+                                "dtype": dtype, "max_abs": max_abs, "rel_l2": rel}) + "\n")
+
+
 def assert_close(u, ref, dtype):
     assert np.all(np.isfinite(u))
     max_abs, rel = errors(u, ref)
+    _report(max_abs, rel, dtype)
     tol = TOL[dtype]
     assert max_abs <= tol["max_abs"] and rel <= tol["rel_l2"], (max_abs, rel)
 
