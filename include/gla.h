@@ -150,7 +150,8 @@ int gla_plan(int B, int H, int grid_h, int grid_w, int d_k, int d_v, int dtype, 
  * layouts and descriptors, on row-major float32 DEVICE arrays:
  *   kind 0  D[128][128] = A[128][64] * B[128][64]^T   (split tf32: each operand is
  *           held as tf32 high + low parts, three products; ~fp32 accuracy)
- *   kind 1  D[64][64]   = A[128][64]^T * B[128][64]   (fp16 operands, the state product)
+ *   kind 1  D[64][64]   = B[128][64]^T * A[128][64]   (fp16 operands, the state product,
+ *           kept transposed: A plays the decayed keys, B the values)
  *   kind 2  D[128][64]  = A[128][128] * B[128][64]    (fp16 operands, P * V)
  *   kind 3  D[128][64]  = A[128][64] * B[64][64]^T    (tf32, the inter-chunk product)
  * Inputs are rounded to the operand type (tf32 or fp16; kind 0 splits them)

@@ -442,7 +442,7 @@ int gla_selftest_mma(int kind, const float *A, const float *B, float *D, void *s
         cudaGetLastError();
         return GLA_ERR_CUDA;
     }
-    kern<<<1, tc::kThreads, tc::kSmemBytes, static_cast<cudaStream_t>(stream)>>>(kind, A, B, D);
+    kern<<<1, tc::kSelfThreads, tc::kSmemBytes, static_cast<cudaStream_t>(stream)>>>(kind, A, B, D);
     if (cudaGetLastError() != cudaSuccess) return GLA_ERR_CUDA;
     return GLA_OK;
 }

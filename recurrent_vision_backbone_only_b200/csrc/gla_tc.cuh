@@ -10,14 +10,16 @@
 // Chunkwise form used here.  A chunk holds n <= 128 consecutive scan
 // positions; b_t is the inclusive in-chunk cumulative sum of
 // lambda_t = log sigma(a_t) / 16 (per key channel), B = b_{n-1}, and r is a
-// per-channel reference (the chunk's middle row).  With Q~ = q (.) e^{b - r},
+// per-channel reference (the chunk's middle row).  The kernel keeps b, B, r
+// in log2 units so every factor below is one ex2.  With Q~ = q (.) e^{b - r},
 // K~ = k (.) e^{r - b}, Ks = k (.) e^{B - b} and the state S_in entering the
 // chunk:
 //   scores   A     = Q~ K~^T   split-tf32: Qh Kh^T + Qh Kl^T + Ql Kh^T, where
 //                    X = Xh + Xl with Xh = tf32(X), Xl = tf32(X - Xh)
 //                    (tcgen05 kind::tf32, A operands Qh/Ql in TMEM, 128x128x64)
 //   masked   P     = d_k^{-1/2} A (.) [s <= t], diagonal A_tt = q_t . k_t in fp32
-//   output   O     = P V + Qh (d_k^{-1/2} Diag(e^{r}) S_in)  (f16 + tf32 MMAs)
+//                    (d_k^{-1/2} = 2^-3 is folded into Q~'s exponent)
+//   output   O     = P V + (Qh + Ql) Diag(e^{r}) S_in   (f16 + tf32 MMAs)
 //   state    S_out = Diag(e^{B}) S_in + Ks^T V       (tcgen05 kind::f16, 64x64x128)
 // Every exponent in Ks, e^{r}, e^{B} is <= 0.  Q~ and K~ carry exponents of
 // either sign bounded by the chunk's decay range about r; they are kept in
@@ -53,10 +55,14 @@ namespace tc {
 
 namespace cg = cooperative_groups;
 
-constexpr int kThreads = 128;
+constexpr int kThreads = 256;      // two threads per chunk row (one per channel half)
+constexpr int kSelfThreads = 128;  // self-test kernel: one thread per row
 constexpr int kC = 128;            // max tokens per chunk (MMA M)
 constexpr int kD = 64;             // head dim handled by this kernel
-constexpr float kHalfRangeSafe = 60.0f;
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLog2Scale = -3.0f;   // log2(d_k^{-1/2}) for d_k = 64, folded into Q~
+// largest |b - r| (log2 units) the tf32 operands carry: 2^86 * 65504 stays finite in fp32
+constexpr float kHalfRangeSafe2 = 86.0f;
 
 // ---- shared memory map (bytes from a 1024-aligned base) ----
 constexpr uint32_t kKL = 0;        // K~ low part  tf32, 2 atoms x [128][128B]
@@ -69,9 +75,10 @@ constexpr uint32_t kTA = 147456;
 constexpr uint32_t kTV = 163840;
 constexpr uint32_t kTG = 180224;
 constexpr uint32_t kMISC = 196608;
+constexpr uint32_t kMiscBytes = 12288;
 constexpr uint32_t kAtom128 = 16384;   // [128 rows][128 B]
 constexpr uint32_t kAtom64 = 8192;     // [64 rows][128 B]
-constexpr size_t kSmemBytes = kMISC + 4096 + 1024;  // + misc + alignment slack
+constexpr size_t kSmemBytes = kMISC + kMiscBytes + 1024;  // + misc + alignment slack
 
 // TMEM columns
 constexpr uint32_t kTmemCols = 512;
@@ -125,12 +132,13 @@ __device__ __forceinline__ void issue_qk(uint32_t sbase, uint32_t tmem) {
         }
     }
 }
-// Sloc[c][j] = sum_s Ks[s][c] V[s][j]  (both operands MN-major, K = 128 rows)
+// Sloc^T[j][c] = sum_s V[s][j] Ks[s][c]  (both operands MN-major, K = 128 rows); the state is
+// kept transposed so each thread owns one value column j and writes S~ rows contiguously.
 __device__ __forceinline__ void issue_state(uint32_t sbase, uint32_t tmem) {
 #pragma unroll
     for (int k = 0; k < 8; ++k) {
-        ptx::mma_f16_ss(tmem + kColSL, ptx::desc_sw128(sbase + kST + k * 2048, kAtom128, 1024),
-                        ptx::desc_sw128(sbase + kTV + k * 2048, kAtom128, 1024), kIdescST, k > 0);
+        ptx::mma_f16_ss(tmem + kColSL, ptx::desc_sw128(sbase + kTV + k * 2048, kAtom128, 1024),
+                        ptx::desc_sw128(sbase + kST + k * 2048, kAtom128, 1024), kIdescST, k > 0);
     }
 }
 // O[t][j] = sum_s P[t][s] V[s][j]
@@ -142,14 +150,17 @@ __device__ __forceinline__ void issue_pv(uint32_t sbase, uint32_t p_base, uint32
                         ptx::desc_sw128(sbase + kTV + k * 2048, kAtom128, 1024), kIdescPV, k > 0);
     }
 }
-// O[t][j] += sum_c Qh[t][c] S~[j][c]
+// O[t][j] += sum_c (Qh + Ql)[t][c] S~[j][c]
 __device__ __forceinline__ void issue_inter(uint32_t sbase, uint32_t tmem, bool accumulate) {
 #pragma unroll
-    for (int k = 0; k < 8; ++k) {
-        const uint32_t soff = (k >> 2) * kAtom64 + (k & 3) * 32;
-        ptx::mma_tf32_ts(tmem + kColO, tmem + kColQH + 8 * k,
-                         ptx::desc_sw128(sbase + kST + soff, 16, 1024), kIdescIN,
-                         accumulate || k > 0);
+    for (int pass = 0; pass < 2; ++pass) {
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+            const uint32_t soff = (k >> 2) * kAtom64 + (k & 3) * 32;
+            ptx::mma_tf32_ts(tmem + kColO, tmem + (pass ? kColQL : kColQH) + 8 * k,
+                             ptx::desc_sw128(sbase + kST + soff, 16, 1024), kIdescIN,
+                             accumulate || pass > 0 || k > 0);
+        }
     }
 }
 
@@ -165,11 +176,16 @@ __device__ __forceinline__ bool wait_phase(uint64_t *bar, uint32_t parity) {
     return true;
 }
 
-__device__ __forceinline__ float log_gamma_fast(float a) {
-    return (fminf(a, 0.0f) - __logf(1.0f + __expf(-fabsf(a)))) * kInvTau;
+// log2 of the retention gate: log2(sigma(a)) / 16, stable for either sign of a.
+__device__ __forceinline__ float log2_gamma(float a) {
+    const float x = ptx::ex2(-fabsf(a) * kLog2e);             // 2^{-|a| log2 e} = e^{-|a|}
+    return (fminf(a, 0.0f) * kLog2e - ptx::lg2(1.0f + x)) * kInvTau;
 }
 
-__device__ __forceinline__ float silu_fast(float g) { return g / (1.0f + __expf(-g)); }
+// SiLU(g) = g / (1 + e^{-g})
+__device__ __forceinline__ float silu_fast(float g) {
+    return g * ptx::rcp(1.0f + ptx::ex2(-g * kLog2e));
+}
 
 __device__ __forceinline__ uint32_t pack_half2(float lo, float hi) {
     const __half2 h = __floats2half2_rn(lo, hi);
@@ -178,23 +194,58 @@ __device__ __forceinline__ uint32_t pack_half2(float lo, float hi) {
 
 // Shared scratch scalars.
 struct Misc {
-    uint64_t mbar[4];
+    uint64_t mbar_mma[2];     // [0] score + state products, [1] P.V + inter products
+    uint64_t mbar_ld[3];      // [0] a tile, [1] q and k tiles, [2] v and g tiles
     uint32_t tmem_base;
-    int slow;             // chunk uses the exact CUDA-core score path
-    int range_err;        // a P entry overflowed fp16
-    int abort;            // a bounded wait expired
-    int rows[kC];         // token row index (b*L + s)*H + h of each chunk row
-    float bref[kD];       // reference r_c (log)
-    float eref[kD];       // e^{r_c}
-    float Bc[kD];         // B_c = b_{n-1,c} (log)
-    float eB[kD];         // e^{B_c}
-    float fB[kD];         // e^{B_c - r_c}
-    float Gs[kD];         // segment total log-decay (exchange)
-    float tot0[kD];       // cumulative sum of the first 64 rows
-    float b0[kD];         // b_{0,c}
-    float w[kD];          // RMSNorm weight
+    int slow;                 // chunk uses the exact CUDA-core score path
+    int range_err;            // a P entry overflowed fp16
+    int abort;                // a bounded wait expired
+    int rows[kC];             // token row index (b*L + s)*H + h of each chunk row
+    alignas(16) float bref[kD];   // reference r_c (log2 units)
+    alignas(16) float eref[kD];   // 2^{r_c}
+    alignas(16) float Bc[kD];     // B_c = b_{n-1,c} (log2)
+    alignas(16) float eB[kD];     // 2^{B_c}
+    alignas(16) float fB[kD];     // 2^{B_c - r_c}
+    alignas(16) float Gs[kD];     // segment total log2-decay (exchange)
+    alignas(16) float b0[kD];     // b_{0,c}
+    alignas(16) float w[kD];      // RMSNorm weight
+    alignas(16) float tot[8][kD]; // per-16-row totals of the gate scan
+    alignas(16) float Gall[16][kD]; // every segment's log2-decay (exchange)
+    alignas(16) float red[2][kC]; // epilogue partial sums of squares (per channel half)
 };
-static_assert(sizeof(Misc) <= 4096, "misc region");
+static_assert(sizeof(Misc) <= kMiscBytes, "misc region");
+
+// Exact scores on CUDA cores for a chunk whose decay range the tf32 operands
+// cannot carry: P[t][s] = d_k^{-1/2} sum_c q_tc k_sc 2^{b_tc - b_sc} (s <= t),
+// written as fp16 into the K~ high-part region.  Rare; kept out of line.
+__device__ __noinline__ void make_p_exact(uint8_t *sm, int t, int ch, int n, float scale,
+                                          int *range_err) {
+    const float *bp = reinterpret_cast<const float *>(sm + kPB);
+    auto bat = [&](int row, int c) { return bp[(off_tf32(kAtom128, row, c >> 2) >> 2) + (c & 3)]; };
+    auto hat = [&](uint32_t tile, int row, int c) {
+        return __half2float(*reinterpret_cast<const __half *>(sm + tile + off_f16(row, c >> 3) + (c & 7) * 2));
+    };
+    int err = 0;
+    for (int s0 = ch * 64; s0 < ch * 64 + 64; s0 += 8) {
+        float v8[8];
+        for (int e = 0; e < 8; ++e) {
+            const int s = s0 + e;
+            float acc = 0.0f;
+            if (s <= t && t < n) {
+                for (int c = 0; c < kD; ++c)
+                    acc = fmaf(hat(kTQ, t, c) * hat(kTK, s, c), exp2f(bat(t, c) - bat(s, c)), acc);
+            }
+            acc *= scale;
+            err |= fabsf(acc) > 65504.0f;
+            v8[e] = acc;
+        }
+        uint4 o;
+        o.x = pack_half2(v8[0], v8[1]); o.y = pack_half2(v8[2], v8[3]);
+        o.z = pack_half2(v8[4], v8[5]); o.w = pack_half2(v8[6], v8[7]);
+        *reinterpret_cast<uint4 *>(sm + kKH + off_f16k128(t, s0 >> 3)) = o;
+    }
+    if (err) *range_err = 1;
+}
 
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1) gla_tc_kernel(const Params p) {
@@ -206,6 +257,9 @@ __global__ void __launch_bounds__(kThreads, 1) gla_tc_kernel(const Params p) {
     Misc &m = *reinterpret_cast<Misc *>(sm + kMISC);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int w4 = warp & 3;          // TMEM lane quarter of this warp
+    const int ch = warp >> 2;         // channel half handled by this thread (row-owner work)
+    const int t = w4 * 32 + lane;     // chunk row owned by this thread
     const int pair = blockIdx.x / p.segs;
     const int rank = blockIdx.x - pair * p.segs;
     const int bb = pair / p.H, hh = pair - bb * p.H;
@@ -224,8 +278,9 @@ __global__ void __launch_bounds__(kThreads, 1) gla_tc_kernel(const Params p) {
         ptx::tmem_relinquish();
     }
     if (tid == 0) {
-        ptx::mbar_init(&m.mbar[0], 1);
-        ptx::mbar_init(&m.mbar[1], 1);
+        ptx::mbar_init(&m.mbar_mma[0], 1);
+        ptx::mbar_init(&m.mbar_mma[1], 1);
+        for (int i = 0; i < 3; ++i) ptx::mbar_init(&m.mbar_ld[i], kThreads);
         ptx::fence_mbarrier_init();
         m.abort = 0;
         m.range_err = 0;
@@ -238,87 +293,127 @@ __global__ void __launch_bounds__(kThreads, 1) gla_tc_kernel(const Params p) {
     __syncthreads();
     ptx::tc_fence_after_sync();
     const uint32_t tmem = m.tmem_base;
-    const uint32_t tmem_warp = tmem + ((uint32_t)(warp * 32) << 16);
-    uint32_t ph0 = 0, ph1 = 0;
+    const uint32_t tmem_warp = tmem + ((uint32_t)(w4 * 32) << 16);
+    uint32_t it = 0;                  // chunk iterations so far (load-barrier parity)
+    uint32_t ph_mma0 = 0, ph_mma1 = 0;
 
-    // state owned by threads with lane < 16: row c = 16*warp + lane, 64 columns
+    // State rows owned by lanes < 16: state column j = 16*w4 + lane (a row of the transposed
+    // state), channels c in [32*ch, 32*ch + 32).
     const bool s_owner = lane < 16;
-    const int s_row = warp * 16 + lane;
-    float S[kD];
+    const int s_row = w4 * 16 + lane;
+    float S[32];
 #pragma unroll
-    for (int j = 0; j < kD; ++j) S[j] = 0.0f;
+    for (int j = 0; j < 32; ++j) S[j] = 0.0f;
+    float Sl[32];
 
-    // ------------------------------------------------------------ helpers
+    auto wait_bar = [&](uint64_t *bar, uint32_t parity) {
+        if (!wait_phase(bar, parity)) m.abort = 1;
+    };
+    // ------------------------------------------------------------ loads
     auto set_rows = [&](int c0, int n) {
         if (tid < n) m.rows[tid] = (bb * p.L + spatial_of(dir, c0 + tid, p.gh, p.gw)) * p.H + hh;
     };
-    // gather one fp16 [n rows][64] tile into the swizzled layout, zero rows >= n
-    auto load_tile = [&](const __half *src, uint32_t dst, int n) {
+    // issue the chunk's gathers (fp16 [n rows][64] tiles, rows >= n zero-filled) into the
+    // swizzled layout; completion is tracked per group on mbar_ld[0..2]
+    auto issue_loads = [&](int n, bool full) {
+        size_t goff[4];
+        uint32_t soff[4], bytes[4];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            const int idx = tid + i * kThreads;
-            const int row = idx >> 3, j = idx & 7;
+        for (int i = 0; i < 4; ++i) {
+            const int row = (tid >> 3) + 32 * i, j = tid & 7;
             const bool ok = row < n;
-            const __half *g = src + (ok ? (size_t)m.rows[row] * kD + j * 8 : 0);
-            ptx::cp_async16(sbase + dst + off_f16(row, j), g, ok ? 16u : 0u);
+            goff[i] = ok ? (size_t)m.rows[row] * kD + j * 8 : 0;
+            soff[i] = sbase + off_f16(row, j);
+            bytes[i] = ok ? 16u : 0u;
         }
+        auto tile = [&](const __half *src, uint32_t dst) {
+#pragma unroll
+            for (int i = 0; i < 4; ++i) ptx::cp_async16(soff[i] + dst, src + goff[i], bytes[i]);
+        };
+        tile(p.a, kTA);
+        ptx::cp_async_mbar_arrive_noinc(&m.mbar_ld[0]);
+        tile(p.k, kTK);
+        if (full) tile(p.q, kTQ);
+        ptx::cp_async_mbar_arrive_noinc(&m.mbar_ld[1]);
+        tile(p.v, kTV);
+        if (full) tile(p.g, kTG);
+        ptx::cp_async_mbar_arrive_noinc(&m.mbar_ld[2]);
     };
-    // column-owner cumulative sum of lambda; writes b (fp32) and per-channel scalars
+    // ------------------------------------------------------------ gate
+    // 16 rows x 2 channels per thread: b = inclusive cumsum of log2(gamma) down the chunk
     auto gate = [&](int n) {
-        const int c = tid & 63, half = tid >> 6;
-        float cs[64];
-        float run = 0.0f;
-        const uint8_t *ta = sm + kTA;
-#pragma unroll 8
-        for (int i = 0; i < 64; ++i) {
-            const int t = half * 64 + i;
-            const __half av = *reinterpret_cast<const __half *>(ta + off_f16(t, c >> 3) + (c & 7) * 2);
-            const float lam = t < n ? log_gamma_fast(__half2float(av)) : 0.0f;
-            run += lam;
-            cs[i] = run;
+        const int cp = tid & 31, tq = tid >> 5;   // channels 2cp, 2cp+1; rows 16tq..16tq+15
+        wait_bar(&m.mbar_ld[0], it & 1);
+        float c0s[16], c1s[16];
+        float r0 = 0.0f, r1 = 0.0f;
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            const int row = tq * 16 + i;
+            const __half2 av = *reinterpret_cast<const __half2 *>(sm + kTA + off_f16(row, cp >> 2) +
+                                                                  (cp & 3) * 4);
+            const float2 af = __half22float2(av);
+            const bool ok = row < n;
+            r0 += ok ? log2_gamma(af.x) : 0.0f;
+            r1 += ok ? log2_gamma(af.y) : 0.0f;
+            c0s[i] = r0;
+            c1s[i] = r1;
         }
-        if (half == 0) {
-            m.tot0[c] = run;
-            m.b0[c] = cs[0];
-        }
+        *reinterpret_cast<float2 *>(&m.tot[tq][2 * cp]) = make_float2(r0, r1);
         __syncthreads();
-        const float add = half ? m.tot0[c] : 0.0f;
-        const int mid = (n - 1) >> 1;
-        float *bp = reinterpret_cast<float *>(sm + kPB);
-#pragma unroll 8
-        for (int i = 0; i < 64; ++i) {
-            const int t = half * 64 + i;
-            const float bt = cs[i] + add;
-            bp[(off_tf32(kAtom128, t, c >> 2) >> 2) + (c & 3)] = bt;
-            if (t == mid) m.bref[c] = bt;
-            if (t == n - 1) m.Bc[c] = bt;
+        float a0 = 0.0f, a1 = 0.0f;
+        for (int q = 0; q < tq; ++q) {
+            const float2 x = *reinterpret_cast<const float2 *>(&m.tot[q][2 * cp]);
+            a0 += x.x;
+            a1 += x.y;
+        }
+        const int c = 2 * cp;
+#pragma unroll
+        for (int i = 0; i < 16; ++i)
+            *reinterpret_cast<float2 *>(sm + kPB + off_tf32(kAtom128, tq * 16 + i, c >> 2) + (c & 3) * 4) =
+                make_float2(c0s[i] + a0, c1s[i] + a1);
+        __syncthreads();
+        if (tid < kD) {
+            const float *bp = reinterpret_cast<const float *>(sm + kPB);
+            auto bat = [&](int row) { return bp[(off_tf32(kAtom128, row, tid >> 2) >> 2) + (tid & 3)]; };
+            const float r = bat((n - 1) >> 1), Bv = bat(n - 1);
+            m.bref[tid] = r;
+            m.Bc[tid] = Bv;
+            if ((bat(0) - r > kHalfRangeSafe2) || (r - Bv > kHalfRangeSafe2)) m.slow = 1;
         }
         __syncthreads();
         if (tid < kD) {
+            if (m.slow) m.bref[tid] = 0.0f;           // slow path: chunk-start reference
             const float r = m.bref[tid], Bv = m.Bc[tid];
-            const bool wide = (m.b0[tid] - r > kHalfRangeSafe) || (r - Bv > kHalfRangeSafe);
-            m.eB[tid] = __expf(Bv);
-            m.fB[tid] = __expf(Bv - r);
-            if (wide) m.slow = 1;
+            m.eB[tid] = ptx::ex2(Bv);
+            m.fB[tid] = ptx::ex2(Bv - r);
+            m.eref[tid] = ptx::ex2(r);
         }
+        __syncthreads();
     };
-    // row-owner operand construction: Q~, K~ (fast path) and Ks; full = false builds Ks only
+    // ------------------------------------------------------------ operands (row t, 32 channels)
+    // fast path: Qh/Ql (TMEM, scaled by d_k^{-1/2}), Kh/Kl (smem tf32), Ks (smem fp16);
+    // slow path: Qh = d_k^{-1/2} q 2^{b}, Ks.  full = false builds Ks only.
     auto build_operands = [&](bool full) {
-        const int t = tid;
         const bool slow = m.slow != 0;
-        const float *bp = reinterpret_cast<const float *>(sm + kPB);
-#pragma unroll 2
-        for (int j = 0; j < 8; ++j) {  // 8 channels per step
+        wait_bar(&m.mbar_ld[1], it & 1);
+#pragma unroll 1
+        for (int jj = 0; jj < 4; ++jj) {
+            const int j = ch * 4 + jj;             // 16 B chunk of 8 channels
             const uint4 kraw = *reinterpret_cast<const uint4 *>(sm + kTK + off_f16(t, j));
-            const uint4 qraw = *reinterpret_cast<const uint4 *>(sm + kTQ + off_f16(t, j));
+            uint4 qraw = make_uint4(0, 0, 0, 0);
+            if (full) qraw = *reinterpret_cast<const uint4 *>(sm + kTQ + off_f16(t, j));
             const __half2 *k2 = reinterpret_cast<const __half2 *>(&kraw);
             const __half2 *q2 = reinterpret_cast<const __half2 *>(&qraw);
-            float bt[8], kv[8], qv[8];
+            float bt[8], rr[8], fb[8], kv[8], qv[8];
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
-                const float4 b4 = *reinterpret_cast<const float4 *>(
-                    reinterpret_cast<const uint8_t *>(bp) + off_tf32(kAtom128, t, 2 * j + h));
-                bt[4 * h + 0] = b4.x; bt[4 * h + 1] = b4.y; bt[4 * h + 2] = b4.z; bt[4 * h + 3] = b4.w;
+                const float4 b4 = *reinterpret_cast<const float4 *>(sm + kPB + off_tf32(kAtom128, t, 2 * j + h));
+                const float4 r4 = *reinterpret_cast<const float4 *>(&m.bref[8 * j + 4 * h]);
+                const float4 f4 = *reinterpret_cast<const float4 *>(slow ? &m.Bc[8 * j + 4 * h]
+                                                                         : &m.fB[8 * j + 4 * h]);
+                bt[4 * h] = b4.x; bt[4 * h + 1] = b4.y; bt[4 * h + 2] = b4.z; bt[4 * h + 3] = b4.w;
+                rr[4 * h] = r4.x; rr[4 * h + 1] = r4.y; rr[4 * h + 2] = r4.z; rr[4 * h + 3] = r4.w;
+                fb[4 * h] = f4.x; fb[4 * h + 1] = f4.y; fb[4 * h + 2] = f4.z; fb[4 * h + 3] = f4.w;
             }
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
@@ -327,27 +422,25 @@ __global__ void __launch_bounds__(kThreads, 1) gla_tc_kernel(const Params p) {
                 kv[2 * e] = kf.x; kv[2 * e + 1] = kf.y;
                 qv[2 * e] = qf.x; qv[2 * e + 1] = qf.y;
             }
+            // tf32 splits: high = low 13 bits cleared, low = exact remainder (the tensor core
+            // drops the low part's own low bits: error <= 2^-20 of the value)
             float ks[8], qh[8], ql[8], kh[8], kl[8];
 #pragma unroll
             for (int e = 0; e < 8; ++e) {
-                const int c = 8 * j + e;
                 if (!slow) {
-                    const float e2 = __expf(m.bref[c] - bt[e]);       // e^{r - b}
-                    ks[e] = kv[e] * e2 * m.fB[c];                   // k e^{B - b}
-                    if (full) {
-                        const float kf = kv[e] * e2;
-                        const float qf = qv[e] * __expf(bt[e] - m.bref[c]);  // q e^{b - r}
-                        kh[e] = ptx::to_tf32(kf);
-                        kl[e] = ptx::to_tf32(kf - kh[e]);
-                        qh[e] = ptx::to_tf32(qf);
-                        ql[e] = ptx::to_tf32(qf - qh[e]);
-                    }
+                    const float kf = kv[e] * ptx::ex2(rr[e] - bt[e]);          // k 2^{r - b}
+                    ks[e] = kf * fb[e];                                         // k 2^{B - b}
+                    const float qf = qv[e] * ptx::ex2(bt[e] - rr[e] + kLog2Scale);  // q 2^{b - r} / 8
+                    kh[e] = ptx::tf32_hi(kf);
+                    kl[e] = kf - kh[e];
+                    qh[e] = ptx::tf32_hi(qf);
+                    ql[e] = qf - qh[e];
                 } else {
-                    ks[e] = kv[e] * __expf(m.Bc[c] - bt[e]);
-                    if (full) {                                      // reference = chunk start
-                        qh[e] = ptx::to_tf32(qv[e] * __expf(bt[e]));
-                        ql[e] = 0.0f;
-                    }
+                    ks[e] = kv[e] * ptx::ex2(fb[e] - bt[e]);      // fb holds B_c here
+                    const float qf = qv[e] * ptx::ex2(bt[e] + kLog2Scale);
+                    qh[e] = ptx::tf32_hi(qf);
+                    ql[e] = qf - qh[e];
+                    kh[e] = kl[e] = 0.0f;
                 }
             }
             uint4 kso;
@@ -370,8 +463,10 @@ __global__ void __launch_bounds__(kThreads, 1) gla_tc_kernel(const Params p) {
         }
         if (full) ptx::tmem_st_wait();
     };
-    // one-thread MMA issue + commit, everyone waits
-    auto mma_round = [&](int which) {  // 0: state only, 1: QK (+state), 2: PV + inter
+    // ------------------------------------------------------------ MMA rounds (one thread issues)
+    // which: 0 = state only, 1 = scores (+ state), 2 = P.V + inter
+    auto mma_round = [&](int which) {
+        if (which < 2) wait_bar(&m.mbar_ld[2], it & 1);   // V is an operand of the state product
         ptx::fence_proxy_async_smem();
         ptx::tc_fence_before_sync();
         __syncthreads();
@@ -379,302 +474,243 @@ __global__ void __launch_bounds__(kThreads, 1) gla_tc_kernel(const Params p) {
             ptx::tc_fence_after_sync();
             if (which == 0) {
                 issue_state(sbase, tmem);
-                ptx::mma_commit(&m.mbar[0]);
+                ptx::mma_commit(&m.mbar_mma[0]);
             } else if (which == 1) {
                 if (!m.slow) issue_qk(sbase, tmem);
                 issue_state(sbase, tmem);
-                ptx::mma_commit(&m.mbar[0]);
+                ptx::mma_commit(&m.mbar_mma[0]);
             } else {
                 issue_pv(sbase, m.slow ? kKH : kPB, tmem);
                 issue_inter(sbase, tmem, true);
-                ptx::mma_commit(&m.mbar[1]);
+                ptx::mma_commit(&m.mbar_mma[1]);
             }
         }
-        uint64_t *bar = which == 2 ? &m.mbar[1] : &m.mbar[0];
-        uint32_t &ph = which == 2 ? ph1 : ph0;
-        if (!wait_phase(bar, ph)) m.abort = 1;
-        ph ^= 1u;
+        if (which == 2) {
+            wait_bar(&m.mbar_mma[1], ph_mma1);
+            ph_mma1 ^= 1u;
+        } else {
+            wait_bar(&m.mbar_mma[0], ph_mma0);
+            ph_mma0 ^= 1u;
+        }
         ptx::tc_fence_after_sync();
     };
-    // Sloc (TMEM, M=64 layout) -> registers of the state owners (whole warps execute the load)
-    auto read_sloc = [&](float (&Sl)[kD]) {
-        float r0[32], r1[32];
-        ptx::tmem_ld32(tmem_warp + kColSL, r0);
-        ptx::tmem_ld32(tmem_warp + kColSL + 32, r1);
+    // transposed chunk state (TMEM, M=64 layout) -> registers of the state owners (warp-wide)
+    auto read_sloc = [&]() {
+        ptx::tmem_ld32(tmem_warp + kColSL + 32 * ch, Sl);
         ptx::tmem_ld_wait();
-#pragma unroll
-        for (int j = 0; j < 32; ++j) {
-            Sl[j] = r0[j];
-            Sl[32 + j] = r1[j];
-        }
     };
-    // masked, scaled scores -> P (fp16, K-major, 2 atoms) in the b region
+    // ------------------------------------------------------------ P (row t, 64 columns)
     auto make_p_fast = [&]() {
-        const int t = tid;
-        int err = 0;
-        // exact diagonal score q_t . k_t (decay factor 1), fp32 from the raw tiles
-        float dq = 0.0f;
+        if (ch == 1 && t < 64) {                       // whole half above the diagonal
+            const uint4 z = make_uint4(0, 0, 0, 0);
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-            const uint4 kraw = *reinterpret_cast<const uint4 *>(sm + kTK + off_f16(t, j));
-            const uint4 qraw = *reinterpret_cast<const uint4 *>(sm + kTQ + off_f16(t, j));
-            const __half2 *k2 = reinterpret_cast<const __half2 *>(&kraw);
-            const __half2 *q2 = reinterpret_cast<const __half2 *>(&qraw);
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const float2 kf = __half22float2(k2[e]), qf = __half22float2(q2[e]);
-                dq = fmaf(qf.x, kf.x, dq);
-                dq = fmaf(qf.y, kf.y, dq);
-            }
+            for (int j = 0; j < 8; ++j) *reinterpret_cast<uint4 *>(sm + kPB + off_f16k128(t, 8 + j)) = z;
+            return;
         }
-#pragma unroll 1
-        for (int blk = 0; blk < 4; ++blk) {
-            float r[32];
-            ptx::tmem_ld32(tmem_warp + kColDS + blk * 32, r);
-            ptx::tmem_ld_wait();
-#pragma unroll
-            for (int j4 = 0; j4 < 4; ++j4) {  // four 16 B chunks of 8 halves
-                float v8[8];
-#pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    const int s = blk * 32 + j4 * 8 + e;
-                    const float x = s < t ? r[j4 * 8 + e] * p.scale : (s == t ? dq * p.scale : 0.0f);
-                    err |= fabsf(x) > 65504.0f;
-                    v8[e] = x;
-                }
-                uint4 o;
-                o.x = pack_half2(v8[0], v8[1]); o.y = pack_half2(v8[2], v8[3]);
-                o.z = pack_half2(v8[4], v8[5]); o.w = pack_half2(v8[6], v8[7]);
-                *reinterpret_cast<uint4 *>(sm + kPB + off_f16k128(t, blk * 4 + j4)) = o;
-            }
-        }
-        if (err) m.range_err = 1;
-    };
-    // exact scores on CUDA cores (reference = each pair's own decay), P into the K~ region
-    auto make_p_slow = [&](int n) {
-        const int t = tid;
-        const float *bp = reinterpret_cast<const float *>(sm + kPB);
-        auto bat = [&](int row, int c) {
-            return bp[(off_tf32(kAtom128, row, c >> 2) >> 2) + (c & 3)];
-        };
-        auto hat = [&](uint32_t tile, int row, int c) {
-            return __half2float(*reinterpret_cast<const __half *>(sm + tile + off_f16(row, c >> 3) +
-                                                                   (c & 7) * 2));
-        };
-        int err = 0;
-        for (int s0 = 0; s0 < kC; s0 += 8) {
-            float v8[8];
-            for (int e = 0; e < 8; ++e) {
-                const int s = s0 + e;
-                float acc = 0.0f;
-                if (s <= t && t < n) {
-                    for (int c = 0; c < kD; ++c)
-                        acc = fmaf(hat(kTQ, t, c) * hat(kTK, s, c), expf(bat(t, c) - bat(s, c)), acc);
-                }
-                acc *= p.scale;
-                err |= fabsf(acc) > 65504.0f;
-                v8[e] = acc;
-            }
-            uint4 o;
-            o.x = pack_half2(v8[0], v8[1]); o.y = pack_half2(v8[2], v8[3]);
-            o.z = pack_half2(v8[4], v8[5]); o.w = pack_half2(v8[6], v8[7]);
-            *reinterpret_cast<uint4 *>(sm + kKH + off_f16k128(t, s0 >> 3)) = o;
-        }
-        if (err) m.range_err = 1;
-    };
-    // S~ = scale * Diag(e^{r}) S_in, tf32 K-major [j][c] (2 atoms of 64 rows)
-    auto write_stilde = [&]() {
-        if (s_owner) {
-            const int c = s_row;
-            const float f = p.scale * m.eref[c];
-            float *st = reinterpret_cast<float *>(sm + kST);
-#pragma unroll 8
-            for (int j = 0; j < kD; ++j)
-                st[(off_tf32(kAtom64, j, c >> 2) >> 2) + (c & 3)] = ptx::to_tf32(S[j] * f);
-        }
-    };
-    // u = SiLU(g) * o / sqrt(mean(o^2) + eps) * w for the chunk's rows
-    auto epilogue = [&](int n) {
-        const int t = tid;
-        float o[64];
-        {
-            float r0[32], r1[32];
-            ptx::tmem_ld32(tmem_warp + kColO, r0);
-            ptx::tmem_ld32(tmem_warp + kColO + 32, r1);
-            ptx::tmem_ld_wait();
-#pragma unroll
-            for (int j = 0; j < 32; ++j) {
-                o[j] = r0[j];
-                o[32 + j] = r1[j];
-            }
-        }
-        float ss = 0.0f;
-#pragma unroll
-        for (int j = 0; j < 64; ++j) ss = fmaf(o[j], o[j], ss);
-        const float inv = rsqrtf(ss * (1.0f / 64.0f) + p.eps);
-        if (t < n) {
-            __half *dst = p.out + (size_t)m.rows[t] * kD;
+        float dq = 0.0f;                               // exact diagonal score q_t . k_t
+        if ((t >> 6) == ch) {
 #pragma unroll
             for (int j = 0; j < 8; ++j) {
+                const uint4 kraw = *reinterpret_cast<const uint4 *>(sm + kTK + off_f16(t, j));
+                const uint4 qraw = *reinterpret_cast<const uint4 *>(sm + kTQ + off_f16(t, j));
+                const __half2 *k2 = reinterpret_cast<const __half2 *>(&kraw);
+                const __half2 *q2 = reinterpret_cast<const __half2 *>(&qraw);
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const float2 kf = __half22float2(k2[e]), qf = __half22float2(q2[e]);
+                    dq = fmaf(qf.x, kf.x, dq);
+                    dq = fmaf(qf.y, kf.y, dq);
+                }
+            }
+            dq *= p.scale;
+        }
+        float amax = 0.0f;
+#pragma unroll 1
+        for (int blk = 0; blk < 2; ++blk) {
+            const int s0 = ch * 64 + blk * 32;
+            uint8_t *dst = sm + kPB;
+            const int jb = ch * 8 + blk * 4;
+            if (s0 > t) {                              // block above the diagonal: zeros
+                const uint4 z = make_uint4(0, 0, 0, 0);
+#pragma unroll
+                for (int j4 = 0; j4 < 4; ++j4) *reinterpret_cast<uint4 *>(dst + off_f16k128(t, jb + j4)) = z;
+                continue;
+            }
+            float r[32];
+            ptx::tmem_ld32(tmem_warp + kColDS + s0, r);
+            ptx::tmem_ld_wait();
+            if (s0 + 31 >= t) {                        // block holding the diagonal
+#pragma unroll
+                for (int e = 0; e < 32; ++e) {
+                    const int s = s0 + e;
+                    r[e] = s < t ? r[e] : (s == t ? dq : 0.0f);
+                }
+            }
+#pragma unroll
+            for (int e = 0; e < 32; ++e) amax = fmaxf(amax, fabsf(r[e]));
+#pragma unroll
+            for (int j4 = 0; j4 < 4; ++j4) {
+                uint4 o;
+                o.x = pack_half2(r[8 * j4], r[8 * j4 + 1]); o.y = pack_half2(r[8 * j4 + 2], r[8 * j4 + 3]);
+                o.z = pack_half2(r[8 * j4 + 4], r[8 * j4 + 5]); o.w = pack_half2(r[8 * j4 + 6], r[8 * j4 + 7]);
+                *reinterpret_cast<uint4 *>(dst + off_f16k128(t, jb + j4)) = o;
+            }
+        }
+        if (amax > 65504.0f) m.range_err = 1;
+    };
+    // S~[j][c] = 2^{r_c} S_in[c][j], tf32 K-major (rows j, 2 atoms of 32 channels)
+    auto write_stilde = [&]() {
+        if (s_owner) {
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const float4 e4 = *reinterpret_cast<const float4 *>(&m.eref[32 * ch + 4 * i]);
+                *reinterpret_cast<float4 *>(sm + kST + off_tf32(kAtom64, s_row, 8 * ch + i)) =
+                    make_float4(ptx::to_tf32(S[4 * i] * e4.x), ptx::to_tf32(S[4 * i + 1] * e4.y),
+                                ptx::to_tf32(S[4 * i + 2] * e4.z), ptx::to_tf32(S[4 * i + 3] * e4.w));
+            }
+        }
+    };
+    // ------------------------------------------------------------ epilogue (row t, 32 channels)
+    auto epilogue = [&](int n) {
+        float o[32];
+        ptx::tmem_ld32(tmem_warp + kColO + 32 * ch, o);
+        ptx::tmem_ld_wait();
+        float ss = 0.0f;
+#pragma unroll
+        for (int j = 0; j < 32; ++j) ss = fmaf(o[j], o[j], ss);
+        m.red[ch][t] = ss;
+        __syncthreads();
+        const float inv = rsqrtf((m.red[0][t] + m.red[1][t]) * (1.0f / 64.0f) + p.eps);
+        wait_bar(&m.mbar_ld[2], it & 1);               // g tile
+        if (t < n) {
+            __half *dst = p.out + (size_t)m.rows[t] * kD + 32 * ch;
+#pragma unroll
+            for (int jj = 0; jj < 4; ++jj) {
+                const int j = ch * 4 + jj;
                 const uint4 graw = *reinterpret_cast<const uint4 *>(sm + kTG + off_f16(t, j));
                 const __half2 *g2 = reinterpret_cast<const __half2 *>(&graw);
+                const float4 wa = *reinterpret_cast<const float4 *>(&m.w[8 * j]);
+                const float4 wb = *reinterpret_cast<const float4 *>(&m.w[8 * j + 4]);
+                const float wv[8] = {wa.x, wa.y, wa.z, wa.w, wb.x, wb.y, wb.z, wb.w};
                 float u[8];
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
                     const float2 gf = __half22float2(g2[e]);
-                    const int c = 8 * j + 2 * e;
-                    u[2 * e] = o[c] * inv * m.w[c] * silu_fast(gf.x);
-                    u[2 * e + 1] = o[c + 1] * inv * m.w[c + 1] * silu_fast(gf.y);
+                    u[2 * e] = o[8 * jj + 2 * e] * inv * wv[2 * e] * silu_fast(gf.x);
+                    u[2 * e + 1] = o[8 * jj + 2 * e + 1] * inv * wv[2 * e + 1] * silu_fast(gf.y);
                 }
                 uint4 pk;
                 pk.x = pack_half2(u[0], u[1]); pk.y = pack_half2(u[2], u[3]);
                 pk.z = pack_half2(u[4], u[5]); pk.w = pack_half2(u[6], u[7]);
-                *reinterpret_cast<uint4 *>(dst + 8 * j) = pk;
+                *reinterpret_cast<uint4 *>(dst + 8 * jj) = pk;
             }
         }
     };
-    auto finish_gate = [&]() {  // per-chunk reference factors after the slow decision
-        __syncthreads();
-        if (tid < kD) {
-            if (m.slow) m.bref[tid] = 0.0f;
-            m.eref[tid] = __expf(m.bref[tid]);
-        }
-        __syncthreads();
-    };
-    auto chunk_bounds = [&](int ci, int &c0, int &n) {
-        c0 = p0 + ci * chunk_len;
-        n = min(chunk_len, p1 - c0);
-    };
-    // fold the chunk's local state into S: S = e^{B} S + Sloc
-    auto fold_sloc = [&](float (&Sl)[kD], bool into_g) {
+    // fold the chunk's local state into S: S = S Diag(2^{B}) + Sloc (transposed form)
+    auto fold_sloc = [&](bool into_g) {
         if (s_owner) {
-            const float e = m.eB[s_row];
 #pragma unroll
-            for (int j = 0; j < kD; ++j) S[j] = fmaf(e, S[j], Sl[j]);
-            if (into_g) m.Gs[s_row] += m.Bc[s_row];
+            for (int i = 0; i < 8; ++i) {
+                const float4 e4 = *reinterpret_cast<const float4 *>(&m.eB[32 * ch + 4 * i]);
+                S[4 * i] = fmaf(e4.x, S[4 * i], Sl[4 * i]);
+                S[4 * i + 1] = fmaf(e4.y, S[4 * i + 1], Sl[4 * i + 1]);
+                S[4 * i + 2] = fmaf(e4.z, S[4 * i + 2], Sl[4 * i + 2]);
+                S[4 * i + 3] = fmaf(e4.w, S[4 * i + 3], Sl[4 * i + 3]);
+            }
         }
+        if (into_g && tid < kD) m.Gs[tid] += m.Bc[tid];
     };
     // cluster-wide scan of (Gs, S) -> S becomes this segment's incoming state
     auto exchange_states = [&]() {
-        float *X = reinterpret_cast<float *>(sm + kST);  // [64][64] fp32, plain row-major
+        float *X = reinterpret_cast<float *>(sm + kST);  // [64 j][64 c] fp32, plain row-major
         __syncthreads();
         if (s_owner) {
 #pragma unroll
-            for (int i = 0; i < 16; ++i) {
-                const int j4 = (i + lane) & 15;
-                *reinterpret_cast<float4 *>(X + s_row * kD + 4 * j4) =
-                    make_float4(S[4 * j4], S[4 * j4 + 1], S[4 * j4 + 2], S[4 * j4 + 3]);
-            }
+            for (int i = 0; i < 8; ++i)
+                *reinterpret_cast<float4 *>(X + s_row * kD + 32 * ch + 4 * i) =
+                    make_float4(S[4 * i], S[4 * i + 1], S[4 * i + 2], S[4 * i + 3]);
         }
         cg::cluster_group cluster = cg::this_cluster();
         cluster.sync();
+        const int segs = p.segs;
+        // every segment's decay, copied once into local shared memory
+        for (int i = tid; i < segs * kD; i += kThreads) {
+            const int r = i / kD, c = i - r * kD;
+            m.Gall[r][c] = ptx::ex2(*cluster.map_shared_rank(&m.Gs[c], r));
+        }
+        __syncthreads();
         const int E = kD * kD;
-        const int per = (E + p.segs - 1) / p.segs;
+        const int per = (E + segs - 1) / segs;
         const int e0 = rank * per, e1 = min(E, e0 + per);
         for (int e = e0 + tid; e < e1; e += kThreads) {
-            const int c = e / kD;
+            const int c = e & (kD - 1);
+            float x[16];
+#pragma unroll
+            for (int r = 0; r < 16; ++r)
+                if (r < segs) x[r] = *cluster.map_shared_rank(X + e, r);
             float run = 0.0f;
-            for (int r = 0; r < p.segs; ++r) {
-                float *Xr = cluster.map_shared_rank(X, r);
-                const float *Gr = cluster.map_shared_rank(m.Gs, r);
-                const float agg = Xr[e];
-                const float dec = __expf(Gr[c]);
-                Xr[e] = run;
-                run = fmaf(dec, run, agg);
+#pragma unroll
+            for (int r = 0; r < 16; ++r) {
+                if (r < segs) {
+                    const float agg = x[r];
+                    x[r] = run;                       // state entering segment r
+                    run = fmaf(m.Gall[r][c], run, agg);
+                }
             }
+#pragma unroll
+            for (int r = 0; r < 16; ++r)
+                if (r < segs) *cluster.map_shared_rank(X + e, r) = x[r];
         }
         cluster.sync();
         if (s_owner) {
 #pragma unroll
-            for (int i = 0; i < 16; ++i) {
-                const int j4 = (i + lane) & 15;
-                const float4 x = *reinterpret_cast<const float4 *>(X + s_row * kD + 4 * j4);
-                S[4 * j4] = x.x; S[4 * j4 + 1] = x.y; S[4 * j4 + 2] = x.z; S[4 * j4 + 3] = x.w;
+            for (int i = 0; i < 8; ++i) {
+                const float4 v = *reinterpret_cast<const float4 *>(X + s_row * kD + 32 * ch + 4 * i);
+                S[4 * i] = v.x; S[4 * i + 1] = v.y; S[4 * i + 2] = v.z; S[4 * i + 3] = v.w;
             }
         }
-        __syncthreads();
-    };
-    // second half of a chunk: P, S~, PV + inter, epilogue; S advances by the chunk
-    auto finish_chunk = [&](int n, float (&Sl)[kD], bool advance) {
-        if (m.slow) make_p_slow(n); else make_p_fast();
-        write_stilde();
-        mma_round(2);
-        epilogue(n);
-        if (advance) fold_sloc(Sl, false);
-        ptx::tc_fence_before_sync();
         __syncthreads();
     };
 
-    float Sl[kD];
-    if (resident) {
-        // ---- one chunk: load all tiles, exchange mid-chunk ----
-        int c0, n;
-        chunk_bounds(0, c0, n);
-        if (n > 0) set_rows(c0, n);
-        if (tid == 0) m.slow = 0;
-        __syncthreads();
-        load_tile(p.k, kTK, n); load_tile(p.a, kTA, n); load_tile(p.v, kTV, n);
-        load_tile(p.q, kTQ, n); load_tile(p.g, kTG, n);
-        ptx::cp_async_commit();
-        ptx::cp_async_wait_all();
-        __syncthreads();
-        gate(n);
-        finish_gate();
-        build_operands(true);
-        mma_round(1);
-        read_sloc(Sl);
-        if (exchange) {
-            fold_sloc(Sl, true);                      // S = 0 * e^{B} + Sloc, Gs = B
-            exchange_states();
-        }
-        finish_chunk(n, Sl, false);
-    } else {
-        // ---- pass 1: state-only fold of this segment (not needed by the last one) ----
-        if (exchange) {
-            if (rank < p.segs - 1) {
-                for (int ci = 0; ci < n_chunks; ++ci) {
-                    int c0, n;
-                    chunk_bounds(ci, c0, n);
-                    __syncthreads();
-                    set_rows(c0, n);
-                    if (tid == 0) m.slow = 0;
-                    __syncthreads();
-                    load_tile(p.k, kTK, n); load_tile(p.a, kTA, n); load_tile(p.v, kTV, n);
-                    ptx::cp_async_commit();
-                    ptx::cp_async_wait_all();
-                    __syncthreads();
-                    gate(n);
-                    finish_gate();
-                    build_operands(false);
-                    mma_round(0);
-                    read_sloc(Sl);
-                    fold_sloc(Sl, true);
-                    ptx::tc_fence_before_sync();
-                    __syncthreads();
-                }
-            }
-            exchange_states();
-        }
-        // ---- pass 2: outputs from the incoming state ----
-        for (int ci = 0; ci < n_chunks; ++ci) {
-            int c0, n;
-            chunk_bounds(ci, c0, n);
+    // ------------------------------------------------------------ schedule
+    // Non-resident segments (several chunks) run a state-only pass first (all ranks but the
+    // last), then the exchange, then the full pass; a resident segment (one chunk) runs the
+    // full pass once and exchanges mid-chunk.  Every CTA exchanges exactly once.
+    const int n_pass1 = (!resident && exchange && rank < p.segs - 1) ? n_chunks : 0;
+    for (int step = 0; step < n_pass1 + n_chunks; ++step) {
+        const bool pass1 = step < n_pass1;
+        const int ci = pass1 ? step : step - n_pass1;
+        if (!pass1 && ci == 0 && !resident && exchange) exchange_states();
+        int n;
+        {
+            const int c0 = p0 + ci * chunk_len;
+            n = min(chunk_len, p1 - c0);
             __syncthreads();
             set_rows(c0, n);
             if (tid == 0) m.slow = 0;
             __syncthreads();
-            load_tile(p.k, kTK, n); load_tile(p.a, kTA, n); load_tile(p.v, kTV, n);
-            load_tile(p.q, kTQ, n); load_tile(p.g, kTG, n);
-            ptx::cp_async_commit();
-            ptx::cp_async_wait_all();
-            __syncthreads();
-            gate(n);
-            finish_gate();
-            build_operands(true);
-            mma_round(1);
-            read_sloc(Sl);
-            finish_chunk(n, Sl, ci + 1 < n_chunks);
         }
+        issue_loads(n, !pass1);
+        gate(n);
+        build_operands(!pass1);
+        mma_round(pass1 ? 0 : 1);
+        read_sloc();
+        if (pass1 || (resident && exchange)) fold_sloc(true);   // S = S 2^{B} + Sloc, Gs += B
+        if (pass1) {
+            ptx::tc_fence_before_sync();
+            __syncthreads();
+            ++it;
+            continue;
+        }
+        if (resident && exchange) exchange_states();
+        if (m.slow) make_p_exact(sm, t, ch, n, p.scale, &m.range_err); else make_p_fast();
+        write_stilde();
+        mma_round(2);
+        epilogue(n);
+        if (ci + 1 < n_chunks) fold_sloc(false);
+        ptx::tc_fence_before_sync();
+        __syncthreads();
+        ++it;
     }
 
     // ---- teardown ----
@@ -688,10 +724,10 @@ __global__ void __launch_bounds__(kThreads, 1) gla_tc_kernel(const Params p) {
 // Runs one of the kernel's four MMA configurations on row-major fp32 inputs
 // (converted to the operand type in the same shared-memory layouts) and
 // writes D row-major: 0 = scores (split tf32, A[128][64] . B[128][64]^T -> [128][128]),
-// 1 = state (f16, A[128][64]^T . B[128][64] -> [64][64]), 2 = PV (f16,
+// 1 = state (f16, B[128][64]^T . A[128][64] -> [64][64]), 2 = PV (f16,
 // A[128][128] . B[128][64] -> [128][64]), 3 = inter (tf32, A[128][64] .
-// B[64][64]^T -> [128][64]).  One CTA of 128 threads.
-__global__ void __launch_bounds__(kThreads, 1)
+// B[64][64]^T -> [128][64]).  One CTA of kSelfThreads = 128 threads.
+__global__ void __launch_bounds__(kSelfThreads, 1)
 gla_tc_selftest_kernel(int kind, const float *A, const float *Bm, float *Dout) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -704,7 +740,7 @@ gla_tc_selftest_kernel(int kind, const float *A, const float *Bm, float *Dout) {
         ptx::tmem_relinquish();
     }
     if (tid == 0) {
-        ptx::mbar_init(&m.mbar[0], 1);
+        ptx::mbar_init(&m.mbar_mma[0], 1);
         ptx::fence_mbarrier_init();
     }
     ptx::tc_fence_before_sync();
@@ -774,9 +810,9 @@ gla_tc_selftest_kernel(int kind, const float *A, const float *Bm, float *Dout) {
         else if (kind == 1) issue_state(sbase, tmem);
         else if (kind == 2) issue_pv(sbase, kPB, tmem);
         else issue_inter(sbase, tmem, false);
-        ptx::mma_commit(&m.mbar[0]);
+        ptx::mma_commit(&m.mbar_mma[0]);
     }
-    wait_phase(&m.mbar[0], 0);
+    wait_phase(&m.mbar_mma[0], 0);
     ptx::tc_fence_after_sync();
     if (kind == 0) {
         for (int blk = 0; blk < 4; ++blk) {

@@ -25,7 +25,7 @@ def tf32_round(x):
 
 CASES = {
     0: ((128, 64), (128, 64), (128, 128), "split", lambda a, b: a @ b.T),
-    1: ((128, 64), (128, 64), (64, 64), "f16", lambda a, b: a.T @ b),
+    1: ((128, 64), (128, 64), (64, 64), "f16", lambda a, b: b.T @ a),
     2: ((128, 128), (128, 64), (128, 64), "f16", lambda a, b: a @ b),
     3: ((128, 64), (64, 64), (128, 64), "tf32", lambda a, b: a @ b.T),
 }
