@@ -88,7 +88,6 @@ constexpr uint32_t kColO = 192;    // output accumulator 128 x 64
 constexpr uint32_t kColQH = 256;   // Q~ high part, tf32 A operand, 128 x 64
 constexpr uint32_t kColQL = 320;   // Q~ low part
 
-constexpr uint32_t kIdescQK = ptx::idesc_make(2, false, false, 128, 128);
 constexpr uint32_t kIdescST = ptx::idesc_make(0, true, true, 64, 64);
 constexpr uint32_t kIdescPV = ptx::idesc_make(0, false, true, 128, 64);
 constexpr uint32_t kIdescIN = ptx::idesc_make(2, false, false, 128, 64);
@@ -118,7 +117,9 @@ __device__ __forceinline__ uint32_t off_f16k128(uint32_t row, uint32_t j) {
 
 // ------------------------------------------------------------ MMA issue (1 thread)
 // scores[t][s] = sum_c Q~[t][c] K~[s][c] as Qh Kh^T + Qh Kl^T + Ql Kh^T
-__device__ __forceinline__ void issue_qk(uint32_t sbase, uint32_t tmem) {
+// Only the first n_cols score columns (the chunk's rows rounded up to 16) are produced.
+__device__ __forceinline__ void issue_qk(uint32_t sbase, uint32_t tmem, int n_cols) {
+    const uint32_t idesc = ptx::idesc_make(2, false, false, 128, (uint32_t)n_cols);
 #pragma unroll
     for (int pass = 0; pass < 3; ++pass) {
         const uint32_t acol = pass == 2 ? kColQL : kColQH;
@@ -127,7 +128,7 @@ __device__ __forceinline__ void issue_qk(uint32_t sbase, uint32_t tmem) {
         for (int k = 0; k < 8; ++k) {
             const uint32_t koff = (k >> 2) * kAtom128 + (k & 3) * 32;
             ptx::mma_tf32_ts(tmem + kColDS, tmem + acol + 8 * k,
-                             ptx::desc_sw128(sbase + bsm + koff, 16, 1024), kIdescQK,
+                             ptx::desc_sw128(sbase + bsm + koff, 16, 1024), idesc,
                              pass > 0 || k > 0);
         }
     }
@@ -194,7 +195,7 @@ __device__ __forceinline__ uint32_t pack_half2(float lo, float hi) {
 
 // Shared scratch scalars.
 struct Misc {
-    uint64_t mbar_mma[2];     // [0] score + state products, [1] P.V + inter products
+    uint64_t mbar_mma[3];     // [0] state product, [1] score products, [2] P.V + inter
     uint64_t mbar_ld[3];      // [0] a tile, [1] q and k tiles, [2] v and g tiles
     uint32_t tmem_base;
     int slow;                 // chunk uses the exact CUDA-core score path
@@ -212,6 +213,7 @@ struct Misc {
     alignas(16) float tot[8][kD]; // per-16-row totals of the gate scan
     alignas(16) float Gall[16][kD]; // every segment's log2-decay (exchange)
     alignas(16) float red[2][kC]; // epilogue partial sums of squares (per channel half)
+    alignas(16) float dqp[2][kC]; // diagonal score q_t . k_t, per channel half
 };
 static_assert(sizeof(Misc) <= kMiscBytes, "misc region");
 
@@ -272,30 +274,21 @@ __global__ void __launch_bounds__(kThreads, 1) gla_tc_kernel(const Params p) {
     const bool exchange = p.segs > 1;
     const bool resident = n_chunks <= 1;
 
-    // ---- setup: TMEM, barriers, weight ----
-    if (warp == 0) {
-        ptx::tmem_alloc(&m.tmem_base, kTmemCols);
-        ptx::tmem_relinquish();
-    }
+    // ---- setup: barriers and weight; TMEM is allocated once the first gathers are in flight
     if (tid == 0) {
-        ptx::mbar_init(&m.mbar_mma[0], 1);
-        ptx::mbar_init(&m.mbar_mma[1], 1);
+        for (int i = 0; i < 3; ++i) ptx::mbar_init(&m.mbar_mma[i], 1);
         for (int i = 0; i < 3; ++i) ptx::mbar_init(&m.mbar_ld[i], kThreads);
         ptx::fence_mbarrier_init();
         m.abort = 0;
         m.range_err = 0;
     }
-    if (tid < kD) {
-        m.w[tid] = p.w[tid];
-        m.Gs[tid] = 0.0f;
-    }
-    ptx::tc_fence_before_sync();
+    if (tid < kD) m.Gs[tid] = 0.0f;
+    // RMSNorm weight: async copy, covered by the first chunk's v/g load group
+    if (tid < kD / 4) ptx::cp_async16(ptx::smem_u32(&m.w[4 * tid]), p.w + 4 * tid, 16);
     __syncthreads();
-    ptx::tc_fence_after_sync();
-    const uint32_t tmem = m.tmem_base;
-    const uint32_t tmem_warp = tmem + ((uint32_t)(w4 * 32) << 16);
+    uint32_t tmem = 0, tmem_warp = 0;
     uint32_t it = 0;                  // chunk iterations so far (load-barrier parity)
-    uint32_t ph_mma0 = 0, ph_mma1 = 0;
+    uint32_t ph_mma[3] = {0, 0, 0};
 
     // State rows owned by lanes < 16: state column j = 16*w4 + lane (a row of the transposed
     // state), channels c in [32*ch, 32*ch + 32).
@@ -395,6 +388,7 @@ __global__ void __launch_bounds__(kThreads, 1) gla_tc_kernel(const Params p) {
     // slow path: Qh = d_k^{-1/2} q 2^{b}, Ks.  full = false builds Ks only.
     auto build_operands = [&](bool full) {
         const bool slow = m.slow != 0;
+        float dqs = 0.0f;                          // partial q_t . k_t over this half's channels
         wait_bar(&m.mbar_ld[1], it & 1);
 #pragma unroll 1
         for (int jj = 0; jj < 4; ++jj) {
@@ -424,6 +418,10 @@ __global__ void __launch_bounds__(kThreads, 1) gla_tc_kernel(const Params p) {
             }
             // tf32 splits: high = low 13 bits cleared, low = exact remainder (the tensor core
             // drops the low part's own low bits: error <= 2^-20 of the value)
+            if (full) {
+#pragma unroll
+                for (int e = 0; e < 8; ++e) dqs = fmaf(qv[e], kv[e], dqs);
+            }
             float ks[8], qh[8], ql[8], kh[8], kl[8];
 #pragma unroll
             for (int e = 0; e < 8; ++e) {
@@ -461,37 +459,22 @@ __global__ void __launch_bounds__(kThreads, 1) gla_tc_kernel(const Params p) {
                 }
             }
         }
-        if (full) ptx::tmem_st_wait();
+        if (full) {
+            m.dqp[ch][t] = dqs;
+            ptx::tmem_st_wait();
+        }
     };
-    // ------------------------------------------------------------ MMA rounds (one thread issues)
-    // which: 0 = state only, 1 = scores (+ state), 2 = P.V + inter
-    auto mma_round = [&](int which) {
-        if (which < 2) wait_bar(&m.mbar_ld[2], it & 1);   // V is an operand of the state product
+    // ------------------------------------------------------------ MMA issue (one thread)
+    // Make every thread's shared-memory operand writes visible to the tensor core, then
+    // let thread 0 issue.
+    auto operands_ready = [&]() {
         ptx::fence_proxy_async_smem();
         ptx::tc_fence_before_sync();
         __syncthreads();
-        if (tid == 0) {
-            ptx::tc_fence_after_sync();
-            if (which == 0) {
-                issue_state(sbase, tmem);
-                ptx::mma_commit(&m.mbar_mma[0]);
-            } else if (which == 1) {
-                if (!m.slow) issue_qk(sbase, tmem);
-                issue_state(sbase, tmem);
-                ptx::mma_commit(&m.mbar_mma[0]);
-            } else {
-                issue_pv(sbase, m.slow ? kKH : kPB, tmem);
-                issue_inter(sbase, tmem, true);
-                ptx::mma_commit(&m.mbar_mma[1]);
-            }
-        }
-        if (which == 2) {
-            wait_bar(&m.mbar_mma[1], ph_mma1);
-            ph_mma1 ^= 1u;
-        } else {
-            wait_bar(&m.mbar_mma[0], ph_mma0);
-            ph_mma0 ^= 1u;
-        }
+    };
+    auto wait_mma = [&](int i) {
+        wait_bar(&m.mbar_mma[i], ph_mma[i]);
+        ph_mma[i] ^= 1u;
         ptx::tc_fence_after_sync();
     };
     // transposed chunk state (TMEM, M=64 layout) -> registers of the state owners (warp-wide)
@@ -500,62 +483,55 @@ __global__ void __launch_bounds__(kThreads, 1) gla_tc_kernel(const Params p) {
         ptx::tmem_ld_wait();
     };
     // ------------------------------------------------------------ P (row t, 64 columns)
-    auto make_p_fast = [&]() {
-        if (ch == 1 && t < 64) {                       // whole half above the diagonal
-            const uint4 z = make_uint4(0, 0, 0, 0);
-#pragma unroll
-            for (int j = 0; j < 8; ++j) *reinterpret_cast<uint4 *>(sm + kPB + off_f16k128(t, 8 + j)) = z;
-            return;
-        }
-        float dq = 0.0f;                               // exact diagonal score q_t . k_t
-        if ((t >> 6) == ch) {
-#pragma unroll
-            for (int j = 0; j < 8; ++j) {
-                const uint4 kraw = *reinterpret_cast<const uint4 *>(sm + kTK + off_f16(t, j));
-                const uint4 qraw = *reinterpret_cast<const uint4 *>(sm + kTQ + off_f16(t, j));
-                const __half2 *k2 = reinterpret_cast<const __half2 *>(&kraw);
-                const __half2 *q2 = reinterpret_cast<const __half2 *>(&qraw);
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const float2 kf = __half22float2(k2[e]), qf = __half22float2(q2[e]);
-                    dq = fmaf(qf.x, kf.x, dq);
-                    dq = fmaf(qf.y, kf.y, dq);
-                }
-            }
-            dq *= p.scale;
-        }
-        float amax = 0.0f;
-#pragma unroll 1
-        for (int blk = 0; blk < 2; ++blk) {
-            const int s0 = ch * 64 + blk * 32;
-            uint8_t *dst = sm + kPB;
-            const int jb = ch * 8 + blk * 4;
-            if (s0 > t) {                              // block above the diagonal: zeros
-                const uint4 z = make_uint4(0, 0, 0, 0);
-#pragma unroll
-                for (int j4 = 0; j4 < 4; ++j4) *reinterpret_cast<uint4 *>(dst + off_f16k128(t, jb + j4)) = z;
-                continue;
-            }
-            float r[32];
+    // P block: columns [s0, s0 + 32) of row t, fp16 into the b region.  The TMEM load is
+    // warp-collective (.sync.aligned): it is skipped only when the whole warp's rows lie above
+    // the block (a warp-uniform test); pad rows t >= n and entries s > t are zeroed per lane.
+    auto p_block = [&](int s0, int n, float dq, float &amax) {
+        uint8_t *dst = sm + kPB;
+        const int jb = s0 >> 3;
+        const bool warp_above = s0 > 32 * w4 + 31;
+        float r[32];
+        if (!warp_above) {
             ptx::tmem_ld32(tmem_warp + kColDS + s0, r);
             ptx::tmem_ld_wait();
-            if (s0 + 31 >= t) {                        // block holding the diagonal
+        }
+        if (warp_above || s0 > t || t >= n) {
+            const uint4 z = make_uint4(0, 0, 0, 0);
 #pragma unroll
-                for (int e = 0; e < 32; ++e) {
-                    const int s = s0 + e;
-                    r[e] = s < t ? r[e] : (s == t ? dq : 0.0f);
-                }
-            }
+            for (int j4 = 0; j4 < 4; ++j4) *reinterpret_cast<uint4 *>(dst + off_f16k128(t, jb + j4)) = z;
+            return;
+        }
+        if (s0 + 31 >= t) {                            // block holding the diagonal
 #pragma unroll
-            for (int e = 0; e < 32; ++e) amax = fmaxf(amax, fabsf(r[e]));
-#pragma unroll
-            for (int j4 = 0; j4 < 4; ++j4) {
-                uint4 o;
-                o.x = pack_half2(r[8 * j4], r[8 * j4 + 1]); o.y = pack_half2(r[8 * j4 + 2], r[8 * j4 + 3]);
-                o.z = pack_half2(r[8 * j4 + 4], r[8 * j4 + 5]); o.w = pack_half2(r[8 * j4 + 6], r[8 * j4 + 7]);
-                *reinterpret_cast<uint4 *>(dst + off_f16k128(t, jb + j4)) = o;
+            for (int e = 0; e < 32; ++e) {
+                const int s = s0 + e;
+                r[e] = s < t ? r[e] : (s == t ? dq : 0.0f);
             }
         }
+#pragma unroll
+        for (int e = 0; e < 32; ++e) amax = fmaxf(amax, fabsf(r[e]));
+#pragma unroll
+        for (int j4 = 0; j4 < 4; ++j4) {
+            uint4 o;
+            o.x = pack_half2(r[8 * j4], r[8 * j4 + 1]); o.y = pack_half2(r[8 * j4 + 2], r[8 * j4 + 3]);
+            o.z = pack_half2(r[8 * j4 + 4], r[8 * j4 + 5]); o.w = pack_half2(r[8 * j4 + 6], r[8 * j4 + 7]);
+            *reinterpret_cast<uint4 *>(dst + off_f16k128(t, jb + j4)) = o;
+        }
+    };
+    // all warps: row t, the 64 columns of this thread's half
+    auto make_p_fast = [&](int n) {
+        const float dq = (m.dqp[0][t] + m.dqp[1][t]) * p.scale;   // exact diagonal score
+        float amax = 0.0f;
+        p_block(ch * 64, n, dq, amax);
+        p_block(ch * 64 + 32, n, dq, amax);
+        if (amax > 65504.0f) m.range_err = 1;
+    };
+    // warps 4..7 only: row t, all 128 columns (the other warps run the state exchange)
+    auto make_p_rows = [&](int n) {
+        const float dq = (m.dqp[0][t] + m.dqp[1][t]) * p.scale;
+        float amax = 0.0f;
+#pragma unroll 1
+        for (int b4 = 0; b4 < 4; ++b4) p_block(b4 * 32, n, dq, amax);
         if (amax > 65504.0f) m.range_err = 1;
     };
     // S~[j][c] = 2^{r_c} S_in[c][j], tf32 K-major (rows j, 2 atoms of 32 channels)
@@ -620,9 +596,11 @@ __global__ void __launch_bounds__(kThreads, 1) gla_tc_kernel(const Params p) {
         }
         if (into_g && tid < kD) m.Gs[tid] += m.Bc[tid];
     };
-    // cluster-wide scan of (Gs, S) -> S becomes this segment's incoming state
-    auto exchange_states = [&]() {
-        float *X = reinterpret_cast<float *>(sm + kST);  // [64 j][64 c] fp32, plain row-major
+    // Cluster-wide scan of the segment aggregates (Gs, S): every segment receives its
+    // incoming state.  Split in two so P can be built while the cluster barrier settles:
+    // xchg_begin publishes this CTA's aggregate, xchg_end scans and reads the result.
+    float *X = reinterpret_cast<float *>(sm + kST);  // [64 j][64 c] fp32, plain row-major
+    auto xchg_begin = [&]() {
         __syncthreads();
         if (s_owner) {
 #pragma unroll
@@ -630,38 +608,52 @@ __global__ void __launch_bounds__(kThreads, 1) gla_tc_kernel(const Params p) {
                 *reinterpret_cast<float4 *>(X + s_row * kD + 32 * ch + 4 * i) =
                     make_float4(S[4 * i], S[4 * i + 1], S[4 * i + 2], S[4 * i + 3]);
         }
-        cg::cluster_group cluster = cg::this_cluster();
-        cluster.sync();
-        const int segs = p.segs;
-        // every segment's decay, copied once into local shared memory
-        for (int i = tid; i < segs * kD; i += kThreads) {
-            const int r = i / kD, c = i - r * kD;
-            m.Gall[r][c] = ptx::ex2(*cluster.map_shared_rank(&m.Gs[c], r));
-        }
-        __syncthreads();
-        const int E = kD * kD;
-        const int per = (E + segs - 1) / segs;
-        const int e0 = rank * per, e1 = min(E, e0 + per);
-        for (int e = e0 + tid; e < e1; e += kThreads) {
-            const int c = e & (kD - 1);
-            float x[16];
-#pragma unroll
-            for (int r = 0; r < 16; ++r)
-                if (r < segs) x[r] = *cluster.map_shared_rank(X + e, r);
-            float run = 0.0f;
-#pragma unroll
-            for (int r = 0; r < 16; ++r) {
-                if (r < segs) {
-                    const float agg = x[r];
-                    x[r] = run;                       // state entering segment r
-                    run = fmaf(m.Gall[r][c], run, agg);
-                }
+        ptx::cluster_arrive();
+    };
+    // Second half of the exchange.  Called by every thread (the cluster barriers count them
+    // all); the DSMEM scan itself runs on warps 0..3 (`scanners`), synchronised among
+    // themselves with named barrier 1, while the other warps are free for other work before
+    // calling in.
+    auto xchg_end = [&](bool scanners) {
+        ptx::cluster_wait();
+        if (scanners) {
+            const int segs = p.segs;
+            const int sid = tid & 127;
+            // every segment's decay, fetched once (16-byte remote loads)
+            for (int i = sid; i < segs * (kD / 4); i += 128) {
+                const int r = i / (kD / 4), c4 = i - r * (kD / 4);
+                const float4 g = ptx::ld_cluster_v4(ptx::mapa(ptx::smem_u32(&m.Gs[4 * c4]), r));
+                *reinterpret_cast<float4 *>(&m.Gall[r][4 * c4]) =
+                    make_float4(ptx::ex2(g.x), ptx::ex2(g.y), ptx::ex2(g.z), ptx::ex2(g.w));
             }
+            ptx::named_bar_sync(1, 128);
+            const int E2 = kD * kD / 2;                   // float2 pairs of the state
+            const int per = (E2 + segs - 1) / segs;
+            const int e0 = rank * per, e1 = min(E2, e0 + per);
+            const uint32_t xbase = ptx::smem_u32(X);
+            for (int e = e0 + sid; e < e1; e += 128) {
+                const int c = (2 * e) & (kD - 1);
+                float2 x[16];
 #pragma unroll
-            for (int r = 0; r < 16; ++r)
-                if (r < segs) *cluster.map_shared_rank(X + e, r) = x[r];
+                for (int r = 0; r < 16; ++r)
+                    if (r < segs) x[r] = ptx::ld_cluster_v2(ptx::mapa(xbase + 8u * e, r));
+                float2 run = make_float2(0.0f, 0.0f);
+#pragma unroll
+                for (int r = 0; r < 16; ++r) {
+                    if (r < segs) {
+                        const float2 agg = x[r];
+                        const float2 g = *reinterpret_cast<const float2 *>(&m.Gall[r][c]);
+                        x[r] = run;                       // state entering segment r
+                        run = make_float2(fmaf(g.x, run.x, agg.x), fmaf(g.y, run.y, agg.y));
+                    }
+                }
+#pragma unroll
+                for (int r = 0; r < 16; ++r)
+                    if (r < segs) ptx::st_cluster_v2(ptx::mapa(xbase + 8u * e, r), x[r]);
+            }
         }
-        cluster.sync();
+        ptx::cluster_arrive();
+        ptx::cluster_wait();
         if (s_owner) {
 #pragma unroll
             for (int i = 0; i < 8; ++i) {
@@ -680,7 +672,10 @@ __global__ void __launch_bounds__(kThreads, 1) gla_tc_kernel(const Params p) {
     for (int step = 0; step < n_pass1 + n_chunks; ++step) {
         const bool pass1 = step < n_pass1;
         const int ci = pass1 ? step : step - n_pass1;
-        if (!pass1 && ci == 0 && !resident && exchange) exchange_states();
+        if (!pass1 && ci == 0 && !resident && exchange) {
+            xchg_begin();
+            xchg_end(warp < 4);
+        }
         int n;
         {
             const int c0 = p0 + ci * chunk_len;
@@ -691,21 +686,67 @@ __global__ void __launch_bounds__(kThreads, 1) gla_tc_kernel(const Params p) {
             __syncthreads();
         }
         issue_loads(n, !pass1);
-        gate(n);
+        if (step == 0 && warp == 0) {                // overlaps the first gathers' latency
+            ptx::tmem_alloc(&m.tmem_base, kTmemCols);
+            ptx::tmem_relinquish();
+            ptx::tc_fence_before_sync();
+        }
+        gate(n);                                     // contains block barriers
+        if (step == 0) {
+            ptx::tc_fence_after_sync();
+            tmem = m.tmem_base;
+            tmem_warp = tmem + ((uint32_t)(w4 * 32) << 16);
+        }
         build_operands(!pass1);
-        mma_round(pass1 ? 0 : 1);
+        wait_bar(&m.mbar_ld[2], it & 1);             // V, an operand of the state product
+        operands_ready();
+        // The state product goes first: the segment aggregate is published while the score
+        // products run.  The issuing thread stalls while its products drain, so the score
+        // products are issued only after this CTA has arrived on the cluster barrier.
+        if (tid == 0) {
+            ptx::tc_fence_after_sync();
+            issue_state(sbase, tmem);
+            ptx::mma_commit(&m.mbar_mma[0]);
+        }
+        wait_mma(0);
         read_sloc();
-        if (pass1 || (resident && exchange)) fold_sloc(true);   // S = S 2^{B} + Sloc, Gs += B
+        const bool mid_xchg = !pass1 && resident && exchange;
+        if (pass1 || mid_xchg) fold_sloc(true);     // S = S 2^{B} + Sloc, Gs += B
         if (pass1) {
             ptx::tc_fence_before_sync();
             __syncthreads();
             ++it;
             continue;
         }
-        if (resident && exchange) exchange_states();
-        if (m.slow) make_p_exact(sm, t, ch, n, p.scale, &m.range_err); else make_p_fast();
+        if (mid_xchg) xchg_begin();
+        if (tid == 0) {
+            if (!m.slow) issue_qk(sbase, tmem, min(kC, (n + 15) & ~15));
+            ptx::mma_commit(&m.mbar_mma[1]);
+        }
+        wait_mma(1);
+        if (m.slow) {
+            make_p_exact(sm, t, ch, n, p.scale, &m.range_err);
+            if (mid_xchg) xchg_end(warp < 4);
+        } else if (mid_xchg) {
+            // warps 4..7 build P while warps 0..3 scan the segment states
+            if (warp >= 4) make_p_rows(n);
+            xchg_end(warp < 4);
+        } else {
+            make_p_fast(n);
+        }
+        operands_ready();
+        if (tid == 0) {
+            ptx::tc_fence_after_sync();
+            issue_pv(sbase, m.slow ? kKH : kPB, tmem);
+        }
         write_stilde();
-        mma_round(2);
+        operands_ready();
+        if (tid == 0) {
+            ptx::tc_fence_after_sync();
+            issue_inter(sbase, tmem, true);
+            ptx::mma_commit(&m.mbar_mma[2]);
+        }
+        wait_mma(2);
         epilogue(n);
         if (ci + 1 < n_chunks) fold_sloc(false);
         ptx::tc_fence_before_sync();
@@ -717,7 +758,7 @@ __global__ void __launch_bounds__(kThreads, 1) gla_tc_kernel(const Params p) {
     __syncthreads();
     if (tid == 0 && m.range_err) raise_status(8 /* GLA_ERR_RANGE */);
     ptx::tc_fence_after_sync();
-    if (warp == 0) ptx::tmem_dealloc(tmem, kTmemCols);
+    if (warp == 0 && n_pass1 + n_chunks > 0) ptx::tmem_dealloc(tmem, kTmemCols);
 }
 
 // ---------------------------------------------------------------- self-test
@@ -806,7 +847,7 @@ gla_tc_selftest_kernel(int kind, const float *A, const float *Bm, float *Dout) {
     __syncthreads();
     if (tid == 0) {
         ptx::tc_fence_after_sync();
-        if (kind == 0) issue_qk(sbase, tmem);
+        if (kind == 0) issue_qk(sbase, tmem, kC);
         else if (kind == 1) issue_state(sbase, tmem);
         else if (kind == 2) issue_pv(sbase, kPB, tmem);
         else issue_inter(sbase, tmem, false);
