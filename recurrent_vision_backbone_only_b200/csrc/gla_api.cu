@@ -106,7 +106,8 @@ struct Plan {
     size_t smem = 0;
     int max_active_clusters = 0;
     cudaLaunchConfig_t cfg{};
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
+    bool pdl = false;          // programmatic dependent launch (tensor-core kernel)
 };
 
 void configure_launch(Plan &pl, int n_pairs, int threads, cudaStream_t st) {
@@ -121,6 +122,11 @@ void configure_launch(Plan &pl, int n_pairs, int threads, cudaStream_t st) {
     pl.attr[0].val.clusterDim.z = 1;
     pl.cfg.attrs = pl.attr;
     pl.cfg.numAttrs = 1;
+    if (pl.pdl) {
+        pl.attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        pl.attr[1].val.programmaticStreamSerializationAllowed = 1;
+        pl.cfg.numAttrs = 2;
+    }
 }
 
 // Pick the segment count (auto when segs <= 0), shrinking it until a cluster
@@ -227,6 +233,7 @@ int run_tc(const Args &x, int chunk, int segs, float eps, cudaStream_t st, const
     pl.kernel = 1;
     pl.chunk = chunk;
     pl.smem = tc::kSmemBytes;
+    pl.pdl = true;
     int rc = make_plan(kern, pl, L, n_pairs, segs, 1, tc::kThreads, st, di);
     if (rc != GLA_OK) return rc;
     if (query) {

@@ -68,14 +68,14 @@ constexpr float kHalfRangeSafe2 = 86.0f;
 constexpr uint32_t kKL = 0;        // K~ low part  tf32, 2 atoms x [128][128B]
 constexpr uint32_t kKH = 32768;    // K~ high part tf32, 2 atoms x [128][128B] (slow path: P)
 constexpr uint32_t kPB = 65536;    // b   fp32 (QT layout), then P fp16 2 atoms x [128][128B]
-constexpr uint32_t kST = 98304;    // Ks fp16 [128][128B] / S~ tf32 2 x [64][128B] / exchange fp32
+constexpr uint32_t kST = 98304;    // Ks fp16 [128][128B] / state exchange fp32 [64][64]
 constexpr uint32_t kTQ = 114688;   // raw tiles, fp16 [128][128B] each
 constexpr uint32_t kTK = 131072;
-constexpr uint32_t kTA = 147456;
+constexpr uint32_t kTA = 147456;   // a tile; after the gate: S~ tf32 2 x [64][128B]
 constexpr uint32_t kTV = 163840;
 constexpr uint32_t kTG = 180224;
 constexpr uint32_t kMISC = 196608;
-constexpr uint32_t kMiscBytes = 12288;
+constexpr uint32_t kMiscBytes = 16384;
 constexpr uint32_t kAtom128 = 16384;   // [128 rows][128 B]
 constexpr uint32_t kAtom64 = 8192;     // [64 rows][128 B]
 constexpr size_t kSmemBytes = kMISC + kMiscBytes + 1024;  // + misc + alignment slack
@@ -84,9 +84,10 @@ constexpr size_t kSmemBytes = kMISC + kMiscBytes + 1024;  // + misc + alignment 
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColDS = 0;     // scores, 128 x 128 fp32
 constexpr uint32_t kColSL = 128;   // chunk state Ks^T V, M=64 layout
-constexpr uint32_t kColO = 192;    // output accumulator 128 x 64
+constexpr uint32_t kColO = 192;    // inter-chunk output accumulator 128 x 64
 constexpr uint32_t kColQH = 256;   // Q~ high part, tf32 A operand, 128 x 64
 constexpr uint32_t kColQL = 320;   // Q~ low part
+constexpr uint32_t kColOP = 384;   // intra-chunk output accumulator (P V) 128 x 64
 
 constexpr uint32_t kIdescST = ptx::idesc_make(0, true, true, 64, 64);
 constexpr uint32_t kIdescPV = ptx::idesc_make(0, false, true, 128, 64);
@@ -147,11 +148,11 @@ __device__ __forceinline__ void issue_pv(uint32_t sbase, uint32_t p_base, uint32
 #pragma unroll
     for (int k = 0; k < 8; ++k) {
         const uint32_t koff = (k >> 2) * kAtom128 + (k & 3) * 32;
-        ptx::mma_f16_ss(tmem + kColO, ptx::desc_sw128(sbase + p_base + koff, 16, 1024),
+        ptx::mma_f16_ss(tmem + kColOP, ptx::desc_sw128(sbase + p_base + koff, 16, 1024),
                         ptx::desc_sw128(sbase + kTV + k * 2048, kAtom128, 1024), kIdescPV, k > 0);
     }
 }
-// O[t][j] += sum_c (Qh + Ql)[t][c] S~[j][c]
+// O[t][j] (+)= sum_c (Qh + Ql)[t][c] S~[j][c], S~ in the a-tile region
 __device__ __forceinline__ void issue_inter(uint32_t sbase, uint32_t tmem, bool accumulate) {
 #pragma unroll
     for (int pass = 0; pass < 2; ++pass) {
@@ -159,7 +160,7 @@ __device__ __forceinline__ void issue_inter(uint32_t sbase, uint32_t tmem, bool 
         for (int k = 0; k < 8; ++k) {
             const uint32_t soff = (k >> 2) * kAtom64 + (k & 3) * 32;
             ptx::mma_tf32_ts(tmem + kColO, tmem + (pass ? kColQL : kColQH) + 8 * k,
-                             ptx::desc_sw128(sbase + kST + soff, 16, 1024), kIdescIN,
+                             ptx::desc_sw128(sbase + kTA + soff, 16, 1024), kIdescIN,
                              accumulate || pass > 0 || k > 0);
         }
     }
@@ -195,7 +196,7 @@ __device__ __forceinline__ uint32_t pack_half2(float lo, float hi) {
 
 // Shared scratch scalars.
 struct Misc {
-    uint64_t mbar_mma[3];     // [0] state product, [1] score products, [2] P.V + inter
+    uint64_t mbar_mma[4];     // [0] state, [1] scores, [2] inter (+ P.V), [3] early P.V
     uint64_t mbar_ld[3];      // [0] a tile, [1] q and k tiles, [2] v and g tiles
     uint32_t tmem_base;
     int slow;                 // chunk uses the exact CUDA-core score path
@@ -211,7 +212,8 @@ struct Misc {
     alignas(16) float b0[kD];     // b_{0,c}
     alignas(16) float w[kD];      // RMSNorm weight
     alignas(16) float tot[8][kD]; // per-16-row totals of the gate scan
-    alignas(16) float Gall[16][kD]; // every segment's log2-decay (exchange)
+    alignas(16) float Gall[16][kD]; // 2^{Gs} of every segment, pushed by each (exchange)
+    alignas(16) float Eall[16][kD]; // 2^{r} of every segment (direct S~ writes)
     alignas(16) float red[2][kC]; // epilogue partial sums of squares (per channel half)
     alignas(16) float dqp[2][kC]; // diagonal score q_t . k_t, per channel half
 };
@@ -274,21 +276,25 @@ __global__ void __launch_bounds__(kThreads, 1) gla_tc_kernel(const Params p) {
     const bool exchange = p.segs > 1;
     const bool resident = n_chunks <= 1;
 
+    // Programmatic dependent launch: the next launch on the stream may start its prologue now;
+    // this grid touches no global memory before the previous grid has completed.
+    ptx::pdl_launch_dependents();
     // ---- setup: barriers and weight; TMEM is allocated once the first gathers are in flight
     if (tid == 0) {
-        for (int i = 0; i < 3; ++i) ptx::mbar_init(&m.mbar_mma[i], 1);
+        for (int i = 0; i < 4; ++i) ptx::mbar_init(&m.mbar_mma[i], 1);
         for (int i = 0; i < 3; ++i) ptx::mbar_init(&m.mbar_ld[i], kThreads);
         ptx::fence_mbarrier_init();
         m.abort = 0;
         m.range_err = 0;
     }
     if (tid < kD) m.Gs[tid] = 0.0f;
+    ptx::pdl_wait_prior_grid();
     // RMSNorm weight: async copy, covered by the first chunk's v/g load group
     if (tid < kD / 4) ptx::cp_async16(ptx::smem_u32(&m.w[4 * tid]), p.w + 4 * tid, 16);
     __syncthreads();
     uint32_t tmem = 0, tmem_warp = 0;
     uint32_t it = 0;                  // chunk iterations so far (load-barrier parity)
-    uint32_t ph_mma[3] = {0, 0, 0};
+    uint32_t ph_mma[4] = {0, 0, 0, 0};
 
     // State rows owned by lanes < 16: state column j = 16*w4 + lane (a row of the transposed
     // state), channels c in [32*ch, 32*ch + 32).
@@ -540,7 +546,7 @@ __global__ void __launch_bounds__(kThreads, 1) gla_tc_kernel(const Params p) {
 #pragma unroll
             for (int i = 0; i < 8; ++i) {
                 const float4 e4 = *reinterpret_cast<const float4 *>(&m.eref[32 * ch + 4 * i]);
-                *reinterpret_cast<float4 *>(sm + kST + off_tf32(kAtom64, s_row, 8 * ch + i)) =
+                *reinterpret_cast<float4 *>(sm + kTA + off_tf32(kAtom64, s_row, 8 * ch + i)) =
                     make_float4(ptx::to_tf32(S[4 * i] * e4.x), ptx::to_tf32(S[4 * i + 1] * e4.y),
                                 ptx::to_tf32(S[4 * i + 2] * e4.z), ptx::to_tf32(S[4 * i + 3] * e4.w));
             }
@@ -548,9 +554,12 @@ __global__ void __launch_bounds__(kThreads, 1) gla_tc_kernel(const Params p) {
     };
     // ------------------------------------------------------------ epilogue (row t, 32 channels)
     auto epilogue = [&](int n) {
-        float o[32];
+        float o[32], op[32];
         ptx::tmem_ld32(tmem_warp + kColO + 32 * ch, o);
+        ptx::tmem_ld32(tmem_warp + kColOP + 32 * ch, op);
         ptx::tmem_ld_wait();
+#pragma unroll
+        for (int j = 0; j < 32; ++j) o[j] += op[j];
         float ss = 0.0f;
 #pragma unroll
         for (int j = 0; j < 32; ++j) ss = fmaf(o[j], o[j], ss);
@@ -602,6 +611,15 @@ __global__ void __launch_bounds__(kThreads, 1) gla_tc_kernel(const Params p) {
     float *X = reinterpret_cast<float *>(sm + kST);  // [64 j][64 c] fp32, plain row-major
     auto xchg_begin = [&]() {
         __syncthreads();
+        // push this segment's decay 2^{Gs} into row `rank` of every CTA's table
+        if (tid < p.segs * (kD / 4)) {
+            const int r = tid / (kD / 4), c4 = tid - r * (kD / 4);
+            const float4 g = *reinterpret_cast<const float4 *>(&m.Gs[4 * c4]);
+            ptx::st_cluster_v4(ptx::mapa(ptx::smem_u32(&m.Gall[rank][4 * c4]), r),
+                               make_float4(ptx::ex2(g.x), ptx::ex2(g.y), ptx::ex2(g.z), ptx::ex2(g.w)));
+            ptx::st_cluster_v4(ptx::mapa(ptx::smem_u32(&m.Eall[rank][4 * c4]), r),
+                               *reinterpret_cast<const float4 *>(&m.eref[4 * c4]));
+        }
         if (s_owner) {
 #pragma unroll
             for (int i = 0; i < 8; ++i)
@@ -614,19 +632,13 @@ __global__ void __launch_bounds__(kThreads, 1) gla_tc_kernel(const Params p) {
     // all); the DSMEM scan itself runs on warps 0..3 (`scanners`), synchronised among
     // themselves with named barrier 1, while the other warps are free for other work before
     // calling in.
-    auto xchg_end = [&](bool scanners) {
+    // direct: the scanners write each segment's S~ = 2^{r} S_in (tf32, the inter product's B
+    // operand) straight into that CTA's a-tile region, and S is not read back (one chunk).
+    auto xchg_end = [&](bool scanners, bool direct) {
         ptx::cluster_wait();
         if (scanners) {
             const int segs = p.segs;
             const int sid = tid & 127;
-            // every segment's decay, fetched once (16-byte remote loads)
-            for (int i = sid; i < segs * (kD / 4); i += 128) {
-                const int r = i / (kD / 4), c4 = i - r * (kD / 4);
-                const float4 g = ptx::ld_cluster_v4(ptx::mapa(ptx::smem_u32(&m.Gs[4 * c4]), r));
-                *reinterpret_cast<float4 *>(&m.Gall[r][4 * c4]) =
-                    make_float4(ptx::ex2(g.x), ptx::ex2(g.y), ptx::ex2(g.z), ptx::ex2(g.w));
-            }
-            ptx::named_bar_sync(1, 128);
             const int E2 = kD * kD / 2;                   // float2 pairs of the state
             const int per = (E2 + segs - 1) / segs;
             const int e0 = rank * per, e1 = min(E2, e0 + per);
@@ -647,14 +659,29 @@ __global__ void __launch_bounds__(kThreads, 1) gla_tc_kernel(const Params p) {
                         run = make_float2(fmaf(g.x, run.x, agg.x), fmaf(g.y, run.y, agg.y));
                     }
                 }
+                if (direct) {
+                    const int j = (2 * e) >> 6;
+                    const uint32_t dst =
+                        ptx::smem_u32(sm + kTA + off_tf32(kAtom64, j, c >> 2) + (c & 3) * 4);
 #pragma unroll
-                for (int r = 0; r < 16; ++r)
-                    if (r < segs) ptx::st_cluster_v2(ptx::mapa(xbase + 8u * e, r), x[r]);
+                    for (int r = 0; r < 16; ++r) {
+                        if (r < segs) {
+                            const float2 f = *reinterpret_cast<const float2 *>(&m.Eall[r][c]);
+                            ptx::st_cluster_v2(ptx::mapa(dst, r),
+                                               make_float2(ptx::to_tf32(f.x * x[r].x),
+                                                           ptx::to_tf32(f.y * x[r].y)));
+                        }
+                    }
+                } else {
+#pragma unroll
+                    for (int r = 0; r < 16; ++r)
+                        if (r < segs) ptx::st_cluster_v2(ptx::mapa(xbase + 8u * e, r), x[r]);
+                }
             }
         }
         ptx::cluster_arrive();
         ptx::cluster_wait();
-        if (s_owner) {
+        if (!direct && s_owner) {
 #pragma unroll
             for (int i = 0; i < 8; ++i) {
                 const float4 v = *reinterpret_cast<const float4 *>(X + s_row * kD + 32 * ch + 4 * i);
@@ -674,7 +701,7 @@ __global__ void __launch_bounds__(kThreads, 1) gla_tc_kernel(const Params p) {
         const int ci = pass1 ? step : step - n_pass1;
         if (!pass1 && ci == 0 && !resident && exchange) {
             xchg_begin();
-            xchg_end(warp < 4);
+            xchg_end(warp < 4, false);
         }
         int n;
         {
@@ -709,8 +736,18 @@ __global__ void __launch_bounds__(kThreads, 1) gla_tc_kernel(const Params p) {
             ptx::mma_commit(&m.mbar_mma[0]);
         }
         wait_mma(0);
-        read_sloc();
         const bool mid_xchg = !pass1 && resident && exchange;
+        // Score products, issued by thread 128 (warp 4 builds P).  With a mid-chunk exchange
+        // they go out after this CTA has published its aggregate, so the issuing warp's stall
+        // does not delay the publication.
+        auto issue_scores = [&]() {
+            if (tid == 128) {
+                if (!m.slow) issue_qk(sbase, tmem, min(kC, (n + 15) & ~15));
+                ptx::mma_commit(&m.mbar_mma[1]);
+            }
+        };
+        if (!pass1 && !mid_xchg) issue_scores();
+        read_sloc();
         if (pass1 || mid_xchg) fold_sloc(true);     // S = S 2^{B} + Sloc, Gs += B
         if (pass1) {
             ptx::tc_fence_before_sync();
@@ -718,34 +755,52 @@ __global__ void __launch_bounds__(kThreads, 1) gla_tc_kernel(const Params p) {
             ++it;
             continue;
         }
-        if (mid_xchg) xchg_begin();
-        if (tid == 0) {
-            if (!m.slow) issue_qk(sbase, tmem, min(kC, (n + 15) & ~15));
-            ptx::mma_commit(&m.mbar_mma[1]);
+        if (mid_xchg) {
+            xchg_begin();
+            issue_scores();
         }
-        wait_mma(1);
+        const bool pv_early = mid_xchg && !m.slow;
         if (m.slow) {
+            wait_mma(1);
             make_p_exact(sm, t, ch, n, p.scale, &m.range_err);
-            if (mid_xchg) xchg_end(warp < 4);
+            if (mid_xchg) xchg_end(warp < 4, true);
         } else if (mid_xchg) {
-            // warps 4..7 build P while warps 0..3 scan the segment states
-            if (warp >= 4) make_p_rows(n);
-            xchg_end(warp < 4);
+            // warps 4..7 wait for the scores, build P and start P.V; warps 0..3 scan the
+            // segment states and write every segment's S~ directly
+            if (warp >= 4) {
+                wait_mma(1);
+                make_p_rows(n);
+                ptx::fence_proxy_async_smem();
+                ptx::tc_fence_before_sync();
+                ptx::named_bar_sync(2, 128);
+                if (tid == 128) {
+                    ptx::tc_fence_after_sync();
+                    issue_pv(sbase, kPB, tmem);
+                    ptx::mma_commit(&m.mbar_mma[3]);
+                }
+            } else {
+                ph_mma[1] ^= 1u;                      // this phase is consumed by warps 4..7
+            }
+            xchg_end(warp < 4, true);
         } else {
+            wait_mma(1);
             make_p_fast(n);
         }
-        operands_ready();
-        if (tid == 0) {
-            ptx::tc_fence_after_sync();
-            issue_pv(sbase, m.slow ? kKH : kPB, tmem);
+        if (!pv_early) {
+            operands_ready();
+            if (tid == 0) {
+                ptx::tc_fence_after_sync();
+                issue_pv(sbase, m.slow ? kKH : kPB, tmem);
+            }
         }
-        write_stilde();
+        if (!mid_xchg) write_stilde();
         operands_ready();
         if (tid == 0) {
             ptx::tc_fence_after_sync();
-            issue_inter(sbase, tmem, true);
+            issue_inter(sbase, tmem, false);
             ptx::mma_commit(&m.mbar_mma[2]);
         }
+        if (pv_early) wait_mma(3);
         wait_mma(2);
         epilogue(n);
         if (ci + 1 < n_chunks) fold_sloc(false);
@@ -840,7 +895,7 @@ gla_tc_selftest_kernel(int kind, const float *A, const float *Bm, float *Dout) {
         put_f16(kTV, t, Bm + t * 64);
     } else {
         put_split_tmem(A + t * 64, false);
-        if (t < 64) put_tf32(kST, kAtom64, t, Bm + t * 64);
+        if (t < 64) put_tf32(kTA, kAtom64, t, Bm + t * 64);
     }
     ptx::fence_proxy_async_smem();
     ptx::tc_fence_before_sync();
@@ -876,8 +931,9 @@ gla_tc_selftest_kernel(int kind, const float *A, const float *Bm, float *Dout) {
         }
     } else {
         float r0[32], r1[32];
-        ptx::tmem_ld32(tmem_warp + kColO, r0);
-        ptx::tmem_ld32(tmem_warp + kColO + 32, r1);
+        const uint32_t col = kind == 2 ? kColOP : kColO;
+        ptx::tmem_ld32(tmem_warp + col, r0);
+        ptx::tmem_ld32(tmem_warp + col + 32, r1);
         ptx::tmem_ld_wait();
         for (int j = 0; j < 32; ++j) {
             Dout[t * 64 + j] = r0[j];
