@@ -49,6 +49,9 @@ def parse():
     ap.add_argument("--cpu-seconds", type=float, default=10.0,
                     help="CPU-oracle sample budget for cpu_baseline / --impl reference")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--workload", default=WORKLOAD,
+                    help="synthetic workload to time (default: the 40x40 headline); the others "
+                         "are reported with their own metric name")
     return ap.parse_args()
 
 
@@ -135,7 +138,7 @@ class ClockSampler:
                 "samples": len(rows)}
 
 
-def cpu_oracle_sample(wl, x, budget_s: float):
+def cpu_oracle_sample(wl, x, budget_s: float, directions=DIRECTIONS):
     """Time the fp64 oracle on whole (direction) passes of the workload until the budget."""
     import numpy as np
     import oracle
@@ -146,7 +149,7 @@ def cpu_oracle_sample(wl, x, budget_s: float):
     passes, tokens = 0, 0
     t0 = time.perf_counter()
     while True:
-        d = DIRECTIONS[passes % len(DIRECTIONS)]
+        d = directions[passes % len(directions)]
         oracle.gla_forward(xs["q"], xs["k"], xs["v"], xs["a"], xs["g"], xs["w"],
                            wl.grid_h, wl.grid_w, d, threads=threads)
         passes += 1
@@ -232,13 +235,14 @@ def run_ours(args, ws, rank, local):
     _b.build()
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
-    wl = synth.WORKLOADS[WORKLOAD]
+    wl = synth.WORKLOADS[args.workload]
     x = synth.make_inputs(wl)
     gh, gw = wl.grid_h, wl.grid_w
+    directions = wl.directions if args.workload != WORKLOAD else DIRECTIONS
 
     # rotating pool of input sets, total larger than L2
     set_bytes = wl.tokens * wl.bytes_per_token
-    n_sets = max(8, math.ceil(2 * L2_BYTES / set_bytes))
+    n_sets = max(2 if set_bytes > L2_BYTES else 8, math.ceil(2 * L2_BYTES / set_bytes))
     base = {n: torch.from_numpy(x[n]).to(dev) for n in ("q", "k", "v", "a", "g")}
     w = torch.from_numpy(x["w"]).to(dev)
     sets = []
@@ -246,10 +250,11 @@ def run_ours(args, ws, rank, local):
         s = {n: base[n].clone() for n in base}
         s["out"] = torch.empty_like(base["v"])
         sets.append(s)
-    launches_per_step = len(DIRECTIONS)
+    launches_per_step = len(directions)
+    dt = torch.float16 if wl.dtype == "f16" else torch.float32
 
     def step(i):
-        for j, d in enumerate(DIRECTIONS):
+        for j, d in enumerate(directions):
             s = sets[(i * launches_per_step + j) % n_sets]
             gla.gla_fwd(s["q"], s["k"], s["v"], s["a"], s["g"], w, s["out"], gh, gw, d)
 
@@ -318,9 +323,9 @@ def run_ours(args, ws, rank, local):
     e2e_steps = max(1, min(args.e2e_steps, K))
     hx = {n: torch.from_numpy(np.ascontiguousarray(x[n])).pin_memory()
           for n in ("q", "k", "v", "a", "g", "w")}
-    hout = torch.empty(tuple(x["v"].shape), dtype=torch.float16).pin_memory()
+    hout = torch.empty(tuple(x["v"].shape), dtype=dt).pin_memory()
     with torch.cuda.stream(stream):
-        for d in DIRECTIONS:  # warm the staging buffers
+        for d in directions:  # warm the staging buffers
             gla.gla_fwd_host(hx["q"], hx["k"], hx["v"], hx["a"], hx["g"], hx["w"], hout, gh, gw,
                              d, stream=stream)
         if ws > 1:
@@ -329,7 +334,7 @@ def run_ours(args, ws, rank, local):
         e1 = torch.cuda.Event(enable_timing=True)
         e0.record(stream)
         for i in range(e2e_steps):
-            for d in DIRECTIONS:
+            for d in directions:
                 gla.gla_fwd_host(hx["q"], hx["k"], hx["v"], hx["a"], hx["g"], hx["w"], hout, gh,
                                  gw, d, stream=stream)
         e1.record(stream)
@@ -348,21 +353,24 @@ def run_ours(args, ws, rank, local):
     if rank != 0:
         return
     clocks = clk.summary()
+    dnames = {0: "L2R", 1: "R2L", 2: "T2B", 3: "B2T", 4: "cycle b%4"}
     line = {
-        "metric": METRIC, "value": value, "unit": "Mtokens/s", "n_gpus": ws, "steps": K,
+        "metric": METRIC if args.workload == WORKLOAD else
+                  "GLA fwd Mtokens/s (B·H·L), %s workload" % wl.name, "value": value, "unit": "Mtokens/s", "n_gpus": ws, "steps": K,
         "warmup": args.warmup, "ms_per_step": max_ms / K, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "f16", "data": "synthetic",
+        "scaling": "weak", "vs_baseline": None, "dtype": wl.dtype, "data": "synthetic",
         "config": {
-            "workload": "%s: %dx%d patch grid (L=%d), B=%d, H=%d, d_k=d_v=%d, fp16 I/O, fp32 "
-                        "accumulation; one step = 4 launches (L2R, R2L, T2B, B2T)"
-                        % (wl.name, gh, gw, wl.L, wl.B, wl.H, wl.d_k),
+            "workload": "%s: %dx%d patch grid (L=%d), B=%d, H=%d, d_k=d_v=%d, %s I/O, fp32 "
+                        "accumulation; one step = %d launch(es) (%s)"
+                        % (wl.name, gh, gw, wl.L, wl.B, wl.H, wl.d_k, wl.dtype, launches_per_step,
+                           ", ".join(dnames[d] for d in directions)),
             "tokens_per_step": tokens_per_step,
             "l2": "rotating pool of %d input sets (%.0f MB > 126 MB L2); no flush kernel"
                   % (n_sets, n_sets * set_bytes / 1e6),
             "timing": "CUDA-graph replays (graphs of %d steps), CUDA events on the launch "
                       "stream; warm-up = %d eager steps + one untimed replay" % (G, args.warmup),
             "parallelism": "replicas" if ws > 1 else "single GPU",
-            "schedule": gla.plan(wl.B, wl.H, gh, gw, wl.d_k, wl.d_v, 0),
+            "schedule": gla.plan(wl.B, wl.H, gh, gw, wl.d_k, wl.d_v, 0 if wl.dtype == "f16" else 1),
         },
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": achieved / peak, "traffic": profile_traffic(),
@@ -375,7 +383,7 @@ def run_ours(args, ws, rank, local):
         "clocks": clocks,
     }
     if ws == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_oracle_sample(wl, x, args.cpu_seconds)
+        line["cpu_baseline"] = cpu_oracle_sample(wl, x, args.cpu_seconds, directions)
     print(json.dumps(line), flush=True)
 
 

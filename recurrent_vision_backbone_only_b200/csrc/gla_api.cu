@@ -129,11 +129,44 @@ void configure_launch(Plan &pl, int n_pairs, int threads, cudaStream_t st) {
     }
 }
 
+// Clusters of `size` CTAs of this launch shape the device holds at once (0 = none).
+template <typename K>
+int active_clusters(K kern, Plan &pl, int n_pairs, int size, int threads, cudaStream_t st) {
+    Plan probe = pl;
+    probe.segs = size;
+    configure_launch(probe, n_pairs, threads, st);
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, kern, &probe.cfg) != cudaSuccess) {
+        cudaGetLastError();
+        n = 0;
+    }
+    return n;
+}
+
+// Tensor-core schedule cost model, relative units (a full 128-token chunk ~ 1): a chunk of
+// n tokens costs 0.45 + 0.55 n/128 (fixed latency chain + per-token work); a segment of
+// one chunk runs resident and adds 0.15 for the exchange; a longer segment that exchanges
+// first runs a state-only pass (~0.4 per chunk) and the exchange (0.2); a launch takes
+// ceil(pairs / resident clusters) waves.
+double tc_cost(int L, int n_pairs, int segs, int active) {
+    if (active <= 0) return 1e30;
+    const int seg_len = ceil_div(L, segs);
+    const int s_eff = ceil_div(L, seg_len);
+    const int chunks = ceil_div(seg_len, 128);
+    const double chunk_len = (double)seg_len / chunks;
+    const double per_chunk = 0.45 + 0.55 * chunk_len / 128.0;
+    double per_cta = chunks * per_chunk;
+    if (s_eff > 1) per_cta += chunks <= 1 ? 0.15 : chunks * 0.4 + 0.2;
+    const int waves = ceil_div(n_pairs, active);
+    return waves * per_cta;
+}
+
 // Pick the segment count (auto when segs <= 0), shrinking it until a cluster
-// fits on the device.  `unit` is the granularity of a segment's length.
+// fits on the device.  `unit` is the granularity of a segment's length.  With a
+// cost model (tensor-core kernel) every cluster size 1..16 is scored instead.
 template <typename K>
 int make_plan(K kern, Plan &pl, int L, int n_pairs, int segs, int unit, int threads,
-              cudaStream_t st, const DeviceInfo &di) {
+              cudaStream_t st, const DeviceInfo &di, bool cost_model = false) {
     if (pl.smem > (size_t)di.max_smem_optin) return GLA_ERR_UNSUPPORTED;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)pl.smem) !=
             cudaSuccess ||
@@ -142,7 +175,38 @@ int make_plan(K kern, Plan &pl, int L, int n_pairs, int segs, int unit, int thre
         return GLA_ERR_CUDA;
     }
     const bool auto_segs = segs <= 0;
-    if (auto_segs) {
+    if (auto_segs && cost_model) {
+        static std::mutex mu;
+        static int cache[64][17];
+        static bool have[64][17] = {};
+        int dev = 0;
+        cudaGetDevice(&dev);
+        double best = 1e30;
+        int best_s = 1;
+        for (int cand = 1; cand <= 16 && cand <= L; ++cand) {
+            const int s_eff = ceil_div(L, ceil_div(L, cand));
+            if (s_eff != cand) continue;           // equal-length segments only
+            int act;
+            {
+                std::lock_guard<std::mutex> lock(mu);
+                if (dev >= 0 && dev < 64 && have[dev][cand]) {
+                    act = cache[dev][cand];
+                } else {
+                    act = active_clusters(kern, pl, n_pairs, cand, threads, st);
+                    if (dev >= 0 && dev < 64) {
+                        cache[dev][cand] = act;
+                        have[dev][cand] = true;
+                    }
+                }
+            }
+            const double c = tc_cost(L, n_pairs, cand, act);
+            if (c < best - 1e-9) {
+                best = c;
+                best_s = cand;
+            }
+        }
+        segs = best_s;
+    } else if (auto_segs) {
         segs = di.sms / n_pairs;
         segs = segs < 1 ? 1 : (segs > 16 ? 16 : segs);
     }
@@ -234,7 +298,7 @@ int run_tc(const Args &x, int chunk, int segs, float eps, cudaStream_t st, const
     pl.chunk = chunk;
     pl.smem = tc::kSmemBytes;
     pl.pdl = true;
-    int rc = make_plan(kern, pl, L, n_pairs, segs, 1, tc::kThreads, st, di);
+    int rc = make_plan(kern, pl, L, n_pairs, segs, 1, tc::kThreads, st, di, true);
     if (rc != GLA_OK) return rc;
     if (query) {
         *query = pl;
