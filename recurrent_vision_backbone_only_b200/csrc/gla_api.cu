@@ -161,6 +161,10 @@ double tc_cost(int L, int n_pairs, int segs, int active) {
     return waves * per_cta;
 }
 
+// The tensor-core kernel's state exchange splits the 64 state rows into ceil(64/segs)-row
+// slices and needs ceil(64/segs) * segs <= 66.
+bool tc_segs_ok(int segs) { return segs == 1 || ceil_div(64, segs) * segs <= tc::kMaxSliceRows; }
+
 // Pick the segment count (auto when segs <= 0), shrinking it until a cluster
 // fits on the device.  `unit` is the granularity of a segment's length.  With a
 // cost model (tensor-core kernel) every cluster size 1..16 is scored instead.
@@ -186,6 +190,7 @@ int make_plan(K kern, Plan &pl, int L, int n_pairs, int segs, int unit, int thre
         for (int cand = 1; cand <= 16 && cand <= L; ++cand) {
             const int s_eff = ceil_div(L, ceil_div(L, cand));
             if (s_eff != cand) continue;           // equal-length segments only
+            if (!tc_segs_ok(cand)) continue;        // state-row slices must fit the buffer
             int act;
             {
                 std::lock_guard<std::mutex> lock(mu);
@@ -228,7 +233,10 @@ int make_plan(K kern, Plan &pl, int L, int n_pairs, int segs, int unit, int thre
         pl.max_active_clusters = n;
         if (n > 0) return GLA_OK;
         if (!auto_segs || pl.segs == 1) return GLA_ERR_UNSUPPORTED;
-        plan_segs((pl.segs + 1) / 2);
+        int next = (pl.segs + 1) / 2;
+        if (cost_model)
+            while (next > 1 && !tc_segs_ok(next)) --next;
+        plan_segs(next);
         configure_launch(pl, n_pairs, threads, st);
     }
 }
@@ -293,6 +301,11 @@ int run_tc(const Args &x, int chunk, int segs, float eps, cudaStream_t st, const
     const int n_pairs = x.B * x.H;
     if (chunk <= 0) chunk = tc::kC;
     if (chunk % 16 != 0 || chunk > tc::kC) return GLA_ERR_UNSUPPORTED;
+    if (segs > 0) {                              // explicit: must fit the exchange slices
+        int s_eff = segs > L ? L : segs;
+        s_eff = ceil_div(L, ceil_div(L, s_eff));
+        if (!tc_segs_ok(s_eff)) return GLA_ERR_UNSUPPORTED;
+    }
     Plan pl;
     pl.kernel = 1;
     pl.chunk = chunk;

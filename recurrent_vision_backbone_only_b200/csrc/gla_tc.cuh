@@ -78,7 +78,13 @@ constexpr uint32_t kMISC = 196608;
 constexpr uint32_t kMiscBytes = 16384;
 constexpr uint32_t kAtom128 = 16384;   // [128 rows][128 B]
 constexpr uint32_t kAtom64 = 8192;     // [64 rows][128 B]
-constexpr size_t kSmemBytes = kMISC + kMiscBytes + 1024;  // + misc + alignment slack
+// exchange receive buffer: [segs][slice rows][64] fp32 aggregate slices
+constexpr uint32_t kRECV = kMISC + kMiscBytes;
+// rows of the 64-row state are split into ceil(64/segs)-row slices; segs must keep
+// ceil(64/segs) * segs <= 70 (kMaxSliceRows)
+constexpr int kMaxSliceRows = 70;
+constexpr uint32_t kRecvBytes = kMaxSliceRows * 256;
+constexpr size_t kSmemBytes = kRECV + kRecvBytes + 1024;  // + alignment slack
 
 // TMEM columns
 constexpr uint32_t kTmemCols = 512;
@@ -179,6 +185,18 @@ __device__ __forceinline__ bool wait_phase(uint64_t *bar, uint32_t parity) {
 }
 
 // log2 of the retention gate: log2(sigma(a)) / 16, stable for either sign of a.
+// Bounded wait with cluster-scope acquire (data pushed by other CTAs of the cluster).
+__device__ __forceinline__ bool wait_cluster_phase(uint64_t *bar, uint32_t parity) {
+    const long long start = clock64();
+    while (!ptx::mbar_try_wait_cluster(bar, parity)) {
+        if (clock64() - start > (1LL << 32)) {
+            raise_status(7 /* GLA_ERR_TIMEOUT */);
+            return false;
+        }
+    }
+    return true;
+}
+
 __device__ __forceinline__ float log2_gamma(float a) {
     const float x = ptx::ex2(-fabsf(a) * kLog2e);             // 2^{-|a| log2 e} = e^{-|a|}
     return (fminf(a, 0.0f) * kLog2e - ptx::lg2(1.0f + x)) * kInvTau;
@@ -198,6 +216,7 @@ __device__ __forceinline__ uint32_t pack_half2(float lo, float hi) {
 struct Misc {
     uint64_t mbar_mma[4];     // [0] state, [1] scores, [2] inter (+ P.V), [3] early P.V
     uint64_t mbar_ld[3];      // [0] a tile, [1] q and k tiles, [2] v and g tiles
+    uint64_t mbar_x[2];       // exchange: [0] aggregates received, [1] S~ / S_in received
     uint32_t tmem_base;
     int slow;                 // chunk uses the exact CUDA-core score path
     int range_err;            // a P entry overflowed fp16
@@ -214,6 +233,7 @@ struct Misc {
     alignas(16) float tot[8][kD]; // per-16-row totals of the gate scan
     alignas(16) float Gall[16][kD]; // 2^{Gs} of every segment, pushed by each (exchange)
     alignas(16) float Eall[16][kD]; // 2^{r} of every segment (direct S~ writes)
+    alignas(16) float eGrow[kD];    // 2^{Gs} of this segment (sent to every CTA)
     alignas(16) float red[2][kC]; // epilogue partial sums of squares (per channel half)
     alignas(16) float dqp[2][kC]; // diagonal score q_t . k_t, per channel half
 };
@@ -288,6 +308,23 @@ __global__ void __launch_bounds__(kThreads, 1) gla_tc_kernel(const Params p) {
         m.range_err = 0;
     }
     if (tid < kD) m.Gs[tid] = 0.0f;
+    // Exchange partition: CTA s scans state rows [s*rows_per, s*rows_per + slice_rows(s)).
+    const int rows_per = exchange ? (kD + p.segs - 1) / p.segs : kD;
+    auto slice_rows = [&](int s_) { return max(0, min(kD, (s_ + 1) * rows_per) - s_ * rows_per); };
+    const int my_rows = exchange ? slice_rows(rank) : 0;
+    if (exchange) {
+        if (tid == 0) {
+            ptx::mbar_init(&m.mbar_x[0], 1);
+            ptx::mbar_init(&m.mbar_x[1], 1);
+            ptx::fence_mbarrier_init();
+            // every segment sends this CTA its aggregate slice and its 2^G and 2^r rows;
+            // every row of this CTA's S~ (or S_in) arrives exactly once
+            ptx::mbar_arrive_expect_tx(&m.mbar_x[0], (uint32_t)(p.segs * (my_rows * 256 + 2 * kD * 4)));
+            ptx::mbar_arrive_expect_tx(&m.mbar_x[1], (uint32_t)(kD * kD * 4));
+        }
+        __syncthreads();
+        ptx::cluster_arrive();        // start-up barrier: waited on before the first push
+    }
     ptx::pdl_wait_prior_grid();
     // RMSNorm weight: async copy, covered by the first chunk's v/g load group
     if (tid < kD / 4) ptx::cp_async16(ptx::smem_u32(&m.w[4 * tid]), p.w + 4 * tid, 16);
@@ -390,30 +427,51 @@ __global__ void __launch_bounds__(kThreads, 1) gla_tc_kernel(const Params p) {
         __syncthreads();
     };
     // ------------------------------------------------------------ operands (row t, 32 channels)
-    // fast path: Qh/Ql (TMEM, scaled by d_k^{-1/2}), Kh/Kl (smem tf32), Ks (smem fp16);
-    // slow path: Qh = d_k^{-1/2} q 2^{b}, Ks.  full = false builds Ks only.
-    auto build_operands = [&](bool full) {
-        const bool slow = m.slow != 0;
-        float dqs = 0.0f;                          // partial q_t . k_t over this half's channels
+    // Decayed keys Ks = k 2^{B - b} (fp16, the state product's A operand).  Built first so
+    // the segment aggregate can be published before the score operands exist.
+    auto build_ks = [&]() {
         wait_bar(&m.mbar_ld[1], it & 1);
 #pragma unroll 1
         for (int jj = 0; jj < 4; ++jj) {
             const int j = ch * 4 + jj;             // 16 B chunk of 8 channels
             const uint4 kraw = *reinterpret_cast<const uint4 *>(sm + kTK + off_f16(t, j));
-            uint4 qraw = make_uint4(0, 0, 0, 0);
-            if (full) qraw = *reinterpret_cast<const uint4 *>(sm + kTQ + off_f16(t, j));
+            const __half2 *k2 = reinterpret_cast<const __half2 *>(&kraw);
+            float ks[8];
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                const float4 b4 = *reinterpret_cast<const float4 *>(sm + kPB + off_tf32(kAtom128, t, 2 * j + h));
+                const float4 B4 = *reinterpret_cast<const float4 *>(&m.Bc[8 * j + 4 * h]);
+                const float2 k01 = __half22float2(k2[2 * h]), k23 = __half22float2(k2[2 * h + 1]);
+                ks[4 * h + 0] = k01.x * ptx::ex2(B4.x - b4.x);
+                ks[4 * h + 1] = k01.y * ptx::ex2(B4.y - b4.y);
+                ks[4 * h + 2] = k23.x * ptx::ex2(B4.z - b4.z);
+                ks[4 * h + 3] = k23.y * ptx::ex2(B4.w - b4.w);
+            }
+            uint4 kso;
+            kso.x = pack_half2(ks[0], ks[1]); kso.y = pack_half2(ks[2], ks[3]);
+            kso.z = pack_half2(ks[4], ks[5]); kso.w = pack_half2(ks[6], ks[7]);
+            *reinterpret_cast<uint4 *>(sm + kST + off_f16(t, j)) = kso;
+        }
+    };
+    // Score operands.  Fast path: Qh/Ql (TMEM, carrying d_k^{-1/2}), Kh/Kl (smem tf32);
+    // slow path: Qh/Ql of d_k^{-1/2} q 2^{b} only.  Also the exact diagonal q_t . k_t.
+    auto build_qk = [&]() {
+        const bool slow = m.slow != 0;
+        float dqs = 0.0f;                          // partial q_t . k_t over this half's channels
+#pragma unroll 1
+        for (int jj = 0; jj < 4; ++jj) {
+            const int j = ch * 4 + jj;
+            const uint4 kraw = *reinterpret_cast<const uint4 *>(sm + kTK + off_f16(t, j));
+            const uint4 qraw = *reinterpret_cast<const uint4 *>(sm + kTQ + off_f16(t, j));
             const __half2 *k2 = reinterpret_cast<const __half2 *>(&kraw);
             const __half2 *q2 = reinterpret_cast<const __half2 *>(&qraw);
-            float bt[8], rr[8], fb[8], kv[8], qv[8];
+            float bt[8], rr[8], kv[8], qv[8];
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
                 const float4 b4 = *reinterpret_cast<const float4 *>(sm + kPB + off_tf32(kAtom128, t, 2 * j + h));
                 const float4 r4 = *reinterpret_cast<const float4 *>(&m.bref[8 * j + 4 * h]);
-                const float4 f4 = *reinterpret_cast<const float4 *>(slow ? &m.Bc[8 * j + 4 * h]
-                                                                         : &m.fB[8 * j + 4 * h]);
                 bt[4 * h] = b4.x; bt[4 * h + 1] = b4.y; bt[4 * h + 2] = b4.z; bt[4 * h + 3] = b4.w;
                 rr[4 * h] = r4.x; rr[4 * h + 1] = r4.y; rr[4 * h + 2] = r4.z; rr[4 * h + 3] = r4.w;
-                fb[4 * h] = f4.x; fb[4 * h + 1] = f4.y; fb[4 * h + 2] = f4.z; fb[4 * h + 3] = f4.w;
             }
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
@@ -422,53 +480,41 @@ __global__ void __launch_bounds__(kThreads, 1) gla_tc_kernel(const Params p) {
                 kv[2 * e] = kf.x; kv[2 * e + 1] = kf.y;
                 qv[2 * e] = qf.x; qv[2 * e + 1] = qf.y;
             }
+#pragma unroll
+            for (int e = 0; e < 8; ++e) dqs = fmaf(qv[e], kv[e], dqs);
             // tf32 splits: high = low 13 bits cleared, low = exact remainder (the tensor core
             // drops the low part's own low bits: error <= 2^-20 of the value)
-            if (full) {
-#pragma unroll
-                for (int e = 0; e < 8; ++e) dqs = fmaf(qv[e], kv[e], dqs);
-            }
-            float ks[8], qh[8], ql[8], kh[8], kl[8];
+            float qh[8], ql[8], kh[8], kl[8];
 #pragma unroll
             for (int e = 0; e < 8; ++e) {
                 if (!slow) {
-                    const float kf = kv[e] * ptx::ex2(rr[e] - bt[e]);          // k 2^{r - b}
-                    ks[e] = kf * fb[e];                                         // k 2^{B - b}
-                    const float qf = qv[e] * ptx::ex2(bt[e] - rr[e] + kLog2Scale);  // q 2^{b - r} / 8
+                    const float kf = kv[e] * ptx::ex2(rr[e] - bt[e]);             // k 2^{r - b}
+                    const float qf = qv[e] * ptx::ex2(bt[e] - rr[e] + kLog2Scale); // q 2^{b - r} / 8
                     kh[e] = ptx::tf32_hi(kf);
                     kl[e] = kf - kh[e];
                     qh[e] = ptx::tf32_hi(qf);
                     ql[e] = qf - qh[e];
                 } else {
-                    ks[e] = kv[e] * ptx::ex2(fb[e] - bt[e]);      // fb holds B_c here
                     const float qf = qv[e] * ptx::ex2(bt[e] + kLog2Scale);
                     qh[e] = ptx::tf32_hi(qf);
                     ql[e] = qf - qh[e];
                     kh[e] = kl[e] = 0.0f;
                 }
             }
-            uint4 kso;
-            kso.x = pack_half2(ks[0], ks[1]); kso.y = pack_half2(ks[2], ks[3]);
-            kso.z = pack_half2(ks[4], ks[5]); kso.w = pack_half2(ks[6], ks[7]);
-            *reinterpret_cast<uint4 *>(sm + kST + off_f16(t, j)) = kso;
-            if (full) {
-                ptx::tmem_st8(tmem_warp + kColQH + 8 * j, qh);
-                ptx::tmem_st8(tmem_warp + kColQL + 8 * j, ql);
-                if (!slow) {
+            ptx::tmem_st8(tmem_warp + kColQH + 8 * j, qh);
+            ptx::tmem_st8(tmem_warp + kColQL + 8 * j, ql);
+            if (!slow) {
 #pragma unroll
-                    for (int h = 0; h < 2; ++h) {
-                        *reinterpret_cast<float4 *>(sm + kKH + off_tf32(kAtom128, t, 2 * j + h)) =
-                            make_float4(kh[4 * h], kh[4 * h + 1], kh[4 * h + 2], kh[4 * h + 3]);
-                        *reinterpret_cast<float4 *>(sm + kKL + off_tf32(kAtom128, t, 2 * j + h)) =
-                            make_float4(kl[4 * h], kl[4 * h + 1], kl[4 * h + 2], kl[4 * h + 3]);
-                    }
+                for (int h = 0; h < 2; ++h) {
+                    *reinterpret_cast<float4 *>(sm + kKH + off_tf32(kAtom128, t, 2 * j + h)) =
+                        make_float4(kh[4 * h], kh[4 * h + 1], kh[4 * h + 2], kh[4 * h + 3]);
+                    *reinterpret_cast<float4 *>(sm + kKL + off_tf32(kAtom128, t, 2 * j + h)) =
+                        make_float4(kl[4 * h], kl[4 * h + 1], kl[4 * h + 2], kl[4 * h + 3]);
                 }
             }
         }
-        if (full) {
-            m.dqp[ch][t] = dqs;
-            ptx::tmem_st_wait();
-        }
+        m.dqp[ch][t] = dqs;
+        ptx::tmem_st_wait();
     };
     // ------------------------------------------------------------ MMA issue (one thread)
     // Make every thread's shared-memory operand writes visible to the tensor core, then
@@ -606,85 +652,91 @@ __global__ void __launch_bounds__(kThreads, 1) gla_tc_kernel(const Params p) {
         if (into_g && tid < kD) m.Gs[tid] += m.Bc[tid];
     };
     // Cluster-wide scan of the segment aggregates (Gs, S): every segment receives its
-    // incoming state.  Split in two so P can be built while the cluster barrier settles:
-    // xchg_begin publishes this CTA's aggregate, xchg_end scans and reads the result.
-    float *X = reinterpret_cast<float *>(sm + kST);  // [64 j][64 c] fp32, plain row-major
+    // incoming state.  Each CTA writes its aggregate to shared memory and moves it with
+    // one bulk copy per scanning CTA (cp.async.bulk into the peer's shared memory, bytes
+    // counted on the peer's mbarrier); a scanner owns a slice of state rows, combines the
+    // segments in order, stages every segment's result in that segment's layout and bulk
+    // copies it back.  Buffers: outgoing aggregate X (Ks region), incoming slices (receive
+    // region), scanner staging (q/k tiles, consumed), results into the a tile (S~, direct)
+    // or the g tile (S_in, before a multi-chunk pass) -- no buffer is written remotely while
+    // one of this CTA's own copies may still read it.
+    float *X = reinterpret_cast<float *>(sm + kST);   // [64 j][64 c] fp32 outgoing aggregate
+    const float *recv = reinterpret_cast<const float *>(sm + kRECV);
     auto xchg_begin = [&]() {
-        __syncthreads();
-        // push this segment's decay 2^{Gs} into row `rank` of every CTA's table
-        if (tid < p.segs * (kD / 4)) {
-            const int r = tid / (kD / 4), c4 = tid - r * (kD / 4);
-            const float4 g = *reinterpret_cast<const float4 *>(&m.Gs[4 * c4]);
-            ptx::st_cluster_v4(ptx::mapa(ptx::smem_u32(&m.Gall[rank][4 * c4]), r),
-                               make_float4(ptx::ex2(g.x), ptx::ex2(g.y), ptx::ex2(g.z), ptx::ex2(g.w)));
-            ptx::st_cluster_v4(ptx::mapa(ptx::smem_u32(&m.Eall[rank][4 * c4]), r),
-                               *reinterpret_cast<const float4 *>(&m.eref[4 * c4]));
-        }
+        __syncthreads();                              // Gs, 2^r and S are final
         if (s_owner) {
 #pragma unroll
             for (int i = 0; i < 8; ++i)
                 *reinterpret_cast<float4 *>(X + s_row * kD + 32 * ch + 4 * i) =
                     make_float4(S[4 * i], S[4 * i + 1], S[4 * i + 2], S[4 * i + 3]);
         }
-        ptx::cluster_arrive();
+        if (tid < kD) m.eGrow[tid] = ptx::ex2(m.Gs[tid]);
+        ptx::fence_proxy_async_smem();                // sources of the bulk copies
+        __syncthreads();
+        ptx::cluster_wait();                          // every CTA's exchange barriers exist
+        if (tid < p.segs) {
+            const int r = tid, rr = slice_rows(r);
+            const uint32_t bar = ptx::mapa(ptx::smem_u32(&m.mbar_x[0]), r);
+            if (rr > 0)
+                ptx::bulk_to_cluster(ptx::mapa(sbase + kRECV + rank * rr * 256, r),
+                                     ptx::smem_u32(X + r * rows_per * kD), rr * 256, bar);
+            ptx::bulk_to_cluster(ptx::mapa(ptx::smem_u32(&m.Gall[rank][0]), r),
+                                 ptx::smem_u32(m.eGrow), kD * 4, bar);
+            ptx::bulk_to_cluster(ptx::mapa(ptx::smem_u32(&m.Eall[rank][0]), r),
+                                 ptx::smem_u32(m.eref), kD * 4, bar);
+        }
     };
-    // Second half of the exchange.  Called by every thread (the cluster barriers count them
-    // all); the DSMEM scan itself runs on warps 0..3 (`scanners`), synchronised among
-    // themselves with named barrier 1, while the other warps are free for other work before
-    // calling in.
-    // direct: the scanners write each segment's S~ = 2^{r} S_in (tf32, the inter product's B
-    // operand) straight into that CTA's a-tile region, and S is not read back (one chunk).
+    // direct: results are S~ = tf32(2^{r} S_in) in the inter product's operand layout, bulk
+    // copied into each segment's a-tile region, and S is not read back (one chunk); otherwise
+    // S_in lands row-major in the g-tile region and is read back into S.
     auto xchg_end = [&](bool scanners, bool direct) {
-        ptx::cluster_wait();
+        const uint32_t stage = kTQ;                   // q and k tiles: consumed, 32 KB
         if (scanners) {
-            const int segs = p.segs;
-            const int sid = tid & 127;
-            const int E2 = kD * kD / 2;                   // float2 pairs of the state
-            const int per = (E2 + segs - 1) / segs;
-            const int e0 = rank * per, e1 = min(E2, e0 + per);
-            const uint32_t xbase = ptx::smem_u32(X);
-            for (int e = e0 + sid; e < e1; e += 128) {
-                const int c = (2 * e) & (kD - 1);
-                float2 x[16];
-#pragma unroll
-                for (int r = 0; r < 16; ++r)
-                    if (r < segs) x[r] = ptx::ld_cluster_v2(ptx::mapa(xbase + 8u * e, r));
+            if (!wait_cluster_phase(&m.mbar_x[0], 0)) m.abort = 1;
+            const int segs = p.segs, r0 = rank * rows_per;
+            for (int idx = tid & 127; idx < my_rows * 32; idx += 128) {
+                const int i = idx >> 5, c = 2 * (idx & 31), j = r0 + i;
                 float2 run = make_float2(0.0f, 0.0f);
-#pragma unroll
-                for (int r = 0; r < 16; ++r) {
-                    if (r < segs) {
-                        const float2 agg = x[r];
-                        const float2 g = *reinterpret_cast<const float2 *>(&m.Gall[r][c]);
-                        x[r] = run;                       // state entering segment r
-                        run = make_float2(fmaf(g.x, run.x, agg.x), fmaf(g.y, run.y, agg.y));
+#pragma unroll 4
+                for (int q = 0; q < segs; ++q) {
+                    const float2 agg = *reinterpret_cast<const float2 *>(recv + (q * my_rows + i) * kD + c);
+                    const float2 g = *reinterpret_cast<const float2 *>(&m.Gall[q][c]);
+                    uint32_t off;
+                    float2 out;
+                    if (direct) {
+                        const float2 f = *reinterpret_cast<const float2 *>(&m.Eall[q][c]);
+                        out = make_float2(ptx::to_tf32(f.x * run.x), ptx::to_tf32(f.y * run.y));
+                        off = q * my_rows * 256 + (c >> 5) * my_rows * 128 + i * 128 +
+                              ((((c & 31) >> 2) ^ (j & 7)) << 4) + (c & 3) * 4;
+                    } else {
+                        out = run;
+                        off = q * my_rows * 256 + i * 256 + c * 4;
                     }
+                    *reinterpret_cast<float2 *>(sm + stage + off) = out;   // state entering q
+                    run = make_float2(fmaf(g.x, run.x, agg.x), fmaf(g.y, run.y, agg.y));
                 }
+            }
+            ptx::fence_proxy_async_smem();
+            ptx::named_bar_sync(1, 128);
+            if ((tid & 127) < segs && my_rows > 0) {
+                const int q = tid & 127;
+                const uint32_t bar = ptx::mapa(ptx::smem_u32(&m.mbar_x[1]), q);
+                const uint32_t src = sbase + stage + q * my_rows * 256;
                 if (direct) {
-                    const int j = (2 * e) >> 6;
-                    const uint32_t dst =
-                        ptx::smem_u32(sm + kTA + off_tf32(kAtom64, j, c >> 2) + (c & 3) * 4);
-#pragma unroll
-                    for (int r = 0; r < 16; ++r) {
-                        if (r < segs) {
-                            const float2 f = *reinterpret_cast<const float2 *>(&m.Eall[r][c]);
-                            ptx::st_cluster_v2(ptx::mapa(dst, r),
-                                               make_float2(ptx::to_tf32(f.x * x[r].x),
-                                                           ptx::to_tf32(f.y * x[r].y)));
-                        }
-                    }
+                    for (int a = 0; a < 2; ++a)
+                        ptx::bulk_to_cluster(ptx::mapa(sbase + kTA + a * kAtom64 + r0 * 128, q),
+                                             src + a * my_rows * 128, my_rows * 128, bar);
                 } else {
-#pragma unroll
-                    for (int r = 0; r < 16; ++r)
-                        if (r < segs) ptx::st_cluster_v2(ptx::mapa(xbase + 8u * e, r), x[r]);
+                    ptx::bulk_to_cluster(ptx::mapa(sbase + kTG + r0 * 256, q), src, my_rows * 256, bar);
                 }
             }
         }
-        ptx::cluster_arrive();
-        ptx::cluster_wait();
+        if (!wait_cluster_phase(&m.mbar_x[1], 0)) m.abort = 1;
         if (!direct && s_owner) {
+            const float *Sin = reinterpret_cast<const float *>(sm + kTG);
 #pragma unroll
             for (int i = 0; i < 8; ++i) {
-                const float4 v = *reinterpret_cast<const float4 *>(X + s_row * kD + 32 * ch + 4 * i);
+                const float4 v = *reinterpret_cast<const float4 *>(Sin + s_row * kD + 32 * ch + 4 * i);
                 S[4 * i] = v.x; S[4 * i + 1] = v.y; S[4 * i + 2] = v.z; S[4 * i + 3] = v.w;
             }
         }
@@ -724,7 +776,7 @@ __global__ void __launch_bounds__(kThreads, 1) gla_tc_kernel(const Params p) {
             tmem = m.tmem_base;
             tmem_warp = tmem + ((uint32_t)(w4 * 32) << 16);
         }
-        build_operands(!pass1);
+        build_ks();
         wait_bar(&m.mbar_ld[2], it & 1);             // V, an operand of the state product
         operands_ready();
         // The state product goes first: the segment aggregate is published while the score
@@ -737,16 +789,6 @@ __global__ void __launch_bounds__(kThreads, 1) gla_tc_kernel(const Params p) {
         }
         wait_mma(0);
         const bool mid_xchg = !pass1 && resident && exchange;
-        // Score products, issued by thread 128 (warp 4 builds P).  With a mid-chunk exchange
-        // they go out after this CTA has published its aggregate, so the issuing warp's stall
-        // does not delay the publication.
-        auto issue_scores = [&]() {
-            if (tid == 128) {
-                if (!m.slow) issue_qk(sbase, tmem, min(kC, (n + 15) & ~15));
-                ptx::mma_commit(&m.mbar_mma[1]);
-            }
-        };
-        if (!pass1 && !mid_xchg) issue_scores();
         read_sloc();
         if (pass1 || mid_xchg) fold_sloc(true);     // S = S 2^{B} + Sloc, Gs += B
         if (pass1) {
@@ -755,14 +797,21 @@ __global__ void __launch_bounds__(kThreads, 1) gla_tc_kernel(const Params p) {
             ++it;
             continue;
         }
-        if (mid_xchg) {
-            xchg_begin();
-            issue_scores();
+        // publish the segment aggregate now: the exchange runs under the score operands,
+        // the score products and P
+        if (mid_xchg) xchg_begin();
+        build_qk();
+        operands_ready();
+        if (tid == 128) {                            // score products, issued by warp 4
+            ptx::tc_fence_after_sync();
+            if (!m.slow) issue_qk(sbase, tmem, min(kC, (n + 15) & ~15));
+            ptx::mma_commit(&m.mbar_mma[1]);
         }
         const bool pv_early = mid_xchg && !m.slow;
         if (m.slow) {
             wait_mma(1);
             make_p_exact(sm, t, ch, n, p.scale, &m.range_err);
+            __syncthreads();                          // q/k tiles read; they stage the scan next
             if (mid_xchg) xchg_end(warp < 4, true);
         } else if (mid_xchg) {
             // warps 4..7 wait for the scores, build P and start P.V; warps 0..3 scan the
