@@ -62,6 +62,21 @@ def dist_env():
     return ws, rank, local
 
 
+def max_over_ranks(value_ms: float, device) -> float:
+    """Max of a per-rank time over the job (the job ends when its slowest rank does)."""
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([value_ms], dtype=torch.float64, device=device)
+    if dist.is_available() and dist.is_initialized() and dist.get_world_size() > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(tokens_per_step: int, steps: int, world_size: int, max_ms: float) -> float:
+    """Whole-job Mtokens/s: every rank's tokens over the slowest rank's time."""
+    return tokens_per_step * world_size * steps / (max_ms / 1e3) / 1e6
+
+
 def measured_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -307,13 +322,10 @@ def run_ours(args, ws, rank, local):
     elapsed_ms = ev0.elapsed_time(ev1)
     if gla.get_status(stream) != 0:
         raise RuntimeError("device status set during the timed region")
-    t = torch.tensor([elapsed_ms], dtype=torch.float64, device=dev)
-    if ws > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    max_ms = float(t.item())
+    max_ms = max_over_ranks(elapsed_ms, dev)
 
     tokens_per_step = wl.tokens * launches_per_step
-    value = tokens_per_step * ws * K / (max_ms / 1e3) / 1e6
+    value = job_throughput(tokens_per_step, K, ws, max_ms)
     launch_s = (elapsed_ms / 1e3) / (K * launches_per_step)
     bytes_per_launch = wl.tokens * wl.bytes_per_token
     peak, peak_kind = measured_peaks()
@@ -339,14 +351,11 @@ def run_ours(args, ws, rank, local):
                                  gw, d, stream=stream)
         e1.record(stream)
     torch.cuda.synchronize()
-    te = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=dev)
-    if ws > 1:
-        dist.all_reduce(te, op=dist.ReduceOp.MAX)
-    e2e_ms = float(te.item())
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), dev)
     h2d = launches_per_step * sum(hx[n].numel() * hx[n].element_size()
                                   for n in ("q", "k", "v", "a", "g", "w"))
     d2h = launches_per_step * hout.numel() * hout.element_size()
-    e2e = {"value": tokens_per_step * ws * e2e_steps / (e2e_ms / 1e3) / 1e6, "unit": "Mtokens/s",
+    e2e = {"value": job_throughput(tokens_per_step, e2e_steps, ws, e2e_ms), "unit": "Mtokens/s",
            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
            "steps": e2e_steps, "ms_per_step": e2e_ms / e2e_steps}
 

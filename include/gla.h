@@ -145,6 +145,16 @@ int gla_plan(int B, int H, int grid_h, int grid_w, int d_k, int d_v, int dtype, 
              int *segments, int *seg_len, int *ctas, int *max_active_clusters);
 
 /*
+ * gla_selftest_timeout -- diagnostic for device-side failure detection: launches a
+ * one-thread kernel that waits, with the kernels' bounded-wait loop but a bound of
+ * `limit_cycles` SM clocks (1 .. 2^34), on a barrier nothing ever signals.  The wait
+ * expires, GLA_ERR_TIMEOUT is latched in the device status word (read it with
+ * gla_get_status) and the kernel returns; the context stays usable.  Asynchronous on
+ * `stream`; GLA_ERR_UNSUPPORTED for a bound out of range.
+ */
+int gla_selftest_timeout(long long limit_cycles, void *stream);
+
+/*
  * gla_selftest_mma -- diagnostic: runs ONE of the tensor-core kernel's four
  * matrix products on a single CTA, with the kernel's own shared-memory
  * layouts and descriptors, on row-major float32 DEVICE arrays:

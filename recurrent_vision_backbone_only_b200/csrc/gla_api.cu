@@ -514,6 +514,16 @@ int gla_plan(int B, int H, int grid_h, int grid_w, int d_k, int d_v, int dtype, 
     return GLA_OK;
 }
 
+int gla_selftest_timeout(long long limit_cycles, void *stream) {
+    if (limit_cycles <= 0 || limit_cycles > (1LL << 34)) return GLA_ERR_UNSUPPORTED;
+    DeviceInfo di;
+    int rc = current_device_info(&di);
+    if (rc != GLA_OK) return rc;
+    tc::gla_timeout_selftest_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(limit_cycles);
+    if (cudaGetLastError() != cudaSuccess) return GLA_ERR_CUDA;
+    return GLA_OK;
+}
+
 int gla_selftest_mma(int kind, const float *A, const float *B, float *D, void *stream) {
     if (!A || !B || !D) return GLA_ERR_NULL;
     if (kind < 0 || kind > 3) return GLA_ERR_UNSUPPORTED;

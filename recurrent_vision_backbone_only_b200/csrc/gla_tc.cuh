@@ -865,6 +865,25 @@ __global__ void __launch_bounds__(kThreads, 1) gla_tc_kernel(const Params p) {
     if (warp == 0 && n_pass1 + n_chunks > 0) ptx::tmem_dealloc(tmem, kTmemCols);
 }
 
+// ------------------------------------------------------------- timeout self-test
+// One thread waits, with the kernel's bounded-wait loop but a caller-given bound, on an
+// mbarrier that nothing ever arrives on: the wait must expire, latch GLA_ERR_TIMEOUT in
+// the device status word and return, leaving the context usable.
+__global__ void gla_timeout_selftest_kernel(long long limit_cycles) {
+    __shared__ __align__(8) uint64_t bar;
+    if (threadIdx.x == 0) {
+        ptx::mbar_init(&bar, 1);
+        ptx::fence_mbarrier_init();
+        const long long start = clock64();
+        while (!ptx::mbar_try_wait(&bar, 0)) {
+            if (clock64() - start > limit_cycles) {
+                raise_status(7 /* GLA_ERR_TIMEOUT */);
+                break;
+            }
+        }
+    }
+}
+
 // ---------------------------------------------------------------- self-test
 // Runs one of the kernel's four MMA configurations on row-major fp32 inputs
 // (converted to the operand type in the same shared-memory layouts) and

@@ -54,6 +54,8 @@ def load() -> ctypes.CDLL:
         lib.gla_status_string.restype = ctypes.c_char_p
         lib.gla_version.argtypes = []
         lib.gla_selftest_mma.argtypes = [i, vp, vp, vp, vp]
+        lib.gla_selftest_timeout.argtypes = [ctypes.c_longlong, vp]
+        lib.gla_selftest_timeout.restype = ctypes.c_int
         ip = ctypes.POINTER(ctypes.c_int)
         lib.gla_plan.argtypes = [i] * 7 + [ip] * 5
         lib.gla_plan.restype = ctypes.c_int

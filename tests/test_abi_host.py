@@ -23,7 +23,8 @@ def lib():
 def test_exports_every_declared_symbol(lib):
     names = gla.header_functions()
     assert {"gla_fwd", "gla_fwd_f32", "gla_fwd_ex", "gla_fwd_host", "gla_get_status",
-            "gla_status_string", "gla_version", "gla_selftest_mma"} <= set(names)
+            "gla_status_string", "gla_version", "gla_selftest_mma", "gla_selftest_timeout",
+            "gla_plan"} <= set(names)
     for n in names:
         assert hasattr(lib, n), n
 
@@ -84,6 +85,23 @@ def test_selftest_rejects_bad_arguments(lib):
     assert f(0, None, 16, 16, None) == 1
     assert f(4, 16, 16, 16, None) == 3
     assert f(-1, 16, 16, 16, None) == 3
+
+
+def test_timeout_selftest_rejects_bad_bound(lib):
+    assert lib.gla_selftest_timeout(0, None) == 3
+    assert lib.gla_selftest_timeout(1 << 40, None) == 3
+
+
+def test_plan_rejects_bad_arguments(lib):
+    ip = ctypes.POINTER(ctypes.c_int)
+    vals = [ctypes.c_int(0) for _ in range(5)]
+    args = [1, 6, 40, 40, 64, 64, 0] + [ctypes.byref(v) for v in vals]
+    bad = list(args)
+    bad[7] = None
+    assert lib.gla_plan(*bad) == 1
+    assert lib.gla_plan(*([1, 6, 40, 40, 64, 48, 0] + args[7:])) == 3
+    assert lib.gla_plan(*([1, 0, 40, 40, 64, 64, 0] + args[7:])) == 2
+    assert lib.gla_plan(*([1, 6, 40, 40, 64, 64, 5] + args[7:])) == 3
 
 
 def test_ex_rejects_bad_schedule(lib):
