@@ -163,7 +163,7 @@ double tc_cost(int L, int n_pairs, int segs, int active) {
 
 // The tensor-core kernel's state exchange splits the 64 state rows into ceil(64/segs)-row
 // slices and needs ceil(64/segs) * segs <= 66.
-bool tc_segs_ok(int segs) { return segs == 1 || ceil_div(64, segs) * segs <= tc::kMaxSliceRows; }
+bool tc_segs_ok(int segs) { return segs == 1 || ceil_div(16, segs) * segs <= tc::kMaxGroupSegs; }
 
 // Pick the segment count (auto when segs <= 0), shrinking it until a cluster
 // fits on the device.  `unit` is the granularity of a segment's length.  With a
@@ -190,7 +190,7 @@ int make_plan(K kern, Plan &pl, int L, int n_pairs, int segs, int unit, int thre
         for (int cand = 1; cand <= 16 && cand <= L; ++cand) {
             const int s_eff = ceil_div(L, ceil_div(L, cand));
             if (s_eff != cand) continue;           // equal-length segments only
-            if (!tc_segs_ok(cand)) continue;        // state-row slices must fit the buffer
+            if (!tc_segs_ok(cand)) continue;        // channel groups must fit the buffer
             int act;
             {
                 std::lock_guard<std::mutex> lock(mu);

@@ -68,22 +68,24 @@ constexpr float kHalfRangeSafe2 = 86.0f;
 constexpr uint32_t kKL = 0;        // K~ low part  tf32, 2 atoms x [128][128B]
 constexpr uint32_t kKH = 32768;    // K~ high part tf32, 2 atoms x [128][128B] (slow path: P)
 constexpr uint32_t kPB = 65536;    // b   fp32 (QT layout), then P fp16 2 atoms x [128][128B]
-constexpr uint32_t kST = 98304;    // Ks fp16 [128][128B] / state exchange fp32 [64][64]
+constexpr uint32_t kST = 98304;    // Ks fp16 [128][128B]
 constexpr uint32_t kTQ = 114688;   // raw tiles, fp16 [128][128B] each
 constexpr uint32_t kTK = 131072;
 constexpr uint32_t kTA = 147456;   // a tile; after the gate: S~ tf32 2 x [64][128B]
 constexpr uint32_t kTV = 163840;
 constexpr uint32_t kTG = 180224;
 constexpr uint32_t kMISC = 196608;
-constexpr uint32_t kMiscBytes = 16384;
+constexpr uint32_t kMiscBytes = 8192;
 constexpr uint32_t kAtom128 = 16384;   // [128 rows][128 B]
 constexpr uint32_t kAtom64 = 8192;     // [64 rows][128 B]
-// exchange receive buffer: [segs][slice rows][64] fp32 aggregate slices
+// State exchange: the 64 key channels form 16 groups of 4; group g is scanned by CTA
+// g % segs.  A scanner receives, per (own group, segment), 64 aggregate rows plus the
+// segment's 2^G and 2^r entries of the group: 66 x 16 B.  A CTA owns ceil((16-r)/segs)
+// groups, so the buffer bounds ceil(16/segs) * segs <= kMaxGroupSegs.
 constexpr uint32_t kRECV = kMISC + kMiscBytes;
-// rows of the 64-row state are split into ceil(64/segs)-row slices; segs must keep
-// ceil(64/segs) * segs <= 70 (kMaxSliceRows)
-constexpr int kMaxSliceRows = 70;
-constexpr uint32_t kRecvBytes = kMaxSliceRows * 256;
+constexpr int kGroupRows = kD + 2;
+constexpr int kMaxGroupSegs = 24;
+constexpr uint32_t kRecvBytes = kMaxGroupSegs * kGroupRows * 16;
 constexpr size_t kSmemBytes = kRECV + kRecvBytes + 1024;  // + alignment slack
 
 // TMEM columns
@@ -231,8 +233,6 @@ struct Misc {
     alignas(16) float b0[kD];     // b_{0,c}
     alignas(16) float w[kD];      // RMSNorm weight
     alignas(16) float tot[8][kD]; // per-16-row totals of the gate scan
-    alignas(16) float Gall[16][kD]; // 2^{Gs} of every segment, pushed by each (exchange)
-    alignas(16) float Eall[16][kD]; // 2^{r} of every segment (direct S~ writes)
     alignas(16) float eGrow[kD];    // 2^{Gs} of this segment (sent to every CTA)
     alignas(16) float red[2][kC]; // epilogue partial sums of squares (per channel half)
     alignas(16) float dqp[2][kC]; // diagonal score q_t . k_t, per channel half
@@ -308,22 +308,20 @@ __global__ void __launch_bounds__(kThreads, 1) gla_tc_kernel(const Params p) {
         m.range_err = 0;
     }
     if (tid < kD) m.Gs[tid] = 0.0f;
-    // Exchange partition: CTA s scans state rows [s*rows_per, s*rows_per + slice_rows(s)).
-    const int rows_per = exchange ? (kD + p.segs - 1) / p.segs : kD;
-    auto slice_rows = [&](int s_) { return max(0, min(kD, (s_ + 1) * rows_per) - s_ * rows_per); };
-    const int my_rows = exchange ? slice_rows(rank) : 0;
+    // Exchange partition: CTA r scans the channel groups g = r, r + segs, ... (< 16).
+    const int my_groups = exchange ? (16 - rank + p.segs - 1) / p.segs : 0;
     if (exchange) {
         if (tid == 0) {
             ptx::mbar_init(&m.mbar_x[0], 1);
             ptx::mbar_init(&m.mbar_x[1], 1);
             ptx::fence_mbarrier_init();
-            // every segment sends this CTA its aggregate slice and its 2^G and 2^r rows;
-            // every row of this CTA's S~ (or S_in) arrives exactly once
-            ptx::mbar_arrive_expect_tx(&m.mbar_x[0], (uint32_t)(p.segs * (my_rows * 256 + 2 * kD * 4)));
+            // every segment sends this CTA, per owned group, 64 aggregate rows and its 2^G and
+            // 2^r entries; every 16 B of this CTA's S~ (or S_in) arrives exactly once
+            ptx::mbar_arrive_expect_tx(&m.mbar_x[0], (uint32_t)(my_groups * p.segs * kGroupRows * 16));
             ptx::mbar_arrive_expect_tx(&m.mbar_x[1], (uint32_t)(kD * kD * 4));
         }
         __syncthreads();
-        ptx::cluster_arrive();        // start-up barrier: waited on before the first push
+        ptx::cluster_arrive();        // start-up barrier: waited on under the first gathers
     }
     ptx::pdl_wait_prior_grid();
     // RMSNorm weight: async copy, covered by the first chunk's v/g load group
@@ -652,82 +650,69 @@ __global__ void __launch_bounds__(kThreads, 1) gla_tc_kernel(const Params p) {
         if (into_g && tid < kD) m.Gs[tid] += m.Bc[tid];
     };
     // Cluster-wide scan of the segment aggregates (Gs, S): every segment receives its
-    // incoming state.  Each CTA writes its aggregate to shared memory and moves it with
-    // one bulk copy per scanning CTA (cp.async.bulk into the peer's shared memory, bytes
-    // counted on the peer's mbarrier); a scanner owns a slice of state rows, combines the
-    // segments in order, stages every segment's result in that segment's layout and bulk
-    // copies it back.  Buffers: outgoing aggregate X (Ks region), incoming slices (receive
-    // region), scanner staging (q/k tiles, consumed), results into the a tile (S~, direct)
-    // or the g tile (S_in, before a multi-chunk pass) -- no buffer is written remotely while
-    // one of this CTA's own copies may still read it.
-    float *X = reinterpret_cast<float *>(sm + kST);   // [64 j][64 c] fp32 outgoing aggregate
-    const float *recv = reinterpret_cast<const float *>(sm + kRECV);
+    // incoming state.  The scan is elementwise per state entry (j, c) with the decay of key
+    // channel c, so it is split by channel groups: scanner r owns groups g = r + lg*segs.
+    // Forward: the state owners store each 4-channel piece of their row straight from
+    // registers into the group's scanner, and 32 threads store the 2^{G} and 2^{r} pieces
+    // (st.async, bytes counted on the receiver's mbar_x[0]); receive layout
+    // [lg][segment][66 rows][4] fp32.  Return: a scanner combines the segments in order and
+    // stores each segment's result, as soon as it is produced, into that segment's operand
+    // region (S~ in the a tile, direct) or row-major into the g tile (S_in, before a
+    // multi-chunk pass), counted on the receiver's mbar_x[1].  Every remote region written is
+    // idle at its owner by then: a CTA's a and g tiles are consumed before it publishes its
+    // aggregate, and results follow the aggregates.
+    bool cluster_ready = false;
+    auto cluster_ready_once = [&]() {                 // every CTA's exchange barriers exist
+        if (!cluster_ready) ptx::cluster_wait();
+        cluster_ready = true;
+    };
+    auto recv_off = [&](int lg, int seg, int row) {
+        return kRECV + (uint32_t)(((lg * p.segs + seg) * kGroupRows + row) * 16);
+    };
     auto xchg_begin = [&]() {
-        __syncthreads();                              // Gs, 2^r and S are final
+        cluster_ready_once();
+        if (tid < kD) m.eGrow[tid] = ptx::ex2(m.Gs[tid]);
+        __syncthreads();                              // 2^G row complete
         if (s_owner) {
 #pragma unroll
-            for (int i = 0; i < 8; ++i)
-                *reinterpret_cast<float4 *>(X + s_row * kD + 32 * ch + 4 * i) =
-                    make_float4(S[4 * i], S[4 * i + 1], S[4 * i + 2], S[4 * i + 3]);
+            for (int i = 0; i < 8; ++i) {
+                const int g = 8 * ch + i, dst = g % p.segs;
+                ptx::st_async_v4(ptx::mapa(sbase + recv_off(g / p.segs, rank, s_row), dst),
+                                 make_float4(S[4 * i], S[4 * i + 1], S[4 * i + 2], S[4 * i + 3]),
+                                 ptx::mapa(ptx::smem_u32(&m.mbar_x[0]), dst));
+            }
         }
-        if (tid < kD) m.eGrow[tid] = ptx::ex2(m.Gs[tid]);
-        ptx::fence_proxy_async_smem();                // sources of the bulk copies
-        __syncthreads();
-        ptx::cluster_wait();                          // every CTA's exchange barriers exist
-        if (tid < p.segs) {
-            const int r = tid, rr = slice_rows(r);
-            const uint32_t bar = ptx::mapa(ptx::smem_u32(&m.mbar_x[0]), r);
-            if (rr > 0)
-                ptx::bulk_to_cluster(ptx::mapa(sbase + kRECV + rank * rr * 256, r),
-                                     ptx::smem_u32(X + r * rows_per * kD), rr * 256, bar);
-            ptx::bulk_to_cluster(ptx::mapa(ptx::smem_u32(&m.Gall[rank][0]), r),
-                                 ptx::smem_u32(m.eGrow), kD * 4, bar);
-            ptx::bulk_to_cluster(ptx::mapa(ptx::smem_u32(&m.Eall[rank][0]), r),
-                                 ptx::smem_u32(m.eref), kD * 4, bar);
+        if (tid < 32) {
+            const int g = tid & 15, which = tid >> 4, dst = g % p.segs;
+            const float *src = which ? m.eref : m.eGrow;
+            ptx::st_async_v4(ptx::mapa(sbase + recv_off(g / p.segs, rank, kD + which), dst),
+                             *reinterpret_cast<const float4 *>(src + 4 * g),
+                             ptx::mapa(ptx::smem_u32(&m.mbar_x[0]), dst));
         }
     };
-    // direct: results are S~ = tf32(2^{r} S_in) in the inter product's operand layout, bulk
-    // copied into each segment's a-tile region, and S is not read back (one chunk); otherwise
-    // S_in lands row-major in the g-tile region and is read back into S.
     auto xchg_end = [&](bool scanners, bool direct) {
-        const uint32_t stage = kTQ;                   // q and k tiles: consumed, 32 KB
         if (scanners) {
             if (!wait_cluster_phase(&m.mbar_x[0], 0)) m.abort = 1;
-            const int segs = p.segs, r0 = rank * rows_per;
-            for (int idx = tid & 127; idx < my_rows * 32; idx += 128) {
-                const int i = idx >> 5, c = 2 * (idx & 31), j = r0 + i;
-                float2 run = make_float2(0.0f, 0.0f);
+            const int segs = p.segs;
+            for (int idx = tid & 127; idx < my_groups * kD; idx += 128) {
+                const int lg = idx >> 6, j = idx & 63, c = 4 * (lg * segs + rank);
+                const uint32_t off = direct ? kTA + (c >> 5) * kAtom64 + j * 128 + ((((c & 31) >> 2) ^ (j & 7)) << 4)
+                                            : kTG + j * 256 + c * 4;
+                const uint32_t laddr = sbase + off, lbar = ptx::smem_u32(&m.mbar_x[1]);
+                float4 run = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
 #pragma unroll 4
                 for (int q = 0; q < segs; ++q) {
-                    const float2 agg = *reinterpret_cast<const float2 *>(recv + (q * my_rows + i) * kD + c);
-                    const float2 g = *reinterpret_cast<const float2 *>(&m.Gall[q][c]);
-                    uint32_t off;
-                    float2 out;
+                    const float4 agg = *reinterpret_cast<const float4 *>(sm + recv_off(lg, q, j));
+                    const float4 g = *reinterpret_cast<const float4 *>(sm + recv_off(lg, q, kD));
+                    float4 out = run;                  // state entering segment q
                     if (direct) {
-                        const float2 f = *reinterpret_cast<const float2 *>(&m.Eall[q][c]);
-                        out = make_float2(ptx::to_tf32(f.x * run.x), ptx::to_tf32(f.y * run.y));
-                        off = q * my_rows * 256 + (c >> 5) * my_rows * 128 + i * 128 +
-                              ((((c & 31) >> 2) ^ (j & 7)) << 4) + (c & 3) * 4;
-                    } else {
-                        out = run;
-                        off = q * my_rows * 256 + i * 256 + c * 4;
+                        const float4 f = *reinterpret_cast<const float4 *>(sm + recv_off(lg, q, kD + 1));
+                        out = make_float4(ptx::to_tf32(f.x * run.x), ptx::to_tf32(f.y * run.y),
+                                          ptx::to_tf32(f.z * run.z), ptx::to_tf32(f.w * run.w));
                     }
-                    *reinterpret_cast<float2 *>(sm + stage + off) = out;   // state entering q
-                    run = make_float2(fmaf(g.x, run.x, agg.x), fmaf(g.y, run.y, agg.y));
-                }
-            }
-            ptx::fence_proxy_async_smem();
-            ptx::named_bar_sync(1, 128);
-            if ((tid & 127) < segs && my_rows > 0) {
-                const int q = tid & 127;
-                const uint32_t bar = ptx::mapa(ptx::smem_u32(&m.mbar_x[1]), q);
-                const uint32_t src = sbase + stage + q * my_rows * 256;
-                if (direct) {
-                    for (int a = 0; a < 2; ++a)
-                        ptx::bulk_to_cluster(ptx::mapa(sbase + kTA + a * kAtom64 + r0 * 128, q),
-                                             src + a * my_rows * 128, my_rows * 128, bar);
-                } else {
-                    ptx::bulk_to_cluster(ptx::mapa(sbase + kTG + r0 * 256, q), src, my_rows * 256, bar);
+                    ptx::st_async_v4(ptx::mapa(laddr, q), out, ptx::mapa(lbar, q));
+                    run = make_float4(fmaf(g.x, run.x, agg.x), fmaf(g.y, run.y, agg.y),
+                                      fmaf(g.z, run.z, agg.z), fmaf(g.w, run.w, agg.w));
                 }
             }
         }
@@ -770,6 +755,7 @@ __global__ void __launch_bounds__(kThreads, 1) gla_tc_kernel(const Params p) {
             ptx::tmem_relinquish();
             ptx::tc_fence_before_sync();
         }
+        if (step == 0 && exchange) cluster_ready_once();   // under the first gathers' latency
         gate(n);                                     // contains block barriers
         if (step == 0) {
             ptx::tc_fence_after_sync();
@@ -811,7 +797,7 @@ __global__ void __launch_bounds__(kThreads, 1) gla_tc_kernel(const Params p) {
         if (m.slow) {
             wait_mma(1);
             make_p_exact(sm, t, ch, n, p.scale, &m.range_err);
-            __syncthreads();                          // q/k tiles read; they stage the scan next
+            __syncthreads();
             if (mid_xchg) xchg_end(warp < 4, true);
         } else if (mid_xchg) {
             // warps 4..7 wait for the scores, build P and start P.V; warps 0..3 scan the

@@ -185,3 +185,28 @@ def test_eps_is_honoured():
         ref = oracle.gla_forward(x["q"], x["k"], x["v"], x["a"], x["g"], x["w"], 8, 8, 0,
                                  eps=eps)
         assert_close(u, ref, "f32")
+
+
+@pytest.mark.parametrize("segs", [2, 5, 7, 12])
+def test_segment_counts_sharing_channel_groups(segs):
+    # the state exchange splits the 16 four-channel groups over the segments; counts that do
+    # not divide 16 give some scanners two or more groups.  chunk 128 keeps each segment in one
+    # chunk (exchange mid-chunk, S~ written directly); chunk 32 gives several chunks per
+    # segment (state-only pass, exchange, S_in read back)
+    wl = synth.WORKLOADS["gtr640"].with_(H=2, grid_h=24, grid_w=37)
+    x = synth.make_inputs(wl, seed=segs)
+    ref = oracle_ref(x, 24, 37, 2)
+    for chunk in (32, 128):
+        assert_close(run_gpu(x, 24, 37, 2, chunk=chunk, segments=segs), ref, "f16")
+
+
+@pytest.mark.parametrize("segs", [13, 14, 15])
+def test_segment_counts_beyond_the_exchange_buffer_are_refused(segs):
+    import torch
+    wl = synth.WORKLOADS["gtr640"].with_(H=1, grid_h=16, grid_w=16)
+    x = synth.make_inputs(wl, seed=1)
+    t = {n: torch_dev(x[n]) for n in ("q", "k", "v", "a", "g", "w")}
+    out = torch.empty_like(t["v"])
+    with pytest.raises(gla.GLAError):
+        gla.gla_fwd_ex(t["q"], t["k"], t["v"], t["a"], t["g"], t["w"], out, 16, 16, 0,
+                       chunk=128, segments=segs)
