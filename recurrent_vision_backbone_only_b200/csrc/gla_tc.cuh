@@ -96,6 +96,7 @@ constexpr uint32_t kColO = 192;    // inter-chunk output accumulator 128 x 64
 constexpr uint32_t kColQH = 256;   // Q~ high part, tf32 A operand, 128 x 64
 constexpr uint32_t kColQL = 320;   // Q~ low part
 constexpr uint32_t kColOP = 384;   // intra-chunk output accumulator (P V) 128 x 64
+constexpr uint32_t kColSG = 448;   // SiLU(g) * w per token and channel, 128 x 64 fp32
 
 constexpr uint32_t kIdescST = ptx::idesc_make(0, true, true, 64, 64);
 constexpr uint32_t kIdescPV = ptx::idesc_make(0, false, true, 128, 64);
@@ -216,7 +217,7 @@ __device__ __forceinline__ uint32_t pack_half2(float lo, float hi) {
 
 // Shared scratch scalars.
 struct Misc {
-    uint64_t mbar_mma[4];     // [0] state, [1] scores, [2] inter (+ P.V), [3] early P.V
+    uint64_t mbar_mma[3];     // [0] state, [1] scores, [2] P.V and inter
     uint64_t mbar_ld[3];      // [0] a tile, [1] q and k tiles, [2] v and g tiles
     uint64_t mbar_x[2];       // exchange: [0] aggregates received, [1] S~ / S_in received
     uint32_t tmem_base;
@@ -301,7 +302,7 @@ __global__ void __launch_bounds__(kThreads, 1) gla_tc_kernel(const Params p) {
     ptx::pdl_launch_dependents();
     // ---- setup: barriers and weight; TMEM is allocated once the first gathers are in flight
     if (tid == 0) {
-        for (int i = 0; i < 4; ++i) ptx::mbar_init(&m.mbar_mma[i], 1);
+        for (int i = 0; i < 3; ++i) ptx::mbar_init(&m.mbar_mma[i], 1);
         for (int i = 0; i < 3; ++i) ptx::mbar_init(&m.mbar_ld[i], kThreads);
         ptx::fence_mbarrier_init();
         m.abort = 0;
@@ -329,7 +330,7 @@ __global__ void __launch_bounds__(kThreads, 1) gla_tc_kernel(const Params p) {
     __syncthreads();
     uint32_t tmem = 0, tmem_warp = 0;
     uint32_t it = 0;                  // chunk iterations so far (load-barrier parity)
-    uint32_t ph_mma[4] = {0, 0, 0, 0};
+    uint32_t ph_mma[3] = {0, 0, 0};
 
     // State rows owned by lanes < 16: state column j = 16*w4 + lane (a row of the transposed
     // state), channels c in [32*ch, 32*ch + 32).
@@ -576,14 +577,6 @@ __global__ void __launch_bounds__(kThreads, 1) gla_tc_kernel(const Params p) {
         p_block(ch * 64 + 32, n, dq, amax);
         if (amax > 65504.0f) m.range_err = 1;
     };
-    // warps 4..7 only: row t, all 128 columns (the other warps run the state exchange)
-    auto make_p_rows = [&](int n) {
-        const float dq = (m.dqp[0][t] + m.dqp[1][t]) * p.scale;
-        float amax = 0.0f;
-#pragma unroll 1
-        for (int b4 = 0; b4 < 4; ++b4) p_block(b4 * 32, n, dq, amax);
-        if (amax > 65504.0f) m.range_err = 1;
-    };
     // S~[j][c] = 2^{r_c} S_in[c][j], tf32 K-major (rows j, 2 atoms of 32 channels)
     auto write_stilde = [&]() {
         if (s_owner) {
@@ -597,6 +590,30 @@ __global__ void __launch_bounds__(kThreads, 1) gla_tc_kernel(const Params p) {
         }
     };
     // ------------------------------------------------------------ epilogue (row t, 32 channels)
+    // SiLU(g) * w for row t, channels [32ch, 32ch + 32), into TMEM (read by the epilogue);
+    // computed while the inter product runs
+    auto prep_sg = [&]() {
+        wait_bar(&m.mbar_ld[2], it & 1);               // g tile
+#pragma unroll
+        for (int jj = 0; jj < 4; ++jj) {
+            const int j = ch * 4 + jj;
+            const uint4 graw = *reinterpret_cast<const uint4 *>(sm + kTG + off_f16(t, j));
+            const __half2 *g2 = reinterpret_cast<const __half2 *>(&graw);
+            const float4 wa = *reinterpret_cast<const float4 *>(&m.w[8 * j]);
+            const float4 wb = *reinterpret_cast<const float4 *>(&m.w[8 * j + 4]);
+            const float wv[8] = {wa.x, wa.y, wa.z, wa.w, wb.x, wb.y, wb.z, wb.w};
+            float sg[8];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const float2 gf = __half22float2(g2[e]);
+                sg[2 * e] = wv[2 * e] * silu_fast(gf.x);
+                sg[2 * e + 1] = wv[2 * e + 1] * silu_fast(gf.y);
+            }
+            ptx::tmem_st8(tmem_warp + kColSG + 8 * j, sg);
+        }
+        ptx::tmem_st_wait();
+    };
+    // u = (O_inter + O_intra) / rms * SiLU(g) * w, row t, 32 channels
     auto epilogue = [&](int n) {
         float o[32], op[32];
         ptx::tmem_ld32(tmem_warp + kColO + 32 * ch, o);
@@ -608,26 +625,17 @@ __global__ void __launch_bounds__(kThreads, 1) gla_tc_kernel(const Params p) {
 #pragma unroll
         for (int j = 0; j < 32; ++j) ss = fmaf(o[j], o[j], ss);
         m.red[ch][t] = ss;
+        ptx::tmem_ld32(tmem_warp + kColSG + 32 * ch, op);
+        ptx::tmem_ld_wait();
         __syncthreads();
         const float inv = rsqrtf((m.red[0][t] + m.red[1][t]) * (1.0f / 64.0f) + p.eps);
-        wait_bar(&m.mbar_ld[2], it & 1);               // g tile
         if (t < n) {
             __half *dst = p.out + (size_t)m.rows[t] * kD + 32 * ch;
 #pragma unroll
             for (int jj = 0; jj < 4; ++jj) {
-                const int j = ch * 4 + jj;
-                const uint4 graw = *reinterpret_cast<const uint4 *>(sm + kTG + off_f16(t, j));
-                const __half2 *g2 = reinterpret_cast<const __half2 *>(&graw);
-                const float4 wa = *reinterpret_cast<const float4 *>(&m.w[8 * j]);
-                const float4 wb = *reinterpret_cast<const float4 *>(&m.w[8 * j + 4]);
-                const float wv[8] = {wa.x, wa.y, wa.z, wa.w, wb.x, wb.y, wb.z, wb.w};
                 float u[8];
 #pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const float2 gf = __half22float2(g2[e]);
-                    u[2 * e] = o[8 * jj + 2 * e] * inv * wv[2 * e] * silu_fast(gf.x);
-                    u[2 * e + 1] = o[8 * jj + 2 * e + 1] * inv * wv[2 * e + 1] * silu_fast(gf.y);
-                }
+                for (int e = 0; e < 8; ++e) u[e] = o[8 * jj + e] * inv * op[8 * jj + e];
                 uint4 pk;
                 pk.x = pack_half2(u[0], u[1]); pk.y = pack_half2(u[2], u[3]);
                 pk.z = pack_half2(u[4], u[5]); pk.w = pack_half2(u[6], u[7]);
@@ -690,32 +698,39 @@ __global__ void __launch_bounds__(kThreads, 1) gla_tc_kernel(const Params p) {
                              ptx::mapa(ptx::smem_u32(&m.mbar_x[0]), dst));
         }
     };
-    auto xchg_end = [&](bool scanners, bool direct) {
-        if (scanners) {
-            if (!wait_cluster_phase(&m.mbar_x[0], 0)) m.abort = 1;
-            const int segs = p.segs;
-            for (int idx = tid & 127; idx < my_groups * kD; idx += 128) {
-                const int lg = idx >> 6, j = idx & 63, c = 4 * (lg * segs + rank);
-                const uint32_t off = direct ? kTA + (c >> 5) * kAtom64 + j * 128 + ((((c & 31) >> 2) ^ (j & 7)) << 4)
-                                            : kTG + j * 256 + c * 4;
-                const uint32_t laddr = sbase + off, lbar = ptx::smem_u32(&m.mbar_x[1]);
-                float4 run = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+    // Scan of the received aggregates by warps 0..3: an item is (owned group, row j); its
+    // chain runs over the segments in order and stores each segment's incoming state as soon
+    // as it is produced.
+    auto xchg_scan = [&](bool direct) {
+        if (warp >= 4) return;                        // warp-uniform
+        if (!wait_cluster_phase(&m.mbar_x[0], 0)) m.abort = 1;
+        const int segs = p.segs;
+        const uint32_t lbar = ptx::smem_u32(&m.mbar_x[1]);
+        for (int idx = tid; idx < my_groups * kD; idx += 128) {
+            const int lg = idx >> 6, j = idx & 63, c = 4 * (lg * segs + rank);
+            const uint32_t off = direct ? kTA + (c >> 5) * kAtom64 + j * 128 + ((((c & 31) >> 2) ^ (j & 7)) << 4)
+                                        : kTG + j * 256 + c * 4;
+            const uint32_t laddr = sbase + off;
+            float4 run = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
 #pragma unroll 4
-                for (int q = 0; q < segs; ++q) {
-                    const float4 agg = *reinterpret_cast<const float4 *>(sm + recv_off(lg, q, j));
-                    const float4 g = *reinterpret_cast<const float4 *>(sm + recv_off(lg, q, kD));
-                    float4 out = run;                  // state entering segment q
-                    if (direct) {
-                        const float4 f = *reinterpret_cast<const float4 *>(sm + recv_off(lg, q, kD + 1));
-                        out = make_float4(ptx::to_tf32(f.x * run.x), ptx::to_tf32(f.y * run.y),
-                                          ptx::to_tf32(f.z * run.z), ptx::to_tf32(f.w * run.w));
-                    }
-                    ptx::st_async_v4(ptx::mapa(laddr, q), out, ptx::mapa(lbar, q));
-                    run = make_float4(fmaf(g.x, run.x, agg.x), fmaf(g.y, run.y, agg.y),
-                                      fmaf(g.z, run.z, agg.z), fmaf(g.w, run.w, agg.w));
+            for (int q = 0; q < segs; ++q) {
+                const float4 agg = *reinterpret_cast<const float4 *>(sm + recv_off(lg, q, j));
+                const float4 g = *reinterpret_cast<const float4 *>(sm + recv_off(lg, q, kD));
+                float4 out = run;                      // state entering segment q
+                if (direct) {
+                    const float4 f = *reinterpret_cast<const float4 *>(sm + recv_off(lg, q, kD + 1));
+                    out = make_float4(ptx::to_tf32(f.x * run.x), ptx::to_tf32(f.y * run.y),
+                                      ptx::to_tf32(f.z * run.z), ptx::to_tf32(f.w * run.w));
                 }
+                ptx::st_async_v4(ptx::mapa(laddr, q), out, ptx::mapa(lbar, q));
+                run = make_float4(fmaf(g.x, run.x, agg.x), fmaf(g.y, run.y, agg.y),
+                                  fmaf(g.z, run.z, agg.z), fmaf(g.w, run.w, agg.w));
             }
         }
+    };
+    // wait for this CTA's incoming state: S~ in the a tile (direct) or S_in in the g tile
+    // (read back into the state owners' registers)
+    auto xchg_wait = [&](bool direct) {
         if (!wait_cluster_phase(&m.mbar_x[1], 0)) m.abort = 1;
         if (!direct && s_owner) {
             const float *Sin = reinterpret_cast<const float *>(sm + kTG);
@@ -738,7 +753,8 @@ __global__ void __launch_bounds__(kThreads, 1) gla_tc_kernel(const Params p) {
         const int ci = pass1 ? step : step - n_pass1;
         if (!pass1 && ci == 0 && !resident && exchange) {
             xchg_begin();
-            xchg_end(warp < 4, false);
+            xchg_scan(false);
+            xchg_wait(false);
         }
         int n;
         {
@@ -768,7 +784,7 @@ __global__ void __launch_bounds__(kThreads, 1) gla_tc_kernel(const Params p) {
         // The state product goes first: the segment aggregate is published while the score
         // products run.  The issuing thread stalls while its products drain, so the score
         // products are issued only after this CTA has arrived on the cluster barrier.
-        if (tid == 0) {
+        if (warp == 0 && ptx::elect_one()) {
             ptx::tc_fence_after_sync();
             issue_state(sbase, tmem);
             ptx::mma_commit(&m.mbar_mma[0]);
@@ -783,62 +799,40 @@ __global__ void __launch_bounds__(kThreads, 1) gla_tc_kernel(const Params p) {
             ++it;
             continue;
         }
-        // publish the segment aggregate now: the exchange runs under the score operands,
-        // the score products and P
+        // publish the segment aggregate now: the exchange runs under the score operands and
+        // the score products
         if (mid_xchg) xchg_begin();
         build_qk();
         operands_ready();
-        if (tid == 128) {                            // score products, issued by warp 4
+        if (warp == 4 && ptx::elect_one()) {         // score products, issued by warp 4
             ptx::tc_fence_after_sync();
             if (!m.slow) issue_qk(sbase, tmem, min(kC, (n + 15) & ~15));
             ptx::mma_commit(&m.mbar_mma[1]);
         }
-        const bool pv_early = mid_xchg && !m.slow;
-        if (m.slow) {
-            wait_mma(1);
-            make_p_exact(sm, t, ch, n, p.scale, &m.range_err);
-            __syncthreads();
-            if (mid_xchg) xchg_end(warp < 4, true);
-        } else if (mid_xchg) {
-            // warps 4..7 wait for the scores, build P and start P.V; warps 0..3 scan the
-            // segment states and write every segment's S~ directly
-            if (warp >= 4) {
-                wait_mma(1);
-                make_p_rows(n);
-                ptx::fence_proxy_async_smem();
-                ptx::tc_fence_before_sync();
-                ptx::named_bar_sync(2, 128);
-                if (tid == 128) {
-                    ptx::tc_fence_after_sync();
-                    issue_pv(sbase, kPB, tmem);
-                    ptx::mma_commit(&m.mbar_mma[3]);
-                }
-            } else {
-                ph_mma[1] ^= 1u;                      // this phase is consumed by warps 4..7
-            }
-            xchg_end(warp < 4, true);
-        } else {
-            wait_mma(1);
-            make_p_fast(n);
-        }
-        if (!pv_early) {
-            operands_ready();
-            if (tid == 0) {
-                ptx::tc_fence_after_sync();
-                issue_pv(sbase, m.slow ? kKH : kPB, tmem);
-            }
-        }
-        if (!mid_xchg) write_stilde();
+        if (mid_xchg) xchg_scan(true);
+        wait_mma(1);
+        if (m.slow) make_p_exact(sm, t, ch, n, p.scale, &m.range_err);
+        else make_p_fast(n);
         operands_ready();
-        if (tid == 0) {
+        if (warp == 0 && ptx::elect_one()) {
+            ptx::tc_fence_after_sync();
+            issue_pv(sbase, m.slow ? kKH : kPB, tmem);
+        }
+        if (mid_xchg) {
+            xchg_wait(true);
+        } else {
+            write_stilde();                          // S~ from the state entering this chunk,
+            if (ci + 1 < n_chunks) fold_sloc(false); // then S = S 2^{B} + Sloc for the next one
+        }
+        operands_ready();
+        if (warp == 0 && ptx::elect_one()) {
             ptx::tc_fence_after_sync();
             issue_inter(sbase, tmem, false);
-            ptx::mma_commit(&m.mbar_mma[2]);
+            ptx::mma_commit(&m.mbar_mma[2]);         // P.V and the inter product
         }
-        if (pv_early) wait_mma(3);
+        prep_sg();
         wait_mma(2);
         epilogue(n);
-        if (ci + 1 < n_chunks) fold_sloc(false);
         ptx::tc_fence_before_sync();
         __syncthreads();
         ++it;
