@@ -590,13 +590,12 @@ __global__ void __launch_bounds__(kThreads, 1) gla_tc_kernel(const Params p) {
         }
     };
     // ------------------------------------------------------------ epilogue (row t, 32 channels)
-    // SiLU(g) * w for row t, channels [32ch, 32ch + 32), into TMEM (read by the epilogue);
-    // computed while the inter product runs
+    // SiLU(g) * w for row t, all 64 channels, into TMEM (read by the epilogue).  Run by one
+    // warp per TMEM lane quarter while the score products execute.
     auto prep_sg = [&]() {
         wait_bar(&m.mbar_ld[2], it & 1);               // g tile
-#pragma unroll
-        for (int jj = 0; jj < 4; ++jj) {
-            const int j = ch * 4 + jj;
+#pragma unroll 2
+        for (int j = 0; j < 8; ++j) {
             const uint4 graw = *reinterpret_cast<const uint4 *>(sm + kTG + off_f16(t, j));
             const __half2 *g2 = reinterpret_cast<const __half2 *>(&graw);
             const float4 wa = *reinterpret_cast<const float4 *>(&m.w[8 * j]);
@@ -613,7 +612,9 @@ __global__ void __launch_bounds__(kThreads, 1) gla_tc_kernel(const Params p) {
         }
         ptx::tmem_st_wait();
     };
-    // u = (O_inter + O_intra) / rms * SiLU(g) * w, row t, 32 channels
+    // u = (O_inter + O_intra) / rms * SiLU(g) * w.  Row t, 32 channels per thread, staged as
+    // fp16 rows in the K~ low-part region (free once the score products completed), then
+    // stored with each group of 8 threads writing one whole 128-byte token row.
     auto epilogue = [&](int n) {
         float o[32], op[32];
         ptx::tmem_ld32(tmem_warp + kColO + 32 * ch, o);
@@ -629,18 +630,23 @@ __global__ void __launch_bounds__(kThreads, 1) gla_tc_kernel(const Params p) {
         ptx::tmem_ld_wait();
         __syncthreads();
         const float inv = rsqrtf((m.red[0][t] + m.red[1][t]) * (1.0f / 64.0f) + p.eps);
-        if (t < n) {
-            __half *dst = p.out + (size_t)m.rows[t] * kD + 32 * ch;
 #pragma unroll
-            for (int jj = 0; jj < 4; ++jj) {
-                float u[8];
+        for (int jj = 0; jj < 4; ++jj) {
+            float u[8];
 #pragma unroll
-                for (int e = 0; e < 8; ++e) u[e] = o[8 * jj + e] * inv * op[8 * jj + e];
-                uint4 pk;
-                pk.x = pack_half2(u[0], u[1]); pk.y = pack_half2(u[2], u[3]);
-                pk.z = pack_half2(u[4], u[5]); pk.w = pack_half2(u[6], u[7]);
-                *reinterpret_cast<uint4 *>(dst + 8 * jj) = pk;
-            }
+            for (int e = 0; e < 8; ++e) u[e] = o[8 * jj + e] * inv * op[8 * jj + e];
+            uint4 pk;
+            pk.x = pack_half2(u[0], u[1]); pk.y = pack_half2(u[2], u[3]);
+            pk.z = pack_half2(u[4], u[5]); pk.w = pack_half2(u[6], u[7]);
+            *reinterpret_cast<uint4 *>(sm + kKL + off_f16(t, 4 * ch + jj)) = pk;
+        }
+        __syncthreads();
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const int row = (tid >> 3) + 32 * i, j = tid & 7;
+            if (row < n)
+                *reinterpret_cast<uint4 *>(p.out + (size_t)m.rows[row] * kD + 8 * j) =
+                    *reinterpret_cast<const uint4 *>(sm + kKL + off_f16(row, j));
         }
     };
     // fold the chunk's local state into S: S = S Diag(2^{B}) + Sloc (transposed form)
@@ -804,12 +810,15 @@ __global__ void __launch_bounds__(kThreads, 1) gla_tc_kernel(const Params p) {
         if (mid_xchg) xchg_begin();
         build_qk();
         operands_ready();
-        if (warp == 4 && ptx::elect_one()) {         // score products, issued by warp 4
+        // score products, issued by warp 7; meanwhile warps 4..6 and 3 (after its share of
+        // the scan) compute SiLU(g) * w for their TMEM lane quarters and warps 0..3 scan
+        if (warp == 7 && ptx::elect_one()) {
             ptx::tc_fence_after_sync();
             if (!m.slow) issue_qk(sbase, tmem, min(kC, (n + 15) & ~15));
             ptx::mma_commit(&m.mbar_mma[1]);
         }
         if (mid_xchg) xchg_scan(true);
+        if (warp == 3 || (warp >= 4 && warp < 7)) prep_sg();
         wait_mma(1);
         if (m.slow) make_p_exact(sm, t, ch, n, p.scale, &m.range_err);
         else make_p_fast(n);
@@ -830,7 +839,6 @@ __global__ void __launch_bounds__(kThreads, 1) gla_tc_kernel(const Params p) {
             issue_inter(sbase, tmem, false);
             ptx::mma_commit(&m.mbar_mma[2]);         // P.V and the inter product
         }
-        prep_sg();
         wait_mma(2);
         epilogue(n);
         ptx::tc_fence_before_sync();
