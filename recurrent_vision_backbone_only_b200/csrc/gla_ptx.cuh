@@ -336,6 +336,20 @@ __device__ __forceinline__ uint64_t desc_sw128(uint32_t saddr, uint32_t lbo_byte
     return d;
 }
 
+// Shared-memory matrix descriptor for a 32-bit MN-major operand: 128-byte rows swizzled in
+// 32-byte granules over 4-row atoms (the only MN-major layout for tf32); lbo = stride between
+// 32-element MN atoms, sbo = stride between 4-row K groups.
+__device__ __forceinline__ uint64_t desc_sw128_b32(uint32_t saddr, uint32_t lbo_bytes,
+                                                   uint32_t sbo_bytes) {
+    uint64_t d = 0;
+    d |= (uint64_t)((saddr >> 4) & 0x3FFFu);
+    d |= (uint64_t)((lbo_bytes >> 4) & 0x3FFFu) << 16;
+    d |= (uint64_t)((sbo_bytes >> 4) & 0x3FFFu) << 32;
+    d |= (uint64_t)1 << 46;
+    d |= (uint64_t)1 << 61;
+    return d;
+}
+
 // Instruction descriptor (dense, fp32 accumulate).  fmt: 0 = f16, 2 = tf32.
 // a_mn / b_mn: operand is MN-major (else K-major).
 __host__ __device__ constexpr uint32_t idesc_make(uint32_t fmt, bool a_mn, bool b_mn, uint32_t M,

@@ -100,7 +100,7 @@ constexpr uint32_t kColSG = 448;   // SiLU(g) * w per token and channel, 128 x 6
 
 constexpr uint32_t kIdescST = ptx::idesc_make(0, true, true, 64, 64);
 constexpr uint32_t kIdescPV = ptx::idesc_make(0, false, true, 128, 64);
-constexpr uint32_t kIdescIN = ptx::idesc_make(2, false, false, 128, 64);
+constexpr uint32_t kIdescIN = ptx::idesc_make(2, false, true, 128, 64);
 
 struct Params {
     const __half *q, *k, *v, *a, *g;
@@ -123,6 +123,20 @@ __device__ __forceinline__ uint32_t off_f16(uint32_t row, uint32_t j) { return p
 // fp16 K-major operand with K = 128 (2 atoms): chunk j of K (0..15).
 __device__ __forceinline__ uint32_t off_f16k128(uint32_t row, uint32_t j) {
     return (j >> 3) * kAtom128 + ptx::sw128(row, j & 7);
+}
+// S~ (the inter product's B operand), tf32 MN-major: one 128-byte row per key channel c
+// holding 32 value columns j, 32-byte granules swizzled by (c & 3) within 4-row groups of
+// 512 bytes; two atoms for j < 32 and j >= 32.  Byte offset of (c, j).
+__device__ __forceinline__ uint32_t off_stilde(uint32_t c, uint32_t j) {
+    return (j >> 5) * kAtom64 + (c >> 2) * 512 + (c & 3) * 128 + ((((j & 31) >> 3) ^ (c & 3)) << 5) +
+           (j & 7) * 4;
+}
+// Row slot of aggregate row j in the exchange receive buffer: a bijection within each
+// 16-row block that keeps a warp's stores of 16 consecutive rows contiguous and makes the
+// scanners' reads of 4 consecutive rows at one channel (8 row quads x 4 channels per warp)
+// hit 32 distinct banks.
+__device__ __forceinline__ uint32_t recv_slot(uint32_t j) {
+    return (j & ~7u) | (j & 4u) | ((j ^ (j >> 2)) & 2u) | ((j ^ (j >> 4)) & 1u);
 }
 
 // ------------------------------------------------------------ MMA issue (1 thread)
@@ -161,15 +175,14 @@ __device__ __forceinline__ void issue_pv(uint32_t sbase, uint32_t p_base, uint32
                         ptx::desc_sw128(sbase + kTV + k * 2048, kAtom128, 1024), kIdescPV, k > 0);
     }
 }
-// O[t][j] (+)= sum_c (Qh + Ql)[t][c] S~[j][c], S~ in the a-tile region
+// O[t][j] (+)= sum_c (Qh + Ql)[t][c] S~[c][j], S~ (MN-major) in the a-tile region
 __device__ __forceinline__ void issue_inter(uint32_t sbase, uint32_t tmem, bool accumulate) {
 #pragma unroll
     for (int pass = 0; pass < 2; ++pass) {
 #pragma unroll
-        for (int k = 0; k < 8; ++k) {
-            const uint32_t soff = (k >> 2) * kAtom64 + (k & 3) * 32;
+        for (int k = 0; k < 8; ++k) {                  // 8 key channels = 8 S~ rows per step
             ptx::mma_tf32_ts(tmem + kColO, tmem + (pass ? kColQL : kColQH) + 8 * k,
-                             ptx::desc_sw128(sbase + kTA + soff, 16, 1024), kIdescIN,
+                             ptx::desc_sw128_b32(sbase + kTA + k * 1024, kAtom64, 512), kIdescIN,
                              accumulate || pass > 0 || k > 0);
         }
     }
@@ -203,6 +216,17 @@ __device__ __forceinline__ bool wait_cluster_phase(uint64_t *bar, uint32_t parit
 __device__ __forceinline__ float log2_gamma(float a) {
     const float x = ptx::ex2(-fabsf(a) * kLog2e);             // 2^{-|a| log2 e} = e^{-|a|}
     return (fminf(a, 0.0f) * kLog2e - ptx::lg2(1.0f + x)) * kInvTau;
+}
+
+// 1/x for a positive normal x on the FMA pipe: Newton-Raphson, y <- y + y (1 - x y), from the
+// seed obtained by subtracting the bit pattern of x from a constant (the exponent is negated
+// and the mantissa linearly approximated: relative error below 6%); three steps square the
+// error each time, to about 1 ulp.  Used where the special-function unit is the busier pipe.
+__device__ __forceinline__ float rcp_nr(float x) {
+    float y = __uint_as_float(0x7EF311C7u - __float_as_uint(x));
+#pragma unroll
+    for (int i = 0; i < 3; ++i) y = fmaf(y, fmaf(-x, y, 1.0f), y);
+    return y;
 }
 
 // SiLU(g) = g / (1 + e^{-g})
@@ -452,8 +476,10 @@ __global__ void __launch_bounds__(kThreads, 1) gla_tc_kernel(const Params p) {
             *reinterpret_cast<uint4 *>(sm + kST + off_f16(t, j)) = kso;
         }
     };
-    // Score operands.  Fast path: Qh/Ql (TMEM, carrying d_k^{-1/2}), Kh/Kl (smem tf32);
-    // slow path: Qh/Ql of d_k^{-1/2} q 2^{b} only.  Also the exact diagonal q_t . k_t.
+    // Score operands.  Fast path: with x = 2^{r - b} (one ex2), Kh/Kl (smem tf32) of K~ = k x
+    // and Qh/Ql (TMEM) of Q~ = q / (8 x) (Newton reciprocal; the rounding of x cancels in each
+    // product q_tc x^-1 k_sc x); slow path: Qh/Ql of d_k^{-1/2} q 2^{b} only.  Also the exact
+    // diagonal q_t . k_t.
     auto build_qk = [&]() {
         const bool slow = m.slow != 0;
         float dqs = 0.0f;                          // partial q_t . k_t over this half's channels
@@ -487,8 +513,9 @@ __global__ void __launch_bounds__(kThreads, 1) gla_tc_kernel(const Params p) {
 #pragma unroll
             for (int e = 0; e < 8; ++e) {
                 if (!slow) {
-                    const float kf = kv[e] * ptx::ex2(rr[e] - bt[e]);             // k 2^{r - b}
-                    const float qf = qv[e] * ptx::ex2(bt[e] - rr[e] + kLog2Scale); // q 2^{b - r} / 8
+                    const float x = ptx::ex2(rr[e] - bt[e]);
+                    const float kf = kv[e] * x;                              // k 2^{r - b}
+                    const float qf = qv[e] * rcp_nr(x) * 0.125f;             // q 2^{b - r} / 8
                     kh[e] = ptx::tf32_hi(kf);
                     kl[e] = kf - kh[e];
                     qh[e] = ptx::tf32_hi(qf);
@@ -577,25 +604,23 @@ __global__ void __launch_bounds__(kThreads, 1) gla_tc_kernel(const Params p) {
         p_block(ch * 64 + 32, n, dq, amax);
         if (amax > 65504.0f) m.range_err = 1;
     };
-    // S~[j][c] = 2^{r_c} S_in[c][j], tf32 K-major (rows j, 2 atoms of 32 channels)
+    // S~[c][j] = tf32(2^{r_c} S[c][j]) from the state owners' registers (value column j, key
+    // channels 32ch..32ch+31); 16 consecutive j per warp fill 64 contiguous bytes of a row
     auto write_stilde = [&]() {
         if (s_owner) {
 #pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                const float4 e4 = *reinterpret_cast<const float4 *>(&m.eref[32 * ch + 4 * i]);
-                *reinterpret_cast<float4 *>(sm + kTA + off_tf32(kAtom64, s_row, 8 * ch + i)) =
-                    make_float4(ptx::to_tf32(S[4 * i] * e4.x), ptx::to_tf32(S[4 * i + 1] * e4.y),
-                                ptx::to_tf32(S[4 * i + 2] * e4.z), ptx::to_tf32(S[4 * i + 3] * e4.w));
+            for (int k = 0; k < 32; ++k) {
+                const int c = 32 * ch + k;
+                *reinterpret_cast<float *>(sm + kTA + off_stilde(c, s_row)) = ptx::to_tf32(S[k] * m.eref[c]);
             }
         }
     };
-    // ------------------------------------------------------------ epilogue (row t, 32 channels)
-    // SiLU(g) * w for row t, all 64 channels, into TMEM (read by the epilogue).  Run by one
-    // warp per TMEM lane quarter while the score products execute.
-    auto prep_sg = [&]() {
+    // SiLU(g) * w for row t, channel chunks [j0, j1) of 8, into TMEM (read by the epilogue).
+    // Run while the score products execute, by warps of this row's TMEM lane quarter.
+    auto prep_sg = [&](int j0, int j1) {
         wait_bar(&m.mbar_ld[2], it & 1);               // g tile
 #pragma unroll 2
-        for (int j = 0; j < 8; ++j) {
+        for (int j = j0; j < j1; ++j) {
             const uint4 graw = *reinterpret_cast<const uint4 *>(sm + kTG + off_f16(t, j));
             const __half2 *g2 = reinterpret_cast<const __half2 *>(&graw);
             const float4 wa = *reinterpret_cast<const float4 *>(&m.w[8 * j]);
@@ -669,10 +694,11 @@ __global__ void __launch_bounds__(kThreads, 1) gla_tc_kernel(const Params p) {
     // Forward: the state owners store each 4-channel piece of their row straight from
     // registers into the group's scanner, and 32 threads store the 2^{G} and 2^{r} pieces
     // (st.async, bytes counted on the receiver's mbar_x[0]); receive layout
-    // [lg][segment][66 rows][4] fp32.  Return: a scanner combines the segments in order and
-    // stores each segment's result, as soon as it is produced, into that segment's operand
-    // region (S~ in the a tile, direct) or row-major into the g tile (S_in, before a
-    // multi-chunk pass), counted on the receiver's mbar_x[1].  Every remote region written is
+    // [lg][segment][66 rows][4] fp32, aggregate row j in slot recv_slot(j), then the 2^{G} and
+    // 2^{r} rows.  Return: a scanner combines the segments in order and stores each segment's
+    // result, as soon as it is produced, into that segment's operand region (S~, MN-major, in
+    // the a tile, direct) or channel-major into the g tile (S_in, before a multi-chunk pass),
+    // counted on the receiver's mbar_x[1].  Every remote region written is
     // idle at its owner by then: a CTA's a and g tiles are consumed before it publishes its
     // aggregate, and results follow the aggregates.
     bool cluster_ready = false;
@@ -691,7 +717,7 @@ __global__ void __launch_bounds__(kThreads, 1) gla_tc_kernel(const Params p) {
 #pragma unroll
             for (int i = 0; i < 8; ++i) {
                 const int g = 8 * ch + i, dst = g % p.segs;
-                ptx::st_async_v4(ptx::mapa(sbase + recv_off(g / p.segs, rank, s_row), dst),
+                ptx::st_async_v4(ptx::mapa(sbase + recv_off(g / p.segs, rank, recv_slot(s_row)), dst),
                                  make_float4(S[4 * i], S[4 * i + 1], S[4 * i + 2], S[4 * i + 3]),
                                  ptx::mapa(ptx::smem_u32(&m.mbar_x[0]), dst));
             }
@@ -704,47 +730,52 @@ __global__ void __launch_bounds__(kThreads, 1) gla_tc_kernel(const Params p) {
                              ptx::mapa(ptx::smem_u32(&m.mbar_x[0]), dst));
         }
     };
-    // Scan of the received aggregates by warps 0..3: an item is (owned group, row j); its
-    // chain runs over the segments in order and stores each segment's incoming state as soon
-    // as it is produced.
+    // Scan of the received aggregates by warps 0..3.  An item is (owned group, key channel c,
+    // quad of value columns j0..j0+3); its chain runs over the segments in order and the state
+    // entering each segment is stored, as one 16-byte piece of that segment's S~ row c (or
+    // S_in row c), as soon as it is produced.  A warp covers 8 quads x 4 channels, i.e. four
+    // whole 128-byte destination rows per store.
     auto xchg_scan = [&](bool direct) {
         if (warp >= 4) return;                        // warp-uniform
         if (!wait_cluster_phase(&m.mbar_x[0], 0)) m.abort = 1;
         const int segs = p.segs;
         const uint32_t lbar = ptx::smem_u32(&m.mbar_x[1]);
         for (int idx = tid; idx < my_groups * kD; idx += 128) {
-            const int lg = idx >> 6, j = idx & 63, c = 4 * (lg * segs + rank);
-            const uint32_t off = direct ? kTA + (c >> 5) * kAtom64 + j * 128 + ((((c & 31) >> 2) ^ (j & 7)) << 4)
-                                        : kTG + j * 256 + c * 4;
-            const uint32_t laddr = sbase + off;
+            const int lg = idx >> 6, jq = (idx >> 2) & 15, cl = idx & 3;
+            const int c = 4 * (lg * segs + rank) + cl, j0 = 4 * jq;
+            const uint32_t laddr = sbase + (direct ? kTA + off_stilde(c, j0) : kTG + c * 256 + j0 * 4);
+            uint32_t rs[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) rs[i] = recv_slot(j0 + i) * 16 + cl * 4;
             float4 run = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
 #pragma unroll 4
             for (int q = 0; q < segs; ++q) {
-                const float4 agg = *reinterpret_cast<const float4 *>(sm + recv_off(lg, q, j));
-                const float4 g = *reinterpret_cast<const float4 *>(sm + recv_off(lg, q, kD));
+                const uint8_t *blk = sm + recv_off(lg, q, 0);
+                const float4 agg = make_float4(*reinterpret_cast<const float *>(blk + rs[0]),
+                                               *reinterpret_cast<const float *>(blk + rs[1]),
+                                               *reinterpret_cast<const float *>(blk + rs[2]),
+                                               *reinterpret_cast<const float *>(blk + rs[3]));
+                const float g = *reinterpret_cast<const float *>(blk + kD * 16 + cl * 4);
                 float4 out = run;                      // state entering segment q
                 if (direct) {
-                    const float4 f = *reinterpret_cast<const float4 *>(sm + recv_off(lg, q, kD + 1));
-                    out = make_float4(ptx::to_tf32(f.x * run.x), ptx::to_tf32(f.y * run.y),
-                                      ptx::to_tf32(f.z * run.z), ptx::to_tf32(f.w * run.w));
+                    const float f = *reinterpret_cast<const float *>(blk + (kD + 1) * 16 + cl * 4);
+                    out = make_float4(ptx::to_tf32(f * run.x), ptx::to_tf32(f * run.y),
+                                      ptx::to_tf32(f * run.z), ptx::to_tf32(f * run.w));
                 }
                 ptx::st_async_v4(ptx::mapa(laddr, q), out, ptx::mapa(lbar, q));
-                run = make_float4(fmaf(g.x, run.x, agg.x), fmaf(g.y, run.y, agg.y),
-                                  fmaf(g.z, run.z, agg.z), fmaf(g.w, run.w, agg.w));
+                run = make_float4(fmaf(g, run.x, agg.x), fmaf(g, run.y, agg.y),
+                                  fmaf(g, run.z, agg.z), fmaf(g, run.w, agg.w));
             }
         }
     };
-    // wait for this CTA's incoming state: S~ in the a tile (direct) or S_in in the g tile
-    // (read back into the state owners' registers)
+    // wait for this CTA's incoming state: S~ in the a tile (direct) or S_in, channel-major, in
+    // the g tile (read back into the state owners' registers)
     auto xchg_wait = [&](bool direct) {
         if (!wait_cluster_phase(&m.mbar_x[1], 0)) m.abort = 1;
-        if (!direct && s_owner) {
+        if (!direct && s_owner) {                    // S_in channel-major [c][j]
             const float *Sin = reinterpret_cast<const float *>(sm + kTG);
 #pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                const float4 v = *reinterpret_cast<const float4 *>(Sin + s_row * kD + 32 * ch + 4 * i);
-                S[4 * i] = v.x; S[4 * i + 1] = v.y; S[4 * i + 2] = v.z; S[4 * i + 3] = v.w;
-            }
+            for (int k = 0; k < 32; ++k) S[k] = Sin[(32 * ch + k) * kD + s_row];
         }
         __syncthreads();
     };
@@ -810,15 +841,16 @@ __global__ void __launch_bounds__(kThreads, 1) gla_tc_kernel(const Params p) {
         if (mid_xchg) xchg_begin();
         build_qk();
         operands_ready();
-        // score products, issued by warp 7; meanwhile warps 4..6 and 3 (after its share of
-        // the scan) compute SiLU(g) * w for their TMEM lane quarters and warps 0..3 scan
+        // score products, issued by warp 7; meanwhile the scanning warps store the segment
+        // states and warps 4..6 and 3 (after its share of the scan) compute SiLU(g) * w for
+        // their TMEM lane quarters
         if (warp == 7 && ptx::elect_one()) {
             ptx::tc_fence_after_sync();
             if (!m.slow) issue_qk(sbase, tmem, min(kC, (n + 15) & ~15));
             ptx::mma_commit(&m.mbar_mma[1]);
         }
         if (mid_xchg) xchg_scan(true);
-        if (warp == 3 || (warp >= 4 && warp < 7)) prep_sg();
+        if (warp == 3 || (warp >= 4 && warp < 7)) prep_sg(0, 8);
         wait_mma(1);
         if (m.slow) make_p_exact(sm, t, ch, n, p.scale, &m.range_err);
         else make_p_fast(n);
@@ -951,7 +983,10 @@ gla_tc_selftest_kernel(int kind, const float *A, const float *Bm, float *Dout) {
         put_f16(kTV, t, Bm + t * 64);
     } else {
         put_split_tmem(A + t * 64, false);
-        if (t < 64) put_tf32(kTA, kAtom64, t, Bm + t * 64);
+        if (t < 64) {                                  // B row j = t, MN-major (S~ layout)
+            for (int c = 0; c < 64; ++c)
+                *reinterpret_cast<float *>(sm + kTA + off_stilde(c, t)) = ptx::to_tf32(Bm[t * 64 + c]);
+        }
     }
     ptx::fence_proxy_async_smem();
     ptx::tc_fence_before_sync();
