@@ -241,6 +241,35 @@ def run_reference(args, ws, rank):
     print(json.dumps(line), flush=True)
 
 
+def launch_floor_us(gla, wl, stream, launches: int):
+    """Per-launch time of the do-nothing kernel launched with gla_fwd's exact shape for this
+    workload (cluster, block, shared memory, programmatic dependent launch), replayed from a
+    CUDA graph like the timed steps: the floor no work inside the kernel can remove.  None
+    when the workload does not use the tensor-core kernel."""
+    import torch
+    try:
+        gla.empty_launch(wl.B, wl.H, wl.grid_h, wl.grid_w, stream=stream)
+    except gla.GLAError:
+        return None
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(stream):
+        with torch.cuda.graph(g, stream=stream):
+            for _ in range(launches):
+                gla.empty_launch(wl.B, wl.H, wl.grid_h, wl.grid_w, stream=stream)
+        g.replay()
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    reps = 5
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        for _ in range(reps):
+            g.replay()
+        e1.record(stream)
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1) * 1e3 / (reps * launches)
+
+
 def run_ours(args, ws, rank, local):
     import numpy as np
     import torch
@@ -359,6 +388,10 @@ def run_ours(args, ws, rank, local):
            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
            "steps": e2e_steps, "ms_per_step": e2e_ms / e2e_steps}
 
+    floor_us = launch_floor_us(gla, wl, stream, G * launches_per_step)
+    if gla.get_status(stream) != 0:
+        raise RuntimeError("device status set by the launch-floor measurement")
+
     if rank != 0:
         return
     clocks = clk.summary()
@@ -386,7 +419,9 @@ def run_ours(args, ws, rank, local):
                      "peak_source": "%s (MEASURED_PEAKS.json hbm_gbs)" % peak_kind
                      if peak_kind == "measured" else "fallback 6.65 TB/s",
                      "bytes_per_launch": bytes_per_launch,
-                     "launch_us": launch_s * 1e6},
+                     "launch_us": launch_s * 1e6,
+                     "launch_floor_us": floor_us,
+                     "launch_floor": "do-nothing kernel, same launch shape, same graph replay"},
         "e2e": e2e,
         "gpu_launches": K * launches_per_step,
         "clocks": clocks,

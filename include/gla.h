@@ -145,6 +145,16 @@ int gla_plan(int B, int H, int grid_h, int grid_w, int d_k, int d_v, int dtype, 
              int *segments, int *seg_len, int *ctas, int *max_active_clusters);
 
 /*
+ * gla_empty_launch -- measurement aid: launches a kernel with exactly the launch shape
+ * gla_fwd uses for fp16 d_k = d_v = 64 at these dimensions (grid, thread-block cluster,
+ * block size, dynamic shared memory, programmatic dependent launch) whose body only
+ * performs the dependent-launch handshake.  Timing a run of these gives the per-launch
+ * floor of that shape.  Asynchronous on `stream`.  GLA_ERR_SHAPE for non-positive
+ * dimensions; GLA_ERR_UNSUPPORTED when those dimensions would not use the tensor-core kernel.
+ */
+int gla_empty_launch(int B, int H, int grid_h, int grid_w, void *stream);
+
+/*
  * gla_selftest_timeout -- diagnostic for device-side failure detection: launches a
  * one-thread kernel that waits, with the kernels' bounded-wait loop but a bound of
  * `limit_cycles` SM clocks (1 .. 2^34), on a barrier nothing ever signals.  The wait

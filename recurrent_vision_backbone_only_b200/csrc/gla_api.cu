@@ -514,6 +514,31 @@ int gla_plan(int B, int H, int grid_h, int grid_w, int d_k, int d_v, int dtype, 
     return GLA_OK;
 }
 
+int gla_empty_launch(int B, int H, int grid_h, int grid_w, void *stream) {
+    if (B <= 0 || H <= 0 || grid_h <= 0 || grid_w <= 0) return GLA_ERR_SHAPE;
+    int kernel = 0, segs = 0, seg_len = 0, ctas = 0, active = 0;
+    int rc = gla_plan(B, H, grid_h, grid_w, 64, 64, 0, &kernel, &segs, &seg_len, &ctas, &active);
+    if (rc != GLA_OK) return rc;
+    if (kernel != 1) return GLA_ERR_UNSUPPORTED;
+    auto kern = tc::gla_empty_kernel;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tc::kSmemBytes) !=
+            cudaSuccess ||
+        cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) != cudaSuccess) {
+        cudaGetLastError();
+        return GLA_ERR_CUDA;
+    }
+    Plan pl;
+    pl.segs = segs;
+    pl.smem = tc::kSmemBytes;
+    pl.pdl = true;
+    configure_launch(pl, B * H, tc::kThreads, static_cast<cudaStream_t>(stream));
+    if (cudaLaunchKernelEx(&pl.cfg, kern) != cudaSuccess) {
+        cudaGetLastError();
+        return GLA_ERR_CUDA;
+    }
+    return GLA_OK;
+}
+
 int gla_selftest_timeout(long long limit_cycles, void *stream) {
     if (limit_cycles <= 0 || limit_cycles > (1LL << 34)) return GLA_ERR_UNSUPPORTED;
     DeviceInfo di;

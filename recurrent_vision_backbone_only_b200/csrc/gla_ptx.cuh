@@ -125,6 +125,11 @@ __device__ __forceinline__ void cp_async_wait_all() {
 __device__ __forceinline__ void cluster_arrive() {
     asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
 }
+// Arrive without release semantics: for a start-up barrier whose only payload is mbarrier
+// initialisation already published by fence.mbarrier_init.release.cluster.
+__device__ __forceinline__ void cluster_arrive_relaxed() {
+    asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
+}
 __device__ __forceinline__ void cluster_wait() {
     asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
 }

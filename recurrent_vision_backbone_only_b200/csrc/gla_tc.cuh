@@ -241,7 +241,7 @@ __device__ __forceinline__ uint32_t pack_half2(float lo, float hi) {
 
 // Shared scratch scalars.
 struct Misc {
-    uint64_t mbar_mma[3];     // [0] state, [1] scores, [2] P.V and inter
+    uint64_t mbar_mma[4];     // [0] state, [1] scores, [2] inter (+ P.V), [3] P.V (one chunk)
     uint64_t mbar_ld[3];      // [0] a tile, [1] q and k tiles, [2] v and g tiles
     uint64_t mbar_x[2];       // exchange: [0] aggregates received, [1] S~ / S_in received
     uint32_t tmem_base;
@@ -326,7 +326,7 @@ __global__ void __launch_bounds__(kThreads, 1) gla_tc_kernel(const Params p) {
     ptx::pdl_launch_dependents();
     // ---- setup: barriers and weight; TMEM is allocated once the first gathers are in flight
     if (tid == 0) {
-        for (int i = 0; i < 3; ++i) ptx::mbar_init(&m.mbar_mma[i], 1);
+        for (int i = 0; i < 4; ++i) ptx::mbar_init(&m.mbar_mma[i], 1);
         for (int i = 0; i < 3; ++i) ptx::mbar_init(&m.mbar_ld[i], kThreads);
         ptx::fence_mbarrier_init();
         m.abort = 0;
@@ -345,8 +345,10 @@ __global__ void __launch_bounds__(kThreads, 1) gla_tc_kernel(const Params p) {
             ptx::mbar_arrive_expect_tx(&m.mbar_x[0], (uint32_t)(my_groups * p.segs * kGroupRows * 16));
             ptx::mbar_arrive_expect_tx(&m.mbar_x[1], (uint32_t)(kD * kD * 4));
         }
-        __syncthreads();
-        ptx::cluster_arrive();        // start-up barrier: waited on under the first gathers
+        // start-up barrier, waited on under the first gathers: its payload is the exchange
+        // barriers' initialisation, published by thread 0's fence.mbarrier_init (thread 0
+        // arrives after it), so the arrive itself needs no release
+        ptx::cluster_arrive_relaxed();
     }
     ptx::pdl_wait_prior_grid();
     // RMSNorm weight: async copy, covered by the first chunk's v/g load group
@@ -354,7 +356,7 @@ __global__ void __launch_bounds__(kThreads, 1) gla_tc_kernel(const Params p) {
     __syncthreads();
     uint32_t tmem = 0, tmem_warp = 0;
     uint32_t it = 0;                  // chunk iterations so far (load-barrier parity)
-    uint32_t ph_mma[3] = {0, 0, 0};
+    uint32_t ph_mma[4] = {0, 0, 0, 0};
 
     // State rows owned by lanes < 16: state column j = 16*w4 + lane (a row of the transposed
     // state), channels c in [32*ch, 32*ch + 32).
@@ -768,11 +770,11 @@ __global__ void __launch_bounds__(kThreads, 1) gla_tc_kernel(const Params p) {
             }
         }
     };
-    // wait for this CTA's incoming state: S~ in the a tile (direct) or S_in, channel-major, in
-    // the g tile (read back into the state owners' registers)
-    auto xchg_wait = [&](bool direct) {
+    // wait for this CTA's incoming state S_in (channel-major, g tile) before a multi-chunk pass
+    // and read it back into the state owners' registers
+    auto xchg_wait_sin = [&]() {
         if (!wait_cluster_phase(&m.mbar_x[1], 0)) m.abort = 1;
-        if (!direct && s_owner) {                    // S_in channel-major [c][j]
+        if (s_owner) {
             const float *Sin = reinterpret_cast<const float *>(sm + kTG);
 #pragma unroll
             for (int k = 0; k < 32; ++k) S[k] = Sin[(32 * ch + k) * kD + s_row];
@@ -791,7 +793,7 @@ __global__ void __launch_bounds__(kThreads, 1) gla_tc_kernel(const Params p) {
         if (!pass1 && ci == 0 && !resident && exchange) {
             xchg_begin();
             xchg_scan(false);
-            xchg_wait(false);
+            xchg_wait_sin();
         }
         int n;
         {
@@ -855,21 +857,34 @@ __global__ void __launch_bounds__(kThreads, 1) gla_tc_kernel(const Params p) {
         if (m.slow) make_p_exact(sm, t, ch, n, p.scale, &m.range_err);
         else make_p_fast(n);
         operands_ready();
-        if (warp == 0 && ptx::elect_one()) {
-            ptx::tc_fence_after_sync();
-            issue_pv(sbase, m.slow ? kKH : kPB, tmem);
-        }
         if (mid_xchg) {
-            xchg_wait(true);
+            // P.V by warp 0; the inter product by warp 4 as soon as S~ has arrived (its bytes
+            // are counted on mbar_x[1]; the proxy fence orders them before the tensor core reads)
+            if (warp == 0 && ptx::elect_one()) {
+                ptx::tc_fence_after_sync();
+                issue_pv(sbase, m.slow ? kKH : kPB, tmem);
+                ptx::mma_commit(&m.mbar_mma[3]);
+            } else if (warp == 4 && ptx::elect_one()) {
+                if (!wait_cluster_phase(&m.mbar_x[1], 0)) m.abort = 1;
+                ptx::fence_proxy_async_smem();
+                ptx::tc_fence_after_sync();
+                issue_inter(sbase, tmem, false);
+                ptx::mma_commit(&m.mbar_mma[2]);
+            }
+            wait_mma(3);
         } else {
+            if (warp == 0 && ptx::elect_one()) {
+                ptx::tc_fence_after_sync();
+                issue_pv(sbase, m.slow ? kKH : kPB, tmem);
+            }
             write_stilde();                          // S~ from the state entering this chunk,
             if (ci + 1 < n_chunks) fold_sloc(false); // then S = S 2^{B} + Sloc for the next one
-        }
-        operands_ready();
-        if (warp == 0 && ptx::elect_one()) {
-            ptx::tc_fence_after_sync();
-            issue_inter(sbase, tmem, false);
-            ptx::mma_commit(&m.mbar_mma[2]);         // P.V and the inter product
+            operands_ready();
+            if (warp == 0 && ptx::elect_one()) {
+                ptx::tc_fence_after_sync();
+                issue_inter(sbase, tmem, false);
+                ptx::mma_commit(&m.mbar_mma[2]);     // P.V and the inter product
+            }
         }
         wait_mma(2);
         epilogue(n);
@@ -883,6 +898,14 @@ __global__ void __launch_bounds__(kThreads, 1) gla_tc_kernel(const Params p) {
     if (tid == 0 && m.range_err) raise_status(8 /* GLA_ERR_RANGE */);
     ptx::tc_fence_after_sync();
     if (warp == 0 && n_pass1 + n_chunks > 0) ptx::tmem_dealloc(tmem, kTmemCols);
+}
+
+// ------------------------------------------------------------- launch floor
+// Does nothing but the programmatic-dependent-launch handshake of gla_tc_kernel; launched
+// with that kernel's exact shape it measures the per-launch cost no work can remove.
+__global__ void __launch_bounds__(kThreads, 1) gla_empty_kernel() {
+    ptx::pdl_launch_dependents();
+    ptx::pdl_wait_prior_grid();
 }
 
 // ------------------------------------------------------------- timeout self-test

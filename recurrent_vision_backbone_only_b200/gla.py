@@ -56,6 +56,8 @@ def load() -> ctypes.CDLL:
         lib.gla_selftest_mma.argtypes = [i, vp, vp, vp, vp]
         lib.gla_selftest_timeout.argtypes = [ctypes.c_longlong, vp]
         lib.gla_selftest_timeout.restype = ctypes.c_int
+        lib.gla_empty_launch.argtypes = [ctypes.c_int] * 4 + [vp]
+        lib.gla_empty_launch.restype = ctypes.c_int
         ip = ctypes.POINTER(ctypes.c_int)
         lib.gla_plan.argtypes = [i] * 7 + [ip] * 5
         lib.gla_plan.restype = ctypes.c_int
@@ -173,6 +175,12 @@ def plan(B: int, H: int, grid_h: int, grid_w: int, d_k: int = 64, d_v: int = 64,
     kernel, segs, seg_len, ctas, mac = (v.value for v in vals)
     return {"kernel": {1: "tensor-core", 2: "cuda-core"}.get(kernel, kernel), "segments": segs,
             "seg_len": seg_len, "ctas": ctas, "max_active_clusters": mac}
+
+
+def empty_launch(B: int, H: int, grid_h: int, grid_w: int, stream=None):
+    """Launch the do-nothing kernel with gla_fwd's exact launch shape for these dimensions
+    (fp16, d_k = d_v = 64): timing a run of these gives the per-launch floor."""
+    _check(load().gla_empty_launch(B, H, grid_h, grid_w, _stream_ptr(stream)), "gla_empty_launch")
 
 
 def get_status(stream=None) -> int:

@@ -24,6 +24,7 @@ def test_exports_every_declared_symbol(lib):
     names = gla.header_functions()
     assert {"gla_fwd", "gla_fwd_f32", "gla_fwd_ex", "gla_fwd_host", "gla_get_status",
             "gla_status_string", "gla_version", "gla_selftest_mma", "gla_selftest_timeout",
+            "gla_empty_launch",
             "gla_plan"} <= set(names)
     for n in names:
         assert hasattr(lib, n), n
@@ -88,6 +89,8 @@ def test_selftest_rejects_bad_arguments(lib):
 
 
 def test_timeout_selftest_rejects_bad_bound(lib):
+    assert lib.gla_empty_launch(0, 6, 40, 40, None) == 2     # GLA_ERR_SHAPE, before any device call
+    assert lib.gla_empty_launch(1, 6, 40, -1, None) == 2
     assert lib.gla_selftest_timeout(0, None) == 3
     assert lib.gla_selftest_timeout(1 << 40, None) == 3
 
