@@ -87,13 +87,14 @@ def measured_peaks():
         return FALLBACK_HBM_GBS, "fallback"
 
 
-def profile_traffic():
-    """dram bytes per launch from the committed ncu summary, if it matches this kernel build."""
+def profile_traffic(workload: str):
+    """dram bytes per launch from the committed ncu summary, if it was taken on this workload
+    and this kernel build."""
     try:
         with open(PROFILE_TRAFFIC) as f:
             d = json.load(f)
         from recurrent_vision_backbone_only_b200 import build as _b
-        if d.get("workload") != WORKLOAD or d.get("lib_sources_digest") != _b.sources_digest():
+        if d.get("workload") != workload or d.get("lib_sources_digest") != _b.sources_digest():
             return None
         return d.get("dram_bytes_per_launch")
     except Exception:
@@ -388,7 +389,8 @@ def run_ours(args, ws, rank, local):
            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
            "steps": e2e_steps, "ms_per_step": e2e_ms / e2e_steps}
 
-    floor_us = launch_floor_us(gla, wl, stream, G * launches_per_step)
+    tc_shape = wl.dtype == "f16" and wl.d_k == 64 and wl.d_v == 64
+    floor_us = launch_floor_us(gla, wl, stream, G * launches_per_step) if tc_shape else None
     if gla.get_status(stream) != 0:
         raise RuntimeError("device status set by the launch-floor measurement")
 
@@ -415,7 +417,7 @@ def run_ours(args, ws, rank, local):
             "schedule": gla.plan(wl.B, wl.H, gh, gw, wl.d_k, wl.d_v, 0 if wl.dtype == "f16" else 1),
         },
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-                     "frac": achieved / peak, "traffic": profile_traffic(),
+                     "frac": achieved / peak, "traffic": profile_traffic(wl.name),
                      "peak_source": "%s (MEASURED_PEAKS.json hbm_gbs)" % peak_kind
                      if peak_kind == "measured" else "fallback 6.65 TB/s",
                      "bytes_per_launch": bytes_per_launch,
