@@ -210,3 +210,26 @@ def test_segment_counts_beyond_the_exchange_buffer_are_refused(segs):
     with pytest.raises(gla.GLAError):
         gla.gla_fwd_ex(t["q"], t["k"], t["v"], t["a"], t["g"], t["w"], out, 16, 16, 0,
                        chunk=128, segments=segs)
+
+
+@pytest.mark.parametrize("segs,chunk", [(3, 128), (16, 128), (5, 32)])
+def test_extreme_gates_with_exchange(segs, chunk):
+    # gates of -30 make a chunk's decay range exceed what the tf32 score operands carry, so
+    # P is evaluated exactly on CUDA cores; combined here with the cluster state exchange
+    # (one chunk per segment: mid-chunk exchange; chunk 32: state-only pass first)
+    wl = synth.WORKLOADS["gtr640"].with_(grid_h=16, grid_w=20, H=2)
+    x = synth.make_inputs(wl, seed=7)
+    rng = np.random.default_rng(7)
+    x["a"] = np.where(rng.random(x["a"].shape) < 0.5, -30.0, 30.0).astype(x["a"].dtype)
+    for d in (1, 3):
+        assert_close(run_gpu(x, 16, 20, d, chunk=chunk, segments=segs), oracle_ref(x, 16, 20, d),
+                     "f16")
+
+
+def test_empty_launch_runs_clean():
+    import torch
+    gla.empty_launch(1, 6, 40, 40)
+    gla.empty_launch(16, 12, 40, 40)
+    torch.cuda.synchronize()
+    assert gla.get_status() == 0
+    assert gla.raw_call("gla_empty_launch", 0, 1, 1, 1, None) == 2      # GLA_ERR_SHAPE
