@@ -248,7 +248,8 @@ struct Misc {
     int slow;                 // chunk uses the exact CUDA-core score path
     int range_err;            // a P entry overflowed fp16
     int abort;                // a bounded wait expired
-    int rows[kC];             // token row index (b*L + s)*H + h of each chunk row
+    int rows[2][kC];          // token row index (b*L + s)*H + h of each chunk row (this chunk
+                              // and, gathered early, the next one)
     alignas(16) float bref[kD];   // reference r_c (log2 units)
     alignas(16) float eref[kD];   // 2^{r_c}
     alignas(16) float Bc[kD];     // B_c = b_{n-1,c} (log2)
@@ -371,19 +372,19 @@ __global__ void __launch_bounds__(kThreads, 1) gla_tc_kernel(const Params p) {
         if (!wait_phase(bar, parity)) m.abort = 1;
     };
     // ------------------------------------------------------------ loads
-    auto set_rows = [&](int c0, int n) {
-        if (tid < n) m.rows[tid] = (bb * p.L + spatial_of(dir, c0 + tid, p.gh, p.gw)) * p.H + hh;
+    auto set_rows = [&](int c0, int n, int rb) {
+        if (tid < n) m.rows[rb][tid] = (bb * p.L + spatial_of(dir, c0 + tid, p.gh, p.gw)) * p.H + hh;
     };
     // issue the chunk's gathers (fp16 [n rows][64] tiles, rows >= n zero-filled) into the
     // swizzled layout; completion is tracked per group on mbar_ld[0..2]
-    auto issue_loads = [&](int n, bool full) {
+    auto issue_loads = [&](int n, bool full, int rb) {
         size_t goff[4];
         uint32_t soff[4], bytes[4];
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
             const int row = (tid >> 3) + 32 * i, j = tid & 7;
             const bool ok = row < n;
-            goff[i] = ok ? (size_t)m.rows[row] * kD + j * 8 : 0;
+            goff[i] = ok ? (size_t)m.rows[rb][row] * kD + j * 8 : 0;
             soff[i] = sbase + off_f16(row, j);
             bytes[i] = ok ? 16u : 0u;
         }
@@ -642,7 +643,7 @@ __global__ void __launch_bounds__(kThreads, 1) gla_tc_kernel(const Params p) {
     // u = (O_inter + O_intra) / rms * SiLU(g) * w.  Row t, 32 channels per thread, staged as
     // fp16 rows in the K~ low-part region (free once the score products completed), then
     // stored with each group of 8 threads writing one whole 128-byte token row.
-    auto epilogue = [&](int n) {
+    auto epilogue = [&](int n, int rb) {
         float o[32], op[32];
         ptx::tmem_ld32(tmem_warp + kColO + 32 * ch, o);
         ptx::tmem_ld32(tmem_warp + kColOP + 32 * ch, op);
@@ -672,7 +673,7 @@ __global__ void __launch_bounds__(kThreads, 1) gla_tc_kernel(const Params p) {
         for (int i = 0; i < 4; ++i) {
             const int row = (tid >> 3) + 32 * i, j = tid & 7;
             if (row < n)
-                *reinterpret_cast<uint4 *>(p.out + (size_t)m.rows[row] * kD + 8 * j) =
+                *reinterpret_cast<uint4 *>(p.out + (size_t)m.rows[rb][row] * kD + 8 * j) =
                     *reinterpret_cast<const uint4 *>(sm + kKL + off_f16(row, j));
         }
     };
@@ -787,6 +788,21 @@ __global__ void __launch_bounds__(kThreads, 1) gla_tc_kernel(const Params p) {
     // last), then the exchange, then the full pass; a resident segment (one chunk) runs the
     // full pass once and exchanges mid-chunk.  Every CTA exchanges exactly once.
     const int n_pass1 = (!resident && exchange && rank < p.segs - 1) ? n_chunks : 0;
+    // Within a pass, the next chunk's gathers are issued as soon as this chunk's tiles are
+    // free (after the state product in the state-only pass, after the last products in the
+    // full pass), into the other row-index buffer; never across the exchange, which writes
+    // S_in into the g tile.
+    int rb = 0;                        // row-index buffer of the current chunk
+    bool preloaded = false;            // its gathers were issued during the previous chunk
+    auto preload_next = [&](int ci, bool full) {
+        if (ci + 1 >= n_chunks) return;
+        const int c1 = p0 + (ci + 1) * chunk_len;
+        const int n1 = min(chunk_len, p1 - c1);
+        set_rows(c1, n1, rb ^ 1);
+        __syncthreads();
+        issue_loads(n1, full, rb ^ 1);
+        preloaded = true;
+    };
     for (int step = 0; step < n_pass1 + n_chunks; ++step) {
         const bool pass1 = step < n_pass1;
         const int ci = pass1 ? step : step - n_pass1;
@@ -799,12 +815,15 @@ __global__ void __launch_bounds__(kThreads, 1) gla_tc_kernel(const Params p) {
         {
             const int c0 = p0 + ci * chunk_len;
             n = min(chunk_len, p1 - c0);
-            __syncthreads();
-            set_rows(c0, n);
-            if (tid == 0) m.slow = 0;
-            __syncthreads();
+            if (!preloaded) {
+                __syncthreads();
+                set_rows(c0, n, rb);
+                __syncthreads();
+                issue_loads(n, !pass1, rb);
+            }
+            preloaded = false;
+            if (tid == 0) m.slow = 0;               // read only after the gate's barriers
         }
-        issue_loads(n, !pass1);
         if (step == 0 && warp == 0) {                // overlaps the first gathers' latency
             ptx::tmem_alloc(&m.tmem_base, kTmemCols);
             ptx::tmem_relinquish();
@@ -830,12 +849,14 @@ __global__ void __launch_bounds__(kThreads, 1) gla_tc_kernel(const Params p) {
         }
         wait_mma(0);
         const bool mid_xchg = !pass1 && resident && exchange;
+        if (pass1) preload_next(ci, false);          // a, k, v consumed
         read_sloc();
         if (pass1 || mid_xchg) fold_sloc(true);     // S = S 2^{B} + Sloc, Gs += B
         if (pass1) {
             ptx::tc_fence_before_sync();
             __syncthreads();
             ++it;
+            rb ^= preloaded ? 1 : 0;
             continue;
         }
         // publish the segment aggregate now: the exchange runs under the score operands and
@@ -844,15 +865,20 @@ __global__ void __launch_bounds__(kThreads, 1) gla_tc_kernel(const Params p) {
         build_qk();
         operands_ready();
         // score products, issued by warp 7; meanwhile the scanning warps store the segment
-        // states and warps 4..6 and 3 (after its share of the scan) compute SiLU(g) * w for
-        // their TMEM lane quarters
+        // states and the other warps compute SiLU(g) * w for their TMEM lane quarters
         if (warp == 7 && ptx::elect_one()) {
             ptx::tc_fence_after_sync();
             if (!m.slow) issue_qk(sbase, tmem, min(kC, (n + 15) & ~15));
             ptx::mma_commit(&m.mbar_mma[1]);
         }
-        if (mid_xchg) xchg_scan(true);
-        if (warp == 3 || (warp >= 4 && warp < 7)) prep_sg(0, 8);
+        if (mid_xchg) {
+            xchg_scan(true);
+            if (warp == 3 || (warp >= 4 && warp < 7)) prep_sg(0, 8);
+        } else if (warp == 3) {                      // no scan: each warp its own channel
+            prep_sg(0, 8);                           // half, warp 3 also the issuing warp's
+        } else if (warp != 7) {
+            prep_sg(4 * ch, 4 * ch + 4);
+        }
         wait_mma(1);
         if (m.slow) make_p_exact(sm, t, ch, n, p.scale, &m.range_err);
         else make_p_fast(n);
@@ -887,10 +913,12 @@ __global__ void __launch_bounds__(kThreads, 1) gla_tc_kernel(const Params p) {
             }
         }
         wait_mma(2);
-        epilogue(n);
+        preload_next(ci, true);                      // every tile consumed (all products done)
+        epilogue(n, rb);
         ptx::tc_fence_before_sync();
         __syncthreads();
         ++it;
+        rb ^= preloaded ? 1 : 0;
     }
 
     // ---- teardown ----
