@@ -69,31 +69,13 @@ __device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t *bar, uint32_t pa
     return ok != 0;
 }
 
-// Asynchronous store into another CTA's shared memory (cluster address); completion is
-// counted in bytes on the destination CTA's mbarrier (also a cluster address).
-__device__ __forceinline__ void st_async_v2(uint32_t addr, float2 v, uint32_t bar) {
-    asm volatile(
-        "st.async.shared::cluster.mbarrier::complete_tx::bytes.v2.f32 [%0], {%1, %2}, [%3];" ::"r"(
-            addr),
-        "f"(v.x), "f"(v.y), "r"(bar)
-        : "memory");
-}
+// 16-byte store into another CTA's shared memory (`addr` from mapa) whose completion counts
+// 16 bytes on that CTA's mbarrier `bar` (also a mapa address).
 __device__ __forceinline__ void st_async_v4(uint32_t addr, float4 v, uint32_t bar) {
     asm volatile(
         "st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.f32 [%0], {%1, %2, %3, %4}, "
         "[%5];" ::"r"(addr),
         "f"(v.x), "f"(v.y), "f"(v.z), "f"(v.w), "r"(bar)
-        : "memory");
-}
-
-// Bulk copy of `bytes` (multiple of 16, 16-byte aligned) from this CTA's shared memory to
-// another CTA's (cluster address), completion counted on the destination's mbarrier.
-__device__ __forceinline__ void bulk_to_cluster(uint32_t dst, uint32_t src, uint32_t bytes,
-                                                uint32_t bar) {
-    asm volatile(
-        "cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, "
-        "[%3];" ::"r"(dst),
-        "r"(src), "r"(bytes), "r"(bar)
         : "memory");
 }
 
@@ -112,24 +94,13 @@ __device__ __forceinline__ void cp_async16(uint32_t dst, const void *src, uint32
                  : "memory");
 }
 
-__device__ __forceinline__ void cp_async_commit() {
-    asm volatile("cp.async.commit_group;" ::: "memory");
-}
-
-__device__ __forceinline__ void cp_async_wait_all() {
-    asm volatile("cp.async.wait_group 0;" ::: "memory");
-}
-
 // ------------------------------------------------------------------- cluster
-// Split cluster barrier: arrive (release this CTA's prior writes) / wait (acquire).
-__device__ __forceinline__ void cluster_arrive() {
-    asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
-}
-// Arrive without release semantics: for a start-up barrier whose only payload is mbarrier
+// Split cluster barrier.  Arrive without release semantics: for a start-up barrier whose only payload is mbarrier
 // initialisation already published by fence.mbarrier_init.release.cluster.
 __device__ __forceinline__ void cluster_arrive_relaxed() {
     asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
 }
+// Wait for every thread of the cluster to have arrived (acquire).
 __device__ __forceinline__ void cluster_wait() {
     asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
@@ -142,12 +113,6 @@ __device__ __forceinline__ void pdl_wait_prior_grid() {
     asm volatile("griddepcontrol.wait;" ::: "memory");
 }
 
-// Named barrier `id` over `count` threads (whole warps).
-__device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t count) {
-    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
-}
-
-// Address of the same shared-memory location in CTA `rank` of the cluster.
 // One lane of the (converged) warp is elected; used to issue single-thread tensor-core work
 // from a warp-uniform branch.
 __device__ __forceinline__ bool elect_one() {
@@ -159,31 +124,11 @@ __device__ __forceinline__ bool elect_one() {
         : "=r"(pred));
     return pred != 0;
 }
+// Address of the same shared-memory location in CTA `rank` of the cluster.
 __device__ __forceinline__ uint32_t mapa(uint32_t saddr, uint32_t rank) {
     uint32_t r;
     asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr), "r"(rank));
     return r;
-}
-__device__ __forceinline__ float2 ld_cluster_v2(uint32_t addr) {
-    float2 v;
-    asm volatile("ld.shared::cluster.v2.f32 {%0,%1}, [%2];" : "=f"(v.x), "=f"(v.y) : "r"(addr) : "memory");
-    return v;
-}
-__device__ __forceinline__ void st_cluster_v2(uint32_t addr, float2 v) {
-    asm volatile("st.shared::cluster.v2.f32 [%0], {%1,%2};" ::"r"(addr), "f"(v.x), "f"(v.y) : "memory");
-}
-__device__ __forceinline__ float4 ld_cluster_v4(uint32_t addr) {
-    float4 v;
-    asm volatile("ld.shared::cluster.v4.f32 {%0,%1,%2,%3}, [%4];"
-                 : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
-                 : "r"(addr)
-                 : "memory");
-    return v;
-}
-__device__ __forceinline__ void st_cluster_v4(uint32_t addr, float4 v) {
-    asm volatile("st.shared::cluster.v4.f32 [%0], {%1,%2,%3,%4};" ::"r"(addr), "f"(v.x), "f"(v.y),
-                 "f"(v.z), "f"(v.w)
-                 : "memory");
 }
 
 // --------------------------------------------------------------------- fences
@@ -230,15 +175,6 @@ __device__ __forceinline__ void mma_f16_ss(uint32_t d_tmem, uint64_t a_desc, uin
         : "memory");
 }
 
-__device__ __forceinline__ void mma_tf32_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
-                                            uint32_t idesc, bool accumulate) {
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::tf32 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"((uint32_t)accumulate)
-        : "memory");
-}
 
 // D[tmem] (+)= A[tmem] * B[smem] (A: M lanes x K columns of 32-bit tf32).
 __device__ __forceinline__ void mma_tf32_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
