@@ -113,6 +113,11 @@ __device__ __forceinline__ void pdl_wait_prior_grid() {
     asm volatile("griddepcontrol.wait;" ::: "memory");
 }
 
+// Named barrier `id` (1..15) over `count` threads (a multiple of 32).
+__device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t count) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+
 // One lane of the (converged) warp is elected; used to issue single-thread tensor-core work
 // from a warp-uniform branch.
 __device__ __forceinline__ bool elect_one() {

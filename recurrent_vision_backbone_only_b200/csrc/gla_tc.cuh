@@ -259,7 +259,6 @@ struct Misc {
     alignas(16) float b0[kD];     // b_{0,c}
     alignas(16) float w[kD];      // RMSNorm weight
     alignas(16) float tot[8][kD]; // per-16-row totals of the gate scan
-    alignas(16) float eGrow[kD];    // 2^{Gs} of this segment (sent to every CTA)
     alignas(16) float red[2][kC]; // epilogue partial sums of squares (per channel half)
     alignas(16) float dqp[2][kC]; // diagonal score q_t . k_t, per channel half
 };
@@ -642,7 +641,8 @@ __global__ void __launch_bounds__(kThreads, 1) gla_tc_kernel(const Params p) {
     };
     // u = (O_inter + O_intra) / rms * SiLU(g) * w.  Row t, 32 channels per thread, staged as
     // fp16 rows in the K~ low-part region (free once the score products completed), then
-    // stored with each group of 8 threads writing one whole 128-byte token row.
+    // stored with each group of 8 threads writing one whole 128-byte token row.  A row's two
+    // halves live in warps w4 and w4 + 4, which synchronise on named barrier 1 + w4 only.
     auto epilogue = [&](int n, int rb) {
         float o[32], op[32];
         ptx::tmem_ld32(tmem_warp + kColO + 32 * ch, o);
@@ -656,7 +656,7 @@ __global__ void __launch_bounds__(kThreads, 1) gla_tc_kernel(const Params p) {
         m.red[ch][t] = ss;
         ptx::tmem_ld32(tmem_warp + kColSG + 32 * ch, op);
         ptx::tmem_ld_wait();
-        __syncthreads();
+        ptx::named_bar_sync(1 + w4, 64);
         const float inv = rsqrtf((m.red[0][t] + m.red[1][t]) * (1.0f / 64.0f) + p.eps);
 #pragma unroll
         for (int jj = 0; jj < 4; ++jj) {
@@ -668,10 +668,11 @@ __global__ void __launch_bounds__(kThreads, 1) gla_tc_kernel(const Params p) {
             pk.z = pack_half2(u[4], u[5]); pk.w = pack_half2(u[6], u[7]);
             *reinterpret_cast<uint4 *>(sm + kKL + off_f16(t, 4 * ch + jj)) = pk;
         }
-        __syncthreads();
+        ptx::named_bar_sync(1 + w4, 64);
+        const int pt = (ch << 5) | lane;                // 0..63 within the warp pair
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-            const int row = (tid >> 3) + 32 * i, j = tid & 7;
+            const int row = 32 * w4 + (pt >> 3) + 8 * i, j = pt & 7;
             if (row < n)
                 *reinterpret_cast<uint4 *>(p.out + (size_t)m.rows[rb][row] * kD + 8 * j) =
                     *reinterpret_cast<const uint4 *>(sm + kKL + off_f16(row, j));
@@ -714,22 +715,34 @@ __global__ void __launch_bounds__(kThreads, 1) gla_tc_kernel(const Params p) {
     };
     auto xchg_begin = [&]() {
         cluster_ready_once();
-        if (tid < kD) m.eGrow[tid] = ptx::ex2(m.Gs[tid]);
-        __syncthreads();                              // 2^G row complete
-        if (s_owner) {
+        // each state row is held by lanes 0..15 (32 channels per warp); lanes 16..31 take the
+        // upper 16 channels of lane - 16's row so every store instruction uses the whole warp
+        float hi[16];
 #pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                const int g = 8 * ch + i, dst = g % p.segs;
-                ptx::st_async_v4(ptx::mapa(sbase + recv_off(g / p.segs, rank, recv_slot(s_row)), dst),
-                                 make_float4(S[4 * i], S[4 * i + 1], S[4 * i + 2], S[4 * i + 3]),
-                                 ptx::mapa(ptx::smem_u32(&m.mbar_x[0]), dst));
-            }
+        for (int k = 0; k < 16; ++k) hi[k] = __shfl_sync(0xffffffffu, S[16 + k], lane & 15);
+        const int row = w4 * 16 + (lane & 15), i0 = lane < 16 ? 0 : 4;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const int g = 8 * ch + i0 + i, dst = g % p.segs;
+            const float4 v = lane < 16 ? make_float4(S[4 * i], S[4 * i + 1], S[4 * i + 2], S[4 * i + 3])
+                                       : make_float4(hi[4 * i], hi[4 * i + 1], hi[4 * i + 2], hi[4 * i + 3]);
+            ptx::st_async_v4(ptx::mapa(sbase + recv_off(g / p.segs, rank, recv_slot(row)), dst), v,
+                             ptx::mapa(ptx::smem_u32(&m.mbar_x[0]), dst));
         }
+        // the group pieces of 2^{G} and 2^{r}.  G of a one-chunk segment is its B (the gate's
+        // row, barrier-separated from here); of a longer segment the sum over its state-only
+        // pass, complete since that pass's last barrier
         if (tid < 32) {
-            const int g = tid & 15, which = tid >> 4, dst = g % p.segs;
-            const float *src = which ? m.eref : m.eGrow;
-            ptx::st_async_v4(ptx::mapa(sbase + recv_off(g / p.segs, rank, kD + which), dst),
-                             *reinterpret_cast<const float4 *>(src + 4 * g),
+            const int g = tid & 15, dst = g % p.segs;
+            float4 v;
+            if (tid < 16) {
+                const float *gs = resident ? m.Bc : m.Gs;
+                v = make_float4(ptx::ex2(gs[4 * g]), ptx::ex2(gs[4 * g + 1]), ptx::ex2(gs[4 * g + 2]),
+                                ptx::ex2(gs[4 * g + 3]));
+            } else {
+                v = *reinterpret_cast<const float4 *>(m.eref + 4 * g);
+            }
+            ptx::st_async_v4(ptx::mapa(sbase + recv_off(g / p.segs, rank, kD + (tid >> 4)), dst), v,
                              ptx::mapa(ptx::smem_u32(&m.mbar_x[0]), dst));
         }
     };
