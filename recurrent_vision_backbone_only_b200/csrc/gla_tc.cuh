@@ -19,7 +19,8 @@
 //                    (tcgen05 kind::tf32, A operands Qh/Ql in TMEM, 128x128x64)
 //   masked   P     = d_k^{-1/2} A (.) [s <= t], diagonal A_tt = q_t . k_t in fp32
 //                    (d_k^{-1/2} = 2^-3 is folded into Q~'s exponent)
-//   output   O     = P V + (Qh + Ql) Diag(e^{r}) S_in   (f16 + tf32 MMAs)
+//   output   O     = P V + (Qh + Ql) S~,  S~ = tf32(Diag(e^{r}) S_in)  (f16 + tf32
+//                    MMAs; S~ is an MN-major operand)
 //   state    S_out = Diag(e^{B}) S_in + Ks^T V       (tcgen05 kind::f16, 64x64x128)
 // Every exponent in Ks, e^{r}, e^{B} is <= 0.  Q~ and K~ carry exponents of
 // either sign bounded by the chunk's decay range about r; they are kept in
@@ -34,26 +35,23 @@
 // Schedule.  A (b, h) scan is cut into `segs` contiguous segments, one CTA
 // each, one thread-block cluster per pair.  Segment aggregates
 // (G = total log-decay, S from a zero start) are combined across the
-// cluster through distributed shared memory, each CTA owning a slice of the
-// d_k x d_v state entries (the combine is elementwise per entry), giving
-// every segment its incoming state.  A segment that fits one chunk keeps its
-// tiles resident and does the exchange mid-chunk; longer segments run a
-// state-only pass, the exchange, then the full pass.
+// cluster through distributed shared memory (the combine is elementwise per
+// state entry with the decay of its key channel, so CTA r scans the 4-channel
+// key groups g = r, r + segs, ...), giving every segment its incoming state.
+// A segment that fits one chunk keeps its tiles resident and does the
+// exchange mid-chunk; longer segments run a state-only pass, the exchange,
+// then the full pass, gathering each next chunk under the current one.
 //
 // Input gathers: 16-byte cp.async per thread, scan row t of the chunk read
 // from the token's spatial position (direction remap folded into the
 // address), written straight into the 128B-swizzled operand layout.
 #pragma once
 
-#include <cooperative_groups.h>
-
 #include "gla_common.cuh"
 #include "gla_ptx.cuh"
 
 namespace gla {
 namespace tc {
-
-namespace cg = cooperative_groups;
 
 constexpr int kThreads = 256;      // two threads per chunk row (one per channel half)
 constexpr int kSelfThreads = 128;  // self-test kernel: one thread per row
@@ -65,15 +63,15 @@ constexpr float kLog2Scale = -3.0f;   // log2(d_k^{-1/2}) for d_k = 64, folded i
 constexpr float kHalfRangeSafe2 = 86.0f;
 
 // ---- shared memory map (bytes from a 1024-aligned base) ----
-constexpr uint32_t kKL = 0;        // K~ low part  tf32, 2 atoms x [128][128B]
+constexpr uint32_t kKL = 0;        // K~ low part  tf32, 2 atoms x [128][128B]; then u staging
 constexpr uint32_t kKH = 32768;    // K~ high part tf32, 2 atoms x [128][128B] (slow path: P)
 constexpr uint32_t kPB = 65536;    // b   fp32 (QT layout), then P fp16 2 atoms x [128][128B]
 constexpr uint32_t kST = 98304;    // Ks fp16 [128][128B]
 constexpr uint32_t kTQ = 114688;   // raw tiles, fp16 [128][128B] each
 constexpr uint32_t kTK = 131072;
-constexpr uint32_t kTA = 147456;   // a tile; after the gate: S~ tf32 2 x [64][128B]
+constexpr uint32_t kTA = 147456;   // a tile; after the gate: S~ tf32 MN-major, 2 x [64 c][128B]
 constexpr uint32_t kTV = 163840;
-constexpr uint32_t kTG = 180224;
+constexpr uint32_t kTG = 180224;   // g tile; before a multi-chunk pass: S_in [64 c][64 j] fp32
 constexpr uint32_t kMISC = 196608;
 constexpr uint32_t kMiscBytes = 8192;
 constexpr uint32_t kAtom128 = 16384;   // [128 rows][128 B]
