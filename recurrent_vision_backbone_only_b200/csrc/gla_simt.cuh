@@ -54,8 +54,23 @@ __host__ __device__ constexpr size_t simt_smem_floats(int dk, int dv, int C) {
     return (size_t)dk * dv + dk + 3 * (size_t)C * dk + 2 * (size_t)C * dv + (size_t)C * C + C;
 }
 
+// N consecutive floats from shared memory (N = 2, 4 or 8; p aligned to min(N, 4) floats)
+template <int N>
+__device__ __forceinline__ void load_run(const float *p, float *out) {
+    if constexpr (N == 2) {
+        const float2 v = *reinterpret_cast<const float2 *>(p);
+        out[0] = v.x; out[1] = v.y;
+    } else {
+#pragma unroll
+        for (int q = 0; q < N / 4; ++q) {
+            const float4 v = *reinterpret_cast<const float4 *>(p + 4 * q);
+            out[4 * q] = v.x; out[4 * q + 1] = v.y; out[4 * q + 2] = v.z; out[4 * q + 3] = v.w;
+        }
+    }
+}
+
 template <typename T, int DK, int DV>
-__global__ void __launch_bounds__(kSimtThreads)
+__global__ void __launch_bounds__(kSimtThreads, 2)
 gla_simt_kernel(const SimtParams p) {
     constexpr int NT = kSimtThreads;
     constexpr int NW = NT / 32;
@@ -118,14 +133,32 @@ gla_simt_kernel(const SimtParams p) {
     };
 
     // S <- Diag(e^{b_last}) S + sum_s (k_s (.) e^{b_last - b_s})^T v_s ; G += b_last.
-    // ks must already hold k_s (.) e^{b_last - b_s}.
+    // ks must already hold k_s (.) e^{b_last - b_s}.  Register-blocked: a 16 x 16 thread grid,
+    // each thread a (DK/16) x (DV/16) tile of S, so every loaded k and v value feeds a row or
+    // column of FMAs.  Each entry still accumulates in the order S e^{b}, s = 0, 1, ...
     auto fold_state = [&](int n) {
-        for (int e = tid; e < DK * DV; e += NT) {
-            const int c = e / DV, j = e - c * DV;
-            float acc = S[e] * expf(bs[(n - 1) * DK + c]);
-            for (int s = 0; s < n; ++s) acc = fmaf(ks[s * DK + c], vs[s * DV + j], acc);
-            S[e] = acc;
+        constexpr int TC = DK / 16, TJ = DV / 16;
+        const int c0 = (tid >> 4) * TC, j0 = (tid & 15) * TJ;
+        float acc[TC][TJ];
+#pragma unroll
+        for (int a = 0; a < TC; ++a) {
+            const float dec = expf(bs[(n - 1) * DK + c0 + a]);
+#pragma unroll
+            for (int b2 = 0; b2 < TJ; ++b2) acc[a][b2] = S[(c0 + a) * DV + j0 + b2] * dec;
         }
+        for (int s = 0; s < n; ++s) {
+            float kr[TC], vr[TJ];
+            load_run<TC>(ks + s * DK + c0, kr);
+            load_run<TJ>(vs + s * DV + j0, vr);
+#pragma unroll
+            for (int a = 0; a < TC; ++a)
+#pragma unroll
+                for (int b2 = 0; b2 < TJ; ++b2) acc[a][b2] = fmaf(kr[a], vr[b2], acc[a][b2]);
+        }
+#pragma unroll
+        for (int a = 0; a < TC; ++a)
+#pragma unroll
+            for (int b2 = 0; b2 < TJ; ++b2) S[(c0 + a) * DV + j0 + b2] = acc[a][b2];
         for (int c = tid; c < DK; c += NT) G[c] += bs[(n - 1) * DK + c];
     };
 
@@ -189,12 +222,51 @@ gla_simt_kernel(const SimtParams p) {
         for (int idx = tid; idx < n * DK; idx += NT) qs[idx] *= expf(bs[idx]);
         scale_keys(n);
         __syncthreads();
-        for (int idx = tid; idx < n * DV; idx += NT) {
-            const int t = idx / DV, j = idx - t * DV;
-            float acc = 0.0f;
-            for (int s = 0; s <= t; ++s) acc = fmaf(As[t * C + s], vs[s * DV + j], acc);
-            for (int c = 0; c < DK; ++c) acc = fmaf(qs[t * DK + c], S[c * DV + j], acc);
-            Os[idx] = acc * p.scale;
+        // O[t][j] = scale (sum_{s<=t} A[t][s] v_s[j] + sum_c q~_t[c] S[c][j]); register-blocked
+        // over 4 value columns and the tokens t = tg, tg + TS, ... of one thread, so each
+        // loaded S row piece serves every token of the thread; each output still accumulates
+        // in the order s = 0..t, then c = 0..DK-1
+        {
+            constexpr int JG = DV / 4, TS = NT / JG, MT = (64 + TS - 1) / TS;
+            const int j0 = (tid % JG) * 4, tg = tid / JG;
+            float acc[MT][4];
+#pragma unroll
+            for (int i = 0; i < MT; ++i)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) acc[i][e] = 0.0f;
+#pragma unroll
+            for (int i = 0; i < MT; ++i) {
+                const int t = tg + i * TS;
+                if (t < n) {
+                    for (int s = 0; s <= t; ++s) {
+                        const float a_ts = As[t * C + s];
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) acc[i][e] = fmaf(a_ts, vs[s * DV + j0 + e], acc[i][e]);
+                    }
+                }
+            }
+            for (int c = 0; c < DK; ++c) {
+                const float4 sr = *reinterpret_cast<const float4 *>(S + c * DV + j0);
+#pragma unroll
+                for (int i = 0; i < MT; ++i) {
+                    const int t = tg + i * TS;
+                    if (t < n) {
+                        const float qv = qs[t * DK + c];
+                        acc[i][0] = fmaf(qv, sr.x, acc[i][0]);
+                        acc[i][1] = fmaf(qv, sr.y, acc[i][1]);
+                        acc[i][2] = fmaf(qv, sr.z, acc[i][2]);
+                        acc[i][3] = fmaf(qv, sr.w, acc[i][3]);
+                    }
+                }
+            }
+#pragma unroll
+            for (int i = 0; i < MT; ++i) {
+                const int t = tg + i * TS;
+                if (t < n) {
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) Os[t * DV + j0 + e] = acc[i][e] * p.scale;
+                }
+            }
         }
         __syncthreads();
         fold_state(n);
