@@ -50,8 +50,12 @@ struct SimtParams {
 
 constexpr int kSimtThreads = 256;
 
+// q, k and b rows are padded to d_k + 4 floats: 16-byte aligned, and rows of different
+// tokens fall in different shared-memory banks (the score loop reads one channel of 16 rows)
+__host__ __device__ constexpr int simt_row(int dk) { return dk + 4; }
+
 __host__ __device__ constexpr size_t simt_smem_floats(int dk, int dv, int C) {
-    return (size_t)dk * dv + dk + 3 * (size_t)C * dk + 2 * (size_t)C * dv + (size_t)C * C + C;
+    return (size_t)dk * dv + dk + 3 * (size_t)C * simt_row(dk) + 3 * (size_t)C * dv + (size_t)C * C + C;
 }
 
 // N consecutive floats from shared memory (N = 2, 4 or 8; p aligned to min(N, 4) floats)
@@ -78,13 +82,15 @@ gla_simt_kernel(const SimtParams p) {
     extern __shared__ float smem[];
     float *S = smem;             // [DK][DV] running state / aggregate / incoming state
     float *G = S + DK * DV;      // [DK] segment log-decay
-    float *qs = G + DK;          // [C][DK]
-    float *ks = qs + C * DK;     // [C][DK]
-    float *bs = ks + C * DK;     // [C][DK] in-chunk cumulative log-decay
-    float *vs = bs + C * DK;     // [C][DV]
+    constexpr int KP = simt_row(DK);   // padded row of q, k, b
+    float *qs = G + DK;          // [C][KP]
+    float *ks = qs + C * KP;     // [C][KP]
+    float *bs = ks + C * KP;     // [C][KP] in-chunk cumulative log-decay
+    float *vs = bs + C * KP;     // [C][DV]
     float *Os = vs + C * DV;     // [C][DV]
     float *As = Os + C * DV;     // [C][C] decay-weighted scores
-    int *rows = reinterpret_cast<int *>(As + C * C);  // [C] token row index (b*L+s)*H+h
+    float *gsm = As + C * C;     // [C][DV] output-gate pre-activation
+    int *rows = reinterpret_cast<int *>(gsm + C * DV);  // [C] token row index (b*L+s)*H+h
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int pair = blockIdx.x / p.segs;
@@ -105,28 +111,76 @@ gla_simt_kernel(const SimtParams p) {
     for (int c = tid; c < DK; c += NT) G[c] = 0.0f;
 
     // Gather the chunk [c0, c0+n) in scan order; b = inclusive cumsum of lambda.
+    // Inputs move in 16-byte pieces: EPP elements, PK (PV) pieces per key (value) row.  Each
+    // batch of pieces is loaded into registers before any is consumed, so a batch costs one
+    // DRAM round trip (global loads cannot be reordered past the shared-memory stores).
+    constexpr int EPP = 16 / (int)sizeof(T);
+    constexpr int PK = DK / EPP, PV = DV / EPP;
+    auto unpack = [&](const uint4 &r, float *o) {
+        if constexpr (sizeof(T) == 2) {
+            const __half2 *h2 = reinterpret_cast<const __half2 *>(&r);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const float2 f = __half22float2(h2[e]);
+                o[2 * e] = f.x;
+                o[2 * e + 1] = f.y;
+            }
+        } else {
+            const float *f = reinterpret_cast<const float *>(&r);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) o[e] = f[e];
+        }
+    };
+    auto ld16 = [](const T *ptr) { return *reinterpret_cast<const uint4 *>(ptr); };
     auto load_chunk = [&](int c0, int n, bool with_q) {
         __syncthreads();
         for (int t = tid; t < n; t += NT)
             rows[t] = (b * p.L + spatial_of(dir, c0 + t, p.gh, p.gw)) * p.H + h;
         __syncthreads();
-        for (int idx = tid; idx < n * DK; idx += NT) {
-            const int t = idx / DK, c = idx - t * DK;
-            const size_t off = (size_t)rows[t] * DK + c;
-            ks[idx] = to_f32(k[off]);
-            bs[idx] = log_gamma(to_f32(a[off]));
-            if (with_q) qs[idx] = to_f32(q[off]);
+        for (int base = 0; base < n * PK; base += NT) {
+            const int pi = base + tid;
+            if (pi < n * PK) {
+                const int t = pi / PK, pc = pi - t * PK;
+                const size_t off = (size_t)rows[t] * DK + pc * EPP;
+                const uint4 kr = ld16(k + off), ar = ld16(a + off);
+                const uint4 qr = with_q ? ld16(q + off) : make_uint4(0, 0, 0, 0);
+                float kf[EPP], af[EPP], qf[EPP];
+                unpack(kr, kf);
+                unpack(ar, af);
+                unpack(qr, qf);
+                const int o = t * KP + pc * EPP;
+#pragma unroll
+                for (int e = 0; e < EPP; ++e) {
+                    ks[o + e] = kf[e];
+                    bs[o + e] = log_gamma(af[e]);
+                    if (with_q) qs[o + e] = qf[e];
+                }
+            }
         }
-        for (int idx = tid; idx < n * DV; idx += NT) {
-            const int t = idx / DV, j = idx - t * DV;
-            vs[idx] = to_f32(v[(size_t)rows[t] * DV + j]);
+        for (int base = 0; base < n * PV; base += NT) {
+            const int pi = base + tid;
+            if (pi < n * PV) {
+                const int t = pi / PV, pc = pi - t * PV;
+                const size_t off = (size_t)rows[t] * DV + pc * EPP;
+                const uint4 vr = ld16(v + off);
+                const uint4 gr = with_q ? ld16(g + off) : make_uint4(0, 0, 0, 0);
+                float vf[EPP], gf[EPP];
+                unpack(vr, vf);
+                unpack(gr, gf);
+                const int o = t * DV + pc * EPP;
+#pragma unroll
+                for (int e = 0; e < EPP; ++e) {
+                    vs[o + e] = vf[e];
+                    if (with_q) gsm[o + e] = gf[e];
+                }
+            }
         }
         __syncthreads();
         for (int c = tid; c < DK; c += NT) {
             float run = 0.0f;
             for (int t = 0; t < n; ++t) {
-                run += bs[t * DK + c];
-                bs[t * DK + c] = run;
+                run += bs[t * KP + c];
+                bs[t * KP + c] = run;
             }
         }
         __syncthreads();
@@ -142,13 +196,13 @@ gla_simt_kernel(const SimtParams p) {
         float acc[TC][TJ];
 #pragma unroll
         for (int a = 0; a < TC; ++a) {
-            const float dec = expf(bs[(n - 1) * DK + c0 + a]);
+            const float dec = expf(bs[(n - 1) * KP + c0 + a]);
 #pragma unroll
             for (int b2 = 0; b2 < TJ; ++b2) acc[a][b2] = S[(c0 + a) * DV + j0 + b2] * dec;
         }
         for (int s = 0; s < n; ++s) {
             float kr[TC], vr[TJ];
-            load_run<TC>(ks + s * DK + c0, kr);
+            load_run<TC>(ks + s * KP + c0, kr);
             load_run<TJ>(vs + s * DV + j0, vr);
 #pragma unroll
             for (int a = 0; a < TC; ++a)
@@ -159,13 +213,13 @@ gla_simt_kernel(const SimtParams p) {
         for (int a = 0; a < TC; ++a)
 #pragma unroll
             for (int b2 = 0; b2 < TJ; ++b2) S[(c0 + a) * DV + j0 + b2] = acc[a][b2];
-        for (int c = tid; c < DK; c += NT) G[c] += bs[(n - 1) * DK + c];
+        for (int c = tid; c < DK; c += NT) G[c] += bs[(n - 1) * KP + c];
     };
 
     auto scale_keys = [&](int n) {
         for (int idx = tid; idx < n * DK; idx += NT) {
-            const int c = idx % DK;
-            ks[idx] *= expf(bs[(n - 1) * DK + c] - bs[idx]);
+            const int t = idx / DK, c = idx - t * DK;
+            ks[t * KP + c] *= expf(bs[(n - 1) * KP + c] - bs[t * KP + c]);
         }
     };
 
@@ -211,62 +265,41 @@ gla_simt_kernel(const SimtParams p) {
             const int t = idx / n, s = idx - t * n;
             float acc = 0.0f;
             if (s <= t) {
-                const float *qt = qs + t * DK, *bt = bs + t * DK;
-                const float *kk = ks + s * DK, *bb = bs + s * DK;
+                const float *qt = qs + t * KP, *bt = bs + t * KP;
+                const float *kk = ks + s * KP, *bb = bs + s * KP;
                 for (int c = 0; c < DK; ++c) acc = fmaf(qt[c] * kk[c], expf(bt[c] - bb[c]), acc);
             }
             As[t * C + s] = acc;
         }
         __syncthreads();
         // q_t (.) e^{b_t} for the inter-chunk term; k_s (.) e^{b_last - b_s} for the state
-        for (int idx = tid; idx < n * DK; idx += NT) qs[idx] *= expf(bs[idx]);
+        for (int idx = tid; idx < n * DK; idx += NT) {
+            const int t = idx / DK, c = idx - t * DK;
+            qs[t * KP + c] *= expf(bs[t * KP + c]);
+        }
         scale_keys(n);
         __syncthreads();
-        // O[t][j] = scale (sum_{s<=t} A[t][s] v_s[j] + sum_c q~_t[c] S[c][j]); register-blocked
-        // over 4 value columns and the tokens t = tg, tg + TS, ... of one thread, so each
-        // loaded S row piece serves every token of the thread; each output still accumulates
-        // in the order s = 0..t, then c = 0..DK-1
-        {
-            constexpr int JG = DV / 4, TS = NT / JG, MT = (64 + TS - 1) / TS;
-            const int j0 = (tid % JG) * 4, tg = tid / JG;
-            float acc[MT][4];
-#pragma unroll
-            for (int i = 0; i < MT; ++i)
-#pragma unroll
-                for (int e = 0; e < 4; ++e) acc[i][e] = 0.0f;
-#pragma unroll
-            for (int i = 0; i < MT; ++i) {
-                const int t = tg + i * TS;
-                if (t < n) {
-                    for (int s = 0; s <= t; ++s) {
-                        const float a_ts = As[t * C + s];
-#pragma unroll
-                        for (int e = 0; e < 4; ++e) acc[i][e] = fmaf(a_ts, vs[s * DV + j0 + e], acc[i][e]);
-                    }
-                }
+        // O[t][j] = scale (sum_{s<=t} A[t][s] v_s[j] + sum_c q~_t[c] S[c][j]), 4 value columns
+        // per work item; each output accumulates in the order s = 0..t, then c = 0..DK-1
+        for (int w = tid; w < n * (DV / 4); w += NT) {
+            const int t = w / (DV / 4), j0 = (w - t * (DV / 4)) * 4;
+            float4 acc = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+            for (int s = 0; s <= t; ++s) {
+                const float a_ts = As[t * C + s];
+                const float4 vr = *reinterpret_cast<const float4 *>(vs + s * DV + j0);
+                acc = make_float4(fmaf(a_ts, vr.x, acc.x), fmaf(a_ts, vr.y, acc.y),
+                                  fmaf(a_ts, vr.z, acc.z), fmaf(a_ts, vr.w, acc.w));
             }
+            const float *qt = qs + t * KP;
+#pragma unroll 4
             for (int c = 0; c < DK; ++c) {
+                const float qv = qt[c];
                 const float4 sr = *reinterpret_cast<const float4 *>(S + c * DV + j0);
-#pragma unroll
-                for (int i = 0; i < MT; ++i) {
-                    const int t = tg + i * TS;
-                    if (t < n) {
-                        const float qv = qs[t * DK + c];
-                        acc[i][0] = fmaf(qv, sr.x, acc[i][0]);
-                        acc[i][1] = fmaf(qv, sr.y, acc[i][1]);
-                        acc[i][2] = fmaf(qv, sr.z, acc[i][2]);
-                        acc[i][3] = fmaf(qv, sr.w, acc[i][3]);
-                    }
-                }
+                acc = make_float4(fmaf(qv, sr.x, acc.x), fmaf(qv, sr.y, acc.y),
+                                  fmaf(qv, sr.z, acc.z), fmaf(qv, sr.w, acc.w));
             }
-#pragma unroll
-            for (int i = 0; i < MT; ++i) {
-                const int t = tg + i * TS;
-                if (t < n) {
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) Os[t * DV + j0 + e] = acc[i][e] * p.scale;
-                }
-            }
+            *reinterpret_cast<float4 *>(Os + t * DV + j0) =
+                make_float4(acc.x * p.scale, acc.y * p.scale, acc.z * p.scale, acc.w * p.scale);
         }
         __syncthreads();
         fold_state(n);
@@ -279,7 +312,7 @@ gla_simt_kernel(const SimtParams p) {
             const float inv = 1.0f / sqrtf(ss / DV + p.eps);
             const size_t base = (size_t)rows[t] * DV;
             for (int j = lane; j < DV; j += 32) {
-                const float u = ot[j] * inv * p.w[j] * silu(to_f32(g[base + j]));
+                const float u = ot[j] * inv * p.w[j] * silu(gsm[t * DV + j]);
                 out[base + j] = from_f32<T>(u);
             }
         }
