@@ -885,12 +885,25 @@ __global__ void __launch_bounds__(kThreads, 1) gla_tc_kernel(const Params p) {
         if (mid_xchg) {
             xchg_scan(true);
             if (warp == 3 || (warp >= 4 && warp < 7)) prep_sg(0, 8);
-        } else if (warp == 3) {                      // no scan: each warp its own channel
-            prep_sg(0, 8);                           // half, warp 3 also the issuing warp's
-        } else if (warp != 7) {
-            prep_sg(4 * ch, 4 * ch + 4);
+        } else {
+            if (warp == 3) prep_sg(0, 8);            // no scan: each warp its own channel half,
+            else if (warp != 7) prep_sg(4 * ch, 4 * ch + 4);   // warp 3 also the issuer's
+            write_stilde();                          // S~ from the state entering this chunk,
+            if (ci + 1 < n_chunks) fold_sloc(false); // then S = S 2^{B} + Sloc for the next one
+            ptx::fence_proxy_async_smem();
         }
         wait_mma(1);
+        if (!mid_xchg) {
+            // the inter product by warp 4 while the others build P (warp 4's rows 0..31 need
+            // no column of P past 31: its share is zero fill)
+            ptx::tc_fence_before_sync();
+            __syncthreads();                         // S~ complete
+            if (warp == 4 && ptx::elect_one()) {
+                ptx::tc_fence_after_sync();
+                issue_inter(sbase, tmem, false);
+                ptx::mma_commit(&m.mbar_mma[2]);
+            }
+        }
         if (m.slow) make_p_exact(sm, t, ch, n, p.scale, &m.range_err);
         else make_p_fast(n);
         operands_ready();
@@ -913,15 +926,9 @@ __global__ void __launch_bounds__(kThreads, 1) gla_tc_kernel(const Params p) {
             if (warp == 0 && ptx::elect_one()) {
                 ptx::tc_fence_after_sync();
                 issue_pv(sbase, m.slow ? kKH : kPB, tmem);
+                ptx::mma_commit(&m.mbar_mma[3]);
             }
-            write_stilde();                          // S~ from the state entering this chunk,
-            if (ci + 1 < n_chunks) fold_sloc(false); // then S = S 2^{B} + Sloc for the next one
-            operands_ready();
-            if (warp == 0 && ptx::elect_one()) {
-                ptx::tc_fence_after_sync();
-                issue_inter(sbase, tmem, false);
-                ptx::mma_commit(&m.mbar_mma[2]);     // P.V and the inter product
-            }
+            wait_mma(3);
         }
         wait_mma(2);
         preload_next(ci, true);                      // every tile consumed (all products done)
