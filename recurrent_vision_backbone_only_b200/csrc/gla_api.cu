@@ -296,7 +296,7 @@ int run_simt(const Args &x, int chunk, int segs, float eps, cudaStream_t st, con
 // fp16 I/O with d_k = d_v = 64.  One cluster of `segs` CTAs per (b, h) pair.
 int run_tc(const Args &x, int chunk, int segs, float eps, cudaStream_t st, const DeviceInfo &di,
            Plan *query) {
-    auto kern = tc::gla_tc_kernel<64>;
+    auto kern = tc::gla_tc_kernel<64, false>;
     const int L = x.gh * x.gw;
     const int n_pairs = x.B * x.H;
     if (chunk <= 0) chunk = tc::kC;
@@ -324,7 +324,19 @@ int run_tc(const Args &x, int chunk, int segs, float eps, cudaStream_t st, const
     p.B = x.B; p.H = x.H; p.gh = x.gh; p.gw = x.gw; p.L = L; p.dir = x.dir;
     p.segs = pl.segs; p.seg_len = pl.seg_len; p.chunk_max = chunk;
     p.eps = eps; p.scale = 0.125f;  // 64^{-1/2}
-    if (cudaLaunchKernelEx(&pl.cfg, kern, p) != cudaSuccess) {
+    // every segment one chunk: the instantiation without the multi-chunk paths (same
+    // resources and launch shape as the one the plan was made for)
+    auto launch = kern;
+    if (pl.seg_len <= chunk) {
+        launch = tc::gla_tc_kernel<64, true>;
+        if (cudaFuncSetAttribute(launch, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)pl.smem) !=
+                cudaSuccess ||
+            cudaFuncSetAttribute(launch, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) != cudaSuccess) {
+            cudaGetLastError();
+            return GLA_ERR_CUDA;
+        }
+    }
+    if (cudaLaunchKernelEx(&pl.cfg, launch, p) != cudaSuccess) {
         cudaGetLastError();
         return GLA_ERR_CUDA;
     }
