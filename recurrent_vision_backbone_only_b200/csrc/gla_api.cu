@@ -324,10 +324,10 @@ int run_tc(const Args &x, int chunk, int segs, float eps, cudaStream_t st, const
     p.B = x.B; p.H = x.H; p.gh = x.gh; p.gw = x.gw; p.L = L; p.dir = x.dir;
     p.segs = pl.segs; p.seg_len = pl.seg_len; p.chunk_max = chunk;
     p.eps = eps; p.scale = 0.125f;  // 64^{-1/2}
-    // every segment one chunk: the instantiation without the multi-chunk paths (same
-    // resources and launch shape as the one the plan was made for)
+    // every segment one chunk and several segments: the instantiation with only the
+    // mid-chunk exchange path (same resources and launch shape as the planned one)
     auto launch = kern;
-    if (pl.seg_len <= chunk) {
+    if (pl.seg_len <= chunk && pl.segs > 1) {
         launch = tc::gla_tc_kernel<64, true>;
         if (cudaFuncSetAttribute(launch, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)pl.smem) !=
                 cudaSuccess ||

@@ -294,10 +294,11 @@ __device__ __noinline__ void make_p_exact(uint8_t *sm, int t, int ch, int n, flo
     if (err) *range_err = 1;
 }
 
-// kOneChunk: every segment of the launch is a single chunk (the host guarantees
-// seg_len <= chunk_max), so the state-only pass, the multi-chunk exchange and the next-chunk
-// gathers are compiled out of that instantiation.
-template <int D, bool kOneChunk>
+// kMid: every segment of the launch is a single chunk and there are several segments (the
+// host guarantees seg_len <= chunk_max and segs > 1): the exchange happens mid-chunk, and the
+// state-only pass, the multi-chunk exchange, the next-chunk gathers and the no-exchange
+// branches are compiled out of that instantiation.
+template <int D, bool kMid>
 __global__ void __launch_bounds__(kThreads, 1) gla_tc_kernel(const Params p) {
     static_assert(D == kD, "tensor-core kernel handles d_k = d_v = 64");
     extern __shared__ uint8_t smem_raw[];
@@ -319,8 +320,8 @@ __global__ void __launch_bounds__(kThreads, 1) gla_tc_kernel(const Params p) {
     const int seg_n = p1 - p0;
     const int n_chunks = seg_n > 0 ? (seg_n + p.chunk_max - 1) / p.chunk_max : 0;
     const int chunk_len = n_chunks > 0 ? (seg_n + n_chunks - 1) / n_chunks : 0;
-    const bool exchange = p.segs > 1;
-    const bool resident = kOneChunk || n_chunks <= 1;
+    const bool exchange = kMid || p.segs > 1;
+    const bool resident = kMid || n_chunks <= 1;
 
     // Programmatic dependent launch: the next launch on the stream may start its prologue now;
     // this grid touches no global memory before the previous grid has completed.
@@ -801,7 +802,7 @@ __global__ void __launch_bounds__(kThreads, 1) gla_tc_kernel(const Params p) {
     // Non-resident segments (several chunks) run a state-only pass first (all ranks but the
     // last), then the exchange, then the full pass; a resident segment (one chunk) runs the
     // full pass once and exchanges mid-chunk.  Every CTA exchanges exactly once.
-    const int n_pass1 = (!kOneChunk && !resident && exchange && rank < p.segs - 1) ? n_chunks : 0;
+    const int n_pass1 = (!kMid && !resident && exchange && rank < p.segs - 1) ? n_chunks : 0;
     // Within a pass, the next chunk's gathers are issued as soon as this chunk's tiles are
     // free (after the state product in the state-only pass, after the last products in the
     // full pass), into the other row-index buffer; never across the exchange, which writes
@@ -820,7 +821,7 @@ __global__ void __launch_bounds__(kThreads, 1) gla_tc_kernel(const Params p) {
     for (int step = 0; step < n_pass1 + n_chunks; ++step) {
         const bool pass1 = step < n_pass1;
         const int ci = pass1 ? step : step - n_pass1;
-        if (!kOneChunk && !pass1 && ci == 0 && !resident && exchange) {
+        if (!kMid && !pass1 && ci == 0 && !resident && exchange) {
             xchg_begin();
             xchg_scan(false);
             xchg_wait_sin();
@@ -862,8 +863,8 @@ __global__ void __launch_bounds__(kThreads, 1) gla_tc_kernel(const Params p) {
             ptx::mma_commit(&m.mbar_mma[0]);
         }
         wait_mma(0);
-        const bool mid_xchg = !pass1 && resident && exchange;
-        if (!kOneChunk && pass1) preload_next(ci, false);   // a, k, v consumed
+        const bool mid_xchg = kMid || (!pass1 && resident && exchange);
+        if (!kMid && pass1) preload_next(ci, false);   // a, k, v consumed
         read_sloc();
         if (pass1 || mid_xchg) fold_sloc(true);     // S = S 2^{B} + Sloc, Gs += B
         if (pass1) {
@@ -892,7 +893,7 @@ __global__ void __launch_bounds__(kThreads, 1) gla_tc_kernel(const Params p) {
             if (warp == 3) prep_sg(0, 8);            // no scan: each warp its own channel half,
             else if (warp != 7) prep_sg(4 * ch, 4 * ch + 4);   // warp 3 also the issuer's
             write_stilde();                          // S~ from the state entering this chunk,
-            if (!kOneChunk && ci + 1 < n_chunks)     // then S = S 2^{B} + Sloc for the next
+            if (!kMid && ci + 1 < n_chunks)          // then S = S 2^{B} + Sloc for the next
                 fold_sloc(false);
             ptx::fence_proxy_async_smem();
         }
@@ -935,7 +936,7 @@ __global__ void __launch_bounds__(kThreads, 1) gla_tc_kernel(const Params p) {
             wait_mma(3);
         }
         wait_mma(2);
-        if (!kOneChunk) preload_next(ci, true);      // every tile consumed (all products done)
+        if (!kMid) preload_next(ci, true);           // every tile consumed (all products done)
         epilogue(n, rb);
         ptx::tc_fence_before_sync();
         __syncthreads();
