@@ -142,11 +142,11 @@ __device__ __forceinline__ uint32_t recv_slot(uint32_t j) {
 // Only the first n_cols score columns (the chunk's rows rounded up to 16) are produced.
 __device__ __forceinline__ void issue_qk(uint32_t sbase, uint32_t tmem, int n_cols) {
     const uint32_t idesc = ptx::idesc_make(2, false, false, 128, (uint32_t)n_cols);
-#pragma unroll
+#pragma unroll 1
     for (int pass = 0; pass < 3; ++pass) {
         const uint32_t acol = pass == 2 ? kColQL : kColQH;
         const uint32_t bsm = pass == 1 ? kKL : kKH;
-#pragma unroll
+#pragma unroll 1
         for (int k = 0; k < 8; ++k) {
             const uint32_t koff = (k >> 2) * kAtom128 + (k & 3) * 32;
             ptx::mma_tf32_ts(tmem + kColDS, tmem + acol + 8 * k,
@@ -158,7 +158,7 @@ __device__ __forceinline__ void issue_qk(uint32_t sbase, uint32_t tmem, int n_co
 // Sloc^T[j][c] = sum_s V[s][j] Ks[s][c]  (both operands MN-major, K = 128 rows); the state is
 // kept transposed so each thread owns one value column j and writes S~ rows contiguously.
 __device__ __forceinline__ void issue_state(uint32_t sbase, uint32_t tmem) {
-#pragma unroll
+#pragma unroll 1
     for (int k = 0; k < 8; ++k) {
         ptx::mma_f16_ss(tmem + kColSL, ptx::desc_sw128(sbase + kTV + k * 2048, kAtom128, 1024),
                         ptx::desc_sw128(sbase + kST + k * 2048, kAtom128, 1024), kIdescST, k > 0);
@@ -166,7 +166,7 @@ __device__ __forceinline__ void issue_state(uint32_t sbase, uint32_t tmem) {
 }
 // O[t][j] = sum_s P[t][s] V[s][j]
 __device__ __forceinline__ void issue_pv(uint32_t sbase, uint32_t p_base, uint32_t tmem) {
-#pragma unroll
+#pragma unroll 1
     for (int k = 0; k < 8; ++k) {
         const uint32_t koff = (k >> 2) * kAtom128 + (k & 3) * 32;
         ptx::mma_f16_ss(tmem + kColOP, ptx::desc_sw128(sbase + p_base + koff, 16, 1024),
@@ -175,9 +175,9 @@ __device__ __forceinline__ void issue_pv(uint32_t sbase, uint32_t p_base, uint32
 }
 // O[t][j] (+)= sum_c (Qh + Ql)[t][c] S~[c][j], S~ (MN-major) in the a-tile region
 __device__ __forceinline__ void issue_inter(uint32_t sbase, uint32_t tmem, bool accumulate) {
-#pragma unroll
+#pragma unroll 1
     for (int pass = 0; pass < 2; ++pass) {
-#pragma unroll
+#pragma unroll 1
         for (int k = 0; k < 8; ++k) {                  // 8 key channels = 8 S~ rows per step
             ptx::mma_tf32_ts(tmem + kColO, tmem + (pass ? kColQL : kColQH) + 8 * k,
                              ptx::desc_sw128_b32(sbase + kTA + k * 1024, kAtom64, 512), kIdescIN,
@@ -604,8 +604,8 @@ __global__ void __launch_bounds__(kThreads, 1) gla_tc_kernel(const Params p) {
     auto make_p_fast = [&](int n) {
         const float dq = (m.dqp[0][t] + m.dqp[1][t]) * p.scale;   // exact diagonal score
         float amax = 0.0f;
-        p_block(ch * 64, n, dq, amax);
-        p_block(ch * 64 + 32, n, dq, amax);
+#pragma unroll 1
+        for (int blk = 0; blk < 2; ++blk) p_block(ch * 64 + 32 * blk, n, dq, amax);
         if (amax > 65504.0f) m.range_err = 1;
     };
     // S~[c][j] = tf32(2^{r_c} S[c][j]) from the state owners' registers (value column j, key
