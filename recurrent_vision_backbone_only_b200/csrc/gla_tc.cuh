@@ -298,6 +298,35 @@ __device__ __noinline__ void make_p_exact(uint8_t *sm, int t, int ch, int n, flo
 // host guarantees seg_len <= chunk_max and segs > 1): the exchange happens mid-chunk, and the
 // state-only pass, the multi-chunk exchange, the next-chunk gathers and the no-exchange
 // branches are compiled out of that instantiation.
+// Score operands of a chunk whose decay range the fast operands cannot carry (row t, 32
+// channels of half ch): Qh/Ql of d_k^{-1/2} q 2^{b} (chunk-start reference; P is then
+// evaluated exactly) into TMEM, and the partial diagonal q_t . k_t.  Rare; kept out of line
+// so the common path stays compact.  Called by whole warps (tcgen05.st is warp-collective).
+__device__ __noinline__ void build_q_exact(uint8_t *sm, int t, int ch, uint32_t tmem_warp, float *dq_out) {
+    float dqs = 0.0f;
+    for (int jj = 0; jj < 4; ++jj) {
+        const int j = ch * 4 + jj;
+        const uint4 kraw = *reinterpret_cast<const uint4 *>(sm + kTK + off_f16(t, j));
+        const uint4 qraw = *reinterpret_cast<const uint4 *>(sm + kTQ + off_f16(t, j));
+        const __half2 *k2 = reinterpret_cast<const __half2 *>(&kraw);
+        const __half2 *q2 = reinterpret_cast<const __half2 *>(&qraw);
+        float qh[8], ql[8];
+        for (int e = 0; e < 8; ++e) {
+            const float kf = e & 1 ? __high2float(k2[e >> 1]) : __low2float(k2[e >> 1]);
+            const float qv = e & 1 ? __high2float(q2[e >> 1]) : __low2float(q2[e >> 1]);
+            const float bt = reinterpret_cast<const float *>(sm + kPB + off_tf32(kAtom128, t, 2 * j + (e >> 2)))[e & 3];
+            dqs = fmaf(qv, kf, dqs);
+            const float qf = qv * ptx::ex2(bt + kLog2Scale);
+            qh[e] = ptx::tf32_hi(qf);
+            ql[e] = qf - qh[e];
+        }
+        ptx::tmem_st8(tmem_warp + kColQH + 8 * j, qh);
+        ptx::tmem_st8(tmem_warp + kColQL + 8 * j, ql);
+    }
+    *dq_out = dqs;
+    ptx::tmem_st_wait();
+}
+
 template <int D, bool kMid>
 __global__ void __launch_bounds__(kThreads, 1) gla_tc_kernel(const Params p) {
     static_assert(D == kD, "tensor-core kernel handles d_k = d_v = 64");
@@ -480,12 +509,15 @@ __global__ void __launch_bounds__(kThreads, 1) gla_tc_kernel(const Params p) {
             *reinterpret_cast<uint4 *>(sm + kST + off_f16(t, j)) = kso;
         }
     };
-    // Score operands.  Fast path: with x = 2^{r - b} (one ex2), Kh/Kl (smem tf32) of K~ = k x
-    // and Qh/Ql (TMEM) of Q~ = q / (8 x) (Newton reciprocal; the rounding of x cancels in each
-    // product q_tc x^-1 k_sc x); slow path: Qh/Ql of d_k^{-1/2} q 2^{b} only.  Also the exact
-    // diagonal q_t . k_t.
+    // Score operands.  With x = 2^{r - b} (one ex2), Kh/Kl (smem tf32) of K~ = k x and Qh/Ql
+    // (TMEM) of Q~ = q / (8 x) (Newton reciprocal; the rounding of x cancels in each product
+    // q_tc x^-1 k_sc x), and the exact diagonal q_t . k_t; a chunk beyond the fast operands'
+    // range takes build_q_exact.
     auto build_qk = [&]() {
-        const bool slow = m.slow != 0;
+        if (m.slow) {                              // CTA-uniform
+            build_q_exact(sm, t, ch, tmem_warp, &m.dqp[ch][t]);
+            return;
+        }
         float dqs = 0.0f;                          // partial q_t . k_t over this half's channels
 #pragma unroll 1
         for (int jj = 0; jj < 4; ++jj) {
@@ -516,31 +548,22 @@ __global__ void __launch_bounds__(kThreads, 1) gla_tc_kernel(const Params p) {
             float qh[8], ql[8], kh[8], kl[8];
 #pragma unroll
             for (int e = 0; e < 8; ++e) {
-                if (!slow) {
-                    const float x = ptx::ex2(rr[e] - bt[e]);
-                    const float kf = kv[e] * x;                              // k 2^{r - b}
-                    const float qf = qv[e] * rcp_nr(x) * 0.125f;             // q 2^{b - r} / 8
-                    kh[e] = ptx::tf32_hi(kf);
-                    kl[e] = kf - kh[e];
-                    qh[e] = ptx::tf32_hi(qf);
-                    ql[e] = qf - qh[e];
-                } else {
-                    const float qf = qv[e] * ptx::ex2(bt[e] + kLog2Scale);
-                    qh[e] = ptx::tf32_hi(qf);
-                    ql[e] = qf - qh[e];
-                    kh[e] = kl[e] = 0.0f;
-                }
+                const float x = ptx::ex2(rr[e] - bt[e]);
+                const float kf = kv[e] * x;                                  // k 2^{r - b}
+                const float qf = qv[e] * rcp_nr(x) * 0.125f;                 // q 2^{b - r} / 8
+                kh[e] = ptx::tf32_hi(kf);
+                kl[e] = kf - kh[e];
+                qh[e] = ptx::tf32_hi(qf);
+                ql[e] = qf - qh[e];
             }
             ptx::tmem_st8(tmem_warp + kColQH + 8 * j, qh);
             ptx::tmem_st8(tmem_warp + kColQL + 8 * j, ql);
-            if (!slow) {
 #pragma unroll
-                for (int h = 0; h < 2; ++h) {
-                    *reinterpret_cast<float4 *>(sm + kKH + off_tf32(kAtom128, t, 2 * j + h)) =
-                        make_float4(kh[4 * h], kh[4 * h + 1], kh[4 * h + 2], kh[4 * h + 3]);
-                    *reinterpret_cast<float4 *>(sm + kKL + off_tf32(kAtom128, t, 2 * j + h)) =
-                        make_float4(kl[4 * h], kl[4 * h + 1], kl[4 * h + 2], kl[4 * h + 3]);
-                }
+            for (int h = 0; h < 2; ++h) {
+                *reinterpret_cast<float4 *>(sm + kKH + off_tf32(kAtom128, t, 2 * j + h)) =
+                    make_float4(kh[4 * h], kh[4 * h + 1], kh[4 * h + 2], kh[4 * h + 3]);
+                *reinterpret_cast<float4 *>(sm + kKL + off_tf32(kAtom128, t, 2 * j + h)) =
+                    make_float4(kl[4 * h], kl[4 * h + 1], kl[4 * h + 2], kl[4 * h + 3]);
             }
         }
         m.dqp[ch][t] = dqs;
@@ -766,7 +789,7 @@ __global__ void __launch_bounds__(kThreads, 1) gla_tc_kernel(const Params p) {
 #pragma unroll
             for (int i = 0; i < 4; ++i) rs[i] = recv_slot(j0 + i) * 16 + cl * 4;
             float4 run = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
-#pragma unroll 4
+#pragma unroll 2
             for (int q = 0; q < segs; ++q) {
                 const uint8_t *blk = sm + recv_off(lg, q, 0);
                 const float4 agg = make_float4(*reinterpret_cast<const float *>(blk + rs[0]),
