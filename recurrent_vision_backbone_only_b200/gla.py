@@ -87,6 +87,16 @@ def _check(rc: int, where: str):
         raise GLAError(rc, where)
 
 
+def _dtype_code(t) -> int:
+    """0 for float16 I/O, 1 for float32 I/O."""
+    import torch
+    if t.dtype == torch.float16:
+        return 0
+    if t.dtype == torch.float32:
+        return 1
+    raise ValueError("q must be float16 or float32, not %s" % t.dtype)
+
+
 def _stream_ptr(stream):
     import torch
     if stream is None:
@@ -140,7 +150,7 @@ def gla_fwd_ex(q, k, v, a, g, w, out, grid_h: int, grid_w: int, direction: int,
     import torch
     B, H, dk, dv = _dims(q, v, grid_h, grid_w)
     _check_tensors(q, k, v, a, g, w, out, q.dtype)
-    dtype = {torch.float16: 0, torch.float32: 1}[q.dtype]
+    dtype = _dtype_code(q)
     args = [ctypes.c_void_p(t.data_ptr()) for t in (q, k, v, a, g, w, out)]
     args += [B, H, grid_h, grid_w, dk, dv, direction, dtype, chunk, segments,
              ctypes.c_float(eps), _stream_ptr(stream)]
@@ -158,7 +168,7 @@ def gla_fwd_host(q, k, v, a, g, w, out, grid_h: int, grid_w: int, direction: int
     for t in (q, k, v, a, g, w, out):
         if t.is_cuda or not t.is_contiguous():
             raise ValueError("gla_fwd_host takes contiguous host tensors")
-    dtype = {torch.float16: 0, torch.float32: 1}[q.dtype]
+    dtype = _dtype_code(q)
     args = [ctypes.c_void_p(t.data_ptr()) for t in (q, k, v, a, g, w, out)]
     args += [int(B), int(H), grid_h, grid_w, int(dk), int(dv), direction, dtype,
              _stream_ptr(stream)]

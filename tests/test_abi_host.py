@@ -127,3 +127,13 @@ def test_binding_raises_when_library_missing(monkeypatch, tmp_path):
     monkeypatch.setattr(gla, "LIB_PATH", os.path.join(str(tmp_path), "missing.so"))
     with pytest.raises(RuntimeError, match="no fallback"):
         gla.load()
+
+
+def test_binding_rejects_unsupported_dtypes_before_any_call():
+    import torch
+    x = torch.zeros(1, 4, 1, 64, dtype=torch.bfloat16)
+    w = torch.zeros(64)
+    with pytest.raises(ValueError):
+        gla.gla_fwd_host(x, x, x, x, x, w, x, 2, 2, 0)
+    with pytest.raises(ValueError):
+        gla.gla_fwd_ex(x, x, x, x, x, w, x, 2, 2, 0)
