@@ -19,7 +19,9 @@ tf32 score operands (high part = the fp32 value with its low 13 mantissa bits cl
 what the tensor core reads; low part = the remainder, read the same way), an exact fp32
 diagonal, fp16 P and decayed keys, tf32 S~, fp32 accumulation, fp16 output.  A single
 tf32 operand per side is shown to miss that tolerance on a first token whose readout
-nearly cancels.
+nearly cancels.  Two alternative state precisions are weighed the same way: an fp16 inter
+product with the segment states exchanged in fp16 stays within the tolerance, bf16 states
+do not.
 """
 import math
 
@@ -229,3 +231,66 @@ def test_broken_factorisations_are_caught(kind):
     _, o_ref = oracle.gla_forward(q, k, v, a, g, w, 12, 20, 1, return_o=True)
     o = chunkwise_o(q, k, v, a, 12, 20, 1, 32, 3, _mutant(kind))
     assert np.max(np.abs(o - o_ref)) > 1.0
+
+
+# ---- alternative state precisions (an fp16 inter product; bf16 states) --------------
+def bf16(x):
+    """Round to bfloat16 (nearest even), returned as fp64."""
+    u = np.ascontiguousarray(x, dtype=np.float32).view(np.uint32).astype(np.uint64)
+    u = (u + 0x7FFF + ((u >> 16) & 1)) & 0xFFFF0000
+    return u.astype(np.uint32).view(np.float32).astype(np.float64)
+
+
+def chunk_f16_inter(q, k, v, lg, S_in):
+    """As chunk_rounded, but the inter product is fp16(q 2^b / sqrt(d_k)) . fp16(S_in):
+    every exponent in it is <= 0, so it suits a single kind::f16 product."""
+    n, dk = q.shape
+    b = np.cumsum(f32(lg).astype(np.float32), axis=0).astype(np.float64)
+    O, S_out, B = chunk_rounded(q, k, v, lg, np.zeros_like(S_in))
+    O = O + f32(f16(q * f32(np.exp2(b)) / math.sqrt(dk)) @ f16(S_in))
+    S_out = f32(S_out + f32(np.exp2(B)[:, None] * S_in))
+    return O, S_out, B
+
+
+def exchanged_in(rnd, monkeypatch):
+    """Run the segment scan with both exchanged states rounded by `rnd`."""
+    def scan(q, k, v, lg, chunk, segs, chunk_fn):
+        L, dk = q.shape
+        seg_len = -(-L // segs)
+        bounds = [(s0, min(L, s0 + seg_len)) for s0 in range(0, L, seg_len)]
+
+        def run(s0, s1, S):
+            outs, G = [], np.zeros(dk)
+            for c0 in range(s0, s1, chunk):
+                c1 = min(s1, c0 + chunk)
+                O, S, B = chunk_fn(q[c0:c1], k[c0:c1], v[c0:c1], lg[c0:c1], S)
+                outs.append(O)
+                G = G + B
+            return np.concatenate(outs), S, G
+
+        incoming, S_in = [], np.zeros((dk, v.shape[1]))
+        for s0, s1 in bounds:
+            incoming.append(rnd(S_in))
+            _, S_agg, G = run(s0, s1, np.zeros_like(S_in))
+            S_in = f32(np.exp2(G)[:, None] * S_in + rnd(S_agg))
+        return np.concatenate([run(s0, s1, S0)[0] for (s0, s1), S0 in zip(bounds, incoming)])
+    monkeypatch.setitem(globals(), "segmented_scan", scan)
+
+
+@pytest.mark.parametrize("rnd,chunk_fn,ok", [(f16, chunk_f16_inter, True),
+                                             (bf16, chunk_rounded, False)])
+def test_state_precision_alternatives(rnd, chunk_fn, ok, monkeypatch):
+    from recurrent_vision_backbone_only_b200 import synth
+    wl = synth.WORKLOADS["gtr640"]
+    x = {n: t.astype(np.float64) for n, t in synth.make_inputs(wl, seed=0).items()}
+    exchanged_in(rnd, monkeypatch)
+    worst = 0.0
+    for direction in (0, 1, 2, 3):
+        ref = oracle.gla_forward(x["q"], x["k"], x["v"], x["a"], x["g"], x["w"],
+                                 wl.grid_h, wl.grid_w, direction)
+        o = chunkwise_o(x["q"], x["k"], x["v"], x["a"], wl.grid_h, wl.grid_w, direction,
+                        128, 16, chunk_fn)
+        max_abs, rel = errors(epilogue_f16(o, x["g"], x["w"]), ref)
+        worst = max(worst, max_abs)
+        assert rel <= 2e-3
+    assert (worst <= 1e-2) == ok, worst
