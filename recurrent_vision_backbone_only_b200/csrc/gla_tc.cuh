@@ -350,7 +350,11 @@ __global__ void __launch_bounds__(kThreads, 1) gla_tc_kernel(const Params p) {
     const int n_chunks = seg_n > 0 ? (seg_n + p.chunk_max - 1) / p.chunk_max : 0;
     const int chunk_len = n_chunks > 0 ? (seg_n + n_chunks - 1) / n_chunks : 0;
     const bool exchange = kMid || p.segs > 1;
-    const bool resident = kMid || n_chunks <= 1;
+    // Residency follows the launch's segment length, not this segment's: a scanner writes
+    // every destination in its own layout (S~ for resident segments, S_in otherwise), so all
+    // CTAs of a cluster must agree.  A shorter last segment of one chunk, in a launch whose
+    // segments span several, takes the multi-chunk path with a single chunk.
+    const bool resident = kMid || p.seg_len <= p.chunk_max;
 
     // Programmatic dependent launch: the next launch on the stream may start its prologue now;
     // this grid touches no global memory before the previous grid has completed.

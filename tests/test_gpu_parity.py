@@ -233,3 +233,16 @@ def test_empty_launch_runs_clean():
     torch.cuda.synchronize()
     assert gla.get_status() == 0
     assert gla.raw_call("gla_empty_launch", 0, 1, 1, 1, None) == 2      # GLA_ERR_SHAPE
+
+
+@pytest.mark.parametrize("gh,gw,chunk,segs", [(16, 20, 32, 9), (42, 50, 128, 16), (42, 50, 0, 0)])
+def test_shorter_last_segment_of_one_chunk(gh, gw, chunk, segs):
+    # segments of several chunks whose last, shorter segment fits one chunk (16x20: 9
+    # segments of 36 tokens with chunk 32, the last of 32; 42x50: 16 segments of 132, the
+    # last of 120; and the automatic plan for 42x50): every CTA of a cluster must take the
+    # same exchange layout
+    wl = synth.WORKLOADS["gtr640"].with_(H=2, grid_h=gh, grid_w=gw)
+    x = synth.make_inputs(wl, seed=gh + gw)
+    for d in (0, 2):
+        assert_close(run_gpu(x, gh, gw, d, chunk=chunk, segments=segs), oracle_ref(x, gh, gw, d),
+                     "f16")
