@@ -38,9 +38,10 @@
 // cluster through distributed shared memory (the combine is elementwise per
 // state entry with the decay of its key channel, so CTA r scans the 4-channel
 // key groups g = r, r + segs, ...), giving every segment its incoming state.
-// A segment that fits one chunk keeps its tiles resident and does the
-// exchange mid-chunk; longer segments run a state-only pass, the exchange,
-// then the full pass, gathering each next chunk under the current one.
+// When the launch's segments fit one chunk, each keeps its tiles resident
+// and does the exchange mid-chunk; otherwise the segments run a state-only
+// pass, the exchange, then the full pass, gathering each next chunk under
+// the current one.
 //
 // Input gathers: 16-byte cp.async per thread, scan row t of the chunk read
 // from the token's spatial position (direction remap folded into the
@@ -826,9 +827,9 @@ __global__ void __launch_bounds__(kThreads, 1) gla_tc_kernel(const Params p) {
     };
 
     // ------------------------------------------------------------ schedule
-    // Non-resident segments (several chunks) run a state-only pass first (all ranks but the
-    // last), then the exchange, then the full pass; a resident segment (one chunk) runs the
-    // full pass once and exchanges mid-chunk.  Every CTA exchanges exactly once.
+    // Non-resident segments run a state-only pass first (all ranks but the last), then the
+    // exchange, then the full pass; a resident segment (one chunk) runs the full pass once
+    // and exchanges mid-chunk.  Every CTA exchanges exactly once.
     const int n_pass1 = (!kMid && !resident && exchange && rank < p.segs - 1) ? n_chunks : 0;
     // Within a pass, the next chunk's gathers are issued as soon as this chunk's tiles are
     // free (after the state product in the state-only pass, after the last products in the
