@@ -110,8 +110,10 @@ int gla_fwd_host(const void *q, const void *k, const void *v,
  * epsilon exposed, for tests: `chunk` = tokens per chunk (0 = the default
  * of the chosen kernel; otherwise a multiple of 16 that the kernel supports,
  * else GLA_ERR_UNSUPPORTED), `segments` = CTAs per (b, h) pair splitting the
- * scan (0 = automatic, else 1..16), `eps` the RMSNorm epsilon.  Every valid
- * choice computes the same operation (up to rounding order).
+ * scan (0 = automatic, else 1..16; the tensor-core kernel refuses 13, 14 and
+ * 15 with GLA_ERR_UNSUPPORTED, as their key-channel groups do not fit its
+ * state-exchange buffer), `eps` the RMSNorm epsilon.  Every valid choice
+ * computes the same operation (up to rounding order).
  */
 int gla_fwd_ex(const void *q, const void *k, const void *v,
                const void *gate_preact, const void *out_gate_preact,

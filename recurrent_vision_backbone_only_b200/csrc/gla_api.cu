@@ -161,8 +161,9 @@ double tc_cost(int L, int n_pairs, int segs, int active) {
     return waves * per_cta;
 }
 
-// The tensor-core kernel's state exchange splits the 64 state rows into ceil(64/segs)-row
-// slices and needs ceil(64/segs) * segs <= 66.
+// The tensor-core kernel's state exchange deals the 16 four-channel key groups out to the
+// segments; a scanner's receive buffer holds ceil(16/segs) groups from every segment, so
+// ceil(16/segs) * segs must not exceed tc::kMaxGroupSegs (24).
 bool tc_segs_ok(int segs) { return segs == 1 || ceil_div(16, segs) * segs <= tc::kMaxGroupSegs; }
 
 // Pick the segment count (auto when segs <= 0), shrinking it until a cluster
