@@ -98,8 +98,9 @@ def chunkwise_o(q, k, v, a, gh, gw, direction, chunk, segs, chunk_fn):
 @pytest.mark.parametrize("direction", [0, 1, 2, 3])
 @pytest.mark.parametrize("chunk,segs,where", [(16, 1, "middle"), (32, 3, "first"),
                                               (64, 16, "middle"), (100, 5, "last"),
-                                              (128, 2, "middle")])
+                                              (128, 2, "middle"), (32, 7, "middle")])
 def test_factorised_form_is_exact(direction, chunk, segs, where):
+    # (32, 7): segments of 35 tokens (two chunks) and a last one of 30 (one chunk)
     rng = np.random.default_rng(7)
     gh, gw = 12, 20
     q, k, v, a, g, w = rand_inputs(rng, 1, gh, gw, 2, 32, 24, a_mean=0.0, a_std=3.0)
