@@ -28,6 +28,8 @@
  * with L = grid_h * grid_w in row-major spatial order (index y*grid_w + x).
  * gate_preact is the full retention-gate pre-activation (x W1 W2 + b) and
  * out_gate_preact is x W_r; both activations are applied inside the call.
+ * Input values must be finite: the kernels do not check them, and an
+ * infinite or NaN element leaves the outputs of its (b, h) pair undefined.
  *
  * Pointers are DEVICE pointers (except in gla_fwd_host), 16-byte aligned,
  * owned by the caller; out must not overlap any input.  gla_fwd,
