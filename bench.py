@@ -49,6 +49,8 @@ def parse():
     ap.add_argument("--cpu-seconds", type=float, default=10.0,
                     help="CPU-oracle sample budget for cpu_baseline / --impl reference")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--kernel", choices=["auto", "tc128", "tc64", "simt"], default="auto",
+                    help="kernel to time (default: the one gla_fwd picks for the workload)")
     ap.add_argument("--workload", default=WORKLOAD,
                     help="synthetic workload to time (default: the 40x40 headline); the others "
                          "are reported with their own metric name")
@@ -316,10 +318,17 @@ def run_ours(args, ws, rank, local):
     launches_per_step = len(directions)
     dt = torch.float16 if wl.dtype == "f16" else torch.float32
 
+    kernel = {"auto": 0, "tc128": gla.KERNEL_TC128, "tc64": gla.KERNEL_TC64,
+              "simt": gla.KERNEL_SIMT}[args.kernel]
+
     def step(i):
         for j, d in enumerate(directions):
             s = sets[(i * launches_per_step + j) % n_sets]
-            gla.gla_fwd(s["q"], s["k"], s["v"], s["a"], s["g"], w, s["out"], gh, gw, d)
+            if kernel:
+                gla.gla_fwd_ex(s["q"], s["k"], s["v"], s["a"], s["g"], w, s["out"], gh, gw, d,
+                               kernel=kernel)
+            else:
+                gla.gla_fwd(s["q"], s["k"], s["v"], s["a"], s["g"], w, s["out"], gh, gw, d)
 
     stream = torch.cuda.Stream(device=dev)
     torch.cuda.synchronize()
@@ -432,7 +441,8 @@ def run_ours(args, ws, rank, local):
             "timing": "CUDA-graph replays (graphs of %d steps), CUDA events on the launch "
                       "stream; warm-up = %d eager steps + one untimed replay" % (G, args.warmup),
             "parallelism": "replicas" if ws > 1 else "single GPU",
-            "schedule": gla.plan(wl.B, wl.H, gh, gw, wl.d_k, wl.d_v, 0 if wl.dtype == "f16" else 1),
+            "schedule": gla.plan(wl.B, wl.H, gh, gw, wl.d_k, wl.d_v, 0 if wl.dtype == "f16" else 1)
+                        if not kernel else {"kernel": gla.KERNEL_NAMES[kernel]},
         },
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": achieved / peak, "traffic": profile_traffic(wl.name),

@@ -2,9 +2,10 @@
  * gla.h -- C ABI of libgla.so, the B200 (sm_100a) key-only gated linear
  * attention (GLA) token mixer of GTR.
  *
- * Operation (GTR paper, arXiv 2609.26590, method section): for every batch
- * element b and head h, over the L = grid_h * grid_w tokens of a patch grid
- * visited in one of four scan directions,
+ * Operation ("GTR: Gated Token Recurrence for Efficient Dense Prediction",
+ * arXiv 2609.26590, method section): for every batch element b and head h,
+ * over the L = grid_h * grid_w tokens of a patch grid visited in one of four
+ * scan directions,
  *
  *     gamma_t = sigma(a_t)^(1/16)                 (key-wise retention gate)
  *     S_t     = Diag(gamma_t) S_{t-1} + k_t^T v_t, S_0 = 0   (d_k x d_v state)
@@ -12,14 +13,14 @@
  *     u_t     = SiLU(g_t) * o_t / sqrt(mean_j(o_tj^2) + eps) * w   (eps = 1e-6)
  *
  * and u_t is written back at the token's ORIGINAL spatial position.  The
- * value-side decay is fixed to one.  The scan directions (same paper, method
- * section, "four scan directions"): 0 = left-to-right (rows top to bottom,
- * each row left to right), 1 = right-to-left (rows top to bottom, each row
- * right to left), 2 = top-to-bottom (columns left to right, each column top
- * to bottom), 3 = bottom-to-top (columns left to right, each column bottom to
- * top); the state carries over from one row/column to the next.  4 =
- * GLA_DIR_CYCLE: batch element b uses direction b % 4 (the paper cycles the
- * four directions across blocks; this batches the four in one launch).
+ * value-side decay is fixed to one.  The scan directions (same section, the
+ * scan-direction paragraph): 0 = left-to-right (rows top to bottom, each row
+ * left to right), 1 = right-to-left (rows top to bottom, each row right to
+ * left), 2 = top-to-bottom (columns left to right, each column top to bottom),
+ * 3 = bottom-to-top (columns left to right, each column bottom to top); the
+ * state carries over from one row/column to the next.  4 = GLA_DIR_CYCLE:
+ * batch element b uses direction b % 4 (the paper cycles the four directions
+ * across blocks; this batches the four in one launch).
  *
  * Layouts: every array is dense and token-major with the head interleaved:
  *     q, k, gate_preact (a):        [B][L][H][d_k]
@@ -71,10 +72,15 @@ enum gla_direction {
 };
 
 /*
- * gla_fwd -- fp16 I/O, fp32 arithmetic.  q, k, v, gate_preact,
- * out_gate_preact and out are IEEE binary16 arrays; rms_weight is float32.
- * `stream` is a cudaStream_t (NULL = legacy default stream).
- * Supported head dims: d_k, d_v in {32, 64, 128}.
+ * gla_fwd -- the operation above with fp16 I/O and fp32 arithmetic.
+ * Defined by the GTR paper's method section: the GLA recurrence paragraph (state,
+ * gate, readout), the output-gate paragraph (SiLU gate times RMSNorm) and the
+ * scan-direction paragraph (four directions, results in the original order).
+ * q, k, v, gate_preact, out_gate_preact and out are IEEE binary16 arrays;
+ * rms_weight is float32.  `stream` is a cudaStream_t (NULL = legacy default
+ * stream).  Supported head dims: d_k, d_v in {32, 64, 128}; d_k = d_v = 64 runs on
+ * the 128-row tensor-core kernel, d_k = d_v = 128 on the 64-row one, the others on
+ * CUDA cores (gla_kernel below).
  */
 int gla_fwd(const void *q, const void *k, const void *v,
             const void *gate_preact, const void *out_gate_preact,
@@ -83,8 +89,9 @@ int gla_fwd(const void *q, const void *k, const void *v,
             int direction, void *stream);
 
 /*
- * gla_fwd_f32 -- the same operation with float32 I/O and float32 arithmetic
- * throughout (CUDA cores; no TF32), for callers that need ~1e-6 agreement.
+ * gla_fwd_f32 -- the same operation (same paragraphs of the GTR method section) with
+ * float32 I/O and float32 arithmetic throughout (CUDA cores; no TF32), for callers
+ * that need ~1e-6 agreement.
  */
 int gla_fwd_f32(const float *q, const float *k, const float *v,
                 const float *gate_preact, const float *out_gate_preact,
@@ -94,12 +101,12 @@ int gla_fwd_f32(const float *q, const float *k, const float *v,
 
 /*
  * gla_fwd_host -- gla_fwd / gla_fwd_f32 on HOST buffers (dtype 0 = fp16,
- * 1 = fp32).  Copies the inputs to device buffers owned by the library
- * (grown on demand, kept between calls, one set per device), runs the
- * operation on `stream`, copies `out` back and synchronises `stream` before
- * returning.  Host buffers in page-locked memory make the copies
- * asynchronous DMA.  Not capturable (it synchronises); not thread-safe for
- * concurrent calls on the same device.
+ * 1 = fp32); the operation of the GTR method section as above.  Copies the
+ * inputs to device buffers owned by the library (grown on demand, kept between
+ * calls, one set per device), runs the operation on `stream`, copies `out` back
+ * and synchronises `stream` before returning.  Host buffers in page-locked
+ * memory make the copies asynchronous DMA.  Not capturable (it synchronises);
+ * not thread-safe for concurrent calls on the same device.
  */
 int gla_fwd_host(const void *q, const void *k, const void *v,
                  const void *gate_preact, const void *out_gate_preact,
@@ -107,27 +114,38 @@ int gla_fwd_host(const void *q, const void *k, const void *v,
                  int B, int H, int grid_h, int grid_w, int d_k, int d_v,
                  int direction, int dtype, void *stream);
 
+/* Kernels gla_fwd_ex can be asked for (gla_plan reports the same ids). */
+enum gla_kernel {
+    GLA_KERNEL_AUTO = 0,   /* the one gla_fwd / gla_fwd_f32 choose                       */
+    GLA_KERNEL_TC128 = 1,  /* tensor cores, 128-row chunks: fp16, d_k = d_v = 64           */
+    GLA_KERNEL_SIMT = 2,   /* CUDA cores: every supported shape, fp16 or fp32              */
+    GLA_KERNEL_TC64 = 3    /* tensor cores, 64-row chunks, TMA loads: fp16, d_k = d_v in   */
+                           /* {64, 128}                                                    */
+};
+
 /*
- * gla_fwd_ex -- gla_fwd / gla_fwd_f32 (dtype 0 / 1) with the schedule and
- * epsilon exposed, for tests: `chunk` = tokens per chunk (0 = the default
- * of the chosen kernel; otherwise a multiple of 16 that the kernel supports,
- * else GLA_ERR_UNSUPPORTED), `segments` = CTAs per (b, h) pair splitting the
- * scan (0 = automatic, else 1..16; the tensor-core kernel refuses 13, 14 and
- * 15 with GLA_ERR_UNSUPPORTED, as their key-channel groups do not fit its
- * state-exchange buffer), `eps` the RMSNorm epsilon.  Every valid choice
- * computes the same operation (up to rounding order).
+ * gla_fwd_ex -- gla_fwd / gla_fwd_f32 (dtype 0 / 1) with the kernel, the schedule
+ * and epsilon exposed, for tests; the operation of the GTR method section as above.
+ * `chunk` = tokens per chunk (0 = the default of the kernel; otherwise a multiple
+ * of 16 that the kernel supports: up to 128 for GLA_KERNEL_TC128, 64 for the others,
+ * else GLA_ERR_UNSUPPORTED), `segments` = CTAs per (b, h) pair splitting the scan
+ * (0 = automatic, else 1..16; GLA_KERNEL_TC128 refuses 13, 14 and 15), `eps` the
+ * RMSNorm epsilon, `kernel` a gla_kernel (GLA_ERR_UNSUPPORTED when that kernel does
+ * not take this dtype or head dim).  Every valid choice computes the same operation
+ * (up to rounding order).
  */
 int gla_fwd_ex(const void *q, const void *k, const void *v,
                const void *gate_preact, const void *out_gate_preact,
                const float *rms_weight, void *out,
                int B, int H, int grid_h, int grid_w, int d_k, int d_v,
                int direction, int dtype, int chunk, int segments, float eps,
-               void *stream);
+               int kernel, void *stream);
 
 /*
  * gla_get_status -- synchronises `stream`, returns the current device's
  * latched device-side status in *device_status (GLA_OK if none) and clears
- * it.  Returns GLA_ERR_CUDA if the synchronisation itself failed.
+ * it.  Returns GLA_ERR_CUDA if the synchronisation itself failed.  The pages
+ * define no error reporting; the status word is this library's own.
  */
 int gla_get_status(void *stream, int *device_status);
 
@@ -140,7 +158,7 @@ int gla_version(void);
 /*
  * gla_plan -- the schedule gla_fwd (dtype 0) / gla_fwd_f32 (dtype 1) would
  * use for these shapes on the current device, without launching anything:
- * *kernel = 1 (tensor-core kernel) or 2 (CUDA-core kernel), *segments = CTAs
+ * *kernel = the gla_kernel it runs (1, 2 or 3), *segments = CTAs
  * (one thread-block cluster) per (b, h) pair, *seg_len = scan positions per
  * segment, *ctas = total CTAs, *max_active_clusters = clusters of that shape
  * the device can hold at once.  Same argument errors as gla_fwd.
@@ -154,7 +172,7 @@ int gla_plan(int B, int H, int grid_h, int grid_w, int d_k, int d_v, int dtype, 
  * block size, dynamic shared memory, programmatic dependent launch) whose body only
  * performs the dependent-launch handshake.  Timing a run of these gives the per-launch
  * floor of that shape.  Asynchronous on `stream`.  GLA_ERR_SHAPE for non-positive
- * dimensions; GLA_ERR_UNSUPPORTED when those dimensions would not use the tensor-core kernel.
+ * dimensions.
  */
 int gla_empty_launch(int B, int H, int grid_h, int grid_w, void *stream);
 
@@ -169,18 +187,57 @@ int gla_empty_launch(int B, int H, int grid_h, int grid_w, void *stream);
 int gla_selftest_timeout(long long limit_cycles, void *stream);
 
 /*
- * gla_selftest_mma -- diagnostic: runs ONE of the tensor-core kernel's four
- * matrix products on a single CTA, with the kernel's own shared-memory
- * layouts and descriptors, on row-major float32 DEVICE arrays:
- *   kind 0  D[128][128] = A[128][64] * B[128][64]^T   (split tf32: each operand is
- *           held as tf32 high + low parts, three products; ~fp32 accuracy)
- *   kind 1  D[64][64]   = B[128][64]^T * A[128][64]   (fp16 operands, the state product,
- *           kept transposed: A plays the decayed keys, B the values)
- *   kind 2  D[128][64]  = A[128][128] * B[128][64]    (fp16 operands, P * V)
- *   kind 3  D[128][64]  = A[128][64] * B[64][64]^T    (tf32, the inter-chunk product)
- * Inputs are rounded to the operand type (tf32 or fp16; kind 0 splits them)
- * on the way in; accumulation is fp32.  Asynchronous on `stream`.  Returns GLA_ERR_UNSUPPORTED
- * for another kind.  Not part of the operation itself.
+ * gla_selftest_fault -- diagnostic for device-side failure detection in the operator's
+ * own tensor-core kernel: runs gla_fwd (fp16, d_k = d_v = d in {64, 128}, `segments`
+ * CTAs per pair or 0 for automatic) with every bounded wait limited to
+ * `wait_limit_cycles` SM clocks (1 .. 2^34) and the tile loads of full-pass chunk
+ * `withheld_chunk` of every segment never issued (-1: none).  A wait on the withheld
+ * tiles expires, GLA_ERR_TIMEOUT is latched, the CTA skips its remaining waits and
+ * products and returns; `out` is then undefined.  Arguments as gla_fwd; asynchronous.
+ */
+int gla_selftest_fault(const void *q, const void *k, const void *v,
+                       const void *gate_preact, const void *out_gate_preact,
+                       const float *rms_weight, void *out,
+                       int B, int H, int grid_h, int grid_w, int d, int direction,
+                       int segments, long long wait_limit_cycles, int withheld_chunk,
+                       void *stream);
+
+/*
+ * gla_selftest_chunk -- diagnostic: runs ONE of the tensor-core kernel's matrix products
+ * for head dim d in {64, 128} on a single CTA, with the kernel's own shared-memory and
+ * TMEM layouts, descriptors and TMEM accesses, on row-major float32 DEVICE arrays:
+ *   kind 0  D[64][64] = A[64][d] * B[64][d]^T   (scores; each operand split into bf16
+ *           high + low parts, three products: ~2^-16 relative)
+ *   kind 1  D[d][d]   = A[64][d]^T * B[64][d]   (fp16 operands, the chunk-state product)
+ *   kind 2  D[64][d]  = A[64][64] * B[64][d]    (fp16 operands, P * V, A held in TMEM)
+ *   kind 3  D[64][d]  = A[64][d] * B[d][d]      (bf16 split, the inter-chunk product)
+ * Inputs are rounded to the operand type on the way in; accumulation is fp32.
+ * Asynchronous on `stream`.  Not part of the operation itself.
+ */
+int gla_selftest_chunk(int d, int kind, const float *A, const float *B, float *D, void *stream);
+
+/*
+ * gla_selftest_load -- diagnostic: loads the five 64-row tiles (q, k, gate_preact, v,
+ * out_gate_preact, fp16 DEVICE arrays laid out as for gla_fwd with d_k = d_v = d in
+ * {64, 128}) of chunk `chunk` of the scan of pair (b, h) = (0, 0) in `direction` (0..3) with
+ * the tensor-core kernel's TMA boxes, and writes them to out[5][64][d] (DEVICE float32) in
+ * tile-row order, with info[0] = the chunk's token count n and info[1 + i] = the spatial
+ * index of tile row i (-1 for rows past the chunk) (DEVICE int[65]).  Chunks are the kernel's
+ * default ones (lines cut into pieces of at most 64 positions).  Asynchronous on `stream`.
+ * Not part of the operation itself.
+ */
+int gla_selftest_load(const void *q, const void *k, const void *gate_preact, const void *v,
+                      const void *out_gate_preact, int B, int H, int grid_h, int grid_w, int d,
+                      int direction, int chunk, float *out, int *info, void *stream);
+
+/*
+ * gla_selftest_mma -- diagnostic: runs ONE of the four matrix products of the previous
+ * 128-row tensor-core kernel on a single CTA, on row-major float32 DEVICE arrays:
+ *   kind 0  D[128][128] = A[128][64] * B[128][64]^T   (split tf32)
+ *   kind 1  D[64][64]   = B[128][64]^T * A[128][64]   (fp16)
+ *   kind 2  D[128][64]  = A[128][128] * B[128][64]    (fp16)
+ *   kind 3  D[128][64]  = A[128][64] * B[64][64]^T    (tf32)
+ * Asynchronous on `stream`.  Returns GLA_ERR_UNSUPPORTED for another kind.
  */
 int gla_selftest_mma(int kind, const float *A, const float *B, float *D, void *stream);
 

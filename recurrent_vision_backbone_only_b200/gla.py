@@ -48,7 +48,7 @@ def load() -> ctypes.CDLL:
         lib.gla_fwd.argtypes = common + [vp]
         lib.gla_fwd_f32.argtypes = common + [vp]
         lib.gla_fwd_host.argtypes = common + [i, vp]
-        lib.gla_fwd_ex.argtypes = common + [i, i, i, f, vp]
+        lib.gla_fwd_ex.argtypes = common + [i, i, i, f, i, vp]
         lib.gla_get_status.argtypes = [vp, ctypes.POINTER(ctypes.c_int)]
         lib.gla_status_string.argtypes = [i]
         lib.gla_status_string.restype = ctypes.c_char_p
@@ -61,6 +61,13 @@ def load() -> ctypes.CDLL:
         ip = ctypes.POINTER(ctypes.c_int)
         lib.gla_plan.argtypes = [i] * 7 + [ip] * 5
         lib.gla_plan.restype = ctypes.c_int
+        ll = ctypes.c_longlong
+        lib.gla_selftest_chunk.argtypes = [i, i, vp, vp, vp, vp]
+        lib.gla_selftest_chunk.restype = ctypes.c_int
+        lib.gla_selftest_load.argtypes = [vp] * 5 + [i] * 7 + [vp, vp, vp]
+        lib.gla_selftest_load.restype = ctypes.c_int
+        lib.gla_selftest_fault.argtypes = [vp] * 7 + [i] * 7 + [ll, i, vp]
+        lib.gla_selftest_fault.restype = ctypes.c_int
         for fn in (lib.gla_fwd, lib.gla_fwd_f32, lib.gla_fwd_host, lib.gla_fwd_ex,
                    lib.gla_get_status, lib.gla_version, lib.gla_selftest_mma):
             fn.restype = ctypes.c_int
@@ -144,16 +151,21 @@ def gla_fwd(q, k, v, a, g, w, out, grid_h: int, grid_w: int, direction: int, str
     return out
 
 
+KERNEL_AUTO, KERNEL_TC128, KERNEL_SIMT, KERNEL_TC64 = 0, 1, 2, 3
+KERNEL_NAMES = {1: "tensor-core 128-row", 2: "cuda-core", 3: "tensor-core 64-row"}
+
+
 def gla_fwd_ex(q, k, v, a, g, w, out, grid_h: int, grid_w: int, direction: int,
-               chunk: int = 0, segments: int = 0, eps: float = 1e-6, stream=None):
-    """gla_fwd with the chunk length, segments per pair and epsilon exposed (tests)."""
+               chunk: int = 0, segments: int = 0, eps: float = 1e-6, kernel: int = 0,
+               stream=None):
+    """gla_fwd with the kernel, chunk length, segments per pair and epsilon exposed (tests)."""
     import torch
     B, H, dk, dv = _dims(q, v, grid_h, grid_w)
     _check_tensors(q, k, v, a, g, w, out, q.dtype)
     dtype = _dtype_code(q)
     args = [ctypes.c_void_p(t.data_ptr()) for t in (q, k, v, a, g, w, out)]
     args += [B, H, grid_h, grid_w, dk, dv, direction, dtype, chunk, segments,
-             ctypes.c_float(eps), _stream_ptr(stream)]
+             ctypes.c_float(eps), kernel, _stream_ptr(stream)]
     _check(load().gla_fwd_ex(*args), "gla_fwd_ex")
     return out
 
@@ -183,7 +195,7 @@ def plan(B: int, H: int, grid_h: int, grid_w: int, d_k: int = 64, d_v: int = 64,
     _check(load().gla_plan(B, H, grid_h, grid_w, d_k, d_v, dtype, *[ctypes.byref(v) for v in vals]),
            "gla_plan")
     kernel, segs, seg_len, ctas, mac = (v.value for v in vals)
-    return {"kernel": {1: "tensor-core", 2: "cuda-core"}.get(kernel, kernel), "segments": segs,
+    return {"kernel": KERNEL_NAMES.get(kernel, kernel), "segments": segs,
             "seg_len": seg_len, "ctas": ctas, "max_active_clusters": mac}
 
 

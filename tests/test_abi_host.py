@@ -57,7 +57,7 @@ def call(fn, ptrs=None, B=1, H=2, gh=4, gw=5, dk=64, dv=64, direction=0, extra=(
 
 @pytest.mark.parametrize("fn,extra", [("gla_fwd", ()), ("gla_fwd_f32", ()),
                                       ("gla_fwd_host", (0,)),
-                                      ("gla_fwd_ex", (0, 0, 0, ctypes.c_float(1e-6)))])
+                                      ("gla_fwd_ex", (0, 0, 0, ctypes.c_float(1e-6), 0))])
 def test_argument_errors(lib, fn, extra):
     for i in range(7):
         ptrs = list(ALIGNED)
@@ -108,10 +108,11 @@ def test_plan_rejects_bad_arguments(lib):
 
 
 def test_ex_rejects_bad_schedule(lib):
-    bad = [(5, 0, 0), (0, 0, 17), (0, -1, 0), (1, 0, -2)]   # dtype, chunk, segments
-    for dtype, chunk, segs in bad:
-        rc = call("gla_fwd_ex", extra=(dtype, chunk, segs, ctypes.c_float(1e-6)))
-        assert rc == 3 or (rc == 9 and dtype in (0, 1)), (dtype, chunk, segs, rc)
+    bad = [(5, 0, 0, 0), (0, 0, 17, 0), (0, -1, 0, 0), (1, 0, -2, 0),   # dtype, chunk, segs,
+           (0, 0, 0, 4), (0, 0, 0, -1), (1, 0, 0, 1), (1, 0, 0, 3)]          # kernel
+    for dtype, chunk, segs, kernel in bad:
+        rc = call("gla_fwd_ex", extra=(dtype, chunk, segs, ctypes.c_float(1e-6), kernel))
+        assert rc == 3, (dtype, chunk, segs, kernel, rc)
 
 
 def test_no_device_is_reported_not_faked(lib):

@@ -3,8 +3,8 @@
 Tolerances (on u, the kernel's final output): fp16 I/O with fp32
 accumulation -- max-abs <= 1e-2 and relative L2 <= 2e-3; fp32 I/O -- max-abs
 <= 1e-5.  Every workload runs at its full size in the launch configuration
-the bench uses; the stress workload (L = 16384, d = 128) is compared on
-sampled (b, h) pairs, each of which the oracle recomputes from scratch.
+the bench uses, and every element of every output is compared with the oracle
+(the stress workload, L = 16384 and d = 128, included).
 """
 import os
 
@@ -24,13 +24,16 @@ def torch_dev(x):
     return torch.from_numpy(np.ascontiguousarray(x)).cuda()
 
 
-def run_gpu(x, gh, gw, direction, chunk=0, segments=0, eps=1e-6):
+TC128, SIMT, TC64 = gla.KERNEL_TC128, gla.KERNEL_SIMT, gla.KERNEL_TC64
+
+
+def run_gpu(x, gh, gw, direction, chunk=0, segments=0, eps=1e-6, kernel=0):
     import torch
     t = {n: torch_dev(x[n]) for n in ("q", "k", "v", "a", "g", "w")}
     out = torch.empty_like(t["v"])
-    if chunk or segments or eps != 1e-6:
+    if chunk or segments or eps != 1e-6 or kernel:
         gla.gla_fwd_ex(t["q"], t["k"], t["v"], t["a"], t["g"], t["w"], out, gh, gw, direction,
-                       chunk=chunk, segments=segments, eps=eps)
+                       chunk=chunk, segments=segments, eps=eps, kernel=kernel)
     else:
         gla.gla_fwd(t["q"], t["k"], t["v"], t["a"], t["g"], t["w"], out, gh, gw, direction)
     torch.cuda.synchronize()
@@ -83,37 +86,37 @@ def test_tiny_fp32(direction):
     assert_close(u2, oracle_ref(x, wl.grid_h, wl.grid_w, direction), "f32")
 
 
+@pytest.mark.parametrize("kernel", [0, TC64])
 @pytest.mark.parametrize("name", ["gtr640", "highres"])
-def test_full_workloads_all_directions(name):
+def test_full_workloads_all_directions(name, kernel):
+    # kernel 0: the one gla_fwd picks (the 128-row tensor-core kernel at d = 64)
     wl = synth.WORKLOADS[name]
     x = synth.make_inputs(wl)
     for d in wl.directions:
-        assert_close(run_gpu(x, wl.grid_h, wl.grid_w, d), oracle_ref(x, wl.grid_h, wl.grid_w, d),
-                     wl.dtype)
+        assert_close(run_gpu(x, wl.grid_h, wl.grid_w, d, kernel=kernel),
+                     oracle_ref(x, wl.grid_h, wl.grid_w, d), wl.dtype)
 
 
-def test_batched_cycle():
+@pytest.mark.parametrize("kernel", [0, TC64])
+def test_batched_cycle(kernel):
     wl = synth.WORKLOADS["batched"]
     x = synth.make_inputs(wl)
-    u = run_gpu(x, wl.grid_h, wl.grid_w, 4)
+    u = run_gpu(x, wl.grid_h, wl.grid_w, 4, kernel=kernel)
     assert_close(u, oracle_ref(x, wl.grid_h, wl.grid_w, 4), wl.dtype)
 
 
 @pytest.mark.parametrize("direction", [2, 3])
-def test_stress_sampled_pairs(direction):
+def test_stress_all_pairs(direction):
+    # every (b, h) pair of the 128x128, d = 128 workload against one oracle call
     wl = synth.WORKLOADS["stress"]
     x = synth.make_inputs(wl)
     u = run_gpu(x, wl.grid_h, wl.grid_w, direction)
-    assert np.all(np.isfinite(u.astype(np.float32)))
-    for b, h in [(0, 0), (1, 5)]:
-        xs = {n: x[n][b:b + 1, :, h:h + 1] for n in ("q", "k", "v", "a", "g")}
-        xs["w"] = x["w"]
-        ref = oracle_ref(xs, wl.grid_h, wl.grid_w, direction)
-        assert_close(u[b:b + 1, :, h:h + 1], ref, wl.dtype)
+    assert_close(u, oracle_ref(x, wl.grid_h, wl.grid_w, direction), wl.dtype)
 
 
-@pytest.mark.parametrize("dtype", ["f16", "f32"])
-def test_chunk_and_segment_invariance(dtype):
+@pytest.mark.parametrize("dtype,kernel", [("f16", TC128), ("f16", TC64), ("f16", SIMT),
+                                          ("f32", SIMT)])
+def test_chunk_and_segment_invariance(dtype, kernel):
     wl = synth.WORKLOADS["gtr640"].with_(H=2, dtype=dtype, grid_h=24, grid_w=37)
     x = synth.make_inputs(wl)
     gh, gw = wl.grid_h, wl.grid_w
@@ -121,7 +124,7 @@ def test_chunk_and_segment_invariance(dtype):
     outs = []
     for chunk in (16, 32, 64):
         for segs in (1, 3, 16):
-            u = run_gpu(x, gh, gw, 1, chunk=chunk, segments=segs)
+            u = run_gpu(x, gh, gw, 1, chunk=chunk, segments=segs, kernel=kernel)
             assert_close(u, ref, dtype)
             outs.append(u.astype(np.float64))
     for u in outs[1:]:
@@ -187,43 +190,61 @@ def test_eps_is_honoured():
         assert_close(u, ref, "f32")
 
 
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("segs", [2, 5, 7, 12, 13, 15, 16])
+def test_segment_counts_64_row_kernel(segs, d):
+    # the state exchange deals key channel c to scanner c % segs: counts that do not divide d
+    # give scanners unequal channel counts.  chunk 64 gives segments of one or two chunks,
+    # chunk 16 segments of several (state-only pass, exchange, full pass)
+    wl = synth.WORKLOADS["gtr640"].with_(H=2, grid_h=24, grid_w=37, d_k=d, d_v=d)
+    x = synth.make_inputs(wl, seed=segs)
+    ref = oracle_ref(x, 24, 37, 2)
+    for chunk in (16, 64):
+        assert_close(run_gpu(x, 24, 37, 2, chunk=chunk, segments=segs, kernel=TC64), ref, "f16")
+
+
 @pytest.mark.parametrize("segs", [2, 5, 7, 12])
-def test_segment_counts_sharing_channel_groups(segs):
-    # the state exchange splits the 16 four-channel groups over the segments; counts that do
-    # not divide 16 give some scanners two or more groups.  chunk 128 keeps each segment in one
-    # chunk (exchange mid-chunk, S~ written directly); chunk 32 gives several chunks per
-    # segment (state-only pass, exchange, S_in read back)
+def test_segment_counts_128_row_kernel(segs):
+    # the 128-row kernel splits the 16 four-channel key groups over the segments; counts that
+    # do not divide 16 give some scanners two or more groups.  chunk 128 keeps each segment in
+    # one chunk (exchange mid-chunk), chunk 32 gives several chunks per segment
     wl = synth.WORKLOADS["gtr640"].with_(H=2, grid_h=24, grid_w=37)
     x = synth.make_inputs(wl, seed=segs)
     ref = oracle_ref(x, 24, 37, 2)
     for chunk in (32, 128):
-        assert_close(run_gpu(x, 24, 37, 2, chunk=chunk, segments=segs), ref, "f16")
+        assert_close(run_gpu(x, 24, 37, 2, chunk=chunk, segments=segs, kernel=TC128), ref, "f16")
 
 
-@pytest.mark.parametrize("segs", [13, 14, 15])
-def test_segment_counts_beyond_the_exchange_buffer_are_refused(segs):
+@pytest.mark.parametrize("kernel,chunk,segs,d", [(TC64, 128, 0, 64), (TC64, 40, 0, 64), (TC64, 64, 17, 64),
+                                                 (TC128, 0, 13, 64), (TC128, 0, 15, 64),
+                                                 (TC128, 144, 0, 64), (TC128, 0, 0, 128)])
+def test_unsupported_schedules_are_refused(kernel, chunk, segs, d):
     import torch
-    wl = synth.WORKLOADS["gtr640"].with_(H=1, grid_h=16, grid_w=16)
+    wl = synth.WORKLOADS["gtr640"].with_(H=1, grid_h=16, grid_w=16, d_k=d, d_v=d)
     x = synth.make_inputs(wl, seed=1)
     t = {n: torch_dev(x[n]) for n in ("q", "k", "v", "a", "g", "w")}
     out = torch.empty_like(t["v"])
     with pytest.raises(gla.GLAError):
         gla.gla_fwd_ex(t["q"], t["k"], t["v"], t["a"], t["g"], t["w"], out, 16, 16, 0,
-                       chunk=128, segments=segs)
+                       chunk=chunk, segments=segs, kernel=kernel)
 
 
-@pytest.mark.parametrize("segs,chunk", [(3, 128), (16, 128), (5, 32)])
-def test_extreme_gates_with_exchange(segs, chunk):
-    # gates of -30 make a chunk's decay range exceed what the tf32 score operands carry, so
-    # P is evaluated exactly on CUDA cores; combined here with the cluster state exchange
-    # (one chunk per segment: mid-chunk exchange; chunk 32: state-only pass first)
-    wl = synth.WORKLOADS["gtr640"].with_(grid_h=16, grid_w=20, H=2)
+@pytest.mark.parametrize("kernel,d,segs,chunk", [(TC64, 64, 3, 64), (TC64, 64, 16, 64),
+                                                 (TC64, 64, 5, 32), (TC64, 128, 3, 64),
+                                                 (TC64, 128, 16, 64), (TC64, 128, 5, 32),
+                                                 (TC128, 64, 3, 128), (TC128, 64, 16, 128),
+                                                 (TC128, 64, 5, 32)])
+def test_extreme_gates_with_exchange(kernel, d, segs, chunk):
+    # gates of -30 make a chunk's decay range exceed what the 16-bit (64-row kernel) or tf32
+    # (128-row kernel) score operands carry, so P is evaluated exactly on CUDA cores; combined
+    # here with the cluster state exchange
+    wl = synth.WORKLOADS["gtr640"].with_(grid_h=16, grid_w=20, H=2, d_k=d, d_v=d)
     x = synth.make_inputs(wl, seed=7)
     rng = np.random.default_rng(7)
     x["a"] = np.where(rng.random(x["a"].shape) < 0.5, -30.0, 30.0).astype(x["a"].dtype)
-    for d in (1, 3):
-        assert_close(run_gpu(x, 16, 20, d, chunk=chunk, segments=segs), oracle_ref(x, 16, 20, d),
-                     "f16")
+    for dr in (1, 3):
+        assert_close(run_gpu(x, 16, 20, dr, chunk=chunk, segments=segs, kernel=kernel),
+                     oracle_ref(x, 16, 20, dr), "f16")
 
 
 def test_empty_launch_runs_clean():
@@ -235,14 +256,16 @@ def test_empty_launch_runs_clean():
     assert gla.raw_call("gla_empty_launch", 0, 1, 1, 1, None) == 2      # GLA_ERR_SHAPE
 
 
-@pytest.mark.parametrize("gh,gw,chunk,segs", [(16, 20, 32, 9), (42, 50, 128, 16), (42, 50, 0, 0)])
-def test_shorter_last_segment_of_one_chunk(gh, gw, chunk, segs):
-    # segments of several chunks whose last, shorter segment fits one chunk (16x20: 9
-    # segments of 36 tokens with chunk 32, the last of 32; 42x50: 16 segments of 132, the
-    # last of 120; and the automatic plan for 42x50): every CTA of a cluster must take the
-    # same exchange layout
+@pytest.mark.parametrize("kernel,gh,gw,chunk,segs", [(TC128, 16, 20, 32, 9), (TC128, 42, 50, 128, 16),
+                                                     (TC128, 42, 50, 0, 0), (TC64, 16, 20, 32, 9),
+                                                     (TC64, 42, 50, 64, 16), (TC64, 42, 50, 0, 0)])
+def test_shorter_last_segment(kernel, gh, gw, chunk, segs):
+    # a last segment shorter than the others (128-row kernel, 16x20: 9 segments of 36 tokens
+    # with chunk 32, the last of 32; 42x50: 16 segments of 132, the last of 120; and the
+    # automatic plan).  For the 128-row kernel every CTA of a cluster must take the same
+    # exchange layout; for the 64-row kernel the last segment holds fewer chunks.
     wl = synth.WORKLOADS["gtr640"].with_(H=2, grid_h=gh, grid_w=gw)
     x = synth.make_inputs(wl, seed=gh + gw)
-    for d in (0, 2):
-        assert_close(run_gpu(x, gh, gw, d, chunk=chunk, segments=segs), oracle_ref(x, gh, gw, d),
-                     "f16")
+    for dr in (0, 2):
+        assert_close(run_gpu(x, gh, gw, dr, chunk=chunk, segments=segs, kernel=kernel),
+                     oracle_ref(x, gh, gw, dr), "f16")
