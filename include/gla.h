@@ -188,19 +188,29 @@ int gla_selftest_timeout(long long limit_cycles, void *stream);
 
 /*
  * gla_selftest_fault -- diagnostic for device-side failure detection in the operator's
- * own tensor-core kernel: runs gla_fwd (fp16, d_k = d_v = d in {64, 128}, `segments`
- * CTAs per pair or 0 for automatic) with every bounded wait limited to
- * `wait_limit_cycles` SM clocks (1 .. 2^34) and the tile loads of full-pass chunk
- * `withheld_chunk` of every segment never issued (-1: none).  A wait on the withheld
- * tiles expires, GLA_ERR_TIMEOUT is latched, the CTA skips its remaining waits and
- * products and returns; `out` is then undefined.  Arguments as gla_fwd; asynchronous.
+ * own tensor-core kernels: runs gla_fwd (fp16, d_k = d_v = d) on `kernel`
+ * (GLA_KERNEL_TC128 with d = 64, or GLA_KERNEL_TC64 with d in {64, 128}; `segments` CTAs
+ * per pair or 0 for automatic) with every bounded wait limited to `wait_limit_cycles` SM
+ * clocks (1 .. 2^34), while the loads of full-pass chunk `withheld_chunk` of every segment
+ * never complete their barrier (-1: none): the 64-row kernel does not issue them, the
+ * 128-row kernel issues the q / k copies without their barrier arrival.  The wait on those
+ * tiles expires, GLA_ERR_TIMEOUT is latched, the CTA skips its remaining waits and products,
+ * drains what is in flight and returns; `out` is then undefined.  Arguments as gla_fwd;
+ * asynchronous.
  */
 int gla_selftest_fault(const void *q, const void *k, const void *v,
                        const void *gate_preact, const void *out_gate_preact,
                        const float *rms_weight, void *out,
                        int B, int H, int grid_h, int grid_w, int d, int direction,
                        int segments, long long wait_limit_cycles, int withheld_chunk,
-                       void *stream);
+                       int kernel, void *stream);
+
+/*
+ * gla_selftest_rcp -- diagnostic: y[i] = the 128-row kernel's Newton-Raphson reciprocal of
+ * x[i] (n DEVICE floats each), for an error-bound test against 1/x.  The pages have no
+ * counterpart; asynchronous on `stream`.
+ */
+int gla_selftest_rcp(const float *x, float *y, int n, void *stream);
 
 /*
  * gla_selftest_chunk -- diagnostic: runs ONE of the tensor-core kernel's matrix products

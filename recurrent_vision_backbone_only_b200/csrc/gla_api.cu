@@ -303,7 +303,7 @@ int run_simt(const Args &x, int chunk, int segs, float eps, cudaStream_t st, con
 // ---------------------------------------------------------- tensor-core path
 // fp16 I/O with d_k = d_v = 64.  One cluster of `segs` CTAs per (b, h) pair.
 int run_tc(const Args &x, int chunk, int segs, float eps, cudaStream_t st, const DeviceInfo &di,
-           Plan *query) {
+           Plan *query, long long wait_limit = 1LL << 32, int fault_chunk = -1) {
     auto kern = tc::gla_tc_kernel<64, false>;
     const int L = x.gh * x.gw;
     const int n_pairs = x.B * x.H;
@@ -332,6 +332,8 @@ int run_tc(const Args &x, int chunk, int segs, float eps, cudaStream_t st, const
     p.B = x.B; p.H = x.H; p.gh = x.gh; p.gw = x.gw; p.L = L; p.dir = x.dir;
     p.segs = pl.segs; p.seg_len = pl.seg_len; p.chunk_max = chunk;
     p.eps = eps; p.scale = 0.125f;  // 64^{-1/2}
+    p.wait_limit = wait_limit;
+    p.fault_chunk = fault_chunk;
     // every segment one chunk and several segments: the instantiation with only the
     // mid-chunk exchange path (same resources and launch shape as the planned one)
     auto launch = kern;
@@ -820,9 +822,11 @@ int gla_selftest_load(const void *q, const void *k, const void *gate_preact, con
 int gla_selftest_fault(const void *q, const void *k, const void *v, const void *gate_preact,
                        const void *out_gate_preact, const float *rms_weight, void *out, int B, int H,
                        int grid_h, int grid_w, int d, int direction, int segments,
-                       long long wait_limit_cycles, int withheld_chunk, void *stream) {
+                       long long wait_limit_cycles, int withheld_chunk, int kernel, void *stream) {
     if (wait_limit_cycles <= 0 || wait_limit_cycles > (1LL << 34)) return GLA_ERR_UNSUPPORTED;
     if (d != 64 && d != 128) return GLA_ERR_UNSUPPORTED;
+    if (kernel != kTc128 && kernel != kTc64) return GLA_ERR_UNSUPPORTED;
+    if (kernel == kTc128 && d != 64) return GLA_ERR_UNSUPPORTED;
     const Args x = make_args(q, k, v, gate_preact, out_gate_preact, rms_weight, out, B, H, grid_h, grid_w,
                              d, d, direction, 2);
     int rc = validate(x);
@@ -832,8 +836,22 @@ int gla_selftest_fault(const void *q, const void *k, const void *v, const void *
     rc = current_device_info(&di);
     if (rc != GLA_OK) return rc;
     const cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (kernel == kTc128) {
+        if (segments > 0 && !tc_segs_ok(segments)) return GLA_ERR_UNSUPPORTED;
+        return run_tc(x, 0, segments, kEps, st, di, nullptr, wait_limit_cycles, withheld_chunk);
+    }
     if (d == 64) return run_chunk<64>(x, 0, segments, kEps, st, di, nullptr, wait_limit_cycles, withheld_chunk);
     return run_chunk<128>(x, 0, segments, kEps, st, di, nullptr, wait_limit_cycles, withheld_chunk);
+}
+
+int gla_selftest_rcp(const float *x, float *y, int n, void *stream) {
+    if (!x || !y) return GLA_ERR_NULL;
+    if (n <= 0) return GLA_ERR_SHAPE;
+    DeviceInfo di;
+    int rc = current_device_info(&di);
+    if (rc != GLA_OK) return rc;
+    tc::gla_rcp_selftest_kernel<<<(n + 255) / 256, 256, 0, static_cast<cudaStream_t>(stream)>>>(x, y, n);
+    return cudaGetLastError() == cudaSuccess ? GLA_OK : GLA_ERR_CUDA;
 }
 
 int gla_selftest_mma(int kind, const float *A, const float *B, float *D, void *stream) {

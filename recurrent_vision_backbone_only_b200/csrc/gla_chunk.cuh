@@ -368,8 +368,9 @@ __device__ __noinline__ void exact_p(const uint8_t *sm, uint32_t stage, uint32_t
 }
 
 // =========================================================================== kernel
+// d = 64: two CTAs per SM, which the register file holds only below 128 registers a thread.
 template <int D>
-__global__ void __launch_bounds__(Cfg<D>::kThreads, D == 64 ? 2 : 1)
+__global__ void __launch_bounds__(Cfg<D>::kThreads, 1) __maxnreg__(D == 64 ? 120 : 128)
     gla_chunk_kernel(const __grid_constant__ Maps maps, const Params p) {
     using C = Cfg<D>;
     extern __shared__ uint8_t smem_raw[];

@@ -110,6 +110,8 @@ struct Params {
     int seg_len;   // scan positions per segment
     int chunk_max; // largest chunk (16..128); a segment is split into equal chunks
     float eps, scale;
+    long long wait_limit;  // bound of every mbarrier wait, SM clocks
+    int fault_chunk;       // test hook: full-pass chunk whose q/k loads never signal (-1: none)
 };
 
 // ------------------------------------------------------- operand addressing
@@ -187,25 +189,31 @@ __device__ __forceinline__ void issue_inter(uint32_t sbase, uint32_t tmem, bool 
     }
 }
 
-// Bounded wait on an mbarrier phase; on expiry latch GLA_ERR_TIMEOUT and return false.
-__device__ __forceinline__ bool wait_phase(uint64_t *bar, uint32_t parity) {
+// Bounded wait on an mbarrier phase, `limit` SM clocks.  Once a wait of the CTA has expired
+// (*abort set) it returns false at once; on expiry it latches GLA_ERR_TIMEOUT and sets *abort.
+__device__ __forceinline__ bool wait_phase(uint64_t *bar, uint32_t parity, long long limit,
+                                           volatile int *abort) {
+    if (*abort) return false;
     const long long start = clock64();
     while (!ptx::mbar_try_wait(bar, parity)) {
-        if (clock64() - start > (1LL << 32)) {
+        if (clock64() - start > limit) {
             raise_status(7 /* GLA_ERR_TIMEOUT */);
+            *abort = 1;
             return false;
         }
     }
     return true;
 }
 
-// log2 of the retention gate: log2(sigma(a)) / 16, stable for either sign of a.
-// Bounded wait with cluster-scope acquire (data pushed by other CTAs of the cluster).
-__device__ __forceinline__ bool wait_cluster_phase(uint64_t *bar, uint32_t parity) {
+// The same with cluster-scope acquire (data pushed by other CTAs of the cluster).
+__device__ __forceinline__ bool wait_cluster_phase(uint64_t *bar, uint32_t parity, long long limit,
+                                                   volatile int *abort) {
+    if (*abort) return false;
     const long long start = clock64();
     while (!ptx::mbar_try_wait_cluster(bar, parity)) {
-        if (clock64() - start > (1LL << 32)) {
+        if (clock64() - start > limit) {
             raise_status(7 /* GLA_ERR_TIMEOUT */);
+            *abort = 1;
             return false;
         }
     }
@@ -217,10 +225,13 @@ __device__ __forceinline__ float log2_gamma(float a) {
     return (fminf(a, 0.0f) * kLog2e - ptx::lg2(1.0f + x)) * kInvTau;
 }
 
-// 1/x for a positive normal x on the FMA pipe: Newton-Raphson, y <- y + y (1 - x y), from the
-// seed obtained by subtracting the bit pattern of x from a constant (the exponent is negated
-// and the mantissa linearly approximated: relative error below 6%); three steps square the
-// error each time, to about 1 ulp.  Used where the special-function unit is the busier pipe.
+// 1/x for a positive normal x on the FMA pipe: Newton-Raphson, y <- y + y (1 - x y), from an
+// integer-subtraction seed.  Reading the float bits of x as an integer, C - bits(x) negates the
+// exponent and replaces the mantissa m in [0, 1) by a linear function of it, so the seed is a
+// piecewise-linear approximation of 1/x on every binade.  C = 0x7EF311C7 is the constant that
+// minimises the seed's largest relative error over a binade (found by a direct search over C:
+// 5.05%); each Newton step squares the error, so three steps reach fp32 rounding.  Used where
+// the special-function unit is the busier pipe.
 __device__ __forceinline__ float rcp_nr(float x) {
     float y = __uint_as_float(0x7EF311C7u - __float_as_uint(x));
 #pragma unroll
@@ -241,6 +252,7 @@ __device__ __forceinline__ uint32_t pack_half2(float lo, float hi) {
 // Shared scratch scalars.
 struct Misc {
     uint64_t mbar_mma[4];     // [0] state, [1] scores, [2] inter (+ P.V), [3] P.V (one chunk)
+    uint64_t mbar_end;        // teardown after an expired wait: products still in flight
     uint64_t mbar_ld[3];      // [0] a tile, [1] q and k tiles, [2] v and g tiles
     uint64_t mbar_x[2];       // exchange: [0] aggregates received, [1] S~ / S_in received
     uint32_t tmem_base;
@@ -363,6 +375,7 @@ __global__ void __launch_bounds__(kThreads, 1) gla_tc_kernel(const Params p) {
     // ---- setup: barriers and weight; TMEM is allocated once the first gathers are in flight
     if (tid == 0) {
         for (int i = 0; i < 4; ++i) ptx::mbar_init(&m.mbar_mma[i], 1);
+        ptx::mbar_init(&m.mbar_end, 3);       // one commit from each MMA-issuing warp (0, 4, 7)
         for (int i = 0; i < 3; ++i) ptx::mbar_init(&m.mbar_ld[i], kThreads);
         ptx::fence_mbarrier_init();
         m.abort = 0;
@@ -403,16 +416,16 @@ __global__ void __launch_bounds__(kThreads, 1) gla_tc_kernel(const Params p) {
     for (int j = 0; j < 32; ++j) S[j] = 0.0f;
     float Sl[32];
 
-    auto wait_bar = [&](uint64_t *bar, uint32_t parity) {
-        if (!wait_phase(bar, parity)) m.abort = 1;
-    };
+    volatile int *abort_flag = &m.abort;
+    auto wait_bar = [&](uint64_t *bar, uint32_t parity) { wait_phase(bar, parity, p.wait_limit, abort_flag); };
     // ------------------------------------------------------------ loads
     auto set_rows = [&](int c0, int n, int rb) {
         if (tid < n) m.rows[rb][tid] = (bb * p.L + spatial_of(dir, c0 + tid, p.gh, p.gw)) * p.H + hh;
     };
     // issue the chunk's gathers (fp16 [n rows][64] tiles, rows >= n zero-filled) into the
     // swizzled layout; completion is tracked per group on mbar_ld[0..2]
-    auto issue_loads = [&](int n, bool full, int rb) {
+    // `withhold`: test hook, the q/k group never signals its barrier (its wait then expires)
+    auto issue_loads = [&](int n, bool full, int rb, bool withhold) {
         size_t goff[4];
         uint32_t soff[4], bytes[4];
 #pragma unroll
@@ -431,7 +444,7 @@ __global__ void __launch_bounds__(kThreads, 1) gla_tc_kernel(const Params p) {
         ptx::cp_async_mbar_arrive_noinc(&m.mbar_ld[0]);
         tile(p.k, kTK);
         if (full) tile(p.q, kTQ);
-        ptx::cp_async_mbar_arrive_noinc(&m.mbar_ld[1]);
+        if (!withhold) ptx::cp_async_mbar_arrive_noinc(&m.mbar_ld[1]);
         tile(p.v, kTV);
         if (full) tile(p.g, kTG);
         ptx::cp_async_mbar_arrive_noinc(&m.mbar_ld[2]);
@@ -783,7 +796,7 @@ __global__ void __launch_bounds__(kThreads, 1) gla_tc_kernel(const Params p) {
     // whole 128-byte destination rows per store.
     auto xchg_scan = [&](bool direct) {
         if (warp >= 4) return;                        // warp-uniform
-        if (!wait_cluster_phase(&m.mbar_x[0], 0)) m.abort = 1;
+        wait_cluster_phase(&m.mbar_x[0], 0, p.wait_limit, abort_flag);
         const int segs = p.segs;
         const uint32_t lbar = ptx::smem_u32(&m.mbar_x[1]);
         for (int idx = tid; idx < my_groups * kD; idx += 128) {
@@ -817,7 +830,7 @@ __global__ void __launch_bounds__(kThreads, 1) gla_tc_kernel(const Params p) {
     // wait for this CTA's incoming state S_in (channel-major, g tile) before a multi-chunk pass
     // and read it back into the state owners' registers
     auto xchg_wait_sin = [&]() {
-        if (!wait_cluster_phase(&m.mbar_x[1], 0)) m.abort = 1;
+        wait_cluster_phase(&m.mbar_x[1], 0, p.wait_limit, abort_flag);
         if (s_owner) {
             const float *Sin = reinterpret_cast<const float *>(sm + kTG);
 #pragma unroll
@@ -843,7 +856,7 @@ __global__ void __launch_bounds__(kThreads, 1) gla_tc_kernel(const Params p) {
         const int n1 = min(chunk_len, p1 - c1);
         set_rows(c1, n1, rb ^ 1);
         __syncthreads();
-        issue_loads(n1, full, rb ^ 1);
+        issue_loads(n1, full, rb ^ 1, full && ci + 1 == p.fault_chunk);
         preloaded = true;
     };
     for (int step = 0; step < n_pass1 + n_chunks; ++step) {
@@ -862,7 +875,7 @@ __global__ void __launch_bounds__(kThreads, 1) gla_tc_kernel(const Params p) {
                 __syncthreads();
                 set_rows(c0, n, rb);
                 __syncthreads();
-                issue_loads(n, !pass1, rb);
+                issue_loads(n, !pass1, rb, !pass1 && ci == p.fault_chunk);
             }
             preloaded = false;
             if (tid == 0) m.slow = 0;               // read only after the gate's barriers
@@ -887,7 +900,7 @@ __global__ void __launch_bounds__(kThreads, 1) gla_tc_kernel(const Params p) {
         // products are issued only after this CTA has arrived on the cluster barrier.
         if (warp == 0 && ptx::elect_one()) {
             ptx::tc_fence_after_sync();
-            issue_state(sbase, tmem);
+            if (!*abort_flag) issue_state(sbase, tmem);
             ptx::mma_commit(&m.mbar_mma[0]);
         }
         wait_mma(0);
@@ -911,7 +924,7 @@ __global__ void __launch_bounds__(kThreads, 1) gla_tc_kernel(const Params p) {
         // states and the other warps compute SiLU(g) * w for their TMEM lane quarters
         if (warp == 7 && ptx::elect_one()) {
             ptx::tc_fence_after_sync();
-            if (!m.slow) issue_qk(sbase, tmem, min(kC, (n + 15) & ~15));
+            if (!m.slow && !*abort_flag) issue_qk(sbase, tmem, min(kC, (n + 15) & ~15));
             ptx::mma_commit(&m.mbar_mma[1]);
         }
         if (mid_xchg) {
@@ -933,7 +946,7 @@ __global__ void __launch_bounds__(kThreads, 1) gla_tc_kernel(const Params p) {
             __syncthreads();                         // S~ complete
             if (warp == 4 && ptx::elect_one()) {
                 ptx::tc_fence_after_sync();
-                issue_inter(sbase, tmem, false);
+                if (!*abort_flag) issue_inter(sbase, tmem, false);
                 ptx::mma_commit(&m.mbar_mma[2]);
             }
         }
@@ -945,20 +958,20 @@ __global__ void __launch_bounds__(kThreads, 1) gla_tc_kernel(const Params p) {
             // are counted on mbar_x[1]; the proxy fence orders them before the tensor core reads)
             if (warp == 0 && ptx::elect_one()) {
                 ptx::tc_fence_after_sync();
-                issue_pv(sbase, m.slow ? kKH : kPB, tmem);
+                if (!*abort_flag) issue_pv(sbase, m.slow ? kKH : kPB, tmem);
                 ptx::mma_commit(&m.mbar_mma[3]);
             } else if (warp == 4 && ptx::elect_one()) {
-                if (!wait_cluster_phase(&m.mbar_x[1], 0)) m.abort = 1;
+                wait_cluster_phase(&m.mbar_x[1], 0, p.wait_limit, abort_flag);
                 ptx::fence_proxy_async_smem();
                 ptx::tc_fence_after_sync();
-                issue_inter(sbase, tmem, false);
+                if (!*abort_flag) issue_inter(sbase, tmem, false);
                 ptx::mma_commit(&m.mbar_mma[2]);
             }
             wait_mma(3);
         } else {
             if (warp == 0 && ptx::elect_one()) {
                 ptx::tc_fence_after_sync();
-                issue_pv(sbase, m.slow ? kKH : kPB, tmem);
+                if (!*abort_flag) issue_pv(sbase, m.slow ? kKH : kPB, tmem);
                 ptx::mma_commit(&m.mbar_mma[3]);
             }
             wait_mma(3);
@@ -974,6 +987,27 @@ __global__ void __launch_bounds__(kThreads, 1) gla_tc_kernel(const Params p) {
 
     // ---- teardown ----
     __syncthreads();
+    if (*abort_flag) {
+        // a wait expired: copies, remote stores and products already in flight land before the
+        // shared memory and TMEM are released (bounded again; the status is already latched)
+        volatile int no_abort = 0;
+        asm volatile("cp.async.wait_all;" ::: "memory");
+        if ((warp == 0 || warp == 4 || warp == 7) && ptx::elect_one()) ptx::mma_commit(&m.mbar_end);
+        if (tid == 0) {
+            wait_phase(&m.mbar_end, 0, p.wait_limit, &no_abort);
+            if (exchange) {
+                wait_cluster_phase(&m.mbar_x[0], 0, p.wait_limit, &no_abort);
+                wait_cluster_phase(&m.mbar_x[1], 0, p.wait_limit, &no_abort);
+            }
+        }
+        __syncthreads();
+    }
+    // every CTA of the cluster reaches this barrier, so none leaves while another may still
+    // store into its shared memory
+    if (exchange) {
+        ptx::cluster_arrive_release();
+        ptx::cluster_wait();
+    }
     if (tid == 0 && m.range_err) raise_status(8 /* GLA_ERR_RANGE */);
     ptx::tc_fence_after_sync();
     if (warp == 0 && n_pass1 + n_chunks > 0) ptx::tmem_dealloc(tmem, kTmemCols);
@@ -1004,6 +1038,13 @@ __global__ void gla_timeout_selftest_kernel(long long limit_cycles) {
             }
         }
     }
+}
+
+// ------------------------------------------------------- reciprocal self-test
+// y[i] = rcp_nr(x[i]): the kernel's Newton reciprocal, for an error-bound test against 1/x.
+__global__ void gla_rcp_selftest_kernel(const float *x, float *y, int n) {
+    const int i = blockIdx.x * blockDim.x + threadIdx.x;
+    if (i < n) y[i] = rcp_nr(x[i]);
 }
 
 // ---------------------------------------------------------------- self-test
@@ -1038,8 +1079,7 @@ gla_tc_selftest_kernel(int kind, const float *A, const float *Bm, float *Dout) {
     auto put_tf32 = [&](uint32_t region, uint32_t atom, int row, const float *src) {
         for (int c4 = 0; c4 < 16; ++c4)
             *reinterpret_cast<float4 *>(sm + region + off_tf32(atom, row, c4)) =
-                make_float4(ptx::to_tf32(src[4 * c4]), ptx::to_tf32(src[4 * c4 + 1]),
-                            ptx::to_tf32(src[4 * c4 + 2]), ptx::to_tf32(src[4 * c4 + 3]));
+                make_float4(src[4 * c4], src[4 * c4 + 1], src[4 * c4 + 2], src[4 * c4 + 3]);
     };
     auto put_f16 = [&](uint32_t region, int row, const float *src) {
         for (int j = 0; j < 8; ++j) {
@@ -1049,13 +1089,16 @@ gla_tc_selftest_kernel(int kind, const float *A, const float *Bm, float *Dout) {
             *reinterpret_cast<uint4 *>(sm + region + off_f16(row, j)) = o;
         }
     };
-    // split a row into tf32 high/low parts: rows of A go to TMEM, rows of B to shared memory
+    // split a row into tf32 high/low parts exactly as the kernel's score operands are built:
+    // high = the value with its low 13 mantissa bits cleared, low = the exact remainder (the
+    // tensor core drops the remainder's own low bits).  Kind 3 (no low part) rounds to tf32.
     auto put_split_tmem = [&](const float *src, bool with_low) {
         for (int j = 0; j < 8; ++j) {
             float h[8], l[8];
             for (int e = 0; e < 8; ++e) {
-                h[e] = ptx::to_tf32(src[8 * j + e]);
-                l[e] = with_low ? ptx::to_tf32(src[8 * j + e] - h[e]) : 0.0f;
+                const float x = src[8 * j + e];
+                h[e] = with_low ? ptx::tf32_hi(x) : ptx::to_tf32(x);
+                l[e] = with_low ? x - h[e] : 0.0f;
             }
             ptx::tmem_st8(tmem_warp + kColQH + 8 * j, h);
             ptx::tmem_st8(tmem_warp + kColQL + 8 * j, l);
@@ -1066,8 +1109,8 @@ gla_tc_selftest_kernel(int kind, const float *A, const float *Bm, float *Dout) {
         put_split_tmem(A + t * 64, true);
         float hi[64], lo[64];
         for (int c = 0; c < 64; ++c) {
-            hi[c] = ptx::to_tf32(Bm[t * 64 + c]);
-            lo[c] = ptx::to_tf32(Bm[t * 64 + c] - hi[c]);
+            hi[c] = ptx::tf32_hi(Bm[t * 64 + c]);
+            lo[c] = Bm[t * 64 + c] - hi[c];
         }
         put_tf32(kKH, kAtom128, t, hi);
         put_tf32(kKL, kAtom128, t, lo);
@@ -1101,7 +1144,8 @@ gla_tc_selftest_kernel(int kind, const float *A, const float *Bm, float *Dout) {
         else issue_inter(sbase, tmem, false);
         ptx::mma_commit(&m.mbar_mma[0]);
     }
-    wait_phase(&m.mbar_mma[0], 0);
+    volatile int no_abort = 0;
+    wait_phase(&m.mbar_mma[0], 0, 1LL << 32, &no_abort);
     ptx::tc_fence_after_sync();
     if (kind == 0) {
         for (int blk = 0; blk < 4; ++blk) {

@@ -66,7 +66,9 @@ def load() -> ctypes.CDLL:
         lib.gla_selftest_chunk.restype = ctypes.c_int
         lib.gla_selftest_load.argtypes = [vp] * 5 + [i] * 7 + [vp, vp, vp]
         lib.gla_selftest_load.restype = ctypes.c_int
-        lib.gla_selftest_fault.argtypes = [vp] * 7 + [i] * 7 + [ll, i, vp]
+        lib.gla_selftest_fault.argtypes = [vp] * 7 + [i] * 7 + [ll, i, i, vp]
+        lib.gla_selftest_rcp.argtypes = [vp, vp, i, vp]
+        lib.gla_selftest_rcp.restype = ctypes.c_int
         lib.gla_selftest_fault.restype = ctypes.c_int
         for fn in (lib.gla_fwd, lib.gla_fwd_f32, lib.gla_fwd_host, lib.gla_fwd_ex,
                    lib.gla_get_status, lib.gla_version, lib.gla_selftest_mma):
@@ -121,18 +123,22 @@ def _dims(q, v, grid_h, grid_w):
     return int(B), int(H), int(dk), int(dv)
 
 
-def _check_tensors(q, k, v, a, g, w, out, dtype):
+def _check_tensors(q, k, v, a, g, w, out, dtype, on_device: bool = True):
+    """Every tensor has the shape, dtype and placement the library reads and writes through its
+    raw pointer (device tensors for gla_fwd*, host tensors for gla_fwd_host)."""
     import torch
+    where = "CUDA" if on_device else "host (CPU)"
     B, L, H, dk = q.shape
     dv = v.shape[-1]
     for name, t, d in (("q", q, dk), ("k", k, dk), ("a", a, dk), ("v", v, dv),
                        ("g", g, dv), ("out", out, dv)):
         if tuple(t.shape) != (B, L, H, d):
             raise ValueError("%s has shape %s, expected %s" % (name, tuple(t.shape), (B, L, H, d)))
-        if t.dtype != dtype or not t.is_cuda or not t.is_contiguous():
-            raise ValueError("%s must be a contiguous CUDA %s tensor" % (name, dtype))
-    if tuple(w.shape) != (dv,) or w.dtype != torch.float32 or not w.is_cuda or not w.is_contiguous():
-        raise ValueError("w must be a contiguous CUDA float32 tensor of shape [d_v]")
+        if t.dtype != dtype or t.is_cuda != on_device or not t.is_contiguous():
+            raise ValueError("%s must be a contiguous %s %s tensor" % (name, where, dtype))
+    if (tuple(w.shape) != (dv,) or w.dtype != torch.float32 or w.is_cuda != on_device
+            or not w.is_contiguous()):
+        raise ValueError("w must be a contiguous %s float32 tensor of shape [d_v]" % where)
 
 
 def gla_fwd(q, k, v, a, g, w, out, grid_h: int, grid_w: int, direction: int, stream=None):
@@ -172,18 +178,11 @@ def gla_fwd_ex(q, k, v, a, g, w, out, grid_h: int, grid_w: int, direction: int,
 
 def gla_fwd_host(q, k, v, a, g, w, out, grid_h: int, grid_w: int, direction: int, stream=None):
     """The same operation on HOST tensors (CPU, ideally pinned); synchronous."""
-    import torch
-    B, L, H, dk = q.shape
-    dv = v.shape[-1]
-    if L != grid_h * grid_w:
-        raise ValueError("L must equal grid_h*grid_w")
-    for t in (q, k, v, a, g, w, out):
-        if t.is_cuda or not t.is_contiguous():
-            raise ValueError("gla_fwd_host takes contiguous host tensors")
+    B, H, dk, dv = _dims(q, v, grid_h, grid_w)
     dtype = _dtype_code(q)
+    _check_tensors(q, k, v, a, g, w, out, q.dtype, on_device=False)
     args = [ctypes.c_void_p(t.data_ptr()) for t in (q, k, v, a, g, w, out)]
-    args += [int(B), int(H), grid_h, grid_w, int(dk), int(dv), direction, dtype,
-             _stream_ptr(stream)]
+    args += [B, H, grid_h, grid_w, dk, dv, direction, dtype, _stream_ptr(stream)]
     _check(load().gla_fwd_host(*args), "gla_fwd_host")
     return out
 

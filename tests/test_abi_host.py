@@ -138,3 +138,26 @@ def test_binding_rejects_unsupported_dtypes_before_any_call():
         gla.gla_fwd_host(x, x, x, x, x, w, x, 2, 2, 0)
     with pytest.raises(ValueError):
         gla.gla_fwd_ex(x, x, x, x, x, w, x, 2, 2, 0)
+
+
+@pytest.mark.parametrize("bad", ["w_fp16", "out_small", "k_other_d", "g_fp32", "v_strided"])
+def test_host_entry_checks_every_tensor_before_any_call(bad):
+    # gla_fwd_host copies whole host buffers by raw pointer: a tensor of the wrong shape or
+    # dtype must be refused in the binding, before the library reads or writes past its end
+    import torch
+    B, H, gh, gw, d = 1, 2, 3, 4, 64
+    L = gh * gw
+    t = {n: torch.zeros(B, L, H, d, dtype=torch.float16) for n in ("q", "k", "v", "a", "g", "out")}
+    w = torch.zeros(d, dtype=torch.float32)
+    if bad == "w_fp16":
+        w = w.half()
+    elif bad == "out_small":
+        t["out"] = torch.zeros(B, L - 1, H, d, dtype=torch.float16)
+    elif bad == "k_other_d":
+        t["k"] = torch.zeros(B, L, H, 32, dtype=torch.float16)
+    elif bad == "g_fp32":
+        t["g"] = t["g"].float()
+    else:
+        t["v"] = torch.zeros(B, L, H, d, dtype=torch.float16)[..., : d // 2]   # not contiguous
+    with pytest.raises(ValueError):
+        gla.gla_fwd_host(t["q"], t["k"], t["v"], t["a"], t["g"], w, t["out"], gh, gw, 0)
