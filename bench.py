@@ -49,7 +49,7 @@ def parse():
     ap.add_argument("--cpu-seconds", type=float, default=10.0,
                     help="CPU-oracle sample budget for cpu_baseline / --impl reference")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--kernel", choices=["auto", "tc128", "tc64", "simt"], default="auto",
+    ap.add_argument("--kernel", choices=["auto", "tc128", "tc64", "pipe64", "simt"], default="auto",
                     help="kernel to time (default: the one gla_fwd picks for the workload)")
     ap.add_argument("--workload", default=WORKLOAD,
                     help="synthetic workload to time (default: the 40x40 headline); the others "
@@ -319,7 +319,7 @@ def run_ours(args, ws, rank, local):
     dt = torch.float16 if wl.dtype == "f16" else torch.float32
 
     kernel = {"auto": 0, "tc128": gla.KERNEL_TC128, "tc64": gla.KERNEL_TC64,
-              "simt": gla.KERNEL_SIMT}[args.kernel]
+              "pipe64": gla.KERNEL_PIPE64, "simt": gla.KERNEL_SIMT}[args.kernel]
 
     def step(i):
         for j, d in enumerate(directions):

@@ -119,8 +119,10 @@ enum gla_kernel {
     GLA_KERNEL_AUTO = 0,   /* the one gla_fwd / gla_fwd_f32 choose                       */
     GLA_KERNEL_TC128 = 1,  /* tensor cores, 128-row chunks: fp16, d_k = d_v = 64           */
     GLA_KERNEL_SIMT = 2,   /* CUDA cores: every supported shape, fp16 or fp32              */
-    GLA_KERNEL_TC64 = 3    /* tensor cores, 64-row chunks, TMA loads: fp16, d_k = d_v in   */
+    GLA_KERNEL_TC64 = 3,   /* tensor cores, 64-row chunks, TMA loads: fp16, d_k = d_v in   */
                            /* {64, 128}                                                    */
+    GLA_KERNEL_PIPE64 = 4  /* the 64-row kernel with two chunks in flight (warp-specialised */
+                           /* teams, 3-stage TMA ring): fp16, d_k = d_v = 64               */
 };
 
 /*
@@ -189,7 +191,8 @@ int gla_selftest_timeout(long long limit_cycles, void *stream);
 /*
  * gla_selftest_fault -- diagnostic for device-side failure detection in the operator's
  * own tensor-core kernels: runs gla_fwd (fp16, d_k = d_v = d) on `kernel`
- * (GLA_KERNEL_TC128 with d = 64, or GLA_KERNEL_TC64 with d in {64, 128}; `segments` CTAs
+ * (GLA_KERNEL_TC128 or GLA_KERNEL_PIPE64 with d = 64, or GLA_KERNEL_TC64 with d in {64, 128};
+ * `segments` CTAs
  * per pair or 0 for automatic) with every bounded wait limited to `wait_limit_cycles` SM
  * clocks (1 .. 2^34), while the loads of full-pass chunk `withheld_chunk` of every segment
  * never complete their barrier (-1: none): the 64-row kernel does not issue them, the
@@ -221,6 +224,8 @@ int gla_selftest_rcp(const float *x, float *y, int n, void *stream);
  *   kind 1  D[d][d]   = A[64][d]^T * B[64][d]   (fp16 operands, the chunk-state product)
  *   kind 2  D[64][d]  = A[64][64] * B[64][d]    (fp16 operands, P * V, A held in TMEM)
  *   kind 3  D[64][d]  = A[64][d] * B[d][d]      (bf16 split, the inter-chunk product)
+ *   kind 4  D[64][64] = A[64][64] * B[64][64]   (fp16, P * V with P from shared memory, the
+ *           pipelined kernel's form; d = 64 only)
  * Inputs are rounded to the operand type on the way in; accumulation is fp32.
  * Asynchronous on `stream`.  Not part of the operation itself.
  */

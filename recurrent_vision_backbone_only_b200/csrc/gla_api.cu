@@ -15,6 +15,7 @@
 
 #include "gla.h"
 #include "gla_chunk.cuh"
+#include "gla_pipe.cuh"
 #include "gla_common.cuh"
 #include "gla_simt.cuh"
 #include "gla_tc.cuh"
@@ -100,8 +101,9 @@ int current_device_info(DeviceInfo *info) {
 int ceil_div(long long a, long long b) { return (int)((a + b - 1) / b); }
 
 // Kernels: 1 = 128-row tensor-core kernel (fp16, d_k = d_v = 64), 2 = CUDA-core kernel (any
-// supported shape, fp16 or fp32), 3 = 64-row tensor-core kernel (fp16, d_k = d_v in {64, 128}).
-enum { kAuto = 0, kTc128 = 1, kSimt = 2, kTc64 = 3 };
+// supported shape, fp16 or fp32), 3 = 64-row tensor-core kernel (fp16, d_k = d_v in {64, 128}),
+// 4 = the 64-row kernel with two chunks in flight (fp16, d_k = d_v = 64).
+enum { kAuto = 0, kTc128 = 1, kSimt = 2, kTc64 = 3, kPipe64 = 4 };
 
 // Launch schedule: `segs` CTAs (one thread-block cluster) per (b, h) pair,
 // each owning `seg_len` consecutive scan positions.
@@ -429,11 +431,13 @@ double chunk_cost(int q, int n_pairs, int segs, int sms, int active1, int active
     return per_cta * 1.4 * ceil_div(n_pairs, active2);
 }
 
-template <int D>
+template <int D, bool kPipe = false>
 int run_chunk(const Args &x, int chunk, int segs, float eps, cudaStream_t st, const DeviceInfo &di,
               Plan *query, long long wait_limit = 1LL << 32, int fault_chunk = -1) {
-    auto kern = ck::gla_chunk_kernel<D>;
+    static_assert(!kPipe || D == 64, "the pipelined kernel handles d = 64");
+    auto kern = kPipe ? ck::gla_pipe_kernel : ck::gla_chunk_kernel<D>;
     using C = ck::Cfg<D>;
+    constexpr int kThreads = kPipe ? ck::PipeCfg::kThreads : C::kThreads;
     const int L = x.gh * x.gw;
     const int n_pairs = x.B * x.H;
     if (chunk <= 0) chunk = ck::kC;
@@ -443,7 +447,7 @@ int run_chunk(const Args &x, int chunk, int segs, float eps, cudaStream_t st, co
     int q = 0;
     for (int dir = 0; dir < 4; ++dir)
         if (x.dir == 4 || x.dir == dir) q = std::max(q, ck::Lines(dir, x.gh, x.gw, chunk).chunks);
-    const size_t smem_max = chunk_smem<D>(true);
+    const size_t smem_max = kPipe ? ck::pipe_smem_bytes() : chunk_smem<D>(true);
     if (smem_max > (size_t)di.max_smem_optin) return GLA_ERR_UNSUPPORTED;
     // all of the unified L1 / shared memory as shared memory, so two d = 64 CTAs fit on an SM
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_max) != cudaSuccess ||
@@ -454,14 +458,15 @@ int run_chunk(const Args &x, int chunk, int segs, float eps, cudaStream_t st, co
         return GLA_ERR_CUDA;
     }
     Plan pl;
-    pl.kernel = kTc64;
+    pl.kernel = kPipe ? kPipe64 : kTc64;
     pl.chunk = chunk;
     pl.pdl = true;
+    auto smem_of = [&](bool spread) { return kPipe ? ck::pipe_smem_bytes() : chunk_smem<D>(spread); };
     auto clusters = [&](int size, bool spread) {
         Plan probe = pl;
         probe.segs = size;
-        probe.smem = chunk_smem<D>(spread);
-        configure_launch(probe, n_pairs, C::kThreads, st);
+        probe.smem = smem_of(spread);
+        configure_launch(probe, n_pairs, kThreads, st);
         int n = 0;
         if (cudaOccupancyMaxActiveClusters(&n, kern, &probe.cfg) != cudaSuccess) {
             cudaGetLastError();
@@ -500,8 +505,8 @@ int run_chunk(const Args &x, int chunk, int segs, float eps, cudaStream_t st, co
     pl.segs = segs;
     pl.seg_len = std::min(L, ceil_div(q, segs) * ck::Lines(x.dir == 4 ? 0 : x.dir, x.gh, x.gw, chunk).clen);
     const bool spread = (long long)n_pairs * pl.segs <= di.sms;
-    pl.smem = chunk_smem<D>(spread);
-    configure_launch(pl, n_pairs, C::kThreads, st);
+    pl.smem = smem_of(spread);
+    configure_launch(pl, n_pairs, kThreads, st);
     pl.max_active_clusters = clusters(pl.segs, spread);
     if (pl.max_active_clusters <= 0) return GLA_ERR_UNSUPPORTED;
     if (query) {
@@ -546,11 +551,12 @@ int run(const Args &x, int dtype, int chunk, int segs, float eps, cudaStream_t s
     int rc = validate(x);
     if (rc != GLA_OK) return rc;
     if (segs < 0 || segs > 16 || chunk < 0 || !(eps >= 0.0f)) return GLA_ERR_UNSUPPORTED;
-    if (kernel < kAuto || kernel > kTc64) return GLA_ERR_UNSUPPORTED;
+    if (kernel < kAuto || kernel > kPipe64) return GLA_ERR_UNSUPPORTED;
     if (kernel == kAuto) kernel = auto_kernel(x, dtype);
     if (kernel == kTc128 && !(dtype == 0 && x.dk == 64 && x.dv == 64)) return GLA_ERR_UNSUPPORTED;
     if (kernel == kTc64 && !(dtype == 0 && x.dk == x.dv && (x.dk == 64 || x.dk == 128)))
         return GLA_ERR_UNSUPPORTED;
+    if (kernel == kPipe64 && !(dtype == 0 && x.dk == 64 && x.dv == 64)) return GLA_ERR_UNSUPPORTED;
     DeviceInfo di;
     rc = current_device_info(&di);
     if (rc != GLA_OK) return rc;
@@ -558,6 +564,7 @@ int run(const Args &x, int dtype, int chunk, int segs, float eps, cudaStream_t s
     if (kernel == kTc64)
         return x.dk == 64 ? run_chunk<64>(x, chunk, segs, eps, st, di, query)
                           : run_chunk<128>(x, chunk, segs, eps, st, di, query);
+    if (kernel == kPipe64) return run_chunk<64, true>(x, chunk, segs, eps, st, di, query);
     if (dtype == 1) return run_simt<float>(x, chunk, segs, eps, st, di, query);
     return run_simt<__half>(x, chunk, segs, eps, st, di, query);
 }
@@ -772,7 +779,7 @@ int gla_selftest_timeout(long long limit_cycles, void *stream) {
 
 int gla_selftest_chunk(int d, int kind, const float *A, const float *B, float *Dm, void *stream) {
     if (!A || !B || !Dm) return GLA_ERR_NULL;
-    if ((d != 64 && d != 128) || kind < 0 || kind > 3) return GLA_ERR_UNSUPPORTED;
+    if ((d != 64 && d != 128) || kind < 0 || kind > 4 || (kind == 4 && d != 64)) return GLA_ERR_UNSUPPORTED;
     DeviceInfo di;
     int rc = current_device_info(&di);
     if (rc != GLA_OK) return rc;
@@ -825,8 +832,8 @@ int gla_selftest_fault(const void *q, const void *k, const void *v, const void *
                        long long wait_limit_cycles, int withheld_chunk, int kernel, void *stream) {
     if (wait_limit_cycles <= 0 || wait_limit_cycles > (1LL << 34)) return GLA_ERR_UNSUPPORTED;
     if (d != 64 && d != 128) return GLA_ERR_UNSUPPORTED;
-    if (kernel != kTc128 && kernel != kTc64) return GLA_ERR_UNSUPPORTED;
-    if (kernel == kTc128 && d != 64) return GLA_ERR_UNSUPPORTED;
+    if (kernel != kTc128 && kernel != kTc64 && kernel != kPipe64) return GLA_ERR_UNSUPPORTED;
+    if ((kernel == kTc128 || kernel == kPipe64) && d != 64) return GLA_ERR_UNSUPPORTED;
     const Args x = make_args(q, k, v, gate_preact, out_gate_preact, rms_weight, out, B, H, grid_h, grid_w,
                              d, d, direction, 2);
     int rc = validate(x);
@@ -840,6 +847,8 @@ int gla_selftest_fault(const void *q, const void *k, const void *v, const void *
         if (segments > 0 && !tc_segs_ok(segments)) return GLA_ERR_UNSUPPORTED;
         return run_tc(x, 0, segments, kEps, st, di, nullptr, wait_limit_cycles, withheld_chunk);
     }
+    if (kernel == kPipe64)
+        return run_chunk<64, true>(x, 0, segments, kEps, st, di, nullptr, wait_limit_cycles, withheld_chunk);
     if (d == 64) return run_chunk<64>(x, 0, segments, kEps, st, di, nullptr, wait_limit_cycles, withheld_chunk);
     return run_chunk<128>(x, 0, segments, kEps, st, di, nullptr, wait_limit_cycles, withheld_chunk);
 }

@@ -926,6 +926,8 @@ __global__ void gla_chunk_empty_kernel() {
 //   kind 1  state   D[D][D]   = A[64][D]^T B[64][D]   fp16 (A as Ks, B as V; MN-major)
 //   kind 2  P V     D[64][D]  = A[64][64] B[64][D]    fp16 (A -> TMEM as P, B as V)
 //   kind 3  inter   D[64][D]  = A[64][D] B[D][D]      bf16 split (A -> TMEM, B as S~)
+//   kind 4  P V     D[64][D]  = A[64][64] B[64][D]    fp16, A from shared memory (K-major, in the
+//                                                      a tile), the pipelined kernel's form
 template <int D>
 __global__ void __launch_bounds__(Cfg<D>::kThreads, 1)
     gla_chunk_selftest_kernel(int kind, const float *A, const float *Bm, float *Dout) {
@@ -991,6 +993,9 @@ __global__ void __launch_bounds__(Cfg<D>::kThreads, 1)
         store_p<D>(tmem_row, ro.hg, pr);
         ptx::tmem_st_wait();
         put_tile_h(stage + C::kTV, Bm);
+    } else if (kind == 4) {
+        put_tile_h(stage + C::kTA, A);            // P[t][s], 64 x 64, K-major (D = 64)
+        put_tile_h(stage + C::kTV, Bm);
     } else {
         put_q(A);
         for (int idx = tid; idx < D * (D / 8); idx += C::kThreads) {
@@ -1010,7 +1015,13 @@ __global__ void __launch_bounds__(Cfg<D>::kThreads, 1)
         if (kind == 0) Mma<D>::scores(sbase, stage, tmem);
         else if (kind == 1) Mma<D>::state(sbase, stage, tmem);
         else if (kind == 2) Mma<D>::pv(sbase, stage, tmem, false);
-        else Mma<D>::inter(sbase, tmem);
+        else if (kind == 4) {
+            const uint64_t a = ptx::desc_sw128(sbase + stage + C::kTA, 16, 1024);
+            const uint64_t b = ptx::desc_sw128(sbase + stage + C::kTV, C::kAtom, 1024);
+#pragma unroll
+            for (int k = 0; k < 4; ++k)
+                ptx::mma_f16_ss(tmem + C::kColO, a + 2 * k, b + 128 * k, ptx::idesc_ab(0, 0, false, true, 64, D), k > 0);
+        } else Mma<D>::inter(sbase, tmem);
         ptx::mma_commit(&m.mbar_o);
     }
     wait_bar(&m.mbar_o, 0, 1LL << 32, &m.abort);

@@ -1,0 +1,695 @@
+// gla_pipe.cuh -- the 64-row tensor-core kernel of gla_chunk.cuh for d_k = d_v = 64 with two
+// chunks in flight: warp-specialised teams and a 3-stage TMA ring.
+//
+// Operation and chunkwise form: as gla_chunk.cuh (GTR paper, arXiv 2609.26590, method
+// section: S_t = Diag(gamma_t) S_{t-1} + k_t^T v_t, o_t = d_k^{-1/2} q_t S_t, u_t = SiLU(g_t) *
+// RMSNorm(o_t) * w), with the same 16-bit products, line-aligned chunks, TMA boxes and cluster
+// state exchange.  Only the schedule differs.
+//
+// Roles (576 threads):
+//   front team  (warps 0-7)   per chunk: gate (cumulative log2-decay b), then the operands Kh,
+//                             Kl, Ks in place over the raw tiles and Q~ into the chunk's TMEM slot;
+//   back team   (warps 8-15)  per chunk: S~ from the carried state, P from the scores (into the
+//                             dead K~-low tile, as the A operand of P V), the state fold, the
+//                             RMSNorm / SiLU epilogue and the stores;
+//   MMA warp    (warp 16)     issues every tcgen05.mma and commit;
+//   load warp   (warp 17)     issues the TMA boxes into a 3-stage ring.
+// Chunk j uses TMEM slot j % 2 -- lanes 16 (j % 2) .. + 16 of every lane quarter, so one M = 64
+// tile of each slot shares the columns of the other -- and smem stage j % 3.  The front team
+// builds chunk j + 1 while the tensor core and the back team finish chunk j.
+//
+// Synchronisation (mbarriers, phase = use count of the slot / stage).  Every chunk completes
+// every slot barrier exactly once (a state-only chunk with no-op arrivals and commits), and every
+// waiter of a barrier waits on each of its phases in turn, so the k-th use of a slot always waits
+// for parity k & 1 and no waiter is ever two phases behind:
+//   ld[s]        TMA bytes of a stage landed                       load warp -> front, back
+//   fdone[p]     gate + operands of the slot's chunk ready         front -> MMA, back
+//   sl, sc, o[p] chunk state / scores / output products done      tcgen05.commit -> back
+//   sx[p]        S~ of the slot's chunk written                    back -> MMA
+//   pfull[p]     P written                                         back -> MMA
+//   slotfree[p]  the back team is done with the slot's chunk       back -> front, MMA
+//   stfree[s]    the stage may be reloaded (2 arrivals)            tcgen05.commit + back -> load
+#pragma once
+
+#include "gla_chunk.cuh"
+
+namespace gla {
+namespace ck {
+
+struct PipeCfg {
+    static constexpr int D = 64;
+    static constexpr int kTeam = 256;                    // threads per team
+    static constexpr int kThreads = 2 * kTeam + 64;      // + MMA warp + load warp
+    static constexpr int kStages = 3;
+    static constexpr uint32_t kAtom = 64 * 128;
+    static constexpr uint32_t kTile = 64 * D * 2;        // 8 KB
+    static constexpr uint32_t kTQ = 0, kTK = kTile, kTA = 2 * kTile, kTV = 3 * kTile, kTG = 4 * kTile;
+    static constexpr uint32_t kStage = 5 * kTile;        // q (-> Ks), k (-> Kh), a (-> Kl -> P), v, g
+    static constexpr uint32_t kB = kStages * kStage;     // b (front team) / exchange rows
+    static constexpr uint32_t kBBytes = 20480;           // >= max(64 x 64 x 4, (D + 15) x D x 4)
+    static constexpr uint32_t kSX0 = kB + kBBytes;       // S~ slot 0 (high | low); S_in (exchange)
+    static constexpr uint32_t kSXBytes = D * D * 4;      // 16 KB per slot
+    static constexpr uint32_t kMisc = kSX0 + 2 * kSXBytes;
+    // TMEM columns; slot p is lanes 16p .. 16p + 15 of every quarter
+    static constexpr uint32_t kColSC = 0, kColO = 64, kColQH = 128, kColQL = 160, kColSL = 192;
+    static constexpr uint32_t kTmemCols = 256;
+    static constexpr int kMaxRecvRows = D + 15;
+};
+
+struct PipeMisc {
+    uint64_t ld[3], stfree[3];
+    uint64_t fdone[2], sl[2], sc[2], sx[2], pfull[2], o[2], slotfree[2];
+    uint64_t end;              // teardown after an expired wait: products in flight
+    uint32_t tmem_base;
+    int abort, range_err;
+    int slow[2];               // per slot: the chunk takes the exact CUDA-core score path
+    alignas(16) float tot[8][64];     // front: gate block totals
+    alignas(16) float b0[64];         // front: b at the first scan position
+    alignas(16) float rref[2][64];    // per slot: reference r (log2)
+    alignas(16) float Bc[2][64];      // per slot: B (log2)
+    alignas(16) float fB[2][64];      // per slot: 2^{B - r}
+    alignas(16) float er[2][64];      // per slot: 2^{r}
+    alignas(16) float eB[2][64];      // per slot: 2^{B}
+    alignas(16) float dqp[2][4][kC];  // per slot: diagonal score partial sums
+    alignas(16) float red[4][kC];     // back: epilogue partial sums of squares
+    alignas(16) float Gs[64];         // back: segment aggregate log2-decay
+    alignas(16) float w[64];          // RMSNorm weight
+    alignas(16) float recvG[PipeCfg::kMaxRecvRows];
+};
+
+constexpr size_t pipe_smem_bytes() { return PipeCfg::kMisc + sizeof(PipeMisc) + 1024; }
+
+__device__ __forceinline__ void team_bar(int id) { ptx::named_bar_sync(id, PipeCfg::kTeam); }
+
+__global__ void __launch_bounds__(PipeCfg::kThreads, 1)
+    gla_pipe_kernel(const __grid_constant__ Maps maps, const Params p) {
+    using C = PipeCfg;
+    constexpr int D = 64;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                              ~uintptr_t(1023));
+    const uint32_t sbase = ptx::smem_u32(sm);
+    PipeMisc &m = *reinterpret_cast<PipeMisc *>(sm + C::kMisc);
+    volatile int *abort_flag = &m.abort;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const bool front = warp < 8, back = warp >= 8 && warp < 16;
+    const bool mma_warp = warp == 16, load_warp = warp == 17;
+    // team roles (front and back alike): row t, channels [16 cg, 16 cg + 16); back: state row sc,
+    // columns [16 cg, + 16)
+    const int wt = warp & 7, qd = warp & 3, hg = wt >> 2, cg = 2 * hg + (lane >> 4);
+    const int t = 16 * qd + (lane & 15);
+    const int ttid = tid & (C::kTeam - 1);           // thread index within its team
+
+    const int pair = blockIdx.x / p.segs;
+    const int rank = blockIdx.x - pair * p.segs;
+    const int bb = pair / p.H, hh = pair - bb * p.H;
+    const int dir = p.dir == 4 ? (bb & 3) : p.dir;
+    const Lines ln(dir, p.gh, p.gw, p.chunk_max);
+    const int seg_chunks = (ln.chunks + p.segs - 1) / p.segs;
+    const int q0 = min(ln.chunks, rank * seg_chunks);
+    const int n2 = min(ln.chunks, q0 + seg_chunks) - q0;
+    const bool exchange = p.segs > 1;
+    const int n1 = (exchange && rank < p.segs - 1) ? n2 : 0;
+    const int N = n1 + n2;                             // chunks processed: state-only, then full
+    const CUtensorMap *tmaps = ln.fam ? maps.col : maps.row;
+
+    ptx::pdl_launch_dependents();
+    if (tid == 0) {
+        for (int i = 0; i < 3; ++i) {
+            ptx::mbar_init(&m.ld[i], 1);
+            ptx::mbar_init(&m.stfree[i], 2);
+        }
+        for (int i = 0; i < 2; ++i) {
+            ptx::mbar_init(&m.fdone[i], 1);
+            ptx::mbar_init(&m.sl[i], 1);
+            ptx::mbar_init(&m.sc[i], 1);
+            ptx::mbar_init(&m.sx[i], 1);
+            ptx::mbar_init(&m.pfull[i], 1);
+            ptx::mbar_init(&m.o[i], 1);
+            ptx::mbar_init(&m.slotfree[i], 1);
+        }
+        ptx::mbar_init(&m.end, 1);
+        ptx::fence_mbarrier_init();
+        m.abort = 0;
+        m.range_err = 0;
+    }
+    if (warp == 0) {
+        ptx::tmem_alloc(&m.tmem_base, C::kTmemCols);
+        ptx::tmem_relinquish();
+    }
+    if (load_warp && lane == 0)
+        for (int i = 0; i < 5; ++i) ptx::prefetch_tmap(&tmaps[i]);
+    if (tid < D) m.Gs[tid] = 0.0f;
+    ptx::tc_fence_before_sync();
+    __syncthreads();
+    ptx::tc_fence_after_sync();
+    const uint32_t tmem = m.tmem_base;
+    ptx::pdl_wait_prior_grid();
+    if (tid < D / 4)
+        *reinterpret_cast<float4 *>(&m.w[4 * tid]) = *reinterpret_cast<const float4 *>(p.w + 4 * tid);
+    __syncthreads();
+
+    // chunk j of the sequence (state-only chunks, then full chunks) -> chunk of the segment
+    struct Chunk {
+        int line, n, lp0;
+        bool full;
+    };
+    auto chunk_of = [&](int j) {
+        const bool full = j >= n1;
+        const int q = q0 + (full ? j - n1 : j);
+        Chunk c;
+        c.line = q / ln.pieces;
+        const int start = (q - c.line * ln.pieces) * ln.clen;
+        c.n = min(ln.clen, ln.len - start);
+        c.lp0 = ln.rev ? ln.len - start - c.n : start;
+        c.full = full;
+        return c;
+    };
+    auto token_row = [&](const Chunk &c, int i) {
+        const int lp = c.lp0 + i;
+        const int s = ln.fam ? lp * p.gw + c.line : c.line * p.gw + lp;
+        return (bb * p.L + s) * p.H + hh;
+    };
+    auto wait = [&](uint64_t *bar, int use) { return wait_bar(bar, (uint32_t)(use & 1), p.wait_limit, abort_flag); };
+    // lanes of this warp's quarter in TMEM slot `slot`
+    auto tmem_rows = [&](int slot) { return tmem + ((uint32_t)(32 * qd + 16 * slot) << 16); };
+
+    // ---------------------------------------------------------------- exchange
+    // All 576 threads: barriers A, B, C; the back team holds the aggregate (S, Gs).
+    float S[16];                                      // back: S[c = sc][16 cg + i]
+#pragma unroll
+    for (int i = 0; i < 16; ++i) S[i] = 0.0f;
+    const int sc = 16 * qd + (lane & 15);
+    auto run_exchange = [&]() {
+        const int segs = p.segs;
+        const int max_own = (D + segs - 1) / segs;
+        const float *recv = reinterpret_cast<const float *>(sm + C::kB);
+        __syncthreads();
+        ptx::cluster_arrive_release();
+        ptx::cluster_wait();
+        if (back && rank < segs - 1) {
+            const int owner = sc % segs, lc = sc / segs;
+            const uint32_t row = (uint32_t)((rank * max_own + lc) * D + 16 * cg) * 4;
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+                ptx::st_cluster_v4(ptx::mapa(sbase + C::kB + row + 16 * i, owner),
+                                   make_float4(S[4 * i], S[4 * i + 1], S[4 * i + 2], S[4 * i + 3]));
+        }
+        if (tid < D && rank < segs - 1) {
+            const int o2 = tid % segs, l2 = tid / segs;
+            ptx::st_cluster_f32(ptx::mapa(ptx::smem_u32(&m.recvG[rank * max_own + l2]), o2), m.Gs[tid]);
+        }
+        ptx::cluster_arrive_release();
+        ptx::cluster_wait();
+        {
+            const int n_own = (D - rank + segs - 1) / segs;
+            const int items = n_own * (D / 4);
+            for (int it = tid; it < items; it += C::kThreads) {
+                const int lc = it / (D / 4), j4 = it - lc * (D / 4);
+                const int c = lc * segs + rank;
+                const uint32_t dst = sbase + C::kSX0 + (uint32_t)(c * D + 4 * j4) * 4;
+                float4 run = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+                for (int q = 0; q < segs; ++q) {
+                    ptx::st_cluster_v4(ptx::mapa(dst, q), run);
+                    if (q + 1 < segs) {
+                        const float g = ptx::ex2(m.recvG[q * max_own + lc]);
+                        const float4 agg = *reinterpret_cast<const float4 *>(recv + (q * max_own + lc) * D + 4 * j4);
+                        run = make_float4(fmaf(g, run.x, agg.x), fmaf(g, run.y, agg.y),
+                                          fmaf(g, run.z, agg.z), fmaf(g, run.w, agg.w));
+                    }
+                }
+            }
+        }
+        ptx::cluster_arrive_release();
+        ptx::cluster_wait();
+        if (back) {
+            const float *sin = reinterpret_cast<const float *>(sm + C::kSX0);
+#pragma unroll
+            for (int i = 0; i < 16; ++i) S[i] = sin[sc * D + 16 * cg + i];
+        }
+        __syncthreads();
+    };
+
+    // =================================================================== load warp
+    if (load_warp) {
+        int last[3] = {-1, -1, -1};                   // last chunk issued into each stage
+        auto load = [&](int j) {
+            const int s = j % 3;
+            if (j >= 3) wait(&m.stfree[s], (j - 3) / 3);
+            if (lane == 0 && !*abort_flag) {
+                const Chunk c = chunk_of(j);
+                const uint32_t mask = c.full ? 0x1Fu : 0x0Eu;
+                ptx::mbar_arrive_expect_tx(&m.ld[s], (uint32_t)__popc(mask) * C::kTile);
+                if (!(c.full && j - n1 == p.fault_chunk)) {
+                    const int y = ln.fam ? c.line * p.H + hh : hh;
+                    const int z = ln.fam ? bb * p.gh + c.lp0 : bb * p.L + c.line * p.gw + c.lp0;
+                    const uint32_t bar = ptx::smem_u32(&m.ld[s]);
+#pragma unroll
+                    for (int x = 0; x < 5; ++x)
+                        if (mask >> x & 1u)
+                            ptx::tma_load_3d(sbase + s * C::kStage + x * C::kTile, &tmaps[x], 0, y, z, bar);
+                }
+                last[s] = j;
+            }
+            __syncwarp();
+        };
+        const int pre = min(N, n1 + 3);             // everything loadable before the exchange
+        for (int j = 0; j < pre; ++j) load(j);
+        if (exchange) run_exchange();
+        for (int j = pre; j < N; ++j) load(j);
+        // teardown: after an expired wait, the boxes already issued land before smem is freed
+        __syncthreads();
+        if (*abort_flag && lane == 0) {
+            volatile int no_abort = 0;
+            for (int s = 0; s < 3; ++s)
+                if (last[s] >= 0) wait_bar(&m.ld[s], (uint32_t)((last[s] / 3) & 1), p.wait_limit, &no_abort);
+        }
+    }
+
+    // ==================================================================== MMA warp
+    else if (mma_warp) {
+        using M = Mma<64>;
+        const uint64_t kh0 = ptx::desc_sw128(sbase + C::kTK, 16, 1024);
+        const uint64_t kl0 = ptx::desc_sw128(sbase + C::kTA, 16, 1024);
+        const uint64_t ks0 = ptx::desc_sw128(sbase + C::kTQ, C::kAtom, 1024);
+        const uint64_t v0 = ptx::desc_sw128(sbase + C::kTV, C::kAtom, 1024);
+        const uint64_t pa0 = ptx::desc_sw128(sbase + C::kTA, 16, 1024);      // P: K-major A
+        constexpr uint32_t kIdPVss = ptx::idesc_ab(0, 0, false, true, 64, 64);
+        auto step = [&](int j) {
+            const int slot = j & 1, s = j % 3;
+            const Chunk c = chunk_of(j);
+            if (j >= 2) wait(&m.slotfree[slot], (j - 2) >> 1);
+            wait(&m.fdone[slot], j >> 1);
+            const bool go = !*abort_flag;
+            if (lane == 0) {
+                ptx::tc_fence_after_sync();
+                const uint32_t stg = (uint32_t)s * C::kStage >> 4;   // descriptor address units
+                const uint32_t lanes = (uint32_t)(16 * slot) << 16;
+                const uint32_t d_sl = tmem + lanes + C::kColSL, d_sc = tmem + lanes + C::kColSC;
+                const uint32_t d_o = tmem + lanes + C::kColO;
+                const uint32_t a_qh = tmem + lanes + C::kColQH, a_ql = tmem + lanes + C::kColQL;
+                if (go) {
+#pragma unroll
+                    for (int k = 0; k < 4; ++k)
+                        ptx::mma_f16_ss(d_sl, ks0 + stg + 128 * k, v0 + stg + 128 * k, M::kIdSL, k > 0);
+                }
+                ptx::mma_commit(&m.sl[slot]);
+                if (c.full && go && !m.slow[slot]) {
+#pragma unroll
+                    for (int pass = 0; pass < 3; ++pass)
+#pragma unroll
+                        for (int k = 0; k < 4; ++k)
+                            ptx::mma_f16_ts(d_sc, (pass == 2 ? a_ql : a_qh) + 8 * k,
+                                            (pass == 1 ? kl0 : kh0) + stg + 2 * k, M::kIdSC, pass > 0 || k > 0);
+                }
+                ptx::mma_commit(&m.sc[slot]);
+            }
+            __syncwarp();
+            if (c.full) {
+                wait(&m.sx[slot], j >> 1);
+                if (lane == 0) {
+                    ptx::tc_fence_after_sync();
+                    const uint32_t lanes = (uint32_t)(16 * slot) << 16;
+                    const uint64_t sxh = ptx::desc_sw128(sbase + C::kSX0 + slot * C::kSXBytes, D * 128, 1024);
+                    const uint64_t sxl = sxh + ((D * D * 2) >> 4);
+                    if (!*abort_flag) {
+#pragma unroll
+                        for (int pass = 0; pass < 3; ++pass)
+#pragma unroll
+                            for (int k = 0; k < 4; ++k)
+                                ptx::mma_f16_ts(tmem + lanes + C::kColO,
+                                                tmem + lanes + (pass == 2 ? C::kColQL : C::kColQH) + 8 * k,
+                                                (pass == 1 ? sxl : sxh) + 128 * k, M::kIdIN, pass > 0 || k > 0);
+                    }
+                }
+                __syncwarp();
+                wait(&m.pfull[slot], j >> 1);
+                if (lane == 0) {
+                    ptx::tc_fence_after_sync();
+                    const uint32_t lanes = (uint32_t)(16 * slot) << 16;
+                    const uint32_t stg = (uint32_t)s * C::kStage >> 4;
+                    if (!*abort_flag) {
+#pragma unroll
+                        for (int k = 0; k < 4; ++k)
+                            ptx::mma_f16_ss(tmem + lanes + C::kColO, pa0 + stg + 2 * k, v0 + stg + 128 * k,
+                                            kIdPVss, true);
+                    }
+                }
+                __syncwarp();
+            } else {
+                wait(&m.sx[slot], j >> 1);              // the back team's no-op arrivals
+                wait(&m.pfull[slot], j >> 1);
+            }
+            if (lane == 0) {
+                ptx::mma_commit(&m.o[slot]);
+                ptx::mma_commit(&m.stfree[s]);     // this chunk's products have read the stage
+            }
+            __syncwarp();
+        };
+        for (int j = 0; j < n1; ++j) step(j);
+        if (exchange) run_exchange();
+        for (int j = n1; j < N; ++j) step(j);
+        __syncthreads();
+        if (*abort_flag && lane == 0) {
+            volatile int no_abort = 0;
+            ptx::mma_commit(&m.end);
+            wait_bar(&m.end, 0, p.wait_limit, &no_abort);
+        }
+    }
+
+    // ================================================================== front team
+    else if (front) {
+        const uint32_t tmem_q = tmem;                 // + slot lanes below
+        // gate: thread (channel pair cp, block pb of 8 scan positions), b into kB (fp32 atoms)
+        auto gate = [&](uint32_t stage, const Chunk &c, int slot) {
+            const int cp = ttid & 31, pb = ttid >> 5, ch = 2 * cp;
+            const int n = c.n, rev = ln.rev;
+            float c0s[8], c1s[8];
+            float r0 = 0.0f, r1 = 0.0f;
+            const uint32_t aoff = stage + C::kTA + (ch & 7) * 2;
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const int pos = pb * 8 + i;
+                const bool ok = pos < n;
+                const int row = ok ? (rev ? n - 1 - pos : pos) : 0;
+                const float2 af = __half22float2(*reinterpret_cast<const __half2 *>(sm + aoff + ptx::sw128(row, ch >> 3)));
+                r0 += ok ? log2_gamma(af.x) : 0.0f;
+                r1 += ok ? log2_gamma(af.y) : 0.0f;
+                c0s[i] = r0;
+                c1s[i] = r1;
+            }
+            *reinterpret_cast<float2 *>(&m.tot[pb][ch]) = make_float2(r0, r1);
+            if (ttid == 0) m.slow[slot] = 0;
+            team_bar(1);
+            float a0 = 0.0f, a1 = 0.0f;
+            for (int q = 0; q < pb; ++q) {
+                const float2 x = *reinterpret_cast<const float2 *>(&m.tot[q][ch]);
+                a0 += x.x;
+                a1 += x.y;
+            }
+            const int rmid = (n - 1) >> 1;
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const int pos = pb * 8 + i;
+                if (pos < n) {
+                    const int row = rev ? n - 1 - pos : pos;
+                    const float2 bv = make_float2(c0s[i] + a0, c1s[i] + a1);
+                    *reinterpret_cast<float2 *>(sm + C::kB + off_f<64>(row, ch >> 2) + (ch & 3) * 4) = bv;
+                    if (pos == rmid) *reinterpret_cast<float2 *>(&m.rref[slot][ch]) = bv;
+                    if (pos == n - 1) *reinterpret_cast<float2 *>(&m.Bc[slot][ch]) = bv;
+                    if (pos == 0) *reinterpret_cast<float2 *>(&m.b0[ch]) = bv;
+                }
+            }
+            team_bar(1);
+            if (ttid < D) {
+                const float Bv = m.Bc[slot][ttid];
+                m.eB[slot][ttid] = ptx::ex2(Bv);
+                if (c.full && (m.b0[ttid] - m.rref[slot][ttid] > kHalfRange || m.rref[slot][ttid] - Bv > kHalfRange))
+                    m.slow[slot] = 1;
+            }
+            team_bar(1);
+            if (c.full && ttid < D) {
+                const float r = m.slow[slot] ? 0.0f : m.rref[slot][ttid];
+                m.rref[slot][ttid] = r;
+                m.fB[slot][ttid] = ptx::ex2(m.Bc[slot][ttid] - r);
+                m.er[slot][ttid] = ptx::ex2(r);
+            }
+            team_bar(1);
+        };
+        auto build_ks = [&](uint32_t stage, const Chunk &c, int slot) {
+            const int n = c.n;
+#pragma unroll
+            for (int jj = 0; jj < 2; ++jj) {
+                const int j = 2 * cg + jj;
+                const uint32_t o = off_h<64>(t, j);
+                const uint4 kraw = *reinterpret_cast<const uint4 *>(sm + stage + C::kTK + o);
+                const __half2 *k2 = reinterpret_cast<const __half2 *>(&kraw);
+                const float4 bA = *reinterpret_cast<const float4 *>(sm + C::kB + off_f<64>(t, 2 * j));
+                const float4 bB = *reinterpret_cast<const float4 *>(sm + C::kB + off_f<64>(t, 2 * j + 1));
+                const float4 BA = *reinterpret_cast<const float4 *>(&m.Bc[slot][8 * j]);
+                const float4 BB = *reinterpret_cast<const float4 *>(&m.Bc[slot][8 * j + 4]);
+                const float bt[8] = {bA.x, bA.y, bA.z, bA.w, bB.x, bB.y, bB.z, bB.w};
+                const float Bt[8] = {BA.x, BA.y, BA.z, BA.w, BB.x, BB.y, BB.z, BB.w};
+                uint32_t ks[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const float2 kf = __half22float2(k2[e]);
+                    const float x0 = t < n ? kf.x * ptx::ex2(Bt[2 * e] - bt[2 * e]) : 0.0f;
+                    const float x1 = t < n ? kf.y * ptx::ex2(Bt[2 * e + 1] - bt[2 * e + 1]) : 0.0f;
+                    ks[e] = pack_h2(x0, x1);
+                }
+                *reinterpret_cast<uint4 *>(sm + stage + C::kTQ + o) = make_uint4(ks[0], ks[1], ks[2], ks[3]);
+            }
+        };
+        // exact scores of a chunk beyond the bf16 operands' range: row t, columns [16 cg, + 16),
+        // fp16 into the a tile (the P slot)
+        auto exact_p_smem = [&](uint32_t stage, const Chunk &c) {
+            const int n = c.n, rev = ln.rev, s0 = 16 * cg;
+            auto hat = [&](uint32_t tile, int row, int ch) {
+                return __half2float(*reinterpret_cast<const __half *>(sm + stage + tile + off_h<64>(row, ch >> 3) + (ch & 7) * 2));
+            };
+            auto bat = [&](int row, int ch) {
+                return *reinterpret_cast<const float *>(sm + C::kB + off_f<64>(row, ch >> 2) + (ch & 3) * 4);
+            };
+            float pv[16];
+            float amax = 0.0f;
+            for (int e = 0; e < 16; ++e) {
+                const int s = s0 + e;
+                const bool causal = rev ? s >= t : s <= t;
+                float acc = 0.0f;
+                if (causal && t < n && s < n)
+                    for (int ch = 0; ch < D; ++ch) {
+                        const float f = s == t ? 1.0f : ptx::ex2(bat(t, ch) - bat(s, ch));
+                        acc = fmaf(hat(C::kTQ, t, ch) * hat(C::kTK, s, ch), f, acc);
+                    }
+                pv[e] = acc * p.scale;
+                amax = fmaxf(amax, fabsf(pv[e]));
+            }
+            if (amax > 65504.0f) m.range_err = 1;
+            team_bar(1);                              // every thread has read the raw a / k / q it needs
+#pragma unroll
+            for (int h = 0; h < 2; ++h)
+                *reinterpret_cast<uint4 *>(sm + stage + C::kTA + off_h<64>(t, 2 * cg + h)) =
+                    make_uint4(pack_h2(pv[8 * h], pv[8 * h + 1]), pack_h2(pv[8 * h + 2], pv[8 * h + 3]),
+                               pack_h2(pv[8 * h + 4], pv[8 * h + 5]), pack_h2(pv[8 * h + 6], pv[8 * h + 7]));
+        };
+        auto build_full = [&](uint32_t stage, const Chunk &c, int slot, bool slow) {
+            const int n = c.n;
+            float dqs = 0.0f;
+            uint32_t qh[8], ql[8];
+#pragma unroll
+            for (int jj = 0; jj < 2; ++jj) {
+                const int j = 2 * cg + jj;
+                const uint32_t o = off_h<64>(t, j);
+                const uint4 kraw = *reinterpret_cast<const uint4 *>(sm + stage + C::kTK + o);
+                const uint4 qraw = *reinterpret_cast<const uint4 *>(sm + stage + C::kTQ + o);
+                const __half2 *k2 = reinterpret_cast<const __half2 *>(&kraw);
+                const __half2 *q2 = reinterpret_cast<const __half2 *>(&qraw);
+                const float4 bA = *reinterpret_cast<const float4 *>(sm + C::kB + off_f<64>(t, 2 * j));
+                const float4 bB = *reinterpret_cast<const float4 *>(sm + C::kB + off_f<64>(t, 2 * j + 1));
+                const float4 rA = *reinterpret_cast<const float4 *>(&m.rref[slot][8 * j]);
+                const float4 rB = *reinterpret_cast<const float4 *>(&m.rref[slot][8 * j + 4]);
+                const float *fsrc = slow ? m.Bc[slot] : m.fB[slot];
+                const float4 fA = *reinterpret_cast<const float4 *>(fsrc + 8 * j);
+                const float4 fBv = *reinterpret_cast<const float4 *>(fsrc + 8 * j + 4);
+                const float bt[8] = {bA.x, bA.y, bA.z, bA.w, bB.x, bB.y, bB.z, bB.w};
+                const float rr[8] = {rA.x, rA.y, rA.z, rA.w, rB.x, rB.y, rB.z, rB.w};
+                const float ff[8] = {fA.x, fA.y, fA.z, fA.w, fBv.x, fBv.y, fBv.z, fBv.w};
+                float kt[8], qt[8], ks[8];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const float2 kf = __half22float2(k2[e]);
+                    const float2 qf = __half22float2(q2[e]);
+                    const float kv[2] = {kf.x, kf.y}, qv[2] = {qf.x, qf.y};
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) {
+                        const int i = 2 * e + h;
+                        dqs = fmaf(qv[h], kv[h], dqs);
+                        qt[i] = qv[h] * ptx::ex2(bt[i] - rr[i]) * p.scale;
+                        if (!slow) {
+                            kt[i] = kv[h] * ptx::ex2(rr[i] - bt[i]);
+                            ks[i] = kt[i] * ff[i];
+                        } else {
+                            kt[i] = 0.0f;
+                            ks[i] = kv[h] * ptx::ex2(ff[i] - bt[i]);
+                        }
+                        if (t >= n) kt[i] = qt[i] = ks[i] = 0.0f;
+                    }
+                }
+                uint32_t kh4[4], kl4[4], ks4[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    split_bf2(kt[2 * e], kt[2 * e + 1], kh4[e], kl4[e]);
+                    split_bf2(qt[2 * e], qt[2 * e + 1], qh[4 * jj + e], ql[4 * jj + e]);
+                    ks4[e] = pack_h2(ks[2 * e], ks[2 * e + 1]);
+                }
+                if (!slow) {
+                    *reinterpret_cast<uint4 *>(sm + stage + C::kTK + o) = make_uint4(kh4[0], kh4[1], kh4[2], kh4[3]);
+                    *reinterpret_cast<uint4 *>(sm + stage + C::kTA + o) = make_uint4(kl4[0], kl4[1], kl4[2], kl4[3]);
+                }
+                *reinterpret_cast<uint4 *>(sm + stage + C::kTQ + o) = make_uint4(ks4[0], ks4[1], ks4[2], ks4[3]);
+            }
+            m.dqp[slot][cg][t] = dqs * p.scale;
+            const uint32_t rows = tmem_q + ((uint32_t)(32 * qd + 16 * slot) << 16);
+            ptx::tmem_st16x2_x8<8>(rows + C::kColQH + 16 * hg, qh);
+            ptx::tmem_st16x2_x8<8>(rows + C::kColQL + 16 * hg, ql);
+            ptx::tmem_st_wait();
+        };
+        auto step = [&](int j) {
+            const int slot = j & 1, s = j % 3;
+            const uint32_t stage = (uint32_t)s * C::kStage;
+            const Chunk c = chunk_of(j);
+            if (j >= 2) wait(&m.slotfree[slot], (j - 2) >> 1);    // back team done with chunk j - 2
+            wait(&m.ld[s], j / 3);
+            ptx::tc_fence_after_sync();
+            gate(stage, c, slot);
+            if (!c.full) {
+                build_ks(stage, c, slot);
+            } else {
+                const bool slow = m.slow[slot] != 0;
+                if (slow) exact_p_smem(stage, c);
+                build_full(stage, c, slot, slow);
+            }
+            ptx::fence_proxy_async_smem();
+            ptx::tc_fence_before_sync();
+            team_bar(1);
+            if (ttid == 0) ptx::mbar_arrive(&m.fdone[slot]);
+        };
+        for (int j = 0; j < n1; ++j) step(j);
+        if (exchange) run_exchange();
+        for (int j = n1; j < N; ++j) step(j);
+        __syncthreads();
+    }
+
+    // =================================================================== back team
+    else if (back) {
+        auto step = [&](int j) {
+            const int slot = j & 1, s = j % 3;
+            const uint32_t stage = (uint32_t)s * C::kStage;
+            const Chunk c = chunk_of(j);
+            const uint32_t rows = tmem_rows(slot);
+            wait(&m.fdone[slot], j >> 1);              // gate scalars, dq, slow flag of chunk j
+            if (c.full) {
+                // S~ = 2^{r} S (state entering chunk j); this slot's S~ was last read by chunk j - 2,
+                // whose output this team waited for
+                {
+                    const float f = m.er[slot][sc];
+                    uint8_t *sx = sm + C::kSX0 + slot * C::kSXBytes;
+#pragma unroll
+                    for (int q = 0; q < 2; ++q) {
+                        uint32_t h[4], l[4];
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) split_bf2(f * S[8 * q + 2 * e], f * S[8 * q + 2 * e + 1], h[e], l[e]);
+                        const uint32_t o = off_sx<64>(sc, 2 * cg + q);
+                        *reinterpret_cast<uint4 *>(sx + o) = make_uint4(h[0], h[1], h[2], h[3]);
+                        *reinterpret_cast<uint4 *>(sx + D * D * 2 + o) = make_uint4(l[0], l[1], l[2], l[3]);
+                    }
+                }
+                ptx::fence_proxy_async_smem();
+                team_bar(2);
+                if (ttid == 0) ptx::mbar_arrive(&m.sx[slot]);
+                wait(&m.sc[slot], j >> 1);              // scores done: the K~-low tile is free
+                ptx::tc_fence_after_sync();
+                if (!m.slow[slot]) {
+                    float dq = 0.0f;
+#pragma unroll
+                    for (int g = 0; g < 4; ++g) dq += m.dqp[slot][g][t];
+                    float r[16];
+                    ptx::tmem_ld16x2_x16<16>(rows + C::kColSC + 32 * hg, r);
+                    ptx::tmem_ld_wait();
+                    const int s0 = 16 * cg, n = c.n, rev = ln.rev;
+                    float amax = 0.0f;
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) {
+                        const int sp = s0 + e;
+                        const bool before = rev ? sp > t : sp < t;
+                        float v = before ? r[e] : (sp == t ? dq : 0.0f);
+                        v = (t < n && sp < n) ? v : 0.0f;
+                        r[e] = v;
+                        amax = fmaxf(amax, fabsf(v));
+                    }
+                    if (amax > 65504.0f) m.range_err = 1;
+#pragma unroll
+                    for (int h = 0; h < 2; ++h)
+                        *reinterpret_cast<uint4 *>(sm + stage + C::kTA + off_h<64>(t, 2 * cg + h)) =
+                            make_uint4(pack_h2(r[8 * h], r[8 * h + 1]), pack_h2(r[8 * h + 2], r[8 * h + 3]),
+                                       pack_h2(r[8 * h + 4], r[8 * h + 5]), pack_h2(r[8 * h + 6], r[8 * h + 7]));
+                }
+                ptx::fence_proxy_async_smem();
+                ptx::tc_fence_before_sync();
+                team_bar(2);
+                if (ttid == 0) ptx::mbar_arrive(&m.pfull[slot]);
+            } else {                                    // state-only chunk: no S~, no P
+                if (ttid == 0) {
+                    ptx::mbar_arrive(&m.sx[slot]);
+                    ptx::mbar_arrive(&m.pfull[slot]);
+                }
+                wait(&m.sc[slot], j >> 1);              // bare commit; keeps the waits in phase
+            }
+            // S = Diag(2^{B}) S + S_loc
+            wait(&m.sl[slot], j >> 1);
+            ptx::tc_fence_after_sync();
+            {
+                float sl[16];
+                ptx::tmem_ld16x2_x16<16>(tmem + ((uint32_t)(32 * qd + 16 * slot) << 16) + C::kColSL + 32 * hg, sl);
+                ptx::tmem_ld_wait();
+                const float e = m.eB[slot][sc];
+#pragma unroll
+                for (int i = 0; i < 16; ++i) S[i] = fmaf(e, S[i], sl[i]);
+            }
+            if (!c.full && ttid < D) m.Gs[ttid] += m.Bc[slot][ttid];
+            wait(&m.o[slot], j >> 1);                   // a state-only chunk's is a bare commit
+            if (c.full) {
+                ptx::tc_fence_after_sync();
+                float o[16];
+                ptx::tmem_ld16x2_x16<16>(rows + C::kColO + 32 * hg, o);
+                ptx::tmem_ld_wait();
+                float ss = 0.0f;
+#pragma unroll
+                for (int jj = 0; jj < 16; ++jj) ss = fmaf(o[jj], o[jj], ss);
+                m.red[cg][t] = ss;
+                team_bar(2);
+                const float inv = rsqrtf((m.red[0][t] + m.red[1][t] + m.red[2][t] + m.red[3][t]) * (1.0f / D) + p.eps);
+                if (t < c.n) {
+                    __half *dst = p.out + (size_t)token_row(c, t) * D + 16 * cg;
+#pragma unroll
+                    for (int jj = 0; jj < 2; ++jj) {
+                        const int jp = 2 * cg + jj;
+                        const uint4 graw = *reinterpret_cast<const uint4 *>(sm + stage + C::kTG + off_h<64>(t, jp));
+                        const __half2 *g2 = reinterpret_cast<const __half2 *>(&graw);
+                        const float4 wa = *reinterpret_cast<const float4 *>(&m.w[8 * jp]);
+                        const float4 wb = *reinterpret_cast<const float4 *>(&m.w[8 * jp + 4]);
+                        const float wv[8] = {wa.x, wa.y, wa.z, wa.w, wb.x, wb.y, wb.z, wb.w};
+                        uint32_t u[4];
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const float2 gf = __half22float2(g2[e]);
+                            u[e] = pack_h2(o[8 * jj + 2 * e] * inv * wv[2 * e] * silu_fast(gf.x),
+                                           o[8 * jj + 2 * e + 1] * inv * wv[2 * e + 1] * silu_fast(gf.y));
+                        }
+                        *reinterpret_cast<uint4 *>(dst + 8 * jj) = make_uint4(u[0], u[1], u[2], u[3]);
+                    }
+                }
+            }
+            ptx::tc_fence_before_sync();
+            team_bar(2);                                // every read of this slot and stage is done
+            if (ttid == 0) {
+                ptx::mbar_arrive(&m.slotfree[slot]);
+                ptx::mbar_arrive(&m.stfree[s]);
+            }
+        };
+        for (int j = 0; j < n1; ++j) step(j);
+        if (exchange) run_exchange();
+        for (int j = n1; j < N; ++j) step(j);
+        __syncthreads();
+    }
+
+    // ---- teardown (every thread arrives here after the role's own teardown barrier)
+    __syncthreads();
+    if (tid == 0 && m.range_err) raise_status(8 /* GLA_ERR_RANGE */);
+    ptx::tc_fence_after_sync();
+    if (warp == 0) ptx::tmem_dealloc(tmem, C::kTmemCols);
+}
+
+}  // namespace ck
+}  // namespace gla

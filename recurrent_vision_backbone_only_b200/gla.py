@@ -157,8 +157,9 @@ def gla_fwd(q, k, v, a, g, w, out, grid_h: int, grid_w: int, direction: int, str
     return out
 
 
-KERNEL_AUTO, KERNEL_TC128, KERNEL_SIMT, KERNEL_TC64 = 0, 1, 2, 3
-KERNEL_NAMES = {1: "tensor-core 128-row", 2: "cuda-core", 3: "tensor-core 64-row"}
+KERNEL_AUTO, KERNEL_TC128, KERNEL_SIMT, KERNEL_TC64, KERNEL_PIPE64 = 0, 1, 2, 3, 4
+KERNEL_NAMES = {1: "tensor-core 128-row", 2: "cuda-core", 3: "tensor-core 64-row",
+                4: "tensor-core 64-row pipelined"}
 
 
 def gla_fwd_ex(q, k, v, a, g, w, out, grid_h: int, grid_w: int, direction: int,

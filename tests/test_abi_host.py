@@ -109,7 +109,7 @@ def test_plan_rejects_bad_arguments(lib):
 
 def test_ex_rejects_bad_schedule(lib):
     bad = [(5, 0, 0, 0), (0, 0, 17, 0), (0, -1, 0, 0), (1, 0, -2, 0),   # dtype, chunk, segs,
-           (0, 0, 0, 4), (0, 0, 0, -1), (1, 0, 0, 1), (1, 0, 0, 3)]          # kernel
+           (0, 0, 0, 5), (0, 0, 0, -1), (1, 0, 0, 1), (1, 0, 0, 3), (1, 0, 0, 4)]   # kernel
     for dtype, chunk, segs, kernel in bad:
         rc = call("gla_fwd_ex", extra=(dtype, chunk, segs, ctypes.c_float(1e-6), kernel))
         assert rc == 3, (dtype, chunk, segs, kernel, rc)

@@ -49,13 +49,13 @@ def lib(cuda_ok):
     return gla.load()
 
 
-@pytest.mark.parametrize("d", [64, 128])
-@pytest.mark.parametrize("kind", [0, 1, 2, 3])
+@pytest.mark.parametrize("d,kind", [(d, k) for d in (64, 128) for k in range(4)] + [(64, 4)])
 def test_selftest_chunk_products(lib, d, kind):
     import torch
     rng = np.random.default_rng(10 * kind + d)
     shapes = {0: ((64, d), (64, d), (64, 64)), 1: ((64, d), (64, d), (d, d)),
-              2: ((64, 64), (64, d), (64, d)), 3: ((64, d), (d, d), (64, d))}
+              2: ((64, 64), (64, d), (64, d)), 3: ((64, d), (d, d), (64, d)),
+              4: ((64, 64), (64, d), (64, d))}
     sa, sb, sd = shapes[kind]
     A = structured(rng, sa, 0)
     B = structured(rng, sb, 1)
@@ -66,7 +66,7 @@ def test_selftest_chunk_products(lib, d, kind):
     torch.cuda.synchronize()
     D = dD.cpu().numpy().astype(np.float64)
     assert np.all(np.isfinite(D))
-    if kind in (1, 2):
+    if kind in (1, 2, 4):
         a16 = A.astype(np.float16).astype(np.float64)
         b16 = B.astype(np.float16).astype(np.float64)
         expect = a16.T @ b16 if kind == 1 else a16 @ b16

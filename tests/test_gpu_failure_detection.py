@@ -40,7 +40,8 @@ def test_bounded_wait_expires_and_context_survives(cuda_ok):
     assert np.max(np.abs(out.cpu().numpy().astype(np.float64) - ref)) < 1e-2
 
 
-@pytest.mark.parametrize("kernel,d,segments", [(gla.KERNEL_TC64, 64, 1), (gla.KERNEL_TC64, 64, 4),
+@pytest.mark.parametrize("kernel,d,segments", [(gla.KERNEL_PIPE64, 64, 1), (gla.KERNEL_PIPE64, 64, 4),
+                                               (gla.KERNEL_TC64, 64, 1), (gla.KERNEL_TC64, 64, 4),
                                                (gla.KERNEL_TC64, 128, 3), (gla.KERNEL_TC128, 64, 1),
                                                (gla.KERNEL_TC128, 64, 4)])
 def test_operator_wait_expires_and_returns_promptly(cuda_ok, kernel, d, segments):

@@ -24,7 +24,7 @@ def torch_dev(x):
     return torch.from_numpy(np.ascontiguousarray(x)).cuda()
 
 
-TC128, SIMT, TC64 = gla.KERNEL_TC128, gla.KERNEL_SIMT, gla.KERNEL_TC64
+TC128, SIMT, TC64, PIPE64 = gla.KERNEL_TC128, gla.KERNEL_SIMT, gla.KERNEL_TC64, gla.KERNEL_PIPE64
 
 
 def run_gpu(x, gh, gw, direction, chunk=0, segments=0, eps=1e-6, kernel=0):
@@ -86,7 +86,7 @@ def test_tiny_fp32(direction):
     assert_close(u2, oracle_ref(x, wl.grid_h, wl.grid_w, direction), "f32")
 
 
-@pytest.mark.parametrize("kernel", [0, TC64])
+@pytest.mark.parametrize("kernel", [0, TC64, PIPE64])
 @pytest.mark.parametrize("name", ["gtr640", "highres"])
 def test_full_workloads_all_directions(name, kernel):
     # kernel 0: the one gla_fwd picks (the 128-row tensor-core kernel at d = 64)
@@ -97,7 +97,7 @@ def test_full_workloads_all_directions(name, kernel):
                      oracle_ref(x, wl.grid_h, wl.grid_w, d), wl.dtype)
 
 
-@pytest.mark.parametrize("kernel", [0, TC64])
+@pytest.mark.parametrize("kernel", [0, TC64, PIPE64])
 def test_batched_cycle(kernel):
     wl = synth.WORKLOADS["batched"]
     x = synth.make_inputs(wl)
@@ -114,8 +114,8 @@ def test_stress_all_pairs(direction):
     assert_close(u, oracle_ref(x, wl.grid_h, wl.grid_w, direction), wl.dtype)
 
 
-@pytest.mark.parametrize("dtype,kernel", [("f16", TC128), ("f16", TC64), ("f16", SIMT),
-                                          ("f32", SIMT)])
+@pytest.mark.parametrize("dtype,kernel", [("f16", TC128), ("f16", TC64), ("f16", PIPE64),
+                                          ("f16", SIMT), ("f32", SIMT)])
 def test_chunk_and_segment_invariance(dtype, kernel):
     wl = synth.WORKLOADS["gtr640"].with_(H=2, dtype=dtype, grid_h=24, grid_w=37)
     x = synth.make_inputs(wl)
@@ -190,9 +190,9 @@ def test_eps_is_honoured():
         assert_close(u, ref, "f32")
 
 
-@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("d,kernel", [(64, TC64), (128, TC64), (64, PIPE64)])
 @pytest.mark.parametrize("segs", [2, 5, 7, 12, 13, 15, 16])
-def test_segment_counts_64_row_kernel(segs, d):
+def test_segment_counts_64_row_kernel(segs, d, kernel):
     # the state exchange deals key channel c to scanner c % segs: counts that do not divide d
     # give scanners unequal channel counts.  chunk 64 gives segments of one or two chunks,
     # chunk 16 segments of several (state-only pass, exchange, full pass)
@@ -200,7 +200,7 @@ def test_segment_counts_64_row_kernel(segs, d):
     x = synth.make_inputs(wl, seed=segs)
     ref = oracle_ref(x, 24, 37, 2)
     for chunk in (16, 64):
-        assert_close(run_gpu(x, 24, 37, 2, chunk=chunk, segments=segs, kernel=TC64), ref, "f16")
+        assert_close(run_gpu(x, 24, 37, 2, chunk=chunk, segments=segs, kernel=kernel), ref, "f16")
 
 
 @pytest.mark.parametrize("segs", [2, 5, 7, 12])
@@ -229,7 +229,9 @@ def test_unsupported_schedules_are_refused(kernel, chunk, segs, d):
                        chunk=chunk, segments=segs, kernel=kernel)
 
 
-@pytest.mark.parametrize("kernel,d,segs,chunk", [(TC64, 64, 3, 64), (TC64, 64, 16, 64),
+@pytest.mark.parametrize("kernel,d,segs,chunk", [(PIPE64, 64, 3, 64), (PIPE64, 64, 16, 64),
+                                                 (PIPE64, 64, 5, 32),
+                                                 (TC64, 64, 3, 64), (TC64, 64, 16, 64),
                                                  (TC64, 64, 5, 32), (TC64, 128, 3, 64),
                                                  (TC64, 128, 16, 64), (TC64, 128, 5, 32),
                                                  (TC128, 64, 3, 128), (TC128, 64, 16, 128),
@@ -257,7 +259,8 @@ def test_empty_launch_runs_clean():
 
 
 @pytest.mark.parametrize("kernel,gh,gw,chunk,segs", [(TC128, 16, 20, 32, 9), (TC128, 42, 50, 128, 16),
-                                                     (TC128, 42, 50, 0, 0), (TC64, 16, 20, 32, 9),
+                                                     (TC128, 42, 50, 0, 0), (PIPE64, 16, 20, 32, 9),
+                                                     (PIPE64, 42, 50, 64, 16), (TC64, 16, 20, 32, 9),
                                                      (TC64, 42, 50, 64, 16), (TC64, 42, 50, 0, 0)])
 def test_shorter_last_segment(kernel, gh, gw, chunk, segs):
     # a last segment shorter than the others (128-row kernel, 16x20: 9 segments of 36 tokens
