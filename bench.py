@@ -54,6 +54,12 @@ def parse():
     ap.add_argument("--workload", default=WORKLOAD,
                     help="synthetic workload to time (default: the 40x40 headline); the others "
                          "are reported with their own metric name")
+    ap.add_argument("--record-traffic", metavar="NCU_CSV",
+                    help="no bench: read an ncu CSV (dram__bytes_read.sum / dram__bytes_write.sum "
+                         "of the kernel --kernel / --workload select) and print the traffic entry "
+                         "for profiles/traffic.json, stamped with this build's sources digest")
+    ap.add_argument("--ncu-command", default="",
+                    help="with --record-traffic: the ncu command line that wrote the CSV")
     return ap.parse_args()
 
 
@@ -89,18 +95,87 @@ def measured_peaks():
         return FALLBACK_HBM_GBS, "fallback"
 
 
-def profile_traffic(workload: str):
-    """dram bytes per launch from the committed ncu summary, if it was taken on this workload
-    and this kernel build."""
+def profile_traffic(workload: str, kernel: str):
+    """DRAM bytes per launch from the committed ncu entries (profiles/traffic.json), if one was
+    taken on this workload, this kernel and this exact kernel build (sources digest); else None."""
     try:
         with open(PROFILE_TRAFFIC) as f:
             d = json.load(f)
         from recurrent_vision_backbone_only_b200 import build as _b
-        if d.get("workload") != workload or d.get("lib_sources_digest") != _b.sources_digest():
-            return None
-        return d.get("dram_bytes_per_launch")
+        digest = _b.sources_digest()
+        for e in d.get("entries", []):
+            if (e.get("workload") == workload and e.get("kernel") == kernel and
+                    e.get("lib_sources_digest") == digest):
+                return e.get("dram_bytes_per_launch")
+        return None
     except Exception:
         return None
+
+
+def read_ncu_csv(path: str):
+    """Launches of an ncu --csv log (details layout: one row per metric; raw layout: one column
+    per metric) as [(kernel name, {metric: value})], in capture order."""
+    import csv
+    with open(path, newline="") as f:
+        lines = [ln for ln in f if ln.startswith('"')]
+    rows = list(csv.reader(lines))
+    if not rows or rows[0][:1] != ["ID"]:
+        raise ValueError("%s: no ncu CSV header" % path)
+    head = rows[0]
+    launches = {}
+    order = []
+    if "Metric Name" in head:
+        i_id, i_k = head.index("ID"), head.index("Kernel Name")
+        i_n, i_v = head.index("Metric Name"), head.index("Metric Value")
+        i_u = head.index("Metric Unit")
+        scale = {"byte": 1, "Kbyte": 1e3, "Mbyte": 1e6, "Gbyte": 1e9}
+        for r in rows[1:]:
+            if len(r) <= i_v:
+                continue
+            key = r[i_id]
+            if key not in launches:
+                launches[key] = (r[i_k], {})
+                order.append(key)
+            v = float(r[i_v].replace(",", ""))
+            launches[key][1][r[i_n]] = v * scale.get(r[i_u], 1)
+    else:
+        units = rows[1]
+        i_id, i_k = head.index("ID"), head.index("Kernel Name")
+        scale = {"byte": 1, "Kbyte": 1e3, "Mbyte": 1e6, "Gbyte": 1e9}
+        for r in rows[2:]:
+            vals = {}
+            for j, name in enumerate(head):
+                if name.startswith(("dram__", "gpu__time")) and j < len(r) and r[j]:
+                    vals[name] = float(r[j].replace(",", "")) * scale.get(units[j], 1)
+            launches[r[i_id]] = (r[i_k], vals)
+            order.append(r[i_id])
+    return [launches[k] for k in order]
+
+
+def record_traffic(args):
+    """Print the profiles/traffic.json entry for the launches of `args.record_traffic`."""
+    import re
+    from recurrent_vision_backbone_only_b200 import build as _b, gla, synth
+    wl = synth.WORKLOADS[args.workload]
+    kid = {"auto": 0, "tc128": gla.KERNEL_TC128, "tc64": gla.KERNEL_TC64,
+           "pipe64": gla.KERNEL_PIPE64, "simt": gla.KERNEL_SIMT}[args.kernel]
+    symbol = {gla.KERNEL_TC128: "gla_tc_kernel", gla.KERNEL_TC64: "gla_chunk_kernel",
+              gla.KERNEL_PIPE64: "gla_pipe_kernel", gla.KERNEL_SIMT: "gla_simt_kernel"}
+    if not kid:
+        raise SystemExit("--record-traffic needs an explicit --kernel")
+    got = [v for k, v in read_ncu_csv(args.record_traffic) if re.search(symbol[kid], k)]
+    got = [v for v in got if "dram__bytes_read.sum" in v and "dram__bytes_write.sum" in v]
+    if not got:
+        raise SystemExit("no %s launch with dram__bytes_read/write.sum in %s"
+                         % (symbol[kid], args.record_traffic))
+    rd = statistics.mean(v["dram__bytes_read.sum"] for v in got)
+    wr = statistics.mean(v["dram__bytes_write.sum"] for v in got)
+    print(json.dumps({"workload": wl.name, "kernel": gla.KERNEL_NAMES[kid],
+                      "lib_sources_digest": _b.sources_digest(), "launches": len(got),
+                      "dram_read_bytes": rd, "dram_write_bytes": wr,
+                      "dram_bytes_per_launch": rd + wr,
+                      "algorithmic_bytes_per_launch": wl.tokens * wl.bytes_per_token,
+                      "command": args.ncu_command}))
 
 
 class ClockSampler:
@@ -320,6 +395,8 @@ def run_ours(args, ws, rank, local):
 
     kernel = {"auto": 0, "tc128": gla.KERNEL_TC128, "tc64": gla.KERNEL_TC64,
               "pipe64": gla.KERNEL_PIPE64, "simt": gla.KERNEL_SIMT}[args.kernel]
+    kernel_name = (gla.KERNEL_NAMES[kernel] if kernel else
+                   gla.plan(wl.B, wl.H, gh, gw, wl.d_k, wl.d_v, 0 if wl.dtype == "f16" else 1)["kernel"])
 
     def step(i):
         for j, d in enumerate(directions):
@@ -445,7 +522,8 @@ def run_ours(args, ws, rank, local):
                         if not kernel else {"kernel": gla.KERNEL_NAMES[kernel]},
         },
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-                     "frac": achieved / peak, "traffic": profile_traffic(wl.name),
+                     "frac": achieved / peak,
+                     "traffic": profile_traffic(wl.name, kernel_name),
                      "peak_source": "%s (MEASURED_PEAKS.json hbm_gbs)" % peak_kind
                      if peak_kind == "measured" else "fallback 6.65 TB/s",
                      "bytes_per_launch": bytes_per_launch,
@@ -464,6 +542,9 @@ def run_ours(args, ws, rank, local):
 def main():
     args = parse()
     ws, rank, local = dist_env()
+    if args.record_traffic:
+        record_traffic(args)
+        return
     if args.impl == "reference":
         run_reference(args, ws, rank)
         return

@@ -246,6 +246,21 @@ int gla_selftest_load(const void *q, const void *k, const void *gate_preact, con
                       int direction, int chunk, float *out, int *info, void *stream);
 
 /*
+ * gla_scan_layout -- host-only (no device work, no CUDA call): the token each tile row of
+ * each chunk holds when `kernel` (GLA_KERNEL_PIPE64 only) runs a scan of a
+ * grid_h x grid_w grid in `direction` (0..3) with chunks of at most `chunk` positions
+ * (0: 64).  Writes spatial[p] = the row-major spatial index (y * grid_w + x) of the token the
+ * kernel's tiles place at scan position p, for p in [0, grid_h * grid_w) (HOST int array of that
+ * length; a position no tile row claims stays -1, one claimed twice returns GLA_ERR_SHAPE),
+ * and *box_rows = the rows per TMA box (64 for line-aligned chunks).  The scan order is the
+ * one of the scan-direction paragraph of the GTR paper's method section (lines in increasing
+ * order, the state carried from one line's end to the next line's start); the test suite
+ * compares this map with the reference's own on the CPU.
+ */
+int gla_scan_layout(int kernel, int grid_h, int grid_w, int direction, int chunk, int *spatial,
+                    int *box_rows);
+
+/*
  * gla_selftest_mma -- diagnostic: runs ONE of the four matrix products of the previous
  * 128-row tensor-core kernel on a single CTA, on row-major float32 DEVICE arrays:
  *   kind 0  D[128][128] = A[128][64] * B[128][64]^T   (split tf32)

@@ -383,28 +383,31 @@ EncodeTiledFn encode_fn() {
 // 3-D views of a token-major fp16 array [B][gh][gw][H][D] whose boxes (64 channels x 1 x 64
 // positions, 128B-swizzled) are 64 consecutive positions of one grid row (row family: view
 // [B gh gw][H][D]) or of one grid column (column family: view [B gh][gw H][D]) of one head.
-bool make_line_map(CUtensorMap *map, const void *base, int fam, int B, int H, int gh, int gw, int D) {
+bool make_line_map(CUtensorMap *map, const void *base, int fam, int B, int H, int gh, int gw, int D,
+                   int rows) {
     EncodeTiledFn fn = encode_fn();
     if (!fn) return false;
     const cuuint64_t mid = fam ? (cuuint64_t)gw * H : (cuuint64_t)H;
     const cuuint64_t outer = fam ? (cuuint64_t)B * gh : (cuuint64_t)B * gh * gw;
     const cuuint64_t dims[3] = {(cuuint64_t)D, mid, outer};
     const cuuint64_t strides[2] = {(cuuint64_t)D * 2, mid * D * 2};
-    const cuuint32_t box[3] = {64, 1, 64};
+    const cuuint32_t box[3] = {64, 1, (cuuint32_t)rows};
     const cuuint32_t estr[3] = {1, 1, 1};
     return fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3, const_cast<void *>(base), dims, strides, box, estr,
               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// Tensor maps of the five inputs for the line families the directions of a launch use.
-bool make_maps(ck::Maps *maps, const void *const src[5], int dir, int B, int H, int gh, int gw, int D) {
+// Tensor maps of the five inputs for the line families the directions of a launch use; boxes
+// of rows[fam] positions (64, or the group height of packed chunks).
+bool make_maps(ck::Maps *maps, const void *const src[5], int dir, int B, int H, int gh, int gw, int D,
+               const int rows[2]) {
     for (int fam = 0; fam < 2; ++fam) {
         const bool used = dir == 4 || (dir >> 1) == fam;
         if (!used) continue;
         CUtensorMap *dst = fam ? maps->col : maps->row;
         for (int i = 0; i < 5; ++i)
-            if (!make_line_map(&dst[i], src[i], fam, B, H, gh, gw, D)) return false;
+            if (!make_line_map(&dst[i], src[i], fam, B, H, gh, gw, D, rows[fam])) return false;
     }
     return true;
 }
@@ -442,11 +445,21 @@ int run_chunk(const Args &x, int chunk, int segs, float eps, cudaStream_t st, co
     const int n_pairs = x.B * x.H;
     if (chunk <= 0) chunk = ck::kC;
     if (chunk % 16 != 0 || chunk > ck::kC) return GLA_ERR_UNSUPPORTED;
-    // chunks per scan: lines are cut into pieces of at most `chunk` positions; a cycling
+    // chunks per scan: the pipelined kernel packs chunks across lines where the line length
+    // allows (hb > 0), the other cuts lines into pieces of at most `chunk` positions; a cycling
     // launch mixes both line families
-    int q = 0;
+    int hb[2] = {0, 0};
+    if (kPipe) {
+        hb[0] = ck::pack_rows(x.gw, chunk);
+        hb[1] = ck::pack_rows(x.gh, chunk);
+    }
+    int q = 0, clen = 0;
     for (int dir = 0; dir < 4; ++dir)
-        if (x.dir == 4 || x.dir == dir) q = std::max(q, ck::Lines(dir, x.gh, x.gw, chunk).chunks);
+        if (x.dir == 4 || x.dir == dir) {
+            const ck::Scan sc(dir, x.gh, x.gw, chunk, hb[dir >> 1]);
+            q = std::max(q, sc.chunks);
+            clen = std::max(clen, sc.cl);
+        }
     const size_t smem_max = kPipe ? ck::pipe_smem_bytes() : chunk_smem<D>(true);
     if (smem_max > (size_t)di.max_smem_optin) return GLA_ERR_UNSUPPORTED;
     // all of the unified L1 / shared memory as shared memory, so two d = 64 CTAs fit on an SM
@@ -503,7 +516,7 @@ int run_chunk(const Args &x, int chunk, int segs, float eps, cudaStream_t st, co
     }
     if (segs > 16) return GLA_ERR_UNSUPPORTED;
     pl.segs = segs;
-    pl.seg_len = std::min(L, ceil_div(q, segs) * ck::Lines(x.dir == 4 ? 0 : x.dir, x.gh, x.gw, chunk).clen);
+    pl.seg_len = std::min(L, ceil_div(q, segs) * clen);
     const bool spread = (long long)n_pairs * pl.segs <= di.sms;
     pl.smem = smem_of(spread);
     configure_launch(pl, n_pairs, kThreads, st);
@@ -515,7 +528,8 @@ int run_chunk(const Args &x, int chunk, int segs, float eps, cudaStream_t st, co
     }
     ck::Maps maps;
     const void *const src[5] = {x.q, x.k, x.a, x.v, x.g};
-    if (!make_maps(&maps, src, x.dir, x.B, x.H, x.gh, x.gw, D)) return GLA_ERR_CUDA;
+    const int rows[2] = {hb[0] > 0 ? hb[0] : 64, hb[1] > 0 ? hb[1] : 64};
+    if (!make_maps(&maps, src, x.dir, x.B, x.H, x.gh, x.gw, D, rows)) return GLA_ERR_CUDA;
     ck::Params p;
     p.out = static_cast<__half *>(x.out);
     p.w = x.w;
@@ -525,6 +539,8 @@ int run_chunk(const Args &x, int chunk, int segs, float eps, cudaStream_t st, co
     p.scale = 1.0f / sqrtf((float)D);
     p.wait_limit = wait_limit;
     p.fault_chunk = fault_chunk;
+    p.hb[0] = hb[0];
+    p.hb[1] = hb[1];
     if (cudaLaunchKernelEx(&pl.cfg, kern, maps, p) != cudaSuccess) {
         cudaGetLastError();
         return GLA_ERR_CUDA;
@@ -796,6 +812,34 @@ int gla_selftest_chunk(int d, int kind, const float *A, const float *B, float *D
     return launch(ck::gla_chunk_selftest_kernel<128>, ck::Cfg<128>::kThreads, ck::smem_bytes<128>());
 }
 
+int gla_scan_layout(int kernel, int grid_h, int grid_w, int direction, int chunk, int *spatial,
+                    int *box_rows) {
+    if (!spatial || !box_rows) return GLA_ERR_NULL;
+    if (kernel != kPipe64) return GLA_ERR_UNSUPPORTED;
+    if (grid_h <= 0 || grid_w <= 0 || (long long)grid_h * grid_w > (1LL << 30)) return GLA_ERR_SHAPE;
+    if (direction < 0 || direction > 3) return GLA_ERR_UNSUPPORTED;
+    if (chunk <= 0) chunk = ck::kC;
+    if (chunk % 16 != 0 || chunk > ck::kC) return GLA_ERR_UNSUPPORTED;
+    const int L = grid_h * grid_w;
+    const int fam = direction >> 1;
+    const int hb = ck::pack_rows(fam ? grid_h : grid_w, chunk);
+    const ck::Scan sc(direction, grid_h, grid_w, chunk, hb);
+    for (int p = 0; p < L; ++p) spatial[p] = -1;
+    for (int q = 0; q < sc.chunks; ++q) {
+        int p0, n;
+        sc.chunk(q, L, p0, n);
+        for (int i = 0; i < n; ++i) {
+            int line, lp;
+            sc.place(p0, n, i, line, lp);
+            const int pos = p0 + sc.row_of(i, n);
+            if (pos < 0 || pos >= L || spatial[pos] != -1) return GLA_ERR_SHAPE;
+            spatial[pos] = fam ? lp * grid_w + line : line * grid_w + lp;
+        }
+    }
+    *box_rows = hb > 0 ? hb : 64;
+    return GLA_OK;
+}
+
 int gla_selftest_load(const void *q, const void *k, const void *gate_preact, const void *v,
                       const void *out_gate_preact, int B, int H, int grid_h, int grid_w, int d,
                       int direction, int chunk, float *out, int *info, void *stream) {
@@ -811,7 +855,8 @@ int gla_selftest_load(const void *q, const void *k, const void *gate_preact, con
     int rc = current_device_info(&di);
     if (rc != GLA_OK) return rc;
     ck::Maps maps;
-    if (!make_maps(&maps, src, direction, B, H, grid_h, grid_w, d)) return GLA_ERR_CUDA;
+    const int rows[2] = {64, 64};
+    if (!make_maps(&maps, src, direction, B, H, grid_h, grid_w, d, rows)) return GLA_ERR_CUDA;
     const cudaStream_t st = static_cast<cudaStream_t>(stream);
     auto launch = [&](auto kern, size_t tile) {
         const size_t smem = 5 * tile + 64 + 1024;

@@ -126,11 +126,13 @@ struct Params {
     float eps, scale;   // RMSNorm epsilon, d_k^{-1/2}
     long long wait_limit;   // bound of every mbarrier wait, SM clocks
     int fault_chunk;        // test hook: full-pass chunk whose loads are not issued (-1: none)
+    int hb[2];              // pipelined kernel: rows per TMA box of packed chunks for the row and
+                            // column families (0: line-aligned chunks, one 64-row box per tile)
 };
 
 // Tensor maps of the five inputs in the two line families: row family [B L][H][D] (box: 64
-// channels x 1 head x 64 consecutive positions of a row), column family [B gh][W H][D] (64
-// consecutive positions of a column).
+// channels x 1 head x 64 -- or, for packed chunks, hb -- consecutive positions of a row),
+// column family [B gh][W H][D] (consecutive positions of a column).
 struct Maps {
     CUtensorMap row[5];     // q, k, a, v, g
     CUtensorMap col[5];

@@ -3,8 +3,17 @@
 //
 // Operation and chunkwise form: as gla_chunk.cuh (GTR paper, arXiv 2609.26590, method
 // section: S_t = Diag(gamma_t) S_{t-1} + k_t^T v_t, o_t = d_k^{-1/2} q_t S_t, u_t = SiLU(g_t) *
-// RMSNorm(o_t) * w), with the same 16-bit products, line-aligned chunks, TMA boxes and cluster
-// state exchange.  Only the schedule differs.
+// RMSNorm(o_t) * w), with the same 16-bit products and cluster state exchange.  The schedule and
+// the chunking differ.
+//
+// Packed chunks.  Chunk q holds the scan positions [q cl, q cl + cl) whatever lines they
+// cross, so every tile row carries a token (a 40-position line no longer leaves 24 of 64 rows
+// empty).  When hb -- the largest power of two <= 64 dividing both the line length and cl -- is
+// at least 8, every aligned group of hb positions lies in one line and its tokens are equally
+// spaced in memory, so a tile is 64 / hb TMA boxes of hb rows.  Each box is loaded in increasing
+// spatial order; in R->L and B->T the scan runs against it, so scan offset i sits in tile row
+// i ^ (hb - 1).  Other line lengths keep line-aligned chunks (one 64-row box, scan offset i in
+// row n - 1 - i when reversed).
 //
 // Roles (576 threads):
 //   front team  (warps 0-7)   per chunk: gate (cumulative log2-decay b), then the operands Kh,
@@ -79,6 +88,67 @@ struct PipeMisc {
 
 constexpr size_t pipe_smem_bytes() { return PipeCfg::kMisc + sizeof(PipeMisc) + 1024; }
 
+// Rows per TMA box of a packed chunk for lines of length `len` and chunks of `cl` positions:
+// the largest power of two <= 64 dividing both, or 0 (line-aligned chunks) when below 8.
+__host__ __device__ inline int pack_rows(int len, int cl) {
+    int hb = 64;
+    while (hb >= 8 && (len % hb != 0 || cl % hb != 0)) hb >>= 1;
+    return hb >= 8 ? hb : 0;
+}
+
+// Chunks of one (b, h) scan.  Packed (hb > 0): chunk q is the scan positions [q cl, q cl + cl);
+// line-aligned (hb = 0): every line is cut into `pieces` equal pieces of at most cl positions.
+struct Scan {
+    int fam;      // 0: lines are grid rows (L->R, R->L), 1: grid columns (T->B, B->T)
+    int rev;      // the scan runs against the spatial order within a line (R->L, B->T)
+    int len;      // line length
+    int hb;       // rows per box of a packed chunk, 0: line-aligned chunks
+    int cl;       // chunk length (the last chunk may be shorter)
+    int pieces;   // line-aligned: chunks per line
+    int chunks;   // chunks per scan
+    __host__ __device__ Scan(int dir, int gh, int gw, int chunk_max, int hb_) {
+        fam = dir >> 1;
+        rev = dir & 1;
+        len = fam ? gh : gw;
+        hb = hb_;
+        if (hb > 0) {
+            cl = chunk_max;
+            pieces = 0;
+            chunks = (gh * gw + cl - 1) / cl;
+        } else {
+            pieces = (len + chunk_max - 1) / chunk_max;
+            cl = (len + pieces - 1) / pieces;
+            chunks = (fam ? gw : gh) * pieces;
+        }
+    }
+    // first scan position and length of chunk q of a scan of L positions
+    __host__ __device__ void chunk(int q, int L, int &p0, int &n) const {
+        if (hb > 0) {
+            p0 = q * cl;
+            n = min(cl, L - p0);
+        } else {
+            const int line = q / pieces, start = (q - line * pieces) * cl;
+            p0 = line * len + start;
+            n = min(cl, len - start);
+        }
+    }
+    // tile row of scan offset i in a chunk of n positions (an involution: also the offset of row i)
+    __host__ __device__ int row_of(int i, int n) const { return rev ? (hb > 0 ? i ^ (hb - 1) : n - 1 - i) : i; }
+    // line and position along it of tile row i of the chunk starting at scan position p0
+    __host__ __device__ void place(int p0, int n, int i, int &line, int &lp) const {
+        if (hb > 0) {
+            const int pg = p0 + (i & ~(hb - 1));
+            line = pg / len;
+            const int o = pg - line * len;
+            lp = (rev ? len - o - hb : o) + (i & (hb - 1));
+        } else {
+            line = p0 / len;
+            const int st = p0 - line * len;
+            lp = (rev ? len - st - n : st) + i;
+        }
+    }
+};
+
 __device__ __forceinline__ void team_bar(int id) { ptx::named_bar_sync(id, PipeCfg::kTeam); }
 
 __global__ void __launch_bounds__(PipeCfg::kThreads, 1)
@@ -104,7 +174,7 @@ __global__ void __launch_bounds__(PipeCfg::kThreads, 1)
     const int rank = blockIdx.x - pair * p.segs;
     const int bb = pair / p.H, hh = pair - bb * p.H;
     const int dir = p.dir == 4 ? (bb & 3) : p.dir;
-    const Lines ln(dir, p.gh, p.gw, p.chunk_max);
+    const Scan ln(dir, p.gh, p.gw, p.chunk_max, p.hb[dir >> 1]);
     const int seg_chunks = (ln.chunks + p.segs - 1) / p.segs;
     const int q0 = min(ln.chunks, rank * seg_chunks);
     const int n2 = min(ln.chunks, q0 + seg_chunks) - q0;
@@ -151,23 +221,20 @@ __global__ void __launch_bounds__(PipeCfg::kThreads, 1)
 
     // chunk j of the sequence (state-only chunks, then full chunks) -> chunk of the segment
     struct Chunk {
-        int line, n, lp0;
+        int p0, n;          // first scan position, positions
         bool full;
     };
     auto chunk_of = [&](int j) {
         const bool full = j >= n1;
-        const int q = q0 + (full ? j - n1 : j);
         Chunk c;
-        c.line = q / ln.pieces;
-        const int start = (q - c.line * ln.pieces) * ln.clen;
-        c.n = min(ln.clen, ln.len - start);
-        c.lp0 = ln.rev ? ln.len - start - c.n : start;
+        ln.chunk(q0 + (full ? j - n1 : j), p.L, c.p0, c.n);
         c.full = full;
         return c;
     };
     auto token_row = [&](const Chunk &c, int i) {
-        const int lp = c.lp0 + i;
-        const int s = ln.fam ? lp * p.gw + c.line : c.line * p.gw + lp;
+        int line, lp;
+        ln.place(c.p0, c.n, i, line, lp);
+        const int s = ln.fam ? lp * p.gw + line : line * p.gw + lp;
         return (bb * p.L + s) * p.H + hh;
     };
     auto wait = [&](uint64_t *bar, int use) { return wait_bar(bar, (uint32_t)(use & 1), p.wait_limit, abort_flag); };
@@ -241,13 +308,21 @@ __global__ void __launch_bounds__(PipeCfg::kThreads, 1)
                 const uint32_t mask = c.full ? 0x1Fu : 0x0Eu;
                 ptx::mbar_arrive_expect_tx(&m.ld[s], (uint32_t)__popc(mask) * C::kTile);
                 if (!(c.full && j - n1 == p.fault_chunk)) {
-                    const int y = ln.fam ? c.line * p.H + hh : hh;
-                    const int z = ln.fam ? bb * p.gh + c.lp0 : bb * p.L + c.line * p.gw + c.lp0;
+                    // one box per group of hb rows (packed) or one 64-row box.  A group past the
+                    // chunk's end reloads the first group's tokens: rows that are masked later
+                    // still hold finite values, and no box leaves the tensor.
+                    const int rows = ln.hb > 0 ? ln.hb : 64;
                     const uint32_t bar = ptx::smem_u32(&m.ld[s]);
+                    for (int i = 0; i < 64; i += rows) {
+                        int line, lp;
+                        ln.place(c.p0, c.n, i < c.n ? i : 0, line, lp);
+                        const int y = ln.fam ? line * p.H + hh : hh;
+                        const int z = ln.fam ? bb * p.gh + lp : bb * p.L + line * p.gw + lp;
+                        const uint32_t dst = sbase + s * C::kStage + (uint32_t)i * 128;
 #pragma unroll
-                    for (int x = 0; x < 5; ++x)
-                        if (mask >> x & 1u)
-                            ptx::tma_load_3d(sbase + s * C::kStage + x * C::kTile, &tmaps[x], 0, y, z, bar);
+                        for (int x = 0; x < 5; ++x)
+                            if (mask >> x & 1u) ptx::tma_load_3d(dst + x * C::kTile, &tmaps[x], 0, y, z, bar);
+                    }
                 }
                 last[s] = j;
             }
@@ -286,7 +361,6 @@ __global__ void __launch_bounds__(PipeCfg::kThreads, 1)
                 const uint32_t stg = (uint32_t)s * C::kStage >> 4;   // descriptor address units
                 const uint32_t lanes = (uint32_t)(16 * slot) << 16;
                 const uint32_t d_sl = tmem + lanes + C::kColSL, d_sc = tmem + lanes + C::kColSC;
-                const uint32_t d_o = tmem + lanes + C::kColO;
                 const uint32_t a_qh = tmem + lanes + C::kColQH, a_ql = tmem + lanes + C::kColQL;
                 if (go) {
 #pragma unroll
@@ -363,7 +437,7 @@ __global__ void __launch_bounds__(PipeCfg::kThreads, 1)
         // gate: thread (channel pair cp, block pb of 8 scan positions), b into kB (fp32 atoms)
         auto gate = [&](uint32_t stage, const Chunk &c, int slot) {
             const int cp = ttid & 31, pb = ttid >> 5, ch = 2 * cp;
-            const int n = c.n, rev = ln.rev;
+            const int n = c.n;
             float c0s[8], c1s[8];
             float r0 = 0.0f, r1 = 0.0f;
             const uint32_t aoff = stage + C::kTA + (ch & 7) * 2;
@@ -371,7 +445,7 @@ __global__ void __launch_bounds__(PipeCfg::kThreads, 1)
             for (int i = 0; i < 8; ++i) {
                 const int pos = pb * 8 + i;
                 const bool ok = pos < n;
-                const int row = ok ? (rev ? n - 1 - pos : pos) : 0;
+                const int row = ok ? ln.row_of(pos, n) : 0;
                 const float2 af = __half22float2(*reinterpret_cast<const __half2 *>(sm + aoff + ptx::sw128(row, ch >> 3)));
                 r0 += ok ? log2_gamma(af.x) : 0.0f;
                 r1 += ok ? log2_gamma(af.y) : 0.0f;
@@ -392,7 +466,7 @@ __global__ void __launch_bounds__(PipeCfg::kThreads, 1)
             for (int i = 0; i < 8; ++i) {
                 const int pos = pb * 8 + i;
                 if (pos < n) {
-                    const int row = rev ? n - 1 - pos : pos;
+                    const int row = ln.row_of(pos, n);
                     const float2 bv = make_float2(c0s[i] + a0, c1s[i] + a1);
                     *reinterpret_cast<float2 *>(sm + C::kB + off_f<64>(row, ch >> 2) + (ch & 3) * 4) = bv;
                     if (pos == rmid) *reinterpret_cast<float2 *>(&m.rref[slot][ch]) = bv;
@@ -444,7 +518,7 @@ __global__ void __launch_bounds__(PipeCfg::kThreads, 1)
         // exact scores of a chunk beyond the bf16 operands' range: row t, columns [16 cg, + 16),
         // fp16 into the a tile (the P slot)
         auto exact_p_smem = [&](uint32_t stage, const Chunk &c) {
-            const int n = c.n, rev = ln.rev, s0 = 16 * cg;
+            const int n = c.n, s0 = 16 * cg, pt = ln.row_of(t, n);
             auto hat = [&](uint32_t tile, int row, int ch) {
                 return __half2float(*reinterpret_cast<const __half *>(sm + stage + tile + off_h<64>(row, ch >> 3) + (ch & 7) * 2));
             };
@@ -455,7 +529,7 @@ __global__ void __launch_bounds__(PipeCfg::kThreads, 1)
             float amax = 0.0f;
             for (int e = 0; e < 16; ++e) {
                 const int s = s0 + e;
-                const bool causal = rev ? s >= t : s <= t;
+                const bool causal = ln.row_of(s, n) <= pt;
                 float acc = 0.0f;
                 if (causal && t < n && s < n)
                     for (int ch = 0; ch < D; ++ch) {
@@ -597,12 +671,12 @@ __global__ void __launch_bounds__(PipeCfg::kThreads, 1)
                     float r[16];
                     ptx::tmem_ld16x2_x16<16>(rows + C::kColSC + 32 * hg, r);
                     ptx::tmem_ld_wait();
-                    const int s0 = 16 * cg, n = c.n, rev = ln.rev;
+                    const int s0 = 16 * cg, n = c.n, pt = ln.row_of(t, n);
                     float amax = 0.0f;
 #pragma unroll
                     for (int e = 0; e < 16; ++e) {
                         const int sp = s0 + e;
-                        const bool before = rev ? sp > t : sp < t;
+                        const bool before = ln.row_of(sp, n) < pt;
                         float v = before ? r[e] : (sp == t ? dq : 0.0f);
                         v = (t < n && sp < n) ? v : 0.0f;
                         r[e] = v;

@@ -66,6 +66,8 @@ def load() -> ctypes.CDLL:
         lib.gla_selftest_chunk.restype = ctypes.c_int
         lib.gla_selftest_load.argtypes = [vp] * 5 + [i] * 7 + [vp, vp, vp]
         lib.gla_selftest_load.restype = ctypes.c_int
+        lib.gla_scan_layout.argtypes = [i] * 5 + [vp, vp]
+        lib.gla_scan_layout.restype = ctypes.c_int
         lib.gla_selftest_fault.argtypes = [vp] * 7 + [i] * 7 + [ll, i, i, vp]
         lib.gla_selftest_rcp.argtypes = [vp, vp, i, vp]
         lib.gla_selftest_rcp.restype = ctypes.c_int
@@ -197,6 +199,19 @@ def plan(B: int, H: int, grid_h: int, grid_w: int, d_k: int = 64, d_v: int = 64,
     kernel, segs, seg_len, ctas, mac = (v.value for v in vals)
     return {"kernel": KERNEL_NAMES.get(kernel, kernel), "segments": segs,
             "seg_len": seg_len, "ctas": ctas, "max_active_clusters": mac}
+
+
+def scan_layout(grid_h: int, grid_w: int, direction: int, chunk: int = 0,
+                kernel: int = KERNEL_PIPE64):
+    """Spatial index of the token the kernel's chunk tiles place at each scan position (host only).
+
+    Returns (spatial: list of grid_h * grid_w ints, box_rows)."""
+    L = grid_h * grid_w
+    buf = (ctypes.c_int * L)()
+    rows = ctypes.c_int(0)
+    _check(load().gla_scan_layout(kernel, grid_h, grid_w, direction, chunk, buf, ctypes.byref(rows)),
+           "gla_scan_layout")
+    return list(buf), rows.value
 
 
 def empty_launch(B: int, H: int, grid_h: int, grid_w: int, stream=None):

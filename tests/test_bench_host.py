@@ -2,6 +2,8 @@
 whether a timed run was throttled, and the roofline denominators and traffic lookup."""
 import json
 
+import pytest
+
 import bench
 
 
@@ -45,16 +47,41 @@ def test_peaks_read_the_measured_file_else_the_fallback(tmp_path, monkeypatch):
     assert bench.measured_peaks() == (bench.FALLBACK_HBM_GBS, "fallback")
 
 
-def test_traffic_is_reported_only_for_its_workload_and_build(tmp_path, monkeypatch):
+def test_traffic_is_reported_only_for_its_workload_kernel_and_build(tmp_path, monkeypatch):
     from recurrent_vision_backbone_only_b200 import build
     p = tmp_path / "traffic.json"
     monkeypatch.setattr(bench, "PROFILE_TRAFFIC", str(p))
-    p.write_text(json.dumps({"workload": "gtr640", "lib_sources_digest": build.sources_digest(),
-                             "dram_bytes_per_launch": 123456}))
-    assert bench.profile_traffic("gtr640") == 123456
-    assert bench.profile_traffic("highres") is None
-    p.write_text(json.dumps({"workload": "gtr640", "lib_sources_digest": "0" * 16,
-                             "dram_bytes_per_launch": 123456}))
-    assert bench.profile_traffic("gtr640") is None          # kernel changed since the capture
+    entry = {"workload": "gtr640", "kernel": "tensor-core 128-row",
+             "lib_sources_digest": build.sources_digest(), "dram_bytes_per_launch": 123456}
+    p.write_text(json.dumps({"entries": [entry]}))
+    assert bench.profile_traffic("gtr640", "tensor-core 128-row") == 123456
+    assert bench.profile_traffic("highres", "tensor-core 128-row") is None
+    assert bench.profile_traffic("gtr640", "tensor-core 64-row pipelined") is None
+    p.write_text(json.dumps({"entries": [dict(entry, lib_sources_digest="0" * 16)]}))
+    assert bench.profile_traffic("gtr640", "tensor-core 128-row") is None   # kernel changed since
     p.unlink()
-    assert bench.profile_traffic("gtr640") is None
+    assert bench.profile_traffic("gtr640", "tensor-core 128-row") is None
+
+
+NCU_DETAILS = """==PROF== Connected to process 1
+"ID","Process ID","Process Name","Host Name","Kernel Name","Context","Stream","Block Size","Grid Size","Device","CC","Section Name","Metric Name","Metric Unit","Metric Value"
+"0","1","python","h","void gla::ck::gla_pipe_kernel(Maps, Params)","1","7","(576, 1, 1)","(192, 1, 1)","0","10.0","Command line profiler metrics","dram__bytes_read.sum","Mbyte","206.02"
+"0","1","python","h","void gla::ck::gla_pipe_kernel(Maps, Params)","1","7","(576, 1, 1)","(192, 1, 1)","0","10.0","Command line profiler metrics","dram__bytes_write.sum","Mbyte","29.07"
+"1","1","python","h","void other_kernel()","1","7","(1, 1, 1)","(1, 1, 1)","0","10.0","Command line profiler metrics","dram__bytes_read.sum","byte","7"
+"1","1","python","h","void other_kernel()","1","7","(1, 1, 1)","(1, 1, 1)","0","10.0","Command line profiler metrics","dram__bytes_write.sum","byte","0"
+"""
+
+
+def test_ncu_csv_reader_and_traffic_entry(tmp_path, capsys):
+    p = tmp_path / "n.csv"
+    p.write_text(NCU_DETAILS)
+    got = bench.read_ncu_csv(str(p))
+    assert [k for k, _ in got] == ["void gla::ck::gla_pipe_kernel(Maps, Params)", "void other_kernel()"]
+    assert got[0][1]["dram__bytes_read.sum"] == pytest.approx(206.02e6)
+    args = bench.argparse.Namespace(record_traffic=str(p), workload="batched", kernel="pipe64",
+                                    ncu_command="ncu ...")
+    bench.record_traffic(args)
+    e = json.loads(capsys.readouterr().out)
+    assert e["workload"] == "batched" and e["kernel"] == "tensor-core 64-row pipelined"
+    assert e["dram_bytes_per_launch"] == pytest.approx(235.09e6)
+    assert e["launches"] == 1
