@@ -4,6 +4,7 @@
 // key-only GLA token mixer of the GTR paper (arXiv 2609.26590, method
 // section).  Every step of the operation runs in the kernels included here;
 // this file only checks arguments, picks launch shapes and launches.
+#include <cmath>
 #include <cstddef>
 #include <cstdint>
 #include <algorithm>
@@ -537,6 +538,7 @@ int run_chunk(const Args &x, int chunk, int segs, float eps, cudaStream_t st, co
     p.segs = pl.segs; p.chunk_max = chunk;
     p.eps = eps;
     p.scale = 1.0f / sqrtf((float)D);
+    p.log2_scale = (float)(-0.5 * std::log2((double)D));
     p.wait_limit = wait_limit;
     p.fault_chunk = fault_chunk;
     p.hb[0] = hb[0];

@@ -124,6 +124,7 @@ struct Params {
     int segs;           // CTAs per (b, h) pair == cluster size
     int chunk_max;      // largest chunk (16..64); lines are cut into equal pieces no longer
     float eps, scale;   // RMSNorm epsilon, d_k^{-1/2}
+    float log2_scale;   // log2(d_k^{-1/2})
     long long wait_limit;   // bound of every mbarrier wait, SM clocks
     int fault_chunk;        // test hook: full-pass chunk whose loads are not issued (-1: none)
     int hb[2];              // pipelined kernel: rows per TMA box of packed chunks for the row and

@@ -75,6 +75,7 @@ struct PipeMisc {
     alignas(16) float tot[8][64];     // front: gate block totals
     alignas(16) float b0[64];         // front: b at the first scan position
     alignas(16) float rref[2][64];    // per slot: reference r (log2)
+    alignas(16) float rq[2][64];      // per slot: r - log2(d_k^{-1/2}) (the query side's reference)
     alignas(16) float Bc[2][64];      // per slot: B (log2)
     alignas(16) float fB[2][64];      // per slot: 2^{B - r}
     alignas(16) float er[2][64];      // per slot: 2^{r}
@@ -134,6 +135,26 @@ struct Scan {
     }
     // tile row of scan offset i in a chunk of n positions (an involution: also the offset of row i)
     __host__ __device__ int row_of(int i, int n) const { return rev ? (hb > 0 ? i ^ (hb - 1) : n - 1 - i) : i; }
+    // Bit e of the result: the token of tile row s0 + e (s0 a multiple of 16, e < 16) precedes
+    // the token of row t in the scan, both rows inside the chunk of n positions.
+    __device__ uint32_t before_mask(int n, int t, int s0) const {
+        auto span = [](int lo, int hi) -> uint32_t {       // bits lo .. hi - 1, clamped to 0..16
+            lo = max(lo, 0);
+            hi = min(hi, 16);
+            return hi > lo ? ((1u << hi) - 1u) & ~((1u << lo) - 1u) : 0u;
+        };
+        if (t >= n) return 0u;
+        if (rev && hb == 0) return span(t - s0 + 1, n - s0);   // line-aligned, reversed: t < s < n
+        // scan offset of row s0 + e is (s0 + e) ^ xm = (s0 ^ (xm & ~15)) + (e ^ x); for rows inside
+        // the chunk a smaller offset implies s < n
+        const int xm = rev ? hb - 1 : 0, x = xm & 15;
+        uint32_t mk = span(0, (t ^ xm) - (s0 ^ (xm & ~15)));   // bits v with v < that bound
+        if (x & 1) mk = ((mk & 0x5555u) << 1) | ((mk >> 1) & 0x5555u);    // bit e <- bit e ^ x
+        if (x & 2) mk = ((mk & 0x3333u) << 2) | ((mk >> 2) & 0x3333u);
+        if (x & 4) mk = ((mk & 0x0F0Fu) << 4) | ((mk >> 4) & 0x0F0Fu);
+        if (x & 8) mk = ((mk & 0x00FFu) << 8) | ((mk >> 8) & 0x00FFu);
+        return mk;
+    }
     // line and position along it of tile row i of the chunk starting at scan position p0
     __host__ __device__ void place(int p0, int n, int i, int &line, int &lp) const {
         if (hb > 0) {
@@ -434,64 +455,74 @@ __global__ void __launch_bounds__(PipeCfg::kThreads, 1)
     // ================================================================== front team
     else if (front) {
         const uint32_t tmem_q = tmem;                 // + slot lanes below
-        // gate: thread (channel pair cp, block pb of 8 scan positions), b into kB (fp32 atoms)
+        // gate: thread (channel pair cp, block pb of 8 scan positions), b into kB (fp32 atoms).
+        // Rows past the chunk get b = +inf: their decayed keys 2^{r - b} k vanish without a
+        // select, and their queries (infinite) only reach score rows and output rows that are
+        // masked or never stored.  Returns whether the chunk takes the exact score path.
         auto gate = [&](uint32_t stage, const Chunk &c, int slot) {
             const int cp = ttid & 31, pb = ttid >> 5, ch = 2 * cp;
             const int n = c.n;
             float c0s[8], c1s[8];
+            int rows[8];
             float r0 = 0.0f, r1 = 0.0f;
             const uint32_t aoff = stage + C::kTA + (ch & 7) * 2;
 #pragma unroll
             for (int i = 0; i < 8; ++i) {
                 const int pos = pb * 8 + i;
                 const bool ok = pos < n;
-                const int row = ok ? ln.row_of(pos, n) : 0;
-                const float2 af = __half22float2(*reinterpret_cast<const __half2 *>(sm + aoff + ptx::sw128(row, ch >> 3)));
+                rows[i] = ok ? ln.row_of(pos, n) : pos;
+                const float2 af = __half22float2(*reinterpret_cast<const __half2 *>(sm + aoff + ptx::sw128(rows[i], ch >> 3)));
                 r0 += ok ? log2_gamma(af.x) : 0.0f;
                 r1 += ok ? log2_gamma(af.y) : 0.0f;
                 c0s[i] = r0;
                 c1s[i] = r1;
             }
             *reinterpret_cast<float2 *>(&m.tot[pb][ch]) = make_float2(r0, r1);
-            if (ttid == 0) m.slow[slot] = 0;
             team_bar(1);
             float a0 = 0.0f, a1 = 0.0f;
-            for (int q = 0; q < pb; ++q) {
-                const float2 x = *reinterpret_cast<const float2 *>(&m.tot[q][ch]);
-                a0 += x.x;
-                a1 += x.y;
-            }
+#pragma unroll
+            for (int q = 0; q < 7; ++q)
+                if (q < pb) {
+                    const float2 x = *reinterpret_cast<const float2 *>(&m.tot[q][ch]);
+                    a0 += x.x;
+                    a1 += x.y;
+                }
             const int rmid = (n - 1) >> 1;
 #pragma unroll
             for (int i = 0; i < 8; ++i) {
                 const int pos = pb * 8 + i;
-                if (pos < n) {
-                    const int row = ln.row_of(pos, n);
-                    const float2 bv = make_float2(c0s[i] + a0, c1s[i] + a1);
-                    *reinterpret_cast<float2 *>(sm + C::kB + off_f<64>(row, ch >> 2) + (ch & 3) * 4) = bv;
-                    if (pos == rmid) *reinterpret_cast<float2 *>(&m.rref[slot][ch]) = bv;
-                    if (pos == n - 1) *reinterpret_cast<float2 *>(&m.Bc[slot][ch]) = bv;
-                    if (pos == 0) *reinterpret_cast<float2 *>(&m.b0[ch]) = bv;
+                const float2 bv = pos < n ? make_float2(c0s[i] + a0, c1s[i] + a1) : make_float2(INFINITY, INFINITY);
+                *reinterpret_cast<float2 *>(sm + C::kB + off_f<64>(rows[i], ch >> 2) + (ch & 3) * 4) = bv;
+                if (pos == rmid) *reinterpret_cast<float2 *>(&m.rref[slot][ch]) = bv;
+                if (pos == n - 1) *reinterpret_cast<float2 *>(&m.Bc[slot][ch]) = bv;
+                if (pos == 0) *reinterpret_cast<float2 *>(&m.b0[ch]) = bv;
+            }
+            team_bar(1);
+            // per key channel: 2^B, the operand range check, and the fast path's 2^{B - r}, 2^r
+            bool oob = false;
+            if (ttid < D) {
+                const float Bv = m.Bc[slot][ttid], r = m.rref[slot][ttid];
+                m.eB[slot][ttid] = ptx::ex2(Bv);
+                if (c.full) {
+                    oob = m.b0[ttid] - r > kHalfRange || r - Bv > kHalfRange;
+                    m.fB[slot][ttid] = ptx::ex2(Bv - r);
+                    m.er[slot][ttid] = ptx::ex2(r);
+                    m.rq[slot][ttid] = r - p.log2_scale;
                 }
             }
-            team_bar(1);
-            if (ttid < D) {
-                const float Bv = m.Bc[slot][ttid];
-                m.eB[slot][ttid] = ptx::ex2(Bv);
-                if (c.full && (m.b0[ttid] - m.rref[slot][ttid] > kHalfRange || m.rref[slot][ttid] - Bv > kHalfRange))
-                    m.slow[slot] = 1;
+            const bool slow = ptx::named_bar_or(1, C::kTeam, oob);
+            if (slow) {                              // rare; r = 0 keeps every exponent <= 0
+                if (ttid < D) {
+                    m.rref[slot][ttid] = 0.0f;
+                    m.er[slot][ttid] = 1.0f;
+                    m.rq[slot][ttid] = -p.log2_scale;
+                }
+                team_bar(1);
             }
-            team_bar(1);
-            if (c.full && ttid < D) {
-                const float r = m.slow[slot] ? 0.0f : m.rref[slot][ttid];
-                m.rref[slot][ttid] = r;
-                m.fB[slot][ttid] = ptx::ex2(m.Bc[slot][ttid] - r);
-                m.er[slot][ttid] = ptx::ex2(r);
-            }
-            team_bar(1);
+            if (ttid == 0) m.slow[slot] = slow;
+            return slow;
         };
-        auto build_ks = [&](uint32_t stage, const Chunk &c, int slot) {
-            const int n = c.n;
+        auto build_ks = [&](uint32_t stage, int slot) {
 #pragma unroll
             for (int jj = 0; jj < 2; ++jj) {
                 const int j = 2 * cg + jj;
@@ -508,9 +539,8 @@ __global__ void __launch_bounds__(PipeCfg::kThreads, 1)
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
                     const float2 kf = __half22float2(k2[e]);
-                    const float x0 = t < n ? kf.x * ptx::ex2(Bt[2 * e] - bt[2 * e]) : 0.0f;
-                    const float x1 = t < n ? kf.y * ptx::ex2(Bt[2 * e + 1] - bt[2 * e + 1]) : 0.0f;
-                    ks[e] = pack_h2(x0, x1);
+                    ks[e] = pack_h2(kf.x * ptx::ex2(Bt[2 * e] - bt[2 * e]),
+                                    kf.y * ptx::ex2(Bt[2 * e + 1] - bt[2 * e + 1]));
                 }
                 *reinterpret_cast<uint4 *>(sm + stage + C::kTQ + o) = make_uint4(ks[0], ks[1], ks[2], ks[3]);
             }
@@ -547,8 +577,7 @@ __global__ void __launch_bounds__(PipeCfg::kThreads, 1)
                     make_uint4(pack_h2(pv[8 * h], pv[8 * h + 1]), pack_h2(pv[8 * h + 2], pv[8 * h + 3]),
                                pack_h2(pv[8 * h + 4], pv[8 * h + 5]), pack_h2(pv[8 * h + 6], pv[8 * h + 7]));
         };
-        auto build_full = [&](uint32_t stage, const Chunk &c, int slot, bool slow) {
-            const int n = c.n;
+        auto build_full = [&](uint32_t stage, int slot, bool slow) {
             float dqs = 0.0f;
             uint32_t qh[8], ql[8];
 #pragma unroll
@@ -563,11 +592,14 @@ __global__ void __launch_bounds__(PipeCfg::kThreads, 1)
                 const float4 bB = *reinterpret_cast<const float4 *>(sm + C::kB + off_f<64>(t, 2 * j + 1));
                 const float4 rA = *reinterpret_cast<const float4 *>(&m.rref[slot][8 * j]);
                 const float4 rB = *reinterpret_cast<const float4 *>(&m.rref[slot][8 * j + 4]);
+                const float4 qA = *reinterpret_cast<const float4 *>(&m.rq[slot][8 * j]);
+                const float4 qB = *reinterpret_cast<const float4 *>(&m.rq[slot][8 * j + 4]);
                 const float *fsrc = slow ? m.Bc[slot] : m.fB[slot];
                 const float4 fA = *reinterpret_cast<const float4 *>(fsrc + 8 * j);
                 const float4 fBv = *reinterpret_cast<const float4 *>(fsrc + 8 * j + 4);
                 const float bt[8] = {bA.x, bA.y, bA.z, bA.w, bB.x, bB.y, bB.z, bB.w};
                 const float rr[8] = {rA.x, rA.y, rA.z, rA.w, rB.x, rB.y, rB.z, rB.w};
+                const float rq[8] = {qA.x, qA.y, qA.z, qA.w, qB.x, qB.y, qB.z, qB.w};
                 const float ff[8] = {fA.x, fA.y, fA.z, fA.w, fBv.x, fBv.y, fBv.z, fBv.w};
                 float kt[8], qt[8], ks[8];
 #pragma unroll
@@ -579,7 +611,7 @@ __global__ void __launch_bounds__(PipeCfg::kThreads, 1)
                     for (int h = 0; h < 2; ++h) {
                         const int i = 2 * e + h;
                         dqs = fmaf(qv[h], kv[h], dqs);
-                        qt[i] = qv[h] * ptx::ex2(bt[i] - rr[i]) * p.scale;
+                        qt[i] = qv[h] * ptx::ex2(bt[i] - rq[i]);
                         if (!slow) {
                             kt[i] = kv[h] * ptx::ex2(rr[i] - bt[i]);
                             ks[i] = kt[i] * ff[i];
@@ -587,7 +619,6 @@ __global__ void __launch_bounds__(PipeCfg::kThreads, 1)
                             kt[i] = 0.0f;
                             ks[i] = kv[h] * ptx::ex2(ff[i] - bt[i]);
                         }
-                        if (t >= n) kt[i] = qt[i] = ks[i] = 0.0f;
                     }
                 }
                 uint32_t kh4[4], kl4[4], ks4[4];
@@ -616,13 +647,12 @@ __global__ void __launch_bounds__(PipeCfg::kThreads, 1)
             if (j >= 2) wait(&m.slotfree[slot], (j - 2) >> 1);    // back team done with chunk j - 2
             wait(&m.ld[s], j / 3);
             ptx::tc_fence_after_sync();
-            gate(stage, c, slot);
+            const bool slow = gate(stage, c, slot);
             if (!c.full) {
-                build_ks(stage, c, slot);
+                build_ks(stage, slot);
             } else {
-                const bool slow = m.slow[slot] != 0;
                 if (slow) exact_p_smem(stage, c);
-                build_full(stage, c, slot, slow);
+                build_full(stage, slot, slow);
             }
             ptx::fence_proxy_async_smem();
             ptx::tc_fence_before_sync();
@@ -668,26 +698,28 @@ __global__ void __launch_bounds__(PipeCfg::kThreads, 1)
                     float dq = 0.0f;
 #pragma unroll
                     for (int g = 0; g < 4; ++g) dq += m.dqp[slot][g][t];
+                    const int s0 = 16 * cg, n = c.n;
+                    const uint32_t mk = ln.before_mask(n, t, s0);
                     float r[16];
                     ptx::tmem_ld16x2_x16<16>(rows + C::kColSC + 32 * hg, r);
                     ptx::tmem_ld_wait();
-                    const int s0 = 16 * cg, n = c.n, pt = ln.row_of(t, n);
                     float amax = 0.0f;
 #pragma unroll
                     for (int e = 0; e < 16; ++e) {
-                        const int sp = s0 + e;
-                        const bool before = ln.row_of(sp, n) < pt;
-                        float v = before ? r[e] : (sp == t ? dq : 0.0f);
-                        v = (t < n && sp < n) ? v : 0.0f;
-                        r[e] = v;
-                        amax = fmaxf(amax, fabsf(v));
+                        r[e] = (mk >> e & 1u) ? r[e] : 0.0f;
+                        amax = fmaxf(amax, fabsf(r[e]));
                     }
+                    const bool diag = t < n && (unsigned)(t - s0) < 16u;    // exact q_t . k_t
+                    if (diag) amax = fmaxf(amax, fabsf(dq));
                     if (amax > 65504.0f) m.range_err = 1;
 #pragma unroll
                     for (int h = 0; h < 2; ++h)
                         *reinterpret_cast<uint4 *>(sm + stage + C::kTA + off_h<64>(t, 2 * cg + h)) =
                             make_uint4(pack_h2(r[8 * h], r[8 * h + 1]), pack_h2(r[8 * h + 2], r[8 * h + 3]),
                                        pack_h2(r[8 * h + 4], r[8 * h + 5]), pack_h2(r[8 * h + 6], r[8 * h + 7]));
+                    if (diag)
+                        *reinterpret_cast<__half *>(sm + stage + C::kTA + off_h<64>(t, t >> 3) + (t & 7) * 2) =
+                            __float2half_rn(dq);
                 }
                 ptx::fence_proxy_async_smem();
                 ptx::tc_fence_before_sync();
