@@ -79,8 +79,9 @@ enum gla_direction {
  * q, k, v, gate_preact, out_gate_preact and out are IEEE binary16 arrays;
  * rms_weight is float32.  `stream` is a cudaStream_t (NULL = legacy default
  * stream).  Supported head dims: d_k, d_v in {32, 64, 128}; d_k = d_v = 64 runs on
- * the 128-row tensor-core kernel, d_k = d_v = 128 on the 64-row one, the others on
- * CUDA cores (gla_kernel below).
+ * the pipelined 64-row tensor-core kernel when B * H is at least the device's SM count,
+ * else on the 128-row one; d_k = d_v = 128 on the 64-row kernel; the others on CUDA
+ * cores (gla_kernel below).
  */
 int gla_fwd(const void *q, const void *k, const void *v,
             const void *gate_preact, const void *out_gate_preact,
@@ -122,7 +123,8 @@ enum gla_kernel {
     GLA_KERNEL_TC64 = 3,   /* tensor cores, 64-row chunks, TMA loads: fp16, d_k = d_v in   */
                            /* {64, 128}                                                    */
     GLA_KERNEL_PIPE64 = 4  /* the 64-row kernel with two chunks in flight (warp-specialised */
-                           /* teams, 3-stage TMA ring): fp16, d_k = d_v = 64               */
+                           /* teams, 3-stage TMA ring, chunks packed across lines, scores   */
+                           /* and inter product in one N = 128 product): fp16, d = 64       */
 };
 
 /*

@@ -553,12 +553,14 @@ int run_chunk(const Args &x, int chunk, int segs, float eps, cudaStream_t st, co
 // ------------------------------------------------------------- dispatch
 constexpr float kEps = 1e-6f;
 
-// The kernel gla_fwd uses: fp32 I/O on CUDA cores; fp16 d = 64 on the 128-row tensor-core
-// kernel (the faster of the two at that head dim on every workload measured), fp16 d = 128 on
-// the 64-row one (the only one that holds its tiles), other head dims on CUDA cores.
-int auto_kernel(const Args &x, int dtype) {
+// The kernel gla_fwd uses: fp32 I/O on CUDA cores; fp16 d = 64 on the pipelined 64-row kernel
+// when the launch has at least one (b, h) pair per SM (throughput-bound: one CTA per pair, two
+// chunks in flight), else on the 128-row kernel (latency-bound: one chunk per segment and a
+// mid-chunk exchange, faster at 40 x 40, even at 80 x 80); fp16 d = 128 on the 64-row kernel
+// (the only one that holds its tiles); other head dims on CUDA cores.
+int auto_kernel(const Args &x, int dtype, const DeviceInfo &di) {
     if (dtype == 1) return kSimt;
-    if (x.dk == 64 && x.dv == 64) return kTc128;
+    if (x.dk == 64 && x.dv == 64) return (long long)x.B * x.H >= di.sms ? kPipe64 : kTc128;
     if (x.dk == 128 && x.dv == 128) return kTc64;
     return kSimt;
 }
@@ -570,7 +572,6 @@ int run(const Args &x, int dtype, int chunk, int segs, float eps, cudaStream_t s
     if (rc != GLA_OK) return rc;
     if (segs < 0 || segs > 16 || chunk < 0 || !(eps >= 0.0f)) return GLA_ERR_UNSUPPORTED;
     if (kernel < kAuto || kernel > kPipe64) return GLA_ERR_UNSUPPORTED;
-    if (kernel == kAuto) kernel = auto_kernel(x, dtype);
     if (kernel == kTc128 && !(dtype == 0 && x.dk == 64 && x.dv == 64)) return GLA_ERR_UNSUPPORTED;
     if (kernel == kTc64 && !(dtype == 0 && x.dk == x.dv && (x.dk == 64 || x.dk == 128)))
         return GLA_ERR_UNSUPPORTED;
@@ -578,6 +579,7 @@ int run(const Args &x, int dtype, int chunk, int segs, float eps, cudaStream_t s
     DeviceInfo di;
     rc = current_device_info(&di);
     if (rc != GLA_OK) return rc;
+    if (kernel == kAuto) kernel = auto_kernel(x, dtype, di);
     if (kernel == kTc128) return run_tc(x, chunk, segs, eps, st, di, query);
     if (kernel == kTc64)
         return x.dk == 64 ? run_chunk<64>(x, chunk, segs, eps, st, di, query)
@@ -769,9 +771,11 @@ int gla_empty_launch(int B, int H, int grid_h, int grid_w, void *stream) {
     Plan pl;
     int rc = run(x, 0, 0, 0, kEps, static_cast<cudaStream_t>(stream), &pl);
     if (rc != GLA_OK) return rc;
-    if (pl.kernel != kTc128 && pl.kernel != kTc64) return GLA_ERR_UNSUPPORTED;
+    if (pl.kernel != kTc128 && pl.kernel != kTc64 && pl.kernel != kPipe64) return GLA_ERR_UNSUPPORTED;
     auto kern = pl.kernel == kTc128 ? tc::gla_empty_kernel : ck::gla_chunk_empty_kernel;
-    const int threads = pl.kernel == kTc128 ? tc::kThreads : ck::Cfg<64>::kThreads;
+    const int threads = pl.kernel == kTc128  ? tc::kThreads
+                        : pl.kernel == kTc64 ? ck::Cfg<64>::kThreads
+                                             : ck::PipeCfg::kThreads;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)pl.smem) != cudaSuccess ||
         cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) != cudaSuccess) {
         cudaGetLastError();

@@ -52,13 +52,14 @@ struct PipeCfg {
     static constexpr int kStages = 3;
     static constexpr uint32_t kAtom = 64 * 128;
     static constexpr uint32_t kTile = 64 * D * 2;        // 8 KB
-    static constexpr uint32_t kTQ = 0, kTK = kTile, kTA = 2 * kTile, kTV = 3 * kTile, kTG = 4 * kTile;
-    static constexpr uint32_t kStage = 5 * kTile;        // q (-> Ks), k (-> Kh), a (-> Kl -> P), v, g
+    // a stage: q (-> Ks), k (-> K~ high), S~^T high, a (-> K~ low -> P), S~^T low, v, g.  K~ and
+    // S~^T of one part are adjacent, so [K~ | S~^T] is ONE K-major operand of 128 rows.
+    static constexpr uint32_t kTQ = 0, kTK = kTile, kTSH = 2 * kTile, kTA = 3 * kTile, kTSL = 4 * kTile;
+    static constexpr uint32_t kTV = 5 * kTile, kTG = 6 * kTile;
+    static constexpr uint32_t kStage = 7 * kTile;
     static constexpr uint32_t kB = kStages * kStage;     // b (front team) / exchange rows
     static constexpr uint32_t kBBytes = 20480;           // >= max(64 x 64 x 4, (D + 15) x D x 4)
-    static constexpr uint32_t kSX0 = kB + kBBytes;       // S~ slot 0 (high | low); S_in (exchange)
-    static constexpr uint32_t kSXBytes = D * D * 4;      // 16 KB per slot
-    static constexpr uint32_t kMisc = kSX0 + 2 * kSXBytes;
+    static constexpr uint32_t kMisc = kB + kBBytes;
     // TMEM columns; slot p is lanes 16p .. 16p + 15 of every quarter
     static constexpr uint32_t kColSC = 0, kColO = 64, kColQH = 128, kColQL = 160, kColSL = 192;
     static constexpr uint32_t kTmemCols = 256;
@@ -67,7 +68,7 @@ struct PipeCfg {
 
 struct PipeMisc {
     uint64_t ld[3], stfree[3];
-    uint64_t fdone[2], sl[2], sc[2], sx[2], pfull[2], o[2], slotfree[2];
+    uint64_t gdone[2], fdone[2], sl[2], sc[2], sx[2], pfull[2], o[2], slotfree[2];
     uint64_t end;              // teardown after an expired wait: products in flight
     uint32_t tmem_base;
     int abort, range_err;
@@ -211,6 +212,7 @@ __global__ void __launch_bounds__(PipeCfg::kThreads, 1)
             ptx::mbar_init(&m.stfree[i], 2);
         }
         for (int i = 0; i < 2; ++i) {
+            ptx::mbar_init(&m.gdone[i], 1);
             ptx::mbar_init(&m.fdone[i], 1);
             ptx::mbar_init(&m.sl[i], 1);
             ptx::mbar_init(&m.sc[i], 1);
@@ -263,25 +265,35 @@ __global__ void __launch_bounds__(PipeCfg::kThreads, 1)
     auto tmem_rows = [&](int slot) { return tmem + ((uint32_t)(32 * qd + 16 * slot) << 16); };
 
     // ---------------------------------------------------------------- exchange
-    // All 576 threads: barriers A, B, C; the back team holds the aggregate (S, Gs).
-    float S[16];                                      // back: S[c = sc][16 cg + i]
+    // All 576 threads: barriers A, B, C; the back team holds the aggregate (S^T, Gs).  The state
+    // is kept transposed, S^T[j][c] (row j = value column, column c = key channel), so it is the
+    // K-major half of the fused operand; the exchange moves rows of S = S^T transposed, staged
+    // through fp32 rows [c][j] in stage 0's S~ tiles (free until the first full chunk).
+    float S[16];                                      // back: S^T[j = sc][c = 16 cg + i]
 #pragma unroll
     for (int i = 0; i < 16; ++i) S[i] = 0.0f;
     const int sc = 16 * qd + (lane & 15);
+    auto srow = [&](int c) -> uint32_t {              // fp32 row c of the [c][j] staging, stage 0
+        return (c < 32 ? C::kTSH : C::kTSL) + (uint32_t)(c & 31) * (D * 4);
+    };
     auto run_exchange = [&]() {
         const int segs = p.segs;
         const int max_own = (D + segs - 1) / segs;
         const float *recv = reinterpret_cast<const float *>(sm + C::kB);
+        if (back) {
+#pragma unroll
+            for (int i = 0; i < 16; ++i) *reinterpret_cast<float *>(sm + srow(16 * cg + i) + 4 * sc) = S[i];
+        }
         __syncthreads();
         ptx::cluster_arrive_release();
         ptx::cluster_wait();
-        if (back && rank < segs - 1) {
+        if (back && rank < segs - 1) {                // row c = sc of S, columns [16 cg, + 16)
             const int owner = sc % segs, lc = sc / segs;
             const uint32_t row = (uint32_t)((rank * max_own + lc) * D + 16 * cg) * 4;
 #pragma unroll
             for (int i = 0; i < 4; ++i)
                 ptx::st_cluster_v4(ptx::mapa(sbase + C::kB + row + 16 * i, owner),
-                                   make_float4(S[4 * i], S[4 * i + 1], S[4 * i + 2], S[4 * i + 3]));
+                                   *reinterpret_cast<const float4 *>(sm + srow(sc) + 64 * cg + 16 * i));
         }
         if (tid < D && rank < segs - 1) {
             const int o2 = tid % segs, l2 = tid / segs;
@@ -295,7 +307,7 @@ __global__ void __launch_bounds__(PipeCfg::kThreads, 1)
             for (int it = tid; it < items; it += C::kThreads) {
                 const int lc = it / (D / 4), j4 = it - lc * (D / 4);
                 const int c = lc * segs + rank;
-                const uint32_t dst = sbase + C::kSX0 + (uint32_t)(c * D + 4 * j4) * 4;
+                const uint32_t dst = sbase + srow(c) + 16 * j4;
                 float4 run = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
                 for (int q = 0; q < segs; ++q) {
                     ptx::st_cluster_v4(ptx::mapa(dst, q), run);
@@ -311,9 +323,8 @@ __global__ void __launch_bounds__(PipeCfg::kThreads, 1)
         ptx::cluster_arrive_release();
         ptx::cluster_wait();
         if (back) {
-            const float *sin = reinterpret_cast<const float *>(sm + C::kSX0);
 #pragma unroll
-            for (int i = 0; i < 16; ++i) S[i] = sin[sc * D + 16 * cg + i];
+            for (int i = 0; i < 16; ++i) S[i] = *reinterpret_cast<const float *>(sm + srow(16 * cg + i) + 4 * sc);
         }
         __syncthreads();
     };
@@ -340,9 +351,10 @@ __global__ void __launch_bounds__(PipeCfg::kThreads, 1)
                         const int y = ln.fam ? line * p.H + hh : hh;
                         const int z = ln.fam ? bb * p.gh + lp : bb * p.L + line * p.gw + lp;
                         const uint32_t dst = sbase + s * C::kStage + (uint32_t)i * 128;
+                        constexpr uint32_t kDst[5] = {C::kTQ, C::kTK, C::kTA, C::kTV, C::kTG};
 #pragma unroll
                         for (int x = 0; x < 5; ++x)
-                            if (mask >> x & 1u) ptx::tma_load_3d(dst + x * C::kTile, &tmaps[x], 0, y, z, bar);
+                            if (mask >> x & 1u) ptx::tma_load_3d(dst + kDst[x], &tmaps[x], 0, y, z, bar);
                     }
                 }
                 last[s] = j;
@@ -365,79 +377,56 @@ __global__ void __launch_bounds__(PipeCfg::kThreads, 1)
     // ==================================================================== MMA warp
     else if (mma_warp) {
         using M = Mma<64>;
-        const uint64_t kh0 = ptx::desc_sw128(sbase + C::kTK, 16, 1024);
-        const uint64_t kl0 = ptx::desc_sw128(sbase + C::kTA, 16, 1024);
+        const uint64_t kh0 = ptx::desc_sw128(sbase + C::kTK, 16, 1024);      // [K~ high | S~^T high]
+        const uint64_t kl0 = ptx::desc_sw128(sbase + C::kTA, 16, 1024);      // [K~ low | S~^T low]
         const uint64_t ks0 = ptx::desc_sw128(sbase + C::kTQ, C::kAtom, 1024);
         const uint64_t v0 = ptx::desc_sw128(sbase + C::kTV, C::kAtom, 1024);
         const uint64_t pa0 = ptx::desc_sw128(sbase + C::kTA, 16, 1024);      // P: K-major A
         constexpr uint32_t kIdPVss = ptx::idesc_ab(0, 0, false, true, 64, 64);
+        constexpr uint32_t kIdFused = ptx::idesc_ab(1, 1, false, false, 64, 128);
         auto step = [&](int j) {
             const int slot = j & 1, s = j % 3;
             const Chunk c = chunk_of(j);
+            const uint32_t stg = (uint32_t)s * C::kStage >> 4;               // descriptor address units
+            const uint32_t lanes = (uint32_t)(16 * slot) << 16;
             if (j >= 2) wait(&m.slotfree[slot], (j - 2) >> 1);
             wait(&m.fdone[slot], j >> 1);
-            const bool go = !*abort_flag;
             if (lane == 0) {
                 ptx::tc_fence_after_sync();
-                const uint32_t stg = (uint32_t)s * C::kStage >> 4;   // descriptor address units
-                const uint32_t lanes = (uint32_t)(16 * slot) << 16;
-                const uint32_t d_sl = tmem + lanes + C::kColSL, d_sc = tmem + lanes + C::kColSC;
-                const uint32_t a_qh = tmem + lanes + C::kColQH, a_ql = tmem + lanes + C::kColQL;
-                if (go) {
+                if (!*abort_flag) {                   // S_loc^T = V^T Ks (both MN-major)
 #pragma unroll
                     for (int k = 0; k < 4; ++k)
-                        ptx::mma_f16_ss(d_sl, ks0 + stg + 128 * k, v0 + stg + 128 * k, M::kIdSL, k > 0);
+                        ptx::mma_f16_ss(tmem + lanes + C::kColSL, v0 + stg + 128 * k, ks0 + stg + 128 * k, M::kIdSL, k > 0);
                 }
                 ptx::mma_commit(&m.sl[slot]);
-                if (c.full && go && !m.slow[slot]) {
+            }
+            __syncwarp();
+            wait(&m.sx[slot], j >> 1);                // S~^T of the chunk (a no-op for a state-only one)
+            if (lane == 0) {
+                ptx::tc_fence_after_sync();
+                if (c.full && !*abort_flag) {
+                    // [scores | inter] = Q~ [K~ | S~^T]^T, bf16 split: Qh Kh + Qh Kl + Ql Kh, N = 128
 #pragma unroll
                     for (int pass = 0; pass < 3; ++pass)
 #pragma unroll
                         for (int k = 0; k < 4; ++k)
-                            ptx::mma_f16_ts(d_sc, (pass == 2 ? a_ql : a_qh) + 8 * k,
-                                            (pass == 1 ? kl0 : kh0) + stg + 2 * k, M::kIdSC, pass > 0 || k > 0);
+                            ptx::mma_f16_ts(tmem + lanes + C::kColSC,
+                                            tmem + lanes + (pass == 2 ? C::kColQL : C::kColQH) + 8 * k,
+                                            (pass == 1 ? kl0 : kh0) + stg + 2 * k, kIdFused, pass > 0 || k > 0);
                 }
                 ptx::mma_commit(&m.sc[slot]);
             }
             __syncwarp();
-            if (c.full) {
-                wait(&m.sx[slot], j >> 1);
-                if (lane == 0) {
-                    ptx::tc_fence_after_sync();
-                    const uint32_t lanes = (uint32_t)(16 * slot) << 16;
-                    const uint64_t sxh = ptx::desc_sw128(sbase + C::kSX0 + slot * C::kSXBytes, D * 128, 1024);
-                    const uint64_t sxl = sxh + ((D * D * 2) >> 4);
-                    if (!*abort_flag) {
-#pragma unroll
-                        for (int pass = 0; pass < 3; ++pass)
-#pragma unroll
-                            for (int k = 0; k < 4; ++k)
-                                ptx::mma_f16_ts(tmem + lanes + C::kColO,
-                                                tmem + lanes + (pass == 2 ? C::kColQL : C::kColQH) + 8 * k,
-                                                (pass == 1 ? sxl : sxh) + 128 * k, M::kIdIN, pass > 0 || k > 0);
-                    }
-                }
-                __syncwarp();
-                wait(&m.pfull[slot], j >> 1);
-                if (lane == 0) {
-                    ptx::tc_fence_after_sync();
-                    const uint32_t lanes = (uint32_t)(16 * slot) << 16;
-                    const uint32_t stg = (uint32_t)s * C::kStage >> 4;
-                    if (!*abort_flag) {
-#pragma unroll
-                        for (int k = 0; k < 4; ++k)
-                            ptx::mma_f16_ss(tmem + lanes + C::kColO, pa0 + stg + 2 * k, v0 + stg + 128 * k,
-                                            kIdPVss, true);
-                    }
-                }
-                __syncwarp();
-            } else {
-                wait(&m.sx[slot], j >> 1);              // the back team's no-op arrivals
-                wait(&m.pfull[slot], j >> 1);
-            }
+            wait(&m.pfull[slot], j >> 1);
             if (lane == 0) {
+                ptx::tc_fence_after_sync();
+                if (c.full && !*abort_flag) {         // O += P V
+#pragma unroll
+                    for (int k = 0; k < 4; ++k)
+                        ptx::mma_f16_ss(tmem + lanes + C::kColO, pa0 + stg + 2 * k, v0 + stg + 128 * k, kIdPVss, true);
+                }
                 ptx::mma_commit(&m.o[slot]);
-                ptx::mma_commit(&m.stfree[s]);     // this chunk's products have read the stage
+                ptx::mma_commit(&m.stfree[s]);        // this chunk's products have read the stage
             }
             __syncwarp();
         };
@@ -648,6 +637,7 @@ __global__ void __launch_bounds__(PipeCfg::kThreads, 1)
             wait(&m.ld[s], j / 3);
             ptx::tc_fence_after_sync();
             const bool slow = gate(stage, c, slot);
+            if (ttid == 0) ptx::mbar_arrive(&m.gdone[slot]);        // r of the chunk: S~ may start
             if (!c.full) {
                 build_ks(stage, slot);
             } else {
@@ -667,32 +657,39 @@ __global__ void __launch_bounds__(PipeCfg::kThreads, 1)
 
     // =================================================================== back team
     else if (back) {
+        // S~^T of chunk i = S^T Diag(2^{r_i}) from the carried state: bf16 high / low parts into
+        // the stage's S~ tiles (K-major rows j, the second half of the fused product's operand)
+        auto prep_sx = [&](int i) {
+            const int slot = i & 1;
+            wait(&m.gdone[slot], i >> 1);               // r of chunk i
+            if (chunk_of(i).full) {
+                uint8_t *stg = sm + (uint32_t)(i % 3) * C::kStage;
+#pragma unroll
+                for (int q = 0; q < 2; ++q) {
+                    const float4 fa = *reinterpret_cast<const float4 *>(&m.er[slot][16 * cg + 8 * q]);
+                    const float4 fb = *reinterpret_cast<const float4 *>(&m.er[slot][16 * cg + 8 * q + 4]);
+                    const float f[8] = {fa.x, fa.y, fa.z, fa.w, fb.x, fb.y, fb.z, fb.w};
+                    uint32_t h[4], l[4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e)
+                        split_bf2(f[2 * e] * S[8 * q + 2 * e], f[2 * e + 1] * S[8 * q + 2 * e + 1], h[e], l[e]);
+                    const uint32_t o = off_h<64>(sc, 2 * cg + q);
+                    *reinterpret_cast<uint4 *>(stg + C::kTSH + o) = make_uint4(h[0], h[1], h[2], h[3]);
+                    *reinterpret_cast<uint4 *>(stg + C::kTSL + o) = make_uint4(l[0], l[1], l[2], l[3]);
+                }
+                ptx::fence_proxy_async_smem();
+                team_bar(2);
+            }
+            if (ttid == 0) ptx::mbar_arrive(&m.sx[slot]);
+        };
         auto step = [&](int j) {
             const int slot = j & 1, s = j % 3;
             const uint32_t stage = (uint32_t)s * C::kStage;
             const Chunk c = chunk_of(j);
             const uint32_t rows = tmem_rows(slot);
             wait(&m.fdone[slot], j >> 1);              // gate scalars, dq, slow flag of chunk j
+            wait(&m.sc[slot], j >> 1);                 // [scores | inter] done (a bare commit if state-only)
             if (c.full) {
-                // S~ = 2^{r} S (state entering chunk j); this slot's S~ was last read by chunk j - 2,
-                // whose output this team waited for
-                {
-                    const float f = m.er[slot][sc];
-                    uint8_t *sx = sm + C::kSX0 + slot * C::kSXBytes;
-#pragma unroll
-                    for (int q = 0; q < 2; ++q) {
-                        uint32_t h[4], l[4];
-#pragma unroll
-                        for (int e = 0; e < 4; ++e) split_bf2(f * S[8 * q + 2 * e], f * S[8 * q + 2 * e + 1], h[e], l[e]);
-                        const uint32_t o = off_sx<64>(sc, 2 * cg + q);
-                        *reinterpret_cast<uint4 *>(sx + o) = make_uint4(h[0], h[1], h[2], h[3]);
-                        *reinterpret_cast<uint4 *>(sx + D * D * 2 + o) = make_uint4(l[0], l[1], l[2], l[3]);
-                    }
-                }
-                ptx::fence_proxy_async_smem();
-                team_bar(2);
-                if (ttid == 0) ptx::mbar_arrive(&m.sx[slot]);
-                wait(&m.sc[slot], j >> 1);              // scores done: the K~-low tile is free
                 ptx::tc_fence_after_sync();
                 if (!m.slow[slot]) {
                     float dq = 0.0f;
@@ -724,26 +721,28 @@ __global__ void __launch_bounds__(PipeCfg::kThreads, 1)
                 ptx::fence_proxy_async_smem();
                 ptx::tc_fence_before_sync();
                 team_bar(2);
-                if (ttid == 0) ptx::mbar_arrive(&m.pfull[slot]);
-            } else {                                    // state-only chunk: no S~, no P
-                if (ttid == 0) {
-                    ptx::mbar_arrive(&m.sx[slot]);
-                    ptx::mbar_arrive(&m.pfull[slot]);
-                }
-                wait(&m.sc[slot], j >> 1);              // bare commit; keeps the waits in phase
             }
-            // S = Diag(2^{B}) S + S_loc
+            if (ttid == 0) ptx::mbar_arrive(&m.pfull[slot]);
+            // S^T = S^T Diag(2^{B}) + S_loc^T
             wait(&m.sl[slot], j >> 1);
             ptx::tc_fence_after_sync();
             {
                 float sl[16];
-                ptx::tmem_ld16x2_x16<16>(tmem + ((uint32_t)(32 * qd + 16 * slot) << 16) + C::kColSL + 32 * hg, sl);
+                ptx::tmem_ld16x2_x16<16>(rows + C::kColSL + 32 * hg, sl);
                 ptx::tmem_ld_wait();
-                const float e = m.eB[slot][sc];
 #pragma unroll
-                for (int i = 0; i < 16; ++i) S[i] = fmaf(e, S[i], sl[i]);
+                for (int q = 0; q < 4; ++q) {
+                    const float4 e = *reinterpret_cast<const float4 *>(&m.eB[slot][16 * cg + 4 * q]);
+                    S[4 * q] = fmaf(e.x, S[4 * q], sl[4 * q]);
+                    S[4 * q + 1] = fmaf(e.y, S[4 * q + 1], sl[4 * q + 1]);
+                    S[4 * q + 2] = fmaf(e.z, S[4 * q + 2], sl[4 * q + 2]);
+                    S[4 * q + 3] = fmaf(e.w, S[4 * q + 3], sl[4 * q + 3]);
+                }
             }
             if (!c.full && ttid < D) m.Gs[ttid] += m.Bc[slot][ttid];
+            // the next chunk's S~ now, so its fused product runs under this chunk's epilogue (the
+            // first full chunk after an exchange waits for the incoming state)
+            if (j + 1 < N && j + 1 != n1) prep_sx(j + 1);
             wait(&m.o[slot], j >> 1);                   // a state-only chunk's is a bare commit
             if (c.full) {
                 ptx::tc_fence_after_sync();
@@ -784,8 +783,10 @@ __global__ void __launch_bounds__(PipeCfg::kThreads, 1)
                 ptx::mbar_arrive(&m.stfree[s]);
             }
         };
+        if (n1 > 0) prep_sx(0);
         for (int j = 0; j < n1; ++j) step(j);
         if (exchange) run_exchange();
+        if (n1 < N) prep_sx(n1);
         for (int j = n1; j < N; ++j) step(j);
         __syncthreads();
     }
