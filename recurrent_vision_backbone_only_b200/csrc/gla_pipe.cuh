@@ -15,12 +15,19 @@
 // i ^ (hb - 1).  Other line lengths keep line-aligned chunks (one 64-row box, scan offset i in
 // row n - 1 - i when reversed).
 //
+// Fused product.  The carried state is kept transposed, S^T[j][c] (S_loc^T = V^T Ks), so
+// S~^T = S^T Diag(2^r) is a K-major operand like K~, and each stage places S~^T right after K~:
+// [K~ | S~^T] is one 128-row operand, and Q~ [K~ | S~^T]^T yields the scores (columns 0-63) and
+// the inter-chunk term Q~ S~ (columns 64-127, the output accumulator) in the same tcgen05.mma
+// (N = 128): per chunk 4 state, 12 fused and 4 P V products.
+//
 // Roles (576 threads):
 //   front team  (warps 0-7)   per chunk: gate (cumulative log2-decay b), then the operands Kh,
 //                             Kl, Ks in place over the raw tiles and Q~ into the chunk's TMEM slot;
-//   back team   (warps 8-15)  per chunk: S~ from the carried state, P from the scores (into the
-//                             dead K~-low tile, as the A operand of P V), the state fold, the
-//                             RMSNorm / SiLU epilogue and the stores;
+//   back team   (warps 8-15)  per chunk: P from the scores (into the dead K~-low tile, as the A
+//                             operand of P V), the state fold, the NEXT chunk's S~^T (so its
+//                             fused product runs under this chunk's epilogue), the RMSNorm /
+//                             SiLU epilogue and the stores;
 //   MMA warp    (warp 16)     issues every tcgen05.mma and commit;
 //   load warp   (warp 17)     issues the TMA boxes into a 3-stage ring.
 // Chunk j uses TMEM slot j % 2 -- lanes 16 (j % 2) .. + 16 of every lane quarter, so one M = 64
@@ -31,10 +38,11 @@
 // every slot barrier exactly once (a state-only chunk with no-op arrivals and commits), and every
 // waiter of a barrier waits on each of its phases in turn, so the k-th use of a slot always waits
 // for parity k & 1 and no waiter is ever two phases behind:
-//   ld[s]        TMA bytes of a stage landed                       load warp -> front, back
+//   ld[s]        TMA bytes of a stage landed                       load warp -> front
+//   gdone[p]     gate scalars (r) of the slot's chunk ready        front -> back (S~^T)
 //   fdone[p]     gate + operands of the slot's chunk ready         front -> MMA, back
-//   sl, sc, o[p] chunk state / scores / output products done      tcgen05.commit -> back
-//   sx[p]        S~ of the slot's chunk written                    back -> MMA
+//   sl, sc, o[p] chunk state / fused / output products done       tcgen05.commit -> back
+//   sx[p]        S~^T of the slot's chunk written                  back -> MMA
 //   pfull[p]     P written                                         back -> MMA
 //   slotfree[p]  the back team is done with the slot's chunk       back -> front, MMA
 //   stfree[s]    the stage may be reloaded (2 arrivals)            tcgen05.commit + back -> load
@@ -566,10 +574,12 @@ __global__ void __launch_bounds__(PipeCfg::kThreads, 1)
                     make_uint4(pack_h2(pv[8 * h], pv[8 * h + 1]), pack_h2(pv[8 * h + 2], pv[8 * h + 3]),
                                pack_h2(pv[8 * h + 4], pv[8 * h + 5]), pack_h2(pv[8 * h + 6], pv[8 * h + 7]));
         };
-        auto build_full = [&](uint32_t stage, int slot, bool slow) {
+        // fast path (decay half-range within the bf16 operands' reach): one 8-channel group per
+        // iteration, the loop kept rolled so the team's hot code stays small
+        auto build_full = [&](uint32_t stage, int slot) {
             float dqs = 0.0f;
-            uint32_t qh[8], ql[8];
-#pragma unroll
+            const uint32_t rows = tmem_q + ((uint32_t)(32 * qd + 16 * slot) << 16);
+#pragma unroll 1
             for (int jj = 0; jj < 2; ++jj) {
                 const int j = 2 * cg + jj;
                 const uint32_t o = off_h<64>(t, j);
@@ -583,50 +593,71 @@ __global__ void __launch_bounds__(PipeCfg::kThreads, 1)
                 const float4 rB = *reinterpret_cast<const float4 *>(&m.rref[slot][8 * j + 4]);
                 const float4 qA = *reinterpret_cast<const float4 *>(&m.rq[slot][8 * j]);
                 const float4 qB = *reinterpret_cast<const float4 *>(&m.rq[slot][8 * j + 4]);
-                const float *fsrc = slow ? m.Bc[slot] : m.fB[slot];
-                const float4 fA = *reinterpret_cast<const float4 *>(fsrc + 8 * j);
-                const float4 fBv = *reinterpret_cast<const float4 *>(fsrc + 8 * j + 4);
+                const float4 fA = *reinterpret_cast<const float4 *>(&m.fB[slot][8 * j]);
+                const float4 fBv = *reinterpret_cast<const float4 *>(&m.fB[slot][8 * j + 4]);
                 const float bt[8] = {bA.x, bA.y, bA.z, bA.w, bB.x, bB.y, bB.z, bB.w};
                 const float rr[8] = {rA.x, rA.y, rA.z, rA.w, rB.x, rB.y, rB.z, rB.w};
                 const float rq[8] = {qA.x, qA.y, qA.z, qA.w, qB.x, qB.y, qB.z, qB.w};
                 const float ff[8] = {fA.x, fA.y, fA.z, fA.w, fBv.x, fBv.y, fBv.z, fBv.w};
-                float kt[8], qt[8], ks[8];
+                uint32_t kh4[4], kl4[4], ks4[4], qh4[4], ql4[4];
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
                     const float2 kf = __half22float2(k2[e]);
                     const float2 qf = __half22float2(q2[e]);
-                    const float kv[2] = {kf.x, kf.y}, qv[2] = {qf.x, qf.y};
-#pragma unroll
-                    for (int h = 0; h < 2; ++h) {
-                        const int i = 2 * e + h;
-                        dqs = fmaf(qv[h], kv[h], dqs);
-                        qt[i] = qv[h] * ptx::ex2(bt[i] - rq[i]);
-                        if (!slow) {
-                            kt[i] = kv[h] * ptx::ex2(rr[i] - bt[i]);
-                            ks[i] = kt[i] * ff[i];
-                        } else {
-                            kt[i] = 0.0f;
-                            ks[i] = kv[h] * ptx::ex2(ff[i] - bt[i]);
-                        }
-                    }
+                    dqs = fmaf(qf.x, kf.x, dqs);
+                    dqs = fmaf(qf.y, kf.y, dqs);
+                    const float q0 = qf.x * ptx::ex2(bt[2 * e] - rq[2 * e]);
+                    const float q1 = qf.y * ptx::ex2(bt[2 * e + 1] - rq[2 * e + 1]);
+                    const float k0 = kf.x * ptx::ex2(rr[2 * e] - bt[2 * e]);
+                    const float k1 = kf.y * ptx::ex2(rr[2 * e + 1] - bt[2 * e + 1]);
+                    split_bf2(k0, k1, kh4[e], kl4[e]);
+                    split_bf2(q0, q1, qh4[e], ql4[e]);
+                    ks4[e] = pack_h2(k0 * ff[2 * e], k1 * ff[2 * e + 1]);
                 }
-                uint32_t kh4[4], kl4[4], ks4[4];
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    split_bf2(kt[2 * e], kt[2 * e + 1], kh4[e], kl4[e]);
-                    split_bf2(qt[2 * e], qt[2 * e + 1], qh[4 * jj + e], ql[4 * jj + e]);
-                    ks4[e] = pack_h2(ks[2 * e], ks[2 * e + 1]);
-                }
-                if (!slow) {
-                    *reinterpret_cast<uint4 *>(sm + stage + C::kTK + o) = make_uint4(kh4[0], kh4[1], kh4[2], kh4[3]);
-                    *reinterpret_cast<uint4 *>(sm + stage + C::kTA + o) = make_uint4(kl4[0], kl4[1], kl4[2], kl4[3]);
-                }
+                *reinterpret_cast<uint4 *>(sm + stage + C::kTK + o) = make_uint4(kh4[0], kh4[1], kh4[2], kh4[3]);
+                *reinterpret_cast<uint4 *>(sm + stage + C::kTA + o) = make_uint4(kl4[0], kl4[1], kl4[2], kl4[3]);
                 *reinterpret_cast<uint4 *>(sm + stage + C::kTQ + o) = make_uint4(ks4[0], ks4[1], ks4[2], ks4[3]);
+                ptx::tmem_st16x2_x4<8>(rows + C::kColQH + 16 * hg + 4 * jj, qh4);
+                ptx::tmem_st16x2_x4<8>(rows + C::kColQL + 16 * hg + 4 * jj, ql4);
             }
             m.dqp[slot][cg][t] = dqs * p.scale;
+            ptx::tmem_st_wait();
+        };
+        // exact-score path (rare): Q~ = q 2^{b} d_k^{-1/2} into TMEM, Ks = k 2^{B - b}; K~ unused
+        auto build_slow = [&](uint32_t stage, int slot) {
+            float dqs = 0.0f;
             const uint32_t rows = tmem_q + ((uint32_t)(32 * qd + 16 * slot) << 16);
-            ptx::tmem_st16x2_x8<8>(rows + C::kColQH + 16 * hg, qh);
-            ptx::tmem_st16x2_x8<8>(rows + C::kColQL + 16 * hg, ql);
+#pragma unroll 1
+            for (int jj = 0; jj < 2; ++jj) {
+                const int j = 2 * cg + jj;
+                const uint32_t o = off_h<64>(t, j);
+                const uint4 kraw = *reinterpret_cast<const uint4 *>(sm + stage + C::kTK + o);
+                const uint4 qraw = *reinterpret_cast<const uint4 *>(sm + stage + C::kTQ + o);
+                const __half2 *k2 = reinterpret_cast<const __half2 *>(&kraw);
+                const __half2 *q2 = reinterpret_cast<const __half2 *>(&qraw);
+                uint32_t ks4[4], qh4[4], ql4[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const float2 kf = __half22float2(k2[e]);
+                    const float2 qf = __half22float2(q2[e]);
+                    dqs = fmaf(qf.x, kf.x, dqs);
+                    dqs = fmaf(qf.y, kf.y, dqs);
+                    float b2[2], B2[2], rq2[2];
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) {
+                        const int ch = 8 * j + 2 * e + h;
+                        b2[h] = *reinterpret_cast<const float *>(sm + C::kB + off_f<64>(t, ch >> 2) + (ch & 3) * 4);
+                        B2[h] = m.Bc[slot][ch];
+                        rq2[h] = m.rq[slot][ch];
+                    }
+                    split_bf2(qf.x * ptx::ex2(b2[0] - rq2[0]), qf.y * ptx::ex2(b2[1] - rq2[1]), qh4[e], ql4[e]);
+                    ks4[e] = pack_h2(kf.x * ptx::ex2(B2[0] - b2[0]), kf.y * ptx::ex2(B2[1] - b2[1]));
+                }
+                *reinterpret_cast<uint4 *>(sm + stage + C::kTQ + o) = make_uint4(ks4[0], ks4[1], ks4[2], ks4[3]);
+                ptx::tmem_st16x2_x4<8>(rows + C::kColQH + 16 * hg + 4 * jj, qh4);
+                ptx::tmem_st16x2_x4<8>(rows + C::kColQL + 16 * hg + 4 * jj, ql4);
+            }
+            m.dqp[slot][cg][t] = dqs * p.scale;
             ptx::tmem_st_wait();
         };
         auto step = [&](int j) {
@@ -641,8 +672,12 @@ __global__ void __launch_bounds__(PipeCfg::kThreads, 1)
             if (!c.full) {
                 build_ks(stage, slot);
             } else {
-                if (slow) exact_p_smem(stage, c);
-                build_full(stage, slot, slow);
+                if (slow) {
+                    exact_p_smem(stage, c);
+                    build_slow(stage, slot);
+                } else {
+                    build_full(stage, slot);
+                }
             }
             ptx::fence_proxy_async_smem();
             ptx::tc_fence_before_sync();
@@ -755,11 +790,17 @@ __global__ void __launch_bounds__(PipeCfg::kThreads, 1)
                 m.red[cg][t] = ss;
                 team_bar(2);
                 const float inv = rsqrtf((m.red[0][t] + m.red[1][t] + m.red[2][t] + m.red[3][t]) * (1.0f / D) + p.eps);
-                if (t < c.n) {
-                    __half *dst = p.out + (size_t)token_row(c, t) * D + 16 * cg;
-#pragma unroll
-                    for (int jj = 0; jj < 2; ++jj) {
-                        const int jp = 2 * cg + jj;
+                // the TMEM loads are warp-collective: every lane takes them, rows past the chunk
+                // only skip the arithmetic and the store
+                const bool live = t < c.n;
+                __half *dst = p.out + (size_t)(live ? token_row(c, t) : 0) * D + 16 * cg;
+#pragma unroll 1
+                for (int jj = 0; jj < 2; ++jj) {
+                    const int jp = 2 * cg + jj;
+                    float o8[8];
+                    ptx::tmem_ld16x2_x8<16>(rows + C::kColO + 32 * hg + 8 * jj, o8);
+                    ptx::tmem_ld_wait();
+                    if (live) {
                         const uint4 graw = *reinterpret_cast<const uint4 *>(sm + stage + C::kTG + off_h<64>(t, jp));
                         const __half2 *g2 = reinterpret_cast<const __half2 *>(&graw);
                         const float4 wa = *reinterpret_cast<const float4 *>(&m.w[8 * jp]);
@@ -769,8 +810,8 @@ __global__ void __launch_bounds__(PipeCfg::kThreads, 1)
 #pragma unroll
                         for (int e = 0; e < 4; ++e) {
                             const float2 gf = __half22float2(g2[e]);
-                            u[e] = pack_h2(o[8 * jj + 2 * e] * inv * wv[2 * e] * silu_fast(gf.x),
-                                           o[8 * jj + 2 * e + 1] * inv * wv[2 * e + 1] * silu_fast(gf.y));
+                            u[e] = pack_h2(o8[2 * e] * inv * wv[2 * e] * silu_fast(gf.x),
+                                           o8[2 * e + 1] * inv * wv[2 * e + 1] * silu_fast(gf.y));
                         }
                         *reinterpret_cast<uint4 *>(dst + 8 * jj) = make_uint4(u[0], u[1], u[2], u[3]);
                     }
