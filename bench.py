@@ -114,7 +114,8 @@ def profile_traffic(workload: str, kernel: str):
 
 def read_ncu_csv(path: str):
     """Launches of an ncu --csv log (details layout: one row per metric; raw layout: one column
-    per metric) as [(kernel name, {metric: value})], in capture order."""
+    per metric) as [(kernel name, {metric: value})], in capture order; the launch's grid size is
+    kept as the pseudo-metric "grid"."""
     import csv
     with open(path, newline="") as f:
         lines = [ln for ln in f if ln.startswith('"')]
@@ -126,6 +127,7 @@ def read_ncu_csv(path: str):
     order = []
     if "Metric Name" in head:
         i_id, i_k = head.index("ID"), head.index("Kernel Name")
+        i_g = head.index("Grid Size") if "Grid Size" in head else None
         i_n, i_v = head.index("Metric Name"), head.index("Metric Value")
         i_u = head.index("Metric Unit")
         scale = {"byte": 1, "Kbyte": 1e3, "Mbyte": 1e6, "Gbyte": 1e9}
@@ -134,16 +136,17 @@ def read_ncu_csv(path: str):
                 continue
             key = r[i_id]
             if key not in launches:
-                launches[key] = (r[i_k], {})
+                launches[key] = (r[i_k], {"grid": r[i_g] if i_g is not None else ""})
                 order.append(key)
             v = float(r[i_v].replace(",", ""))
             launches[key][1][r[i_n]] = v * scale.get(r[i_u], 1)
     else:
         units = rows[1]
         i_id, i_k = head.index("ID"), head.index("Kernel Name")
+        i_g = head.index("Grid Size") if "Grid Size" in head else None
         scale = {"byte": 1, "Kbyte": 1e3, "Mbyte": 1e6, "Gbyte": 1e9}
         for r in rows[2:]:
-            vals = {}
+            vals = {"grid": r[i_g] if i_g is not None else ""}
             for j, name in enumerate(head):
                 if name.startswith(("dram__", "gpu__time")) and j < len(r) and r[j]:
                     vals[name] = float(r[j].replace(",", "")) * scale.get(units[j], 1)
@@ -168,10 +171,16 @@ def record_traffic(args):
     if not got:
         raise SystemExit("no %s launch with dram__bytes_read/write.sum in %s"
                          % (symbol[kid], args.record_traffic))
-    rd = statistics.mean(v["dram__bytes_read.sum"] for v in got)
-    wr = statistics.mean(v["dram__bytes_write.sum"] for v in got)
+    # one gla_fwd call may issue two launches (a partial wave split off): per call, the mean
+    # over launches of each grid shape, summed over the shapes
+    shapes = sorted({v.get("grid", "") for v in got})
+    rd = sum(statistics.mean(v["dram__bytes_read.sum"] for v in got if v.get("grid", "") == g)
+             for g in shapes)
+    wr = sum(statistics.mean(v["dram__bytes_write.sum"] for v in got if v.get("grid", "") == g)
+             for g in shapes)
     print(json.dumps({"workload": wl.name, "kernel": gla.KERNEL_NAMES[kid],
                       "lib_sources_digest": _b.sources_digest(), "launches": len(got),
+                      "launch_shapes": shapes,
                       "dram_read_bytes": rd, "dram_write_bytes": wr,
                       "dram_bytes_per_launch": rd + wr,
                       "algorithmic_bytes_per_launch": wl.tokens * wl.bytes_per_token,
@@ -397,6 +406,12 @@ def run_ours(args, ws, rank, local):
               "pipe64": gla.KERNEL_PIPE64, "simt": gla.KERNEL_SIMT}[args.kernel]
     kernel_name = (gla.KERNEL_NAMES[kernel] if kernel else
                    gla.plan(wl.B, wl.H, gh, gw, wl.d_k, wl.d_v, 0 if wl.dtype == "f16" else 1)["kernel"])
+    # kernel launches per gla_fwd call: two when the library splits off a partial wave (its
+    # plan then has more CTAs than pairs x segments); gla_fwd_ex with an explicit kernel and
+    # automatic segments splits the same way
+    _pl = gla.plan(wl.B, wl.H, gh, gw, wl.d_k, wl.d_v, 0 if wl.dtype == "f16" else 1)
+    calls_split = (_pl["kernel"] == kernel_name and
+                   _pl["ctas"] > wl.B * wl.H * _pl["segments"])
 
     def step(i):
         for j, d in enumerate(directions):
@@ -531,7 +546,7 @@ def run_ours(args, ws, rank, local):
                      "launch_floor_us": floor_us,
                      "launch_floor": "do-nothing kernel, same launch shape, same graph replay"},
         "e2e": e2e,
-        "gpu_launches": K * launches_per_step,
+        "gpu_launches": K * launches_per_step * (2 if calls_split else 1),
         "clocks": clocks,
     }
     if ws == 1 and not args.no_cpu_baseline:

@@ -79,9 +79,11 @@ enum gla_direction {
  * q, k, v, gate_preact, out_gate_preact and out are IEEE binary16 arrays;
  * rms_weight is float32.  `stream` is a cudaStream_t (NULL = legacy default
  * stream).  Supported head dims: d_k, d_v in {32, 64, 128}; d_k = d_v = 64 runs on
- * the pipelined 64-row tensor-core kernel when B * H is at least the device's SM count,
- * else on the 128-row one; d_k = d_v = 128 on the 64-row kernel; the others on CUDA
- * cores (gla_kernel below).
+ * the pipelined 64-row tensor-core kernel when B * H is at least the device's SM count or
+ * grid_h * grid_w >= 4096, else on the 128-row one; d_k = d_v = 128 on the 64-row kernel;
+ * the others on CUDA cores (gla_kernel below).  A call may issue two kernel launches: when
+ * the pipelined kernel's pairs exceed a whole number of waves, the last partial wave's pairs
+ * run as a second launch with several CTAs per pair.
  */
 int gla_fwd(const void *q, const void *k, const void *v,
             const void *gate_preact, const void *out_gate_preact,
@@ -162,10 +164,11 @@ int gla_version(void);
 /*
  * gla_plan -- the schedule gla_fwd (dtype 0) / gla_fwd_f32 (dtype 1) would
  * use for these shapes on the current device, without launching anything:
- * *kernel = the gla_kernel it runs (1, 2 or 3), *segments = CTAs
- * (one thread-block cluster) per (b, h) pair, *seg_len = scan positions per
- * segment, *ctas = total CTAs, *max_active_clusters = clusters of that shape
- * the device can hold at once.  Same argument errors as gla_fwd.
+ * *kernel = the gla_kernel it runs (1 to 4), *segments = CTAs (one
+ * thread-block cluster) per (b, h) pair, *seg_len = scan positions per
+ * segment, *ctas = total CTAs (of both launches when the call is split; then
+ * *segments and *seg_len describe the first), *max_active_clusters = clusters
+ * of that shape the device can hold at once.  Same argument errors as gla_fwd.
  */
 int gla_plan(int B, int H, int grid_h, int grid_w, int d_k, int d_v, int dtype, int *kernel,
              int *segments, int *seg_len, int *ctas, int *max_active_clusters);

@@ -115,6 +115,9 @@ struct Plan {
     int chunk = 0;             // tokens per chunk (CUDA-core) / largest chunk (tensor-core)
     size_t smem = 0;
     int max_active_clusters = 0;
+    int ctas = 0;              // CTAs of all launches
+    int tail_pairs = 0;        // pipelined kernel: pairs of a second launch (0: none) ...
+    int tail_segs = 0;         // ... with this many segments per pair
     cudaLaunchConfig_t cfg{};
     cudaLaunchAttribute attr[2];
     bool pdl = false;          // programmatic dependent launch (tensor-core kernel)
@@ -488,6 +491,7 @@ int run_chunk(const Args &x, int chunk, int segs, float eps, cudaStream_t st, co
         }
         return n;
     };
+    const bool auto_segs = segs <= 0;
     if (segs <= 0) {
         static std::mutex mu;
         static int cache[64][2][17];
@@ -516,13 +520,33 @@ int run_chunk(const Args &x, int chunk, int segs, float eps, cudaStream_t st, co
         segs = best_s;
     }
     if (segs > 16) return GLA_ERR_UNSUPPORTED;
+    // Throughput launches of the pipelined kernel (one CTA per pair, more pairs than the device
+    // holds) end with a partial wave.  Whole waves stay one CTA per pair; the remaining pairs go
+    // to a second launch that cuts each into segments, so they fill the device instead of a
+    // fraction of it.  The second launch waits for the first (dependent launch), which ends
+    // with its whole waves.
+    int head_pairs = n_pairs;
+    if (kPipe && auto_segs && segs == 1) {
+        const int wave = clusters(1, false);          // resident one-CTA clusters
+        const int rem = wave > 0 ? n_pairs % wave : 0;
+        if (wave > 0 && n_pairs > wave && rem > 0 && 2 * rem <= wave) {
+            int s2 = std::min(std::min(16, q), wave / rem);
+            while (s2 > 1 && (ceil_div(q, ceil_div(q, s2)) != s2 || clusters(s2, false) < rem)) --s2;
+            if (s2 > 1) {
+                head_pairs = n_pairs - rem;
+                pl.tail_pairs = rem;
+                pl.tail_segs = s2;
+            }
+        }
+    }
     pl.segs = segs;
     pl.seg_len = std::min(L, ceil_div(q, segs) * clen);
     const bool spread = (long long)n_pairs * pl.segs <= di.sms;
     pl.smem = smem_of(spread);
-    configure_launch(pl, n_pairs, kThreads, st);
+    configure_launch(pl, head_pairs, kThreads, st);
     pl.max_active_clusters = clusters(pl.segs, spread);
     if (pl.max_active_clusters <= 0) return GLA_ERR_UNSUPPORTED;
+    pl.ctas = head_pairs * pl.segs + pl.tail_pairs * pl.tail_segs;
     if (query) {
         *query = pl;
         return GLA_OK;
@@ -543,9 +567,21 @@ int run_chunk(const Args &x, int chunk, int segs, float eps, cudaStream_t st, co
     p.fault_chunk = fault_chunk;
     p.hb[0] = hb[0];
     p.hb[1] = hb[1];
+    p.pair0 = 0;
     if (cudaLaunchKernelEx(&pl.cfg, kern, maps, p) != cudaSuccess) {
         cudaGetLastError();
         return GLA_ERR_CUDA;
+    }
+    if (pl.tail_pairs > 0) {
+        Plan tail = pl;
+        tail.segs = pl.tail_segs;
+        configure_launch(tail, pl.tail_pairs, kThreads, st);
+        p.segs = tail.segs;
+        p.pair0 = head_pairs;
+        if (cudaLaunchKernelEx(&tail.cfg, kern, maps, p) != cudaSuccess) {
+            cudaGetLastError();
+            return GLA_ERR_CUDA;
+        }
     }
     return GLA_OK;
 }
@@ -555,12 +591,15 @@ constexpr float kEps = 1e-6f;
 
 // The kernel gla_fwd uses: fp32 I/O on CUDA cores; fp16 d = 64 on the pipelined 64-row kernel
 // when the launch has at least one (b, h) pair per SM (throughput-bound: one CTA per pair, two
-// chunks in flight), else on the 128-row kernel (latency-bound: one chunk per segment and a
-// mid-chunk exchange, faster at 40 x 40, even at 80 x 80); fp16 d = 128 on the 64-row kernel
-// (the only one that holds its tiles); other head dims on CUDA cores.
+// chunks in flight) or scans of at least 4096 positions (segments of many chunks: 80 x 80 with
+// 10 segments per pair measured 71.6 us against 73.5 us), else on the 128-row kernel
+// (latency-bound: one chunk per segment and a mid-chunk exchange; 40 x 40 measured 11.9 us
+// against 28 us); fp16 d = 128 on the 64-row kernel (the only one that holds its tiles); other
+// head dims on CUDA cores.
 int auto_kernel(const Args &x, int dtype, const DeviceInfo &di) {
     if (dtype == 1) return kSimt;
-    if (x.dk == 64 && x.dv == 64) return (long long)x.B * x.H >= di.sms ? kPipe64 : kTc128;
+    if (x.dk == 64 && x.dv == 64)
+        return ((long long)x.B * x.H >= di.sms || (long long)x.gh * x.gw >= 4096) ? kPipe64 : kTc128;
     if (x.dk == 128 && x.dv == 128) return kTc64;
     return kSimt;
 }
@@ -750,7 +789,7 @@ int gla_plan(int B, int H, int grid_h, int grid_w, int d_k, int d_v, int dtype, 
     *kernel = pl.kernel;
     *segments = pl.segs;
     *seg_len = pl.seg_len;
-    *ctas = B * H * pl.segs;
+    *ctas = pl.ctas > 0 ? pl.ctas : B * H * pl.segs;
     *max_active_clusters = pl.max_active_clusters;
     return GLA_OK;
 }

@@ -129,6 +129,8 @@ struct Params {
     int fault_chunk;        // test hook: full-pass chunk whose loads are not issued (-1: none)
     int hb[2];              // pipelined kernel: rows per TMA box of packed chunks for the row and
                             // column families (0: line-aligned chunks, one 64-row box per tile)
+    int pair0;              // pipelined kernel: first (b, h) pair of this launch (a launch may
+                            // cover a suffix of the pairs)
 };
 
 // Tensor maps of the five inputs in the two line families: row family [B L][H][D] (box: 64

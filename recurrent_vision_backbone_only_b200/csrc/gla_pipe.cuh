@@ -200,8 +200,8 @@ __global__ void __launch_bounds__(PipeCfg::kThreads, 1)
     const int t = 16 * qd + (lane & 15);
     const int ttid = tid & (C::kTeam - 1);           // thread index within its team
 
-    const int pair = blockIdx.x / p.segs;
-    const int rank = blockIdx.x - pair * p.segs;
+    const int rank = blockIdx.x % p.segs;
+    const int pair = p.pair0 + blockIdx.x / p.segs;
     const int bb = pair / p.H, hh = pair - bb * p.H;
     const int dir = p.dir == 4 ? (bb & 3) : p.dir;
     const Scan ln(dir, p.gh, p.gw, p.chunk_max, p.hb[dir >> 1]);

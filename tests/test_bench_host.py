@@ -67,6 +67,10 @@ NCU_DETAILS = """==PROF== Connected to process 1
 "ID","Process ID","Process Name","Host Name","Kernel Name","Context","Stream","Block Size","Grid Size","Device","CC","Section Name","Metric Name","Metric Unit","Metric Value"
 "0","1","python","h","void gla::ck::gla_pipe_kernel(Maps, Params)","1","7","(576, 1, 1)","(192, 1, 1)","0","10.0","Command line profiler metrics","dram__bytes_read.sum","Mbyte","206.02"
 "0","1","python","h","void gla::ck::gla_pipe_kernel(Maps, Params)","1","7","(576, 1, 1)","(192, 1, 1)","0","10.0","Command line profiler metrics","dram__bytes_write.sum","Mbyte","29.07"
+"2","1","python","h","void gla::ck::gla_pipe_kernel(Maps, Params)","1","7","(576, 1, 1)","(132, 1, 1)","0","10.0","Command line profiler metrics","dram__bytes_read.sum","Mbyte","50"
+"2","1","python","h","void gla::ck::gla_pipe_kernel(Maps, Params)","1","7","(576, 1, 1)","(132, 1, 1)","0","10.0","Command line profiler metrics","dram__bytes_write.sum","Mbyte","10"
+"3","1","python","h","void gla::ck::gla_pipe_kernel(Maps, Params)","1","7","(576, 1, 1)","(192, 1, 1)","0","10.0","Command line profiler metrics","dram__bytes_read.sum","Mbyte","206.02"
+"3","1","python","h","void gla::ck::gla_pipe_kernel(Maps, Params)","1","7","(576, 1, 1)","(192, 1, 1)","0","10.0","Command line profiler metrics","dram__bytes_write.sum","Mbyte","29.07"
 "1","1","python","h","void other_kernel()","1","7","(1, 1, 1)","(1, 1, 1)","0","10.0","Command line profiler metrics","dram__bytes_read.sum","byte","7"
 "1","1","python","h","void other_kernel()","1","7","(1, 1, 1)","(1, 1, 1)","0","10.0","Command line profiler metrics","dram__bytes_write.sum","byte","0"
 """
@@ -76,12 +80,14 @@ def test_ncu_csv_reader_and_traffic_entry(tmp_path, capsys):
     p = tmp_path / "n.csv"
     p.write_text(NCU_DETAILS)
     got = bench.read_ncu_csv(str(p))
-    assert [k for k, _ in got] == ["void gla::ck::gla_pipe_kernel(Maps, Params)", "void other_kernel()"]
+    assert [k for k, _ in got][:2] == ["void gla::ck::gla_pipe_kernel(Maps, Params)"] * 2
     assert got[0][1]["dram__bytes_read.sum"] == pytest.approx(206.02e6)
+    assert got[1][1]["grid"] == "(132, 1, 1)"
     args = bench.argparse.Namespace(record_traffic=str(p), workload="batched", kernel="pipe64",
                                     ncu_command="ncu ...")
     bench.record_traffic(args)
     e = json.loads(capsys.readouterr().out)
     assert e["workload"] == "batched" and e["kernel"] == "tensor-core 64-row pipelined"
-    assert e["dram_bytes_per_launch"] == pytest.approx(235.09e6)
-    assert e["launches"] == 1
+    # a call = one launch of each grid shape: (206.02 + 29.07) + (50 + 10) MB
+    assert e["dram_bytes_per_launch"] == pytest.approx(295.09e6)
+    assert e["launches"] == 3 and len(e["launch_shapes"]) == 2

@@ -89,12 +89,33 @@ def test_tiny_fp32(direction):
 @pytest.mark.parametrize("kernel", [0, TC64, PIPE64])
 @pytest.mark.parametrize("name", ["gtr640", "highres"])
 def test_full_workloads_all_directions(name, kernel):
-    # kernel 0: the one gla_fwd picks (the 128-row tensor-core kernel at d = 64)
+    # kernel 0: the one gla_fwd picks (128-row kernel at 40 x 40, pipelined at 80 x 80)
     wl = synth.WORKLOADS[name]
     x = synth.make_inputs(wl)
     for d in wl.directions:
         assert_close(run_gpu(x, wl.grid_h, wl.grid_w, d, kernel=kernel),
                      oracle_ref(x, wl.grid_h, wl.grid_w, d), wl.dtype)
+
+
+def test_batched_plan_splits_the_partial_wave():
+    # 192 pairs on the pipelined kernel: whole waves one CTA per pair, the remainder in segments
+    import torch
+    wl = synth.WORKLOADS["batched"]
+    pl = gla.plan(wl.B, wl.H, wl.grid_h, wl.grid_w, wl.d_k, wl.d_v, 0)
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    pairs = wl.B * wl.H
+    assert pl["kernel"] == gla.KERNEL_NAMES[PIPE64]
+    if pairs > sms and 2 * (pairs % sms) <= sms:
+        assert pl["ctas"] > pairs
+
+
+@pytest.mark.parametrize("B,H", [(3, 53), (1, 149), (5, 40)])
+def test_partial_wave_split_parity(B, H):
+    # pair counts just above and around a wave: the tail launch starts mid-batch
+    wl = synth.WORKLOADS["batched"].with_(B=B, H=H, grid_h=16, grid_w=24)
+    x = synth.make_inputs(wl)
+    u = run_gpu(x, wl.grid_h, wl.grid_w, 4, kernel=PIPE64)
+    assert_close(u, oracle_ref(x, wl.grid_h, wl.grid_w, 4), wl.dtype)
 
 
 @pytest.mark.parametrize("kernel", [0, TC64, PIPE64])
