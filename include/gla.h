@@ -41,6 +41,13 @@
  * launched; a launch failure returns GLA_ERR_CUDA (the CUDA error is consumed).
  * Device-side faults detected by the kernels (GLA_ERR_TIMEOUT, GLA_ERR_RANGE)
  * are latched in a per-device status word read by gla_get_status().
+ *
+ * Checked build: libgla_checked.so is compiled from the same sources with
+ * -DGLA_CHECKED.  It exports the same calls; in it every computed index that
+ * addresses device or shared memory (gathered and stored token rows, TMA box
+ * coordinates, remote exchange rows, chunk geometry) is checked against its
+ * buffer first, and a violation latches GLA_ERR_CHECK and skips the access.
+ * It stands in for a memory checker on hardware where none can run.
  */
 #ifndef GLA_H_
 #define GLA_H_
@@ -60,7 +67,9 @@ enum gla_status {
     GLA_ERR_CUDA = 6,        /* CUDA launch/runtime error                        */
     GLA_ERR_TIMEOUT = 7,     /* device: a bounded wait ran out                   */
     GLA_ERR_RANGE = 8,       /* device: an intermediate left the operand range   */
-    GLA_ERR_NO_DEVICE = 9    /* no usable sm_100 device                          */
+    GLA_ERR_NO_DEVICE = 9,   /* no usable sm_100 device                          */
+    GLA_ERR_CHECK = 10       /* device: an index check failed (the checked build,  */
+                             /* libgla_checked.so, only; the access was skipped)  */
 };
 
 enum gla_direction {

@@ -18,6 +18,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libgla.so")
+LIB_CHECKED = os.path.join(PKG, "libgla_checked.so")   # -DGLA_CHECKED: index-checked kernels
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",
@@ -51,23 +52,23 @@ def nvcc() -> str:
     return "nvcc"
 
 
-def build(force: bool = False, verbose: bool = False, extra=()) -> str:
-    """Compile libgla.so if stale; return its path."""
+def build(force: bool = False, verbose: bool = False, extra=(), checked: bool = False) -> str:
+    """Compile libgla.so (checked: libgla_checked.so, with -DGLA_CHECKED) if stale; return its path."""
+    lib = LIB_CHECKED if checked else LIB
     srcs = _sources()
-    if (not force and os.path.exists(LIB) and
-            all(os.path.getmtime(s) <= os.path.getmtime(LIB) for s in srcs)):
-        return LIB
-    tmp = LIB + ".tmp%d" % os.getpid()
-    cmd = [nvcc(), *NVCC_FLAGS, *extra, "-I", INCLUDE, "-I", CSRC,
-           os.path.join(CSRC, "gla_api.cu"), "-o", tmp]
+    if (not force and os.path.exists(lib) and
+            all(os.path.getmtime(s) <= os.path.getmtime(lib) for s in srcs)):
+        return lib
+    tmp = lib + ".tmp%d" % os.getpid()
+    cmd = [nvcc(), *NVCC_FLAGS, *(["-DGLA_CHECKED"] if checked else []), *extra, "-I", INCLUDE,
+           "-I", CSRC, os.path.join(CSRC, "gla_api.cu"), "-o", tmp]
     if verbose:
         print(" ".join(cmd), file=sys.stderr)
     subprocess.check_call(cmd)
-    os.replace(tmp, LIB)
-    return LIB
+    os.replace(tmp, lib)
+    return lib
 
 
 if __name__ == "__main__":
-    build(force="--force" in sys.argv, verbose=True,
-          extra=["-Xptxas", "-v"] if "--ptxas-v" in sys.argv else [])
-    print(LIB)
+    print(build(force="--force" in sys.argv, verbose=True, checked="--checked" in sys.argv,
+                extra=["-Xptxas", "-v"] if "--ptxas-v" in sys.argv else []))

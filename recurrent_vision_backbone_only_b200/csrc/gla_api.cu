@@ -760,6 +760,7 @@ const char *gla_status_string(int code) {
     case GLA_ERR_ALIAS: return "GLA_ERR_ALIAS: out overlaps an input";
     case GLA_ERR_CUDA: return "GLA_ERR_CUDA: CUDA runtime or launch error";
     case GLA_ERR_TIMEOUT: return "GLA_ERR_TIMEOUT: a bounded device wait ran out";
+    case GLA_ERR_CHECK: return "GLA_ERR_CHECK: an index check of the checked build failed";
     case GLA_ERR_RANGE: return "GLA_ERR_RANGE: an intermediate left the supported operand range";
     case GLA_ERR_NO_DEVICE: return "GLA_ERR_NO_DEVICE: no usable sm_100 device is current";
     default: return "unknown gla status";

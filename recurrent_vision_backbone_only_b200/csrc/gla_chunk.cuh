@@ -464,6 +464,10 @@ __global__ void __launch_bounds__(Cfg<D>::kThreads, 1) __maxnreg__(D == 64 ? 120
         // [B gh][W H][D] at (channel, line H + h, b gh + lp0)
         const int y = ln.fam ? c.line * p.H + hh : hh;
         const int z = ln.fam ? bb * p.gh + c.lp0 : bb * p.L + c.line * p.gw + c.lp0;
+        // a box starts inside its view (it may run past the line's end: those rows are masked)
+        if (!GLA_CHECK(y >= 0 && y < (ln.fam ? p.gw * p.H : p.H) && z >= 0 &&
+                       z < (ln.fam ? p.B * p.gh : p.B * p.L) && c.lp0 >= 0 && c.lp0 + c.n <= ln.len))
+            return true;
         const uint32_t b = ptx::smem_u32(bar);
         const uint32_t toff[5] = {dst_stage + C::kTQ, dst_stage + C::kTK, dst_stage + C::kTA,
                                   dst_stage + C::kTV, C::kG};
@@ -723,8 +727,9 @@ __global__ void __launch_bounds__(Cfg<D>::kThreads, 1) __maxnreg__(D == 64 ? 120
 #pragma unroll
         for (int g = 0; g < C::kTPR; ++g) tot += m.red[g][t];
         const float inv = rsqrtf(tot * (1.0f / D) + p.eps);
-        if (t < c.n) {
-            __half *dst = p.out + (size_t)token_row(c, t) * D + 16 * ro.cg;
+        const int orow = t < c.n ? token_row(c, t) : 0;
+        if (t < c.n && GLA_CHECK(orow >= 0 && orow < p.B * p.L * p.H)) {
+            __half *dst = p.out + (size_t)orow * D + 16 * ro.cg;
 #pragma unroll
             for (int jj = 0; jj < 2; ++jj) {
                 const int j = 2 * ro.cg + jj;
@@ -798,7 +803,8 @@ __global__ void __launch_bounds__(Cfg<D>::kThreads, 1) __maxnreg__(D == 64 ? 120
         __syncthreads();
         ptx::cluster_arrive_release();
         ptx::cluster_wait();
-        if (rank < segs - 1) {
+        if (rank < segs - 1 && GLA_CHECK((rank + 1) * max_own <= C::kMaxRecvRows &&
+                                          (uint32_t)(C::kMaxRecvRows * D * 4) <= C::kRecvBytes)) {
             const int owner = ro.sc % segs, lc = ro.sc / segs;
             const uint32_t row = (uint32_t)((rank * max_own + lc) * D + ro.sj0) * 4;
 #pragma unroll
@@ -819,6 +825,7 @@ __global__ void __launch_bounds__(Cfg<D>::kThreads, 1) __maxnreg__(D == 64 ? 120
             for (int it = tid; it < items; it += C::kThreads) {
                 const int lc = it / (D / 4), j4 = it - lc * (D / 4);
                 const int c = lc * segs + rank;
+                if (!GLA_CHECK(c < D && (segs - 1) * max_own + lc < C::kMaxRecvRows)) continue;
                 const uint32_t dst = sbase + C::kSX + (uint32_t)(c * D + 4 * j4) * 4;   // S_in fp32 [c][j]
                 float4 run = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
                 for (int q = 0; q < segs; ++q) {

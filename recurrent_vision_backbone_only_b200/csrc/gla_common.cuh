@@ -25,6 +25,19 @@ __device__ __forceinline__ void raise_status(int code) {
     atomicCAS(&g_status, 0, code);
 }
 
+// Index checks of the checked build (compiled with -DGLA_CHECKED into libgla_checked.so): a
+// computed index outside its buffer latches GLA_ERR_CHECK (10) and the caller skips the access
+// instead of making it.  The release build compiles every check to `true`.
+#ifdef GLA_CHECKED
+__device__ __forceinline__ bool gla_check(bool ok) {
+    if (!ok) raise_status(10 /* GLA_ERR_CHECK */);
+    return ok;
+}
+#define GLA_CHECK(cond) ::gla::gla_check(cond)
+#else
+#define GLA_CHECK(cond) true
+#endif
+
 // Scan position p -> row-major spatial index y*gw + x.
 //   0 L->R: row y = p / gw, x = p % gw
 //   1 R->L: row y = p / gw, x = gw-1 - p % gw

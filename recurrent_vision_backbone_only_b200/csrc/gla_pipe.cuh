@@ -259,6 +259,7 @@ __global__ void __launch_bounds__(PipeCfg::kThreads, 1)
         const bool full = j >= n1;
         Chunk c;
         ln.chunk(q0 + (full ? j - n1 : j), p.L, c.p0, c.n);
+        if (!GLA_CHECK(c.n >= 1 && c.n <= 64 && c.p0 >= 0 && c.p0 + c.n <= p.L)) c.n = 1;
         c.full = full;
         return c;
     };
@@ -298,12 +299,14 @@ __global__ void __launch_bounds__(PipeCfg::kThreads, 1)
         if (back && rank < segs - 1) {                // row c = sc of S, columns [16 cg, + 16)
             const int owner = sc % segs, lc = sc / segs;
             const uint32_t row = (uint32_t)((rank * max_own + lc) * D + 16 * cg) * 4;
+            if (GLA_CHECK(rank * max_own + lc < C::kMaxRecvRows && (rank + 1) * max_own <= C::kMaxRecvRows &&
+                          (uint32_t)(C::kMaxRecvRows * D * 4) <= C::kBBytes))
 #pragma unroll
             for (int i = 0; i < 4; ++i)
                 ptx::st_cluster_v4(ptx::mapa(sbase + C::kB + row + 16 * i, owner),
                                    *reinterpret_cast<const float4 *>(sm + srow(sc) + 64 * cg + 16 * i));
         }
-        if (tid < D && rank < segs - 1) {
+        if (tid < D && rank < segs - 1 && GLA_CHECK(rank * max_own + tid / segs < C::kMaxRecvRows)) {
             const int o2 = tid % segs, l2 = tid / segs;
             ptx::st_cluster_f32(ptx::mapa(ptx::smem_u32(&m.recvG[rank * max_own + l2]), o2), m.Gs[tid]);
         }
@@ -315,6 +318,7 @@ __global__ void __launch_bounds__(PipeCfg::kThreads, 1)
             for (int it = tid; it < items; it += C::kThreads) {
                 const int lc = it / (D / 4), j4 = it - lc * (D / 4);
                 const int c = lc * segs + rank;
+                if (!GLA_CHECK(c < D && (segs - 1) * max_own + lc < C::kMaxRecvRows)) continue;
                 const uint32_t dst = sbase + srow(c) + 16 * j4;
                 float4 run = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
                 for (int q = 0; q < segs; ++q) {
@@ -358,6 +362,11 @@ __global__ void __launch_bounds__(PipeCfg::kThreads, 1)
                         ln.place(c.p0, c.n, i < c.n ? i : 0, line, lp);
                         const int y = ln.fam ? line * p.H + hh : hh;
                         const int z = ln.fam ? bb * p.gh + lp : bb * p.L + line * p.gw + lp;
+                        // a box starts inside its view; a packed group stays inside its line
+                        if (!GLA_CHECK(y >= 0 && y < (ln.fam ? p.gw * p.H : p.H) && z >= 0 &&
+                                       z < (ln.fam ? p.B * p.gh : p.B * p.L) && lp >= 0 &&
+                                       (ln.hb == 0 || lp + rows <= ln.len)))
+                            continue;
                         const uint32_t dst = sbase + s * C::kStage + (uint32_t)i * 128;
                         constexpr uint32_t kDst[5] = {C::kTQ, C::kTK, C::kTA, C::kTV, C::kTG};
 #pragma unroll
@@ -792,8 +801,9 @@ __global__ void __launch_bounds__(PipeCfg::kThreads, 1)
                 const float inv = rsqrtf((m.red[0][t] + m.red[1][t] + m.red[2][t] + m.red[3][t]) * (1.0f / D) + p.eps);
                 // the TMEM loads are warp-collective: every lane takes them, rows past the chunk
                 // only skip the arithmetic and the store
-                const bool live = t < c.n;
-                __half *dst = p.out + (size_t)(live ? token_row(c, t) : 0) * D + 16 * cg;
+                const int orow = t < c.n ? token_row(c, t) : 0;
+                const bool live = t < c.n && GLA_CHECK(orow >= 0 && orow < p.B * p.L * p.H);
+                __half *dst = p.out + (size_t)(live ? orow : 0) * D + 16 * cg;
 #pragma unroll 1
                 for (int jj = 0; jj < 2; ++jj) {
                     const int jp = 2 * cg + jj;

@@ -134,8 +134,10 @@ gla_simt_kernel(const SimtParams p) {
     auto ld16 = [](const T *ptr) { return *reinterpret_cast<const uint4 *>(ptr); };
     auto load_chunk = [&](int c0, int n, bool with_q) {
         __syncthreads();
-        for (int t = tid; t < n; t += NT)
-            rows[t] = (b * p.L + spatial_of(dir, c0 + t, p.gh, p.gw)) * p.H + h;
+        for (int t = tid; t < n; t += NT) {
+            const int r = (b * p.L + spatial_of(dir, c0 + t, p.gh, p.gw)) * p.H + h;
+            rows[t] = GLA_CHECK(c0 + t < p.L && r >= 0 && r < p.B * p.L * p.H) ? r : 0;
+        }
         __syncthreads();
         for (int base = 0; base < n * PK; base += NT) {
             const int pi = base + tid;

@@ -420,7 +420,11 @@ __global__ void __launch_bounds__(kThreads, 1) gla_tc_kernel(const Params p) {
     auto wait_bar = [&](uint64_t *bar, uint32_t parity) { wait_phase(bar, parity, p.wait_limit, abort_flag); };
     // ------------------------------------------------------------ loads
     auto set_rows = [&](int c0, int n, int rb) {
-        if (tid < n) m.rows[rb][tid] = (bb * p.L + spatial_of(dir, c0 + tid, p.gh, p.gw)) * p.H + hh;
+        if (tid < n) {
+            const int r = (bb * p.L + spatial_of(dir, c0 + tid, p.gh, p.gw)) * p.H + hh;
+            // a gathered or stored token row lies inside the arrays (row 0 stands in otherwise)
+            m.rows[rb][tid] = GLA_CHECK(c0 + tid < p.L && r >= 0 && r < p.B * p.L * p.H) ? r : 0;
+        }
     };
     // issue the chunk's gathers (fp16 [n rows][64] tiles, rows >= n zero-filled) into the
     // swizzled layout; completion is tracked per group on mbar_ld[0..2]
@@ -754,7 +758,9 @@ __global__ void __launch_bounds__(kThreads, 1) gla_tc_kernel(const Params p) {
         cluster_ready = true;
     };
     auto recv_off = [&](int lg, int seg, int row) {
-        return kRECV + (uint32_t)(((lg * p.segs + seg) * kGroupRows + row) * 16);
+        const uint32_t o = (uint32_t)(((lg * p.segs + seg) * kGroupRows + row) * 16);
+        // a receive slot lies inside the receive region (its first slot stands in otherwise)
+        return kRECV + (GLA_CHECK(row < kGroupRows && o + 16 <= kRecvBytes) ? o : 0u);
     };
     auto xchg_begin = [&]() {
         cluster_ready_once();

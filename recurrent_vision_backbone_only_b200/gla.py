@@ -18,12 +18,15 @@ from typing import Optional
 
 PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(PKG, "libgla.so")
+# the same library with every computed index checked before use (-DGLA_CHECKED)
+LIB_CHECKED_PATH = os.path.join(PKG, "libgla_checked.so")
 HEADER = os.path.join(os.path.dirname(PKG), "include", "gla.h")
 
 GLA_OK = 0
 STATUS_NAMES = {0: "GLA_OK", 1: "GLA_ERR_NULL", 2: "GLA_ERR_SHAPE", 3: "GLA_ERR_UNSUPPORTED",
                 4: "GLA_ERR_DIRECTION", 5: "GLA_ERR_ALIAS", 6: "GLA_ERR_CUDA",
-                7: "GLA_ERR_TIMEOUT", 8: "GLA_ERR_RANGE", 9: "GLA_ERR_NO_DEVICE"}
+                7: "GLA_ERR_TIMEOUT", 8: "GLA_ERR_RANGE", 9: "GLA_ERR_NO_DEVICE",
+                10: "GLA_ERR_CHECK"}
 DIR_L2R, DIR_R2L, DIR_T2B, DIR_B2T, DIR_CYCLE = 0, 1, 2, 3, 4
 
 _lib = None

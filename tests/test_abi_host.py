@@ -30,10 +30,13 @@ def test_exports_every_declared_symbol(lib):
         assert hasattr(lib, n), n
 
 
-def test_exports_via_nm():
+@pytest.mark.parametrize("checked", [False, True])
+def test_exports_via_nm(checked):
+    # the release library and its index-checked twin (-DGLA_CHECKED) export the same calls
     import subprocess
-    build.build()
-    out = subprocess.run(["nm", "-D", "--defined-only", gla.LIB_PATH], capture_output=True,
+    path = build.build(checked=checked)
+    assert path == (gla.LIB_CHECKED_PATH if checked else gla.LIB_PATH)
+    out = subprocess.run(["nm", "-D", "--defined-only", path], capture_output=True,
                          text=True, check=True).stdout
     exported = {line.split()[-1] for line in out.splitlines() if line.strip()}
     for n in gla.header_functions():
@@ -42,7 +45,7 @@ def test_exports_via_nm():
 
 def test_version_and_strings(lib):
     assert lib.gla_version() >= 100
-    for code in range(10):
+    for code in range(11):
         s = gla.status_string(code)
         assert s.startswith(gla.STATUS_NAMES[code])
     assert "unknown" in gla.status_string(99)
