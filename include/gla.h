@@ -266,7 +266,8 @@ int gla_selftest_load(const void *q, const void *k, const void *gate_preact, con
  * (0: 64).  Writes spatial[p] = the row-major spatial index (y * grid_w + x) of the token the
  * kernel's tiles place at scan position p, for p in [0, grid_h * grid_w) (HOST int array of that
  * length; a position no tile row claims stays -1, one claimed twice returns GLA_ERR_SHAPE),
- * and *box_rows = the rows per TMA box (64 for line-aligned chunks).  The scan order is the
+ * and *box_rows = the rows per TMA box (64 for line-aligned chunks; a forward row scan,
+ * direction 0, loads whole chunks of consecutive token rows).  The scan order is the
  * one of the scan-direction paragraph of the GTR paper's method section (lines in increasing
  * order, the state carried from one line's end to the next line's start); the test suite
  * compares this map with the reference's own on the CPU.

@@ -454,8 +454,8 @@ int run_chunk(const Args &x, int chunk, int segs, float eps, cudaStream_t st, co
     // launch mixes both line families
     int hb[2] = {0, 0};
     if (kPipe) {
-        hb[0] = ck::pack_rows(x.gw, chunk);
-        hb[1] = ck::pack_rows(x.gh, chunk);
+        hb[0] = ck::box_rows(x.dir, 0, x.gh, x.gw, chunk);
+        hb[1] = ck::box_rows(x.dir, 1, x.gh, x.gw, chunk);
     }
     int q = 0, clen = 0;
     for (int dir = 0; dir < 4; ++dir)
@@ -868,7 +868,7 @@ int gla_scan_layout(int kernel, int grid_h, int grid_w, int direction, int chunk
     if (chunk % 16 != 0 || chunk > ck::kC) return GLA_ERR_UNSUPPORTED;
     const int L = grid_h * grid_w;
     const int fam = direction >> 1;
-    const int hb = ck::pack_rows(fam ? grid_h : grid_w, chunk);
+    const int hb = ck::box_rows(direction, fam, grid_h, grid_w, chunk);
     const ck::Scan sc(direction, grid_h, grid_w, chunk, hb);
     for (int p = 0; p < L; ++p) spatial[p] = -1;
     for (int q = 0; q < sc.chunks; ++q) {

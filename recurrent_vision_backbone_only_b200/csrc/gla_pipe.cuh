@@ -106,6 +106,19 @@ __host__ __device__ inline int pack_rows(int len, int cl) {
     return hb >= 8 ? hb : 0;
 }
 
+// Rows per TMA box for line family `fam` of a launch in direction `dir` (4: cycling).  A
+// forward row scan alone (dir 0) visits the token rows in memory order, so a chunk of cl
+// positions is consecutive rows whatever lines it spans and needs no line-bounded groups: boxes
+// of the largest power of two dividing cl.  Otherwise packed groups within a line (pack_rows).
+__host__ __device__ inline int box_rows(int dir, int fam, int gh, int gw, int cl) {
+    if (fam == 0 && dir == 0) {
+        int hb = 64;
+        while (cl % hb != 0) hb >>= 1;
+        return hb;
+    }
+    return pack_rows(fam ? gh : gw, cl);
+}
+
 // Chunks of one (b, h) scan.  Packed (hb > 0): chunk q is the scan positions [q cl, q cl + cl);
 // line-aligned (hb = 0): every line is cut into `pieces` equal pieces of at most cl positions.
 struct Scan {
@@ -113,6 +126,8 @@ struct Scan {
     int rev;      // the scan runs against the spatial order within a line (R->L, B->T)
     int len;      // line length
     int hb;       // rows per box of a packed chunk, 0: line-aligned chunks
+    bool contig;  // packed forward row scan (L->R): a chunk is consecutive token rows whatever
+                  // lines it spans, so its boxes need not stop at a line's end
     int cl;       // chunk length (the last chunk may be shorter)
     int pieces;   // line-aligned: chunks per line
     int chunks;   // chunks per scan
@@ -121,6 +136,7 @@ struct Scan {
         rev = dir & 1;
         len = fam ? gh : gw;
         hb = hb_;
+        contig = hb > 0 && fam == 0 && rev == 0;
         if (hb > 0) {
             cl = chunk_max;
             pieces = 0;
@@ -347,32 +363,40 @@ __global__ void __launch_bounds__(PipeCfg::kThreads, 1)
         auto load = [&](int j) {
             const int s = j % 3;
             if (j >= 3) wait(&m.stfree[s], (j - 3) / 3);
-            if (lane == 0 && !*abort_flag) {
+            // lane 0 decides (the abort flag may change under the warp) and sets the byte count;
+            // the lanes then issue the boxes
+            const bool go = __shfl_sync(0xffffffffu, lane == 0 ? (int)!*abort_flag : 0, 0) != 0;
+            if (go) {
                 const Chunk c = chunk_of(j);
                 const uint32_t mask = c.full ? 0x1Fu : 0x0Eu;
-                ptx::mbar_arrive_expect_tx(&m.ld[s], (uint32_t)__popc(mask) * C::kTile);
+                if (lane == 0) ptx::mbar_arrive_expect_tx(&m.ld[s], (uint32_t)__popc(mask) * C::kTile);
+                __syncwarp();
                 if (!(c.full && j - n1 == p.fault_chunk)) {
                     // one box per group of hb rows (packed) or one 64-row box.  A group past the
                     // chunk's end reloads the first group's tokens: rows that are masked later
                     // still hold finite values, and no box leaves the tensor.
                     const int rows = ln.hb > 0 ? ln.hb : 64;
                     const uint32_t bar = ptx::smem_u32(&m.ld[s]);
-                    for (int i = 0; i < 64; i += rows) {
+                    constexpr uint32_t kDst[5] = {C::kTQ, C::kTK, C::kTA, C::kTV, C::kTG};
+                    auto box = [&](int i, int x) {        // tile x, tile rows [i, i + rows)
                         int line, lp;
                         ln.place(c.p0, c.n, i < c.n ? i : 0, line, lp);
                         const int y = ln.fam ? line * p.H + hh : hh;
                         const int z = ln.fam ? bb * p.gh + lp : bb * p.L + line * p.gw + lp;
                         // a box starts inside its view; a packed group stays inside its line
+                        // (except in a forward row scan, whose positions are contiguous rows)
                         if (!GLA_CHECK(y >= 0 && y < (ln.fam ? p.gw * p.H : p.H) && z >= 0 &&
                                        z < (ln.fam ? p.B * p.gh : p.B * p.L) && lp >= 0 &&
-                                       (ln.hb == 0 || lp + rows <= ln.len)))
-                            continue;
-                        const uint32_t dst = sbase + s * C::kStage + (uint32_t)i * 128;
-                        constexpr uint32_t kDst[5] = {C::kTQ, C::kTK, C::kTA, C::kTV, C::kTG};
+                                       (ln.hb == 0 || ln.contig || lp + rows <= ln.len)))
+                            return;
+                        ptx::tma_load_3d(sbase + s * C::kStage + (uint32_t)i * 128 + kDst[x], &tmaps[x], 0, y, z, bar);
+                    };
+                    // one group per lane, its tiles in turn (measured at least as fast as one box
+                    // per lane, and faster when a chunk has more boxes than the warp has lanes)
+                    for (int i = lane * rows; i < 64; i += 32 * rows)
 #pragma unroll
                         for (int x = 0; x < 5; ++x)
-                            if (mask >> x & 1u) ptx::tma_load_3d(dst + kDst[x], &tmaps[x], 0, y, z, bar);
-                    }
+                            if (mask >> x & 1u) box(i, x);
                 }
                 last[s] = j;
             }

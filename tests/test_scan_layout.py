@@ -30,7 +30,17 @@ def test_layout_matches_the_oracle_scan_order(grid, chunk):
                                              ((8, 8), 16, 8)])
 def test_box_height(grid, chunk, rows):
     """Packed chunks where the line length has a power-of-two factor >= 8 in common with the
-    chunk length; 64-row boxes (line-aligned chunks) otherwise."""
+    chunk length; 64-row boxes (line-aligned chunks) otherwise (shown on R->L, which packs
+    within lines)."""
+    gh, gw = grid
+    assert gla.scan_layout(gh, gw, 1, chunk)[1] == rows
+
+
+@pytest.mark.parametrize("grid,chunk,rows", [((40, 40), 0, 64), ((24, 37), 0, 64), ((7, 5), 32, 32),
+                                             ((40, 40), 48, 16)])
+def test_forward_row_scans_load_whole_chunks(grid, chunk, rows):
+    """L->R visits token rows in memory order: a chunk is consecutive rows across lines, loaded
+    in boxes of the largest power of two dividing the chunk length."""
     gh, gw = grid
     assert gla.scan_layout(gh, gw, 0, chunk)[1] == rows
 
