@@ -110,3 +110,29 @@ def gla_forward(q, k, v, a, g, w, grid_h: int, grid_w: int, direction: int,
     if rc != 0:
         raise RuntimeError("gla_oracle_fwd failed with code %d" % rc)
     return (out, o) if return_o else out
+
+
+GATE_RANK = 16
+
+
+def gate_projection(x, w1, w2, b):
+    """Retention-gate pre-activation a = x W1 W2 + b, fp64.
+
+    GTR paper (arXiv 2609.26590), method section, GLA recurrence paragraph: the gate is
+    gamma_t = sigma(x_t W_alpha^(1) W_alpha^(2) + b_alpha)^(1/tau), a low-rank projection of
+    rank r = 16 "following GLA".  Reading taken here (the paragraph writes one head, d_k key
+    channels): as in GLA, one first factor W1 [d][r] is shared by the heads and the second factor
+    W2 [r][H d_k] maps to every head's key channels, with one bias per key channel.
+
+    x [T][d] (T tokens, d the model width), w1 [d][r], w2 [r][n], b [n]  ->  a [T][n], with
+    n = H d_k laid out head-major, i.e. exactly the gate_preact layout [B][L][H][d_k] of the
+    operator.  Two library matmuls in the paragraph's order; no reassociation.
+    """
+    x64 = np.asarray(x, dtype=np.float64)
+    w1_64 = np.asarray(w1, dtype=np.float64)
+    w2_64 = np.asarray(w2, dtype=np.float64)
+    b64 = np.asarray(b, dtype=np.float64)
+    if x64.ndim != 2 or w1_64.shape[0] != x64.shape[1] or w2_64.shape[0] != w1_64.shape[1] \
+            or b64.shape != (w2_64.shape[1],):
+        raise ValueError("gate_projection: shapes x [T][d], w1 [d][r], w2 [r][n], b [n] expected")
+    return (x64 @ w1_64) @ w2_64 + b64
