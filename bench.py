@@ -37,6 +37,20 @@ DIRECTIONS = (0, 1, 2, 3)
 L2_BYTES = 126 * 1024 * 1024
 FALLBACK_HBM_GBS = 6650.0
 PROFILE_TRAFFIC = os.path.join(ROOT, "profiles", "traffic.json")
+GATE_KERNEL = "gate projection (tcgen05)"
+GATE_RANK = 16
+
+
+def gate_shape(wl, d_model: int):
+    """(tokens, d_model, n_out) of the gate projection feeding the workload's operator."""
+    return wl.B * wl.L, d_model, wl.H * wl.d_k
+
+
+def gate_bytes(wl, d_model: int) -> int:
+    """Algorithmic HBM bytes of one projection: x read and a written once (fp16), the weights
+    (fp16) and bias (fp32) read once."""
+    T, d, n = gate_shape(wl, d_model)
+    return 2 * T * d + 2 * T * n + 2 * GATE_RANK * (d + n) + 4 * n
 
 
 def parse():
@@ -54,6 +68,12 @@ def parse():
     ap.add_argument("--workload", default=WORKLOAD,
                     help="synthetic workload to time (default: the 40x40 headline); the others "
                          "are reported with their own metric name")
+    ap.add_argument("--op", choices=["gla", "gate"], default="gla",
+                    help="gla: the operator (default); gate: the retention gate's low-rank "
+                         "projection a = x W1 W2 + b over the workload's tokens (B*L), its output "
+                         "width H*d_k, model width --d-model")
+    ap.add_argument("--d-model", type=int, default=384,
+                    help="with --op gate: the model width d (GTR-L: 384)")
     ap.add_argument("--record-traffic", metavar="NCU_CSV",
                     help="no bench: read an ncu CSV (dram__bytes_read.sum / dram__bytes_write.sum "
                          "of the kernel --kernel / --workload select) and print the traffic entry "
@@ -160,6 +180,21 @@ def record_traffic(args):
     import re
     from recurrent_vision_backbone_only_b200 import build as _b, gla, synth
     wl = synth.WORKLOADS[args.workload]
+    if getattr(args, "op", "gla") == "gate":
+        got = [v for k, v in read_ncu_csv(args.record_traffic) if re.search("gla_gate_kernel", k)]
+        got = [v for v in got if "dram__bytes_read.sum" in v and "dram__bytes_write.sum" in v]
+        if not got:
+            raise SystemExit("no gla_gate_kernel launch with dram bytes in %s" % args.record_traffic)
+        rd = statistics.mean(v["dram__bytes_read.sum"] for v in got)
+        wr = statistics.mean(v["dram__bytes_write.sum"] for v in got)
+        print(json.dumps({"workload": wl.name, "kernel": GATE_KERNEL,
+                          "lib_sources_digest": _b.sources_digest(), "launches": len(got),
+                          "launch_shapes": sorted({v.get("grid", "") for v in got}),
+                          "dram_read_bytes": rd, "dram_write_bytes": wr,
+                          "dram_bytes_per_launch": rd + wr,
+                          "algorithmic_bytes_per_launch": gate_bytes(wl, args.d_model),
+                          "command": args.ncu_command}))
+        return
     kid = {"auto": 0, "tc128": gla.KERNEL_TC128, "tc64": gla.KERNEL_TC64,
            "pipe64": gla.KERNEL_PIPE64, "simt": gla.KERNEL_SIMT}[args.kernel]
     symbol = {gla.KERNEL_TC128: "gla_tc_kernel", gla.KERNEL_TC64: "gla_chunk_kernel",
@@ -554,6 +589,150 @@ def run_ours(args, ws, rank, local):
     print(json.dumps(line), flush=True)
 
 
+def run_gate(args, ws, rank, local):
+    """Time gla_gate_proj (the retention gate's low-rank projection) on the workload's tokens."""
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+    from recurrent_vision_backbone_only_b200 import build as _b, gla, synth
+
+    _b.build()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    wl = synth.WORKLOADS[args.workload]
+    T, d, n = gate_shape(wl, args.d_model)
+    inp = synth.make_gate_inputs(T, d, n, seed=wl.seed)
+    w1, w2, b = (torch.from_numpy(inp[k]).to(dev) for k in ("w1", "w2", "b"))
+    set_bytes = 2 * T * (d + n)
+    n_sets = max(2 if set_bytes > L2_BYTES else 8, math.ceil(2 * L2_BYTES / set_bytes))
+    x0 = torch.from_numpy(inp["x"]).to(dev)
+    sets = [(x0.clone(), torch.empty((T, n), dtype=torch.float16, device=dev)) for _ in range(n_sets)]
+
+    def step(i):
+        xs, a = sets[i % n_sets]
+        gla.gate_proj(xs, w1, w2, b, a)
+
+    stream = torch.cuda.Stream(device=dev)
+    torch.cuda.synchronize()
+    with torch.cuda.stream(stream):
+        for i in range(args.warmup):
+            step(i)
+    if gla.get_status(stream) != 0:
+        raise RuntimeError("device status set during warm-up")
+    K = args.steps
+    G = min(K, 100)
+    with torch.cuda.stream(stream):
+        g_main = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g_main, stream=stream):
+            for i in range(G):
+                step(i)
+        g_rem = None
+        if K % G:
+            g_rem = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g_rem, stream=stream):
+                for i in range(K % G):
+                    step(i)
+        g_main.replay()
+        if g_rem is not None:
+            g_rem.replay()
+    torch.cuda.synchronize()
+    plan = [g_main] * (K // G) + ([g_rem] if g_rem is not None else [])
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if ws > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        with torch.cuda.stream(stream):
+            ev0.record(stream)
+            for gr in plan:
+                gr.replay()
+            ev1.record(stream)
+        torch.cuda.synchronize()
+    if ws > 1:
+        dist.barrier()
+    if gla.get_status(stream) != 0:
+        raise RuntimeError("device status set during the timed region")
+    max_ms = max_over_ranks(ev0.elapsed_time(ev1), dev)
+    value = job_throughput(T, K, ws, max_ms)
+    launch_s = max_ms / 1e3 / K
+    peak, peak_kind = measured_peaks()
+    achieved = gate_bytes(wl, d) / launch_s / 1e9
+
+    # e2e: x from pinned host memory, the projection, a back to pinned host memory
+    e2e_steps = max(1, min(args.e2e_steps, K))
+    hx = torch.from_numpy(inp["x"]).pin_memory()
+    ha = torch.empty((T, n), dtype=torch.float16).pin_memory()
+    xs, a = sets[0]
+    with torch.cuda.stream(stream):
+        xs.copy_(hx, non_blocking=True)
+        gla.gate_proj(xs, w1, w2, b, a)
+        ha.copy_(a, non_blocking=True)
+        if ws > 1:
+            dist.barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(e2e_steps):
+            xs.copy_(hx, non_blocking=True)
+            gla.gate_proj(xs, w1, w2, b, a)
+            ha.copy_(a, non_blocking=True)
+        e1.record(stream)
+    torch.cuda.synchronize()
+    if gla.get_status(stream) != 0:
+        raise RuntimeError("device status set during the e2e region")
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), dev)
+    if rank != 0:
+        return
+    line = {
+        "metric": "gate projection Mtokens/s (B·L), %s workload" % wl.name, "value": value,
+        "unit": "Mtokens/s", "n_gpus": ws, "steps": K, "warmup": args.warmup,
+        "ms_per_step": max_ms / K, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f16", "data": "synthetic",
+        "config": {
+            "workload": "%s tokens: a = x W1 W2 + b, tokens=%d (B=%d x %dx%d), d_model=%d, rank=%d, "
+                        "n_out=H*d_k=%d, fp16 I/O, fp32 accumulation; one step = 1 launch"
+                        % (wl.name, T, wl.B, wl.grid_h, wl.grid_w, d, GATE_RANK, n),
+            "tokens_per_step": T,
+            "l2": "rotating pool of %d x/a sets (%.0f MB > 126 MB L2); no flush kernel"
+                  % (n_sets, n_sets * set_bytes / 1e6),
+            "timing": "CUDA-graph replays (graphs of %d steps), CUDA events on the launch stream"
+                      % G,
+            "parallelism": "replicas" if ws > 1 else "single GPU",
+        },
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                     "frac": achieved / peak, "traffic": profile_traffic(wl.name, GATE_KERNEL),
+                     "peak_source": "%s (MEASURED_PEAKS.json hbm_gbs)" % peak_kind
+                     if peak_kind == "measured" else "fallback 6.65 TB/s",
+                     "bytes_per_launch": gate_bytes(wl, d), "launch_us": launch_s * 1e6},
+        "e2e": {"value": job_throughput(T, e2e_steps, ws, e2e_ms), "unit": "Mtokens/s",
+                "h2d_bytes_per_step": hx.numel() * 2, "d2h_bytes_per_step": ha.numel() * 2,
+                "steps": e2e_steps, "ms_per_step": e2e_ms / e2e_steps},
+        "gpu_launches": K,
+        "clocks": clk.summary(),
+    }
+    if ws == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_gate_sample(inp, args.cpu_seconds)
+    print(json.dumps(line), flush=True)
+
+
+def cpu_gate_sample(inp, budget_s: float):
+    """The oracle's gate projection (fp64) timed on the host over repeated whole-input calls
+    until about a tenth of the budget has passed."""
+    import oracle
+    x, w1, w2, b = (inp[k].astype("float64") for k in ("x", "w1", "w2", "b"))
+    t0 = time.perf_counter()
+    calls = 0
+    while True:
+        oracle.gate_projection(x, w1, w2, b)
+        calls += 1
+        el = time.perf_counter() - t0
+        if el >= budget_s / 10:
+            break
+    return {"value": calls * x.shape[0] / el / 1e6, "unit": "Mtokens/s",
+            "cores": os.cpu_count(), "kind": "oracle",
+            "sample": "%d whole-input calls of the fp64 oracle (numpy matmuls, %d tokens each)"
+                      % (calls, x.shape[0])}
+
+
 def main():
     args = parse()
     ws, rank, local = dist_env()
@@ -571,7 +750,7 @@ def main():
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=torch.device("cuda", local))
     try:
-        run_ours(args, ws, rank, local)
+        (run_gate if args.op == "gate" else run_ours)(args, ws, rank, local)
     finally:
         if ws > 1:
             import torch.distributed as dist

@@ -260,6 +260,24 @@ int gla_selftest_load(const void *q, const void *k, const void *gate_preact, con
                       int direction, int chunk, float *out, int *info, void *stream);
 
 /*
+ * gla_gate_proj -- the retention gate's pre-activation, the input gate_preact of gla_fwd:
+ *     a[t][c] = sum_j (sum_i x[t][i] w1[i][j]) w2[j][c] + bias[c]
+ * GTR paper's method section, GLA recurrence paragraph: gamma_t = sigma(x_t W_alpha^(1)
+ * W_alpha^(2) + b_alpha)^(1/tau), a low-rank projection of rank r = 16 "following GLA" -- read
+ * as GLA builds it: one first factor shared by the heads, a second factor onto every head's
+ * key channels.  x: [tokens][d_model] fp16 (token-major, tokens = B * L), w1: [d_model][rank]
+ * fp16, w2: [rank][n_out] fp16 (n_out = H * d_k, head-major), bias: [n_out] float32, a:
+ * [tokens][n_out] fp16 -- the [B][L][H][d_k] layout gla_fwd reads.  DEVICE pointers, 16-byte
+ * aligned, caller-owned; a must not overlap an input (GLA_ERR_ALIAS).  rank must be 16,
+ * d_model a multiple of 64 up to 1024, n_out a multiple of 128 up to 1024, else
+ * GLA_ERR_UNSUPPORTED.  tcgen05 tensor cores: x W1 with fp32 accumulation, that product split
+ * into fp16 high and low parts for the second factor, fp16 output.  Asynchronous on `stream`;
+ * an intermediate above the fp16 range latches GLA_ERR_RANGE.
+ */
+int gla_gate_proj(const void *x, const void *w1, const void *w2, const float *bias, void *a,
+                  int tokens, int d_model, int rank, int n_out, void *stream);
+
+/*
  * gla_scan_layout -- host-only (no device work, no CUDA call): the token each tile row of
  * each chunk holds when `kernel` (GLA_KERNEL_PIPE64 only) runs a scan of a
  * grid_h x grid_w grid in `direction` (0..3) with chunks of at most `chunk` positions

@@ -17,6 +17,7 @@
 #include "gla.h"
 #include "gla_chunk.cuh"
 #include "gla_pipe.cuh"
+#include "gla_gate.cuh"
 #include "gla_common.cuh"
 #include "gla_simt.cuh"
 #include "gla_tc.cuh"
@@ -856,6 +857,81 @@ int gla_selftest_chunk(int d, int kind, const float *A, const float *B, float *D
     };
     if (d == 64) return launch(ck::gla_chunk_selftest_kernel<64>, ck::Cfg<64>::kThreads, ck::smem_bytes<64>());
     return launch(ck::gla_chunk_selftest_kernel<128>, ck::Cfg<128>::kThreads, ck::smem_bytes<128>());
+}
+
+int gla_gate_proj(const void *x, const void *w1, const void *w2, const float *bias, void *a,
+                  int tokens, int d_model, int rank, int n_out, void *stream) {
+    if (!x || !w1 || !w2 || !bias || !a) return GLA_ERR_NULL;
+    if (tokens <= 0 || d_model <= 0 || n_out <= 0) return GLA_ERR_SHAPE;
+    if ((long long)tokens * std::max(d_model, n_out) > (1LL << 40)) return GLA_ERR_SHAPE;
+    if (rank != gla::gp::kRank || d_model % 64 != 0 || d_model > gla::gp::kMaxD ||
+        n_out % (int)gla::gp::kChunkN != 0 || n_out > gla::gp::kMaxN)
+        return GLA_ERR_UNSUPPORTED;
+    const void *const ptrs[5] = {x, w1, w2, bias, a};
+    for (const void *ptr : ptrs)
+        if (reinterpret_cast<uintptr_t>(ptr) & 15u) return GLA_ERR_UNSUPPORTED;
+    const uintptr_t ab = reinterpret_cast<uintptr_t>(a), ae = ab + (size_t)tokens * n_out * 2;
+    const size_t sizes[4] = {(size_t)tokens * d_model * 2, (size_t)d_model * rank * 2, (size_t)rank * n_out * 2,
+                             (size_t)n_out * 4};
+    for (int i = 0; i < 4; ++i) {
+        const uintptr_t pb = reinterpret_cast<uintptr_t>(ptrs[i]), pe = pb + sizes[i];
+        if (pb < ae && ab < pe) return GLA_ERR_ALIAS;
+    }
+    DeviceInfo di;
+    int rc = current_device_info(&di);
+    if (rc != GLA_OK) return rc;
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return GLA_ERR_CUDA;
+    // x [tokens][d_model] and a [tokens][n_out] as 3-D maps {width, 1, tokens}, boxes of 64
+    // channels x 128 tokens, 128-byte swizzle (the MMA operand / staging layout)
+    CUtensorMap xmap, amap;
+    const cuuint32_t box[3] = {64, 1, (cuuint32_t)gla::gp::kTileM};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    const struct { CUtensorMap *map; void *base; int width; } maps[2] = {
+        {&xmap, const_cast<void *>(x), d_model}, {&amap, a, n_out}};
+    for (const auto &mp : maps) {
+        const cuuint64_t dims[3] = {(cuuint64_t)mp.width, 1, (cuuint64_t)tokens};
+        const cuuint64_t strides[2] = {(cuuint64_t)mp.width * 2, (cuuint64_t)mp.width * 2};
+        if (fn(mp.map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3, mp.base, dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return GLA_ERR_CUDA;
+    }
+    const size_t smem = gla::gp::gate_smem_bytes();
+    if (smem > (size_t)di.max_smem_optin) return GLA_ERR_UNSUPPORTED;
+    if (cudaFuncSetAttribute(gla::gp::gla_gate_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+        cudaSuccess) {
+        cudaGetLastError();
+        return GLA_ERR_CUDA;
+    }
+    gla::gp::GateParams p;
+    p.w1 = static_cast<const __half *>(w1);
+    p.w2 = static_cast<const __half *>(w2);
+    p.b = bias;
+    p.T = tokens;
+    p.d = d_model;
+    p.n = n_out;
+    p.wait_limit = 1LL << 32;
+    // column groups: split each tile's output chunks only while tiles leave SMs idle
+    const int tiles = (tokens + gla::gp::kTileM - 1) / gla::gp::kTileM;
+    const int nchunks = n_out / (int)gla::gp::kChunkN;
+    p.groups = std::max(1, std::min(nchunks, di.sms / tiles));
+    const int items = tiles * p.groups;
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3((unsigned)std::min(items, di.sms), 1, 1);
+    cfg.blockDim = dim3(gla::gp::kThreads, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = static_cast<cudaStream_t>(stream);
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, gla::gp::gla_gate_kernel, xmap, amap, p) != cudaSuccess) {
+        cudaGetLastError();
+        return GLA_ERR_CUDA;
+    }
+    return GLA_OK;
 }
 
 int gla_scan_layout(int kernel, int grid_h, int grid_w, int direction, int chunk, int *spatial,

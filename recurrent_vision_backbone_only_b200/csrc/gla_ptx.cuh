@@ -100,6 +100,11 @@ __device__ __forceinline__ void cp_async16(uint32_t dst, const void *src, uint32
                  : "memory");
 }
 
+// Wait for all of this thread's cp.async copies.
+__device__ __forceinline__ void cp_async_wait_all() {
+    asm volatile("cp.async.wait_all;" ::: "memory");
+}
+
 // ------------------------------------------------------------------- cluster
 // Split cluster barrier.  Arrive without release semantics: for a start-up barrier whose only payload is mbarrier
 // initialisation already published by fence.mbarrier_init.release.cluster.
@@ -407,17 +412,6 @@ __host__ __device__ constexpr uint32_t idesc_ab(uint32_t a_fmt, uint32_t b_fmt, 
 }
 
 // ----------------------------------------------------------------------- TMA
-// Four rows of a 2-D tensor map (rows r0..r3, inner coordinate x) into 4 consecutive
-// shared-memory rows at dst, completing `bytes` on the mbarrier (tile::gather4; the map's box is
-// one row high).  The swizzle of the map applies to the destination rows.
-__device__ __forceinline__ void tma_gather4(uint32_t dst, const void *tmap, int x, int r0, int r1,
-                                            int r2, int r3, uint32_t bar) {
-    asm volatile(
-        "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
-        " [%0], [%1, {%2, %3, %4, %5, %6}], [%7];" ::"r"(dst),
-        "l"(tmap), "r"(x), "r"(r0), "r"(r1), "r"(r2), "r"(r3), "r"(bar)
-        : "memory");
-}
 // Box of a 3-D tensor map at coordinates (x, y, z) into shared memory at dst (tile mode),
 // completing its bytes on the mbarrier.  Elements outside the tensor are filled with zeros.
 __device__ __forceinline__ void tma_load_3d(uint32_t dst, const void *tmap, int x, int y, int z, uint32_t bar) {
@@ -426,6 +420,25 @@ __device__ __forceinline__ void tma_load_3d(uint32_t dst, const void *tmap, int 
         " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(dst),
         "l"(tmap), "r"(x), "r"(y), "r"(z), "r"(bar)
         : "memory");
+}
+// Box of shared memory at src into a 3-D tensor map at (x, y, z) (tile mode), tracked in this
+// thread's bulk async-group; rows outside the tensor are not written.
+__device__ __forceinline__ void tma_store_3d(const void *tmap, uint32_t src, int x, int y, int z) {
+    asm volatile("cp.async.bulk.tensor.3d.global.shared::cta.tile.bulk_group [%0, {%2, %3, %4}], [%1];"
+                 ::"l"(tmap), "r"(src), "r"(x), "r"(y), "r"(z)
+                 : "memory");
+}
+__device__ __forceinline__ void bulk_commit_group() {
+    asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+// Wait until at most N of this thread's bulk groups still read their shared-memory source.
+template <int N>
+__device__ __forceinline__ void bulk_wait_group_read() {
+    asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory");
+}
+// Wait until all of this thread's bulk groups have completed (writes performed).
+__device__ __forceinline__ void bulk_wait_group_all() {
+    asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
 }
 __device__ __forceinline__ void prefetch_tmap(const void *tmap) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(tmap) : "memory");

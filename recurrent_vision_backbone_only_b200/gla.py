@@ -71,6 +71,8 @@ def load() -> ctypes.CDLL:
         lib.gla_selftest_load.restype = ctypes.c_int
         lib.gla_scan_layout.argtypes = [i] * 5 + [vp, vp]
         lib.gla_scan_layout.restype = ctypes.c_int
+        lib.gla_gate_proj.argtypes = [vp] * 5 + [i] * 4 + [vp]
+        lib.gla_gate_proj.restype = ctypes.c_int
         lib.gla_selftest_fault.argtypes = [vp] * 7 + [i] * 7 + [ll, i, i, vp]
         lib.gla_selftest_rcp.argtypes = [vp, vp, i, vp]
         lib.gla_selftest_rcp.restype = ctypes.c_int
@@ -215,6 +217,28 @@ def scan_layout(grid_h: int, grid_w: int, direction: int, chunk: int = 0,
     _check(load().gla_scan_layout(kernel, grid_h, grid_w, direction, chunk, buf, ctypes.byref(rows)),
            "gla_scan_layout")
     return list(buf), rows.value
+
+
+def gate_proj(x, w1, w2, bias, a, stream=None):
+    """a = x W1 W2 + bias (the retention gate's pre-activation, gla_fwd's gate_preact).
+
+    x [tokens, d_model] fp16, w1 [d_model, 16] fp16, w2 [16, n_out] fp16, bias [n_out] fp32,
+    a [tokens, n_out] fp16; CUDA tensors, contiguous.  Any leading dims of x / a are tokens."""
+    import torch
+    tokens = x.numel() // x.shape[-1] if x.dim() else 0
+    d_model, rank, n_out = x.shape[-1], w1.shape[-1], w2.shape[-1]
+    for t, dt, shape in ((x, torch.float16, None), (w1, torch.float16, (d_model, rank)),
+                         (w2, torch.float16, (rank, n_out)), (bias, torch.float32, (n_out,)),
+                         (a, torch.float16, None)):
+        if not (t.is_cuda and t.is_contiguous() and t.dtype == dt):
+            raise ValueError("gate_proj: contiguous CUDA tensors of the documented dtypes expected")
+        if shape is not None and tuple(t.shape) != shape:
+            raise ValueError("gate_proj: shape %s expected, got %s" % (shape, tuple(t.shape)))
+    if a.numel() != tokens * n_out or a.shape[-1] != n_out:
+        raise ValueError("gate_proj: a must hold [tokens, n_out]")
+    _check(load().gla_gate_proj(*[ctypes.c_void_p(t.data_ptr()) for t in (x, w1, w2, bias, a)],
+                                tokens, d_model, rank, n_out, _stream_ptr(stream)), "gla_gate_proj")
+    return a
 
 
 def empty_launch(B: int, H: int, grid_h: int, grid_w: int, stream=None):

@@ -108,3 +108,26 @@ def make_inputs(wl: Workload, seed: int | None = None) -> Dict[str, np.ndarray]:
     w = (np.float32(1.0) + np.float32(wl.w_std) *
          rng.standard_normal(size=(dv,), dtype=np.float32)).astype(np.float32)
     return {"q": q, "k": k, "v": v, "a": a, "g": g, "w": w}
+
+
+def make_gate_inputs(tokens: int, d_model: int, n_out: int, rank: int = 16, seed: int = 0,
+                     x_std: float = 1.0, b_mean: float = 2.0, b_std: float = 0.5) -> Dict[str, np.ndarray]:
+    """Draw the retention gate's projection inputs: x [tokens][d_model], w1 [d_model][rank],
+    w2 [rank][n_out] (fp16) and b [n_out] (fp32).
+
+    x is the block's normalised input, N(0, x_std); w1 ~ N(0, 1/d_model) and w2 ~ N(0, 1/rank)
+    keep the product near unit scale, and b ~ N(b_mean, b_std) puts the pre-activation where the
+    recurrence workloads draw it (mean 2: per-step retention sigma(2)^(1/16) ~ 0.992).  Draw
+    order: x, w1, w2, b.
+    """
+    rng = np.random.Generator(np.random.PCG64(seed))
+
+    def normal(shape, mean, std, dt):
+        x = rng.standard_normal(size=shape, dtype=np.float32)
+        return (x * np.float32(std) + np.float32(mean)).astype(dt)
+
+    x = normal((tokens, d_model), 0.0, x_std, np.float16)
+    w1 = normal((d_model, rank), 0.0, d_model ** -0.5, np.float16)
+    w2 = normal((rank, n_out), 0.0, rank ** -0.5, np.float16)
+    b = normal((n_out,), b_mean, b_std, np.float32)
+    return {"x": x, "w1": w1, "w2": w2, "b": b}

@@ -164,3 +164,26 @@ def test_host_entry_checks_every_tensor_before_any_call(bad):
         t["v"] = torch.zeros(B, L, H, d, dtype=torch.float16)[..., : d // 2]   # not contiguous
     with pytest.raises(ValueError):
         gla.gla_fwd_host(t["q"], t["k"], t["v"], t["a"], t["g"], w, t["out"], gh, gw, 0)
+
+
+def test_gate_projection_argument_errors(lib):
+    def gate(ptrs=ALIGNED[:5], T=128, d=128, r=16, n=128):
+        args = [ctypes.c_void_p(p) if p is not None else None for p in ptrs]
+        return gla.raw_call("gla_gate_proj", *args, T, d, r, n, None)
+    for i in range(5):
+        ptrs = list(ALIGNED[:5])
+        ptrs[i] = None
+        assert gate(ptrs) == 1                             # GLA_ERR_NULL
+    for kw in (dict(T=0), dict(d=-64), dict(n=0), dict(T=(1 << 31) - 1, d=1024)):
+        assert gate(**kw) == 2                             # GLA_ERR_SHAPE
+    for kw in (dict(r=8), dict(r=32), dict(d=96), dict(d=2048), dict(n=64), dict(n=2048)):
+        assert gate(**kw) == 3                             # GLA_ERR_UNSUPPORTED
+    mis = list(ALIGNED[:5])
+    mis[1] += 4
+    assert gate(mis) == 3                                  # misaligned w1
+    alias = list(ALIGNED[:5])
+    alias[4] = alias[0] + 64                               # a overlaps x
+    assert gate(alias) == 5                                # GLA_ERR_ALIAS
+    import torch
+    if not torch.cuda.is_available():
+        assert gate() == 9                                 # GLA_ERR_NO_DEVICE, nothing faked

@@ -91,3 +91,24 @@ def test_ncu_csv_reader_and_traffic_entry(tmp_path, capsys):
     # a call = one launch of each grid shape: (206.02 + 29.07) + (50 + 10) MB
     assert e["dram_bytes_per_launch"] == pytest.approx(295.09e6)
     assert e["launches"] == 3 and len(e["launch_shapes"]) == 2
+
+
+def test_gate_bytes_and_traffic_entry(tmp_path, capsys):
+    from recurrent_vision_backbone_only_b200 import synth
+    wl = synth.WORKLOADS["batched"]
+    assert bench.gate_shape(wl, 384) == (16 * 1600, 384, 12 * 64)
+    # x read once, a written once (fp16), W1 / W2 (fp16) and b (fp32) read once
+    assert bench.gate_bytes(wl, 384) == 25600 * 384 * 2 + 25600 * 768 * 2 + 16 * 384 * 2 \
+        + 16 * 768 * 2 + 768 * 4
+    csv = NCU_DETAILS.replace("void gla::ck::gla_pipe_kernel(Maps, Params)",
+                              "void gla::gp::gla_gate_kernel(CUtensorMap_st, GateParams)")
+    p = tmp_path / "g.csv"
+    p.write_text(csv)
+    args = bench.argparse.Namespace(record_traffic=str(p), workload="batched", kernel="auto",
+                                    op="gate", d_model=384, ncu_command="ncu ...")
+    bench.record_traffic(args)
+    e = json.loads(capsys.readouterr().out)
+    assert e["kernel"] == bench.GATE_KERNEL and e["launches"] == 3
+    # one launch per call: the mean over launches
+    assert e["dram_bytes_per_launch"] == pytest.approx((2 * 235.09e6 + 60e6) / 3)
+    assert e["algorithmic_bytes_per_launch"] == bench.gate_bytes(wl, 384)

@@ -4,7 +4,8 @@ Every computed index that addresses memory -- gathered and stored token rows, TM
 coordinates, remote exchange rows, chunk geometry -- is checked before use in that build, and
 a violation latches GLA_ERR_CHECK instead of touching memory.  These cases run every kernel
 over the shapes whose index arithmetic differs (ragged and packed grids, reversed and cycling
-directions, 1 to 16 segments, a partial-wave split, d = 32 / 64 / 128, fp16 and fp32) and
+directions, 1 to 16 segments, a partial-wave split, d = 32 / 64 / 128, fp16 and fp32, and the
+gate projection's ragged tiles and column groups) and
 require that no check fires and that the results still match the oracle.  This stands in for
 a device memory checker, which cannot run on this hardware.
 """
@@ -93,3 +94,17 @@ def test_fp32_cuda_cores():
     for direction in (0, 3, 4):
         u = run_checked(x, 12, 9, direction, 0)
         check(u, x, 12, 9, direction, "f32")
+
+
+@pytest.mark.parametrize("T,d,n", [(300, 64, 128), (1600, 384, 384), (5000, 128, 640), (40000, 128, 256)])
+def test_gate_projection(T, d, n):
+    import torch
+    inp = synth.make_gate_inputs(T, d, n, seed=T)
+    t = [torch.from_numpy(np.ascontiguousarray(inp[k])).cuda() for k in ("x", "w1", "w2", "b")]
+    a = torch.empty((T, n), dtype=torch.float16, device="cuda")
+    gla.gate_proj(*t, a)
+    status = gla.get_status()
+    assert status == 0, gla.status_string(status)
+    ref = oracle.gate_projection(*(inp[k].astype(np.float64) for k in ("x", "w1", "w2", "b")))
+    d_ = a.cpu().numpy().astype(np.float64) - ref
+    assert np.max(np.abs(d_)) <= 1e-2 and np.linalg.norm(d_) <= 2e-3 * np.linalg.norm(ref)
