@@ -897,8 +897,9 @@ int gla_gate_proj(const void *x, const void *w1, const void *w2, const float *bi
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
             return GLA_ERR_CUDA;
     }
-    const size_t smem = gla::gp::gate_smem_bytes();
-    if (smem > (size_t)di.max_smem_optin) return GLA_ERR_UNSUPPORTED;
+    const gla::gp::GateLayout lay = gla::gp::gate_layout(d_model, n_out, (size_t)di.max_smem_optin);
+    if (lay.stages < 3) return GLA_ERR_UNSUPPORTED;
+    const size_t smem = lay.bytes;
     if (cudaFuncSetAttribute(gla::gp::gla_gate_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
         cudaSuccess) {
         cudaGetLastError();
@@ -911,14 +912,13 @@ int gla_gate_proj(const void *x, const void *w1, const void *w2, const float *bi
     p.T = tokens;
     p.d = d_model;
     p.n = n_out;
+    p.lay = lay;
     p.wait_limit = 1LL << 32;
-    // column groups: split each tile's output chunks only while tiles leave SMs idle
-    const int tiles = (tokens + gla::gp::kTileM - 1) / gla::gp::kTileM;
-    const int nchunks = n_out / (int)gla::gp::kChunkN;
-    p.groups = std::max(1, std::min(nchunks, di.sms / tiles));
-    const int items = tiles * p.groups;
+    // one CTA per SM, each taking an equal contiguous range of the (tile, output chunk) units
+    const long long units = (long long)((tokens + gla::gp::kTileM - 1) / gla::gp::kTileM) *
+                            (n_out / (int)gla::gp::kChunkN);
     cudaLaunchConfig_t cfg{};
-    cfg.gridDim = dim3((unsigned)std::min(items, di.sms), 1, 1);
+    cfg.gridDim = dim3((unsigned)std::min<long long>(units, di.sms), 1, 1);
     cfg.blockDim = dim3(gla::gp::kThreads, 1, 1);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = static_cast<cudaStream_t>(stream);

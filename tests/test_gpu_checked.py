@@ -5,7 +5,7 @@ coordinates, remote exchange rows, chunk geometry -- is checked before use in th
 a violation latches GLA_ERR_CHECK instead of touching memory.  These cases run every kernel
 over the shapes whose index arithmetic differs (ragged and packed grids, reversed and cycling
 directions, 1 to 16 segments, a partial-wave split, d = 32 / 64 / 128, fp16 and fp32, and the
-gate projection's ragged tiles and column groups) and
+gate projection's ragged tiles and split unit ranges) and
 require that no check fires and that the results still match the oracle.  This stands in for
 a device memory checker, which cannot run on this hardware.
 """

@@ -45,8 +45,9 @@ def check(a, inp):
     assert np.linalg.norm(d) <= 2e-3 * np.linalg.norm(ref)
 
 
-# Tiles are split into column groups while they leave SMs idle (148 SMs): 1600 tokens = 13
-# tiles x 3 groups, 129 tokens = 2 tiles x 8 groups, 6400 tokens = 50 tiles x 2 groups.
+# Each CTA takes a contiguous range of the (128-token tile, 128-column chunk) units: ranges
+# start and end inside tiles, and short inputs give one unit per CTA (1600 tokens: 13 tiles x 3
+# chunks = 39 CTAs; 129 tokens: 2 x 8 = 16 CTAs).
 @pytest.mark.parametrize("T,d,n", [
     (1600, 384, 384),        # GTR-L at 640 px: 40x40 tokens, width 384, 6 heads of 64
     (300, 64, 128),          # ragged last tile (300 = 2 x 128 + 44)
@@ -54,7 +55,7 @@ def check(a, inp):
     (127, 192, 256),
     (129, 1024, 1024),       # widest model and output
     (6400, 192, 256),
-    (5000, 128, 640),        # 40 tiles in 3 column groups of 2, 2 and 1 output chunks
+    (5000, 128, 640),        # 40 tiles x 5 chunks over 148 CTAs: ranges of 1 or 2 units
 ])
 def test_gate_matches_oracle(T, d, n):
     inp = synth.make_gate_inputs(T, d, n, seed=T + d + n)
@@ -64,8 +65,8 @@ def test_gate_matches_oracle(T, d, n):
 
 
 def test_more_tiles_than_sms():
-    # persistent CTAs loop over tiles: 40,000 tokens = 313 tiles on at most 148 CTAs, with the
-    # X ring wrapping many times and both TMEM output buffers reused
+    # 40,000 tokens = 313 tiles x 3 chunks on 148 CTAs: ranges of 6 or 7 units over 3 or 4
+    # tiles each, the X ring wrapping many times and both TMEM output buffers reused
     inp = synth.make_gate_inputs(40000, 128, 384, seed=5)
     a, status = run_gate(inp["x"], inp["w1"], inp["w2"], inp["b"])
     assert status == 0, gla.status_string(status)
