@@ -136,3 +136,40 @@ def gate_projection(x, w1, w2, b):
             or b64.shape != (w2_64.shape[1],):
         raise ValueError("gate_projection: shapes x [T][d], w1 [d][r], w2 [r][n], b [n] expected")
     return (x64 @ w1_64) @ w2_64 + b64
+
+
+SSWIGLU_KERNEL = 3
+
+
+def spatial_swiglu_mix(value, gate, conv_w, conv_b, grid_h, grid_w):
+    """Spatial SwiGLU's token mixing step, fp64: h = SiLU(gate) * (DWConv3x3(value) + conv_b).
+
+    GTR paper (arXiv 2609.26590), method section, Spatial SwiGLU paragraph: the value branch is
+    reshaped to the 2-D patch grid, passed through a 3x3 depthwise convolution and restored to
+    sequence order; the gating branch stays tokenwise.  The block's equation itself is missing
+    from the text; reading taken: SwiGLU's SiLU-activated gating branch multiplies the
+    convolved value branch, the convolution being a framework depthwise Conv2d (per-channel
+    3x3 cross-correlation, zero padding of one token, one bias per channel).
+
+    value, gate [B][L][C] with L = grid_h * grid_w row-major (s = y * grid_w + x),
+    conv_w [C][3][3], conv_b [C]  ->  h [B][L][C].  The nine taps are summed in the order
+    (dy, dx) = (-1,-1), (-1,0), ..., (1,1) over a zero-padded copy of the grid.
+    """
+    v = np.asarray(value, dtype=np.float64)
+    g = np.asarray(gate, dtype=np.float64)
+    w = np.asarray(conv_w, dtype=np.float64)
+    b = np.asarray(conv_b, dtype=np.float64)
+    if v.ndim != 3 or g.shape != v.shape or v.shape[1] != grid_h * grid_w:
+        raise ValueError("spatial_swiglu_mix: value, gate [B][grid_h*grid_w][C] expected")
+    B, L, C = v.shape
+    if w.shape != (C, SSWIGLU_KERNEL, SSWIGLU_KERNEL) or b.shape != (C,):
+        raise ValueError("spatial_swiglu_mix: conv_w [C][3][3], conv_b [C] expected")
+    grid = v.reshape(B, grid_h, grid_w, C)
+    padded = np.zeros((B, grid_h + 2, grid_w + 2, C), dtype=np.float64)
+    padded[:, 1:grid_h + 1, 1:grid_w + 1, :] = grid
+    conv = np.broadcast_to(b, (B, grid_h, grid_w, C)).copy()
+    for dy in (-1, 0, 1):
+        for dx in (-1, 0, 1):
+            conv += w[:, dy + 1, dx + 1] * padded[:, 1 + dy:1 + dy + grid_h, 1 + dx:1 + dx + grid_w, :]
+    silu = g / (1.0 + np.exp(-g))
+    return silu * conv.reshape(B, L, C)
