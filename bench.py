@@ -39,11 +39,20 @@ FALLBACK_HBM_GBS = 6650.0
 PROFILE_TRAFFIC = os.path.join(ROOT, "profiles", "traffic.json")
 GATE_KERNEL = "gate projection (tcgen05)"
 GATE_RANK = 16
+SSWIGLU_KERNEL = "spatial swiglu mix"
+SSWIGLU_EXPANSION = 4
 
 
 def gate_shape(wl, d_model: int):
     """(tokens, d_model, n_out) of the gate projection feeding the workload's operator."""
     return wl.B * wl.L, d_model, wl.H * wl.d_k
+
+
+def sswiglu_bytes(wl, d_model: int) -> int:
+    """Algorithmic HBM bytes of one Spatial SwiGLU mixing step: value and gate read and h
+    written once (fp16), the taps and bias (fp32) read once."""
+    C = SSWIGLU_EXPANSION * d_model
+    return 3 * 2 * wl.B * wl.L * C + 4 * 10 * C
 
 
 def gate_bytes(wl, d_model: int) -> int:
@@ -68,12 +77,13 @@ def parse():
     ap.add_argument("--workload", default=WORKLOAD,
                     help="synthetic workload to time (default: the 40x40 headline); the others "
                          "are reported with their own metric name")
-    ap.add_argument("--op", choices=["gla", "gate"], default="gla",
+    ap.add_argument("--op", choices=["gla", "gate", "sswiglu"], default="gla",
                     help="gla: the operator (default); gate: the retention gate's low-rank "
                          "projection a = x W1 W2 + b over the workload's tokens (B*L), its output "
-                         "width H*d_k, model width --d-model")
+                         "width H*d_k, model width --d-model; sswiglu: Spatial SwiGLU's "
+                         "dwconv + gating step on the workload's grid, 4 x d_model channels")
     ap.add_argument("--d-model", type=int, default=384,
-                    help="with --op gate: the model width d (GTR-L: 384)")
+                    help="with --op gate / sswiglu: the model width d (GTR-L: 384)")
     ap.add_argument("--record-traffic", metavar="NCU_CSV",
                     help="no bench: read an ncu CSV (dram__bytes_read.sum / dram__bytes_write.sum "
                          "of the kernel --kernel / --workload select) and print the traffic entry "
@@ -180,19 +190,22 @@ def record_traffic(args):
     import re
     from recurrent_vision_backbone_only_b200 import build as _b, gla, synth
     wl = synth.WORKLOADS[args.workload]
-    if getattr(args, "op", "gla") == "gate":
-        got = [v for k, v in read_ncu_csv(args.record_traffic) if re.search("gla_gate_kernel", k)]
+    op = getattr(args, "op", "gla")
+    if op in ("gate", "sswiglu"):
+        symbol, kname, alg = {"gate": ("gla_gate_kernel", GATE_KERNEL, gate_bytes),
+                              "sswiglu": ("gla_sswiglu_kernel", SSWIGLU_KERNEL, sswiglu_bytes)}[op]
+        got = [v for k, v in read_ncu_csv(args.record_traffic) if re.search(symbol, k)]
         got = [v for v in got if "dram__bytes_read.sum" in v and "dram__bytes_write.sum" in v]
         if not got:
-            raise SystemExit("no gla_gate_kernel launch with dram bytes in %s" % args.record_traffic)
+            raise SystemExit("no %s launch with dram bytes in %s" % (symbol, args.record_traffic))
         rd = statistics.mean(v["dram__bytes_read.sum"] for v in got)
         wr = statistics.mean(v["dram__bytes_write.sum"] for v in got)
-        print(json.dumps({"workload": wl.name, "kernel": GATE_KERNEL,
+        print(json.dumps({"workload": wl.name, "kernel": kname,
                           "lib_sources_digest": _b.sources_digest(), "launches": len(got),
                           "launch_shapes": sorted({v.get("grid", "") for v in got}),
                           "dram_read_bytes": rd, "dram_write_bytes": wr,
                           "dram_bytes_per_launch": rd + wr,
-                          "algorithmic_bytes_per_launch": gate_bytes(wl, args.d_model),
+                          "algorithmic_bytes_per_launch": alg(wl, args.d_model),
                           "command": args.ncu_command}))
         return
     kid = {"auto": 0, "tc128": gla.KERNEL_TC128, "tc64": gla.KERNEL_TC64,
@@ -589,9 +602,88 @@ def run_ours(args, ws, rank, local):
     print(json.dumps(line), flush=True)
 
 
-def run_gate(args, ws, rank, local):
-    """Time gla_gate_proj (the retention gate's low-rank projection) on the workload's tokens."""
-    import numpy as np
+class AuxOp:
+    """One of the steps next to the operator, timed like it: `step(i)` launches on the current
+    stream with device-resident input set i mod the pool, `e2e_step()` copies a host input
+    set in, launches, and copies the result out."""
+
+    def __init__(self, **kw):
+        self.__dict__.update(kw)
+
+
+def gate_op(args, wl, dev):
+    """gla_gate_proj (the retention gate's low-rank projection) on the workload's tokens."""
+    import torch
+    from recurrent_vision_backbone_only_b200 import gla, synth
+    T, d, n = gate_shape(wl, args.d_model)
+    inp = synth.make_gate_inputs(T, d, n, seed=wl.seed)
+    w1, w2, b = (torch.from_numpy(inp[k]).to(dev) for k in ("w1", "w2", "b"))
+    set_bytes = 2 * T * (d + n)
+    n_sets = max(2 if set_bytes > L2_BYTES else 8, math.ceil(2 * L2_BYTES / set_bytes))
+    x0 = torch.from_numpy(inp["x"]).to(dev)
+    sets = [(x0.clone(), torch.empty((T, n), dtype=torch.float16, device=dev)) for _ in range(n_sets)]
+    hx = torch.from_numpy(inp["x"]).pin_memory()
+    ha = torch.empty((T, n), dtype=torch.float16).pin_memory()
+
+    def step(i):
+        xs, a = sets[i % n_sets]
+        gla.gate_proj(xs, w1, w2, b, a)
+
+    def e2e_step():
+        xs, a = sets[0]
+        xs.copy_(hx, non_blocking=True)
+        gla.gate_proj(xs, w1, w2, b, a)
+        ha.copy_(a, non_blocking=True)
+
+    return AuxOp(
+        name="gate", kernel=GATE_KERNEL, tokens=T, bytes_per_launch=gate_bytes(wl, d), step=step,
+        e2e_step=e2e_step, h2d=hx.numel() * 2, d2h=ha.numel() * 2, n_sets=n_sets, set_bytes=set_bytes,
+        metric="gate projection Mtokens/s (B·L), %s workload" % wl.name,
+        workload="%s tokens: a = x W1 W2 + b, tokens=%d (B=%d x %dx%d), d_model=%d, rank=%d, "
+                 "n_out=H*d_k=%d, fp16 I/O, fp32 accumulation; one step = 1 launch"
+                 % (wl.name, T, wl.B, wl.grid_h, wl.grid_w, d, GATE_RANK, n),
+        cpu=lambda budget: cpu_gate_sample(inp, budget))
+
+
+def sswiglu_op(args, wl, dev):
+    """gla_sswiglu (Spatial SwiGLU's dwconv + gating step) on the workload's grid, with
+    channels = expansion 4 x the model width."""
+    import torch
+    from recurrent_vision_backbone_only_b200 import gla, synth
+    B, gh, gw, C = wl.B, wl.grid_h, wl.grid_w, SSWIGLU_EXPANSION * args.d_model
+    inp = synth.make_sswiglu_inputs(B, gh, gw, C, seed=wl.seed)
+    cw, cb = (torch.from_numpy(inp[k]).to(dev) for k in ("conv_w", "conv_b"))
+    set_bytes = 3 * B * gh * gw * C * 2
+    n_sets = max(2 if set_bytes > L2_BYTES else 8, math.ceil(2 * L2_BYTES / set_bytes))
+    v0, g0 = (torch.from_numpy(inp[k]).to(dev) for k in ("value", "gate"))
+    sets = [(v0.clone(), g0.clone(), torch.empty_like(v0)) for _ in range(n_sets)]
+    hv, hg = (torch.from_numpy(inp[k]).pin_memory() for k in ("value", "gate"))
+    hh = torch.empty(tuple(hv.shape), dtype=torch.float16).pin_memory()
+
+    def step(i):
+        v, g, h = sets[i % n_sets]
+        gla.sswiglu(v, g, cw, cb, h, gh, gw)
+
+    def e2e_step():
+        v, g, h = sets[0]
+        v.copy_(hv, non_blocking=True)
+        g.copy_(hg, non_blocking=True)
+        gla.sswiglu(v, g, cw, cb, h, gh, gw)
+        hh.copy_(h, non_blocking=True)
+
+    return AuxOp(
+        name="sswiglu", kernel=SSWIGLU_KERNEL, tokens=B * gh * gw, bytes_per_launch=sswiglu_bytes(wl, args.d_model),
+        step=step, e2e_step=e2e_step, h2d=2 * hv.numel() * 2, d2h=hh.numel() * 2, n_sets=n_sets,
+        set_bytes=set_bytes,
+        metric="Spatial SwiGLU mix Mtokens/s (B·L), %s workload" % wl.name,
+        workload="%s grid: h = SiLU(gate) * (DWConv3x3(value) + b), B=%d, %dx%d, channels=%d "
+                 "(expansion %d x d_model %d), fp16 I/O, fp32 arithmetic; one step = 1 launch"
+                 % (wl.name, B, gh, gw, C, SSWIGLU_EXPANSION, args.d_model),
+        cpu=lambda budget: cpu_sswiglu_sample(inp, gh, gw, budget))
+
+
+def run_aux(args, ws, rank, local):
+    """Time one of the steps next to the operator (--op gate / sswiglu) like the operator."""
     import torch
     import torch.distributed as dist
     from recurrent_vision_backbone_only_b200 import build as _b, gla, synth
@@ -600,23 +692,13 @@ def run_gate(args, ws, rank, local):
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
     wl = synth.WORKLOADS[args.workload]
-    T, d, n = gate_shape(wl, args.d_model)
-    inp = synth.make_gate_inputs(T, d, n, seed=wl.seed)
-    w1, w2, b = (torch.from_numpy(inp[k]).to(dev) for k in ("w1", "w2", "b"))
-    set_bytes = 2 * T * (d + n)
-    n_sets = max(2 if set_bytes > L2_BYTES else 8, math.ceil(2 * L2_BYTES / set_bytes))
-    x0 = torch.from_numpy(inp["x"]).to(dev)
-    sets = [(x0.clone(), torch.empty((T, n), dtype=torch.float16, device=dev)) for _ in range(n_sets)]
-
-    def step(i):
-        xs, a = sets[i % n_sets]
-        gla.gate_proj(xs, w1, w2, b, a)
+    op = {"gate": gate_op, "sswiglu": sswiglu_op}[args.op](args, wl, dev)
 
     stream = torch.cuda.Stream(device=dev)
     torch.cuda.synchronize()
     with torch.cuda.stream(stream):
         for i in range(args.warmup):
-            step(i)
+            op.step(i)
     if gla.get_status(stream) != 0:
         raise RuntimeError("device status set during warm-up")
     K = args.steps
@@ -625,13 +707,13 @@ def run_gate(args, ws, rank, local):
         g_main = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g_main, stream=stream):
             for i in range(G):
-                step(i)
+                op.step(i)
         g_rem = None
         if K % G:
             g_rem = torch.cuda.CUDAGraph()
             with torch.cuda.graph(g_rem, stream=stream):
                 for i in range(K % G):
-                    step(i)
+                    op.step(i)
         g_main.replay()
         if g_rem is not None:
             g_rem.replay()
@@ -653,28 +735,21 @@ def run_gate(args, ws, rank, local):
     if gla.get_status(stream) != 0:
         raise RuntimeError("device status set during the timed region")
     max_ms = max_over_ranks(ev0.elapsed_time(ev1), dev)
-    value = job_throughput(T, K, ws, max_ms)
+    value = job_throughput(op.tokens, K, ws, max_ms)
     launch_s = max_ms / 1e3 / K
     peak, peak_kind = measured_peaks()
-    achieved = gate_bytes(wl, d) / launch_s / 1e9
+    achieved = op.bytes_per_launch / launch_s / 1e9
 
-    # e2e: x from pinned host memory, the projection, a back to pinned host memory
+    # e2e: inputs from pinned host memory, the launch, the result back to pinned host memory
     e2e_steps = max(1, min(args.e2e_steps, K))
-    hx = torch.from_numpy(inp["x"]).pin_memory()
-    ha = torch.empty((T, n), dtype=torch.float16).pin_memory()
-    xs, a = sets[0]
     with torch.cuda.stream(stream):
-        xs.copy_(hx, non_blocking=True)
-        gla.gate_proj(xs, w1, w2, b, a)
-        ha.copy_(a, non_blocking=True)
+        op.e2e_step()
         if ws > 1:
             dist.barrier()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(stream)
         for _ in range(e2e_steps):
-            xs.copy_(hx, non_blocking=True)
-            gla.gate_proj(xs, w1, w2, b, a)
-            ha.copy_(a, non_blocking=True)
+            op.e2e_step()
         e1.record(stream)
     torch.cuda.synchronize()
     if gla.get_status(stream) != 0:
@@ -683,34 +758,32 @@ def run_gate(args, ws, rank, local):
     if rank != 0:
         return
     line = {
-        "metric": "gate projection Mtokens/s (B·L), %s workload" % wl.name, "value": value,
+        "metric": op.metric, "value": value,
         "unit": "Mtokens/s", "n_gpus": ws, "steps": K, "warmup": args.warmup,
         "ms_per_step": max_ms / K, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f16", "data": "synthetic",
         "config": {
-            "workload": "%s tokens: a = x W1 W2 + b, tokens=%d (B=%d x %dx%d), d_model=%d, rank=%d, "
-                        "n_out=H*d_k=%d, fp16 I/O, fp32 accumulation; one step = 1 launch"
-                        % (wl.name, T, wl.B, wl.grid_h, wl.grid_w, d, GATE_RANK, n),
-            "tokens_per_step": T,
-            "l2": "rotating pool of %d x/a sets (%.0f MB > 126 MB L2); no flush kernel"
-                  % (n_sets, n_sets * set_bytes / 1e6),
+            "workload": op.workload,
+            "tokens_per_step": op.tokens,
+            "l2": "rotating pool of %d input/output sets (%.0f MB > 126 MB L2); no flush kernel"
+                  % (op.n_sets, op.n_sets * op.set_bytes / 1e6),
             "timing": "CUDA-graph replays (graphs of %d steps), CUDA events on the launch stream"
                       % G,
             "parallelism": "replicas" if ws > 1 else "single GPU",
         },
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-                     "frac": achieved / peak, "traffic": profile_traffic(wl.name, GATE_KERNEL),
+                     "frac": achieved / peak, "traffic": profile_traffic(wl.name, op.kernel),
                      "peak_source": "%s (MEASURED_PEAKS.json hbm_gbs)" % peak_kind
                      if peak_kind == "measured" else "fallback 6.65 TB/s",
-                     "bytes_per_launch": gate_bytes(wl, d), "launch_us": launch_s * 1e6},
-        "e2e": {"value": job_throughput(T, e2e_steps, ws, e2e_ms), "unit": "Mtokens/s",
-                "h2d_bytes_per_step": hx.numel() * 2, "d2h_bytes_per_step": ha.numel() * 2,
+                     "bytes_per_launch": op.bytes_per_launch, "launch_us": launch_s * 1e6},
+        "e2e": {"value": job_throughput(op.tokens, e2e_steps, ws, e2e_ms), "unit": "Mtokens/s",
+                "h2d_bytes_per_step": op.h2d, "d2h_bytes_per_step": op.d2h,
                 "steps": e2e_steps, "ms_per_step": e2e_ms / e2e_steps},
         "gpu_launches": K,
         "clocks": clk.summary(),
     }
     if ws == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_gate_sample(inp, args.cpu_seconds)
+        line["cpu_baseline"] = op.cpu(args.cpu_seconds)
     print(json.dumps(line), flush=True)
 
 
@@ -733,6 +806,26 @@ def cpu_gate_sample(inp, budget_s: float):
                       % (calls, x.shape[0])}
 
 
+def cpu_sswiglu_sample(inp, gh: int, gw: int, budget_s: float):
+    """The oracle's Spatial SwiGLU mixing step (fp64 numpy) on the first image, repeated until
+    about a tenth of the budget has passed."""
+    import oracle
+    v, g, w, b = (inp[k][:1].astype("float64") if k in ("value", "gate") else inp[k].astype("float64")
+                  for k in ("value", "gate", "conv_w", "conv_b"))
+    t0 = time.perf_counter()
+    calls = 0
+    while True:
+        oracle.spatial_swiglu_mix(v, g, w, b, gh, gw)
+        calls += 1
+        el = time.perf_counter() - t0
+        if el >= budget_s / 10:
+            break
+    return {"value": calls * gh * gw / el / 1e6, "unit": "Mtokens/s", "cores": os.cpu_count(),
+            "kind": "oracle",
+            "sample": "%d calls of the fp64 oracle (numpy) on one %dx%d image of %d channels"
+                      % (calls, gh, gw, v.shape[2])}
+
+
 def main():
     args = parse()
     ws, rank, local = dist_env()
@@ -750,7 +843,7 @@ def main():
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=torch.device("cuda", local))
     try:
-        (run_gate if args.op == "gate" else run_ours)(args, ws, rank, local)
+        (run_ours if args.op == "gla" else run_aux)(args, ws, rank, local)
     finally:
         if ws > 1:
             import torch.distributed as dist

@@ -278,6 +278,23 @@ int gla_gate_proj(const void *x, const void *w1, const void *w2, const float *bi
                   int tokens, int d_model, int rank, int n_out, void *stream);
 
 /*
+ * gla_sswiglu -- Spatial SwiGLU's token mixing step, fused:
+ *     h[b][y][x][c] = SiLU(gate[b][y][x][c]) *
+ *                     (conv_b[c] + sum_{i,j=0..2} conv_w[c][i][j] value[b][y+i-1][x+j-1][c])
+ * GTR paper's method section, Spatial SwiGLU paragraph: the value branch is reshaped to the
+ * 2-D patch grid, convolved 3x3 depthwise and restored to sequence order; the gating branch
+ * stays tokenwise.  Read as a framework depthwise Conv2d (cross-correlation, zero padding of
+ * one token, per-channel bias) times SiLU of the gating branch.  value, gate, h: [batch]
+ * [grid_h * grid_w][channels] fp16, row-major grid (s = y * grid_w + x), 16-byte aligned;
+ * conv_w [channels][3][3] and conv_b [channels] float32.  DEVICE pointers, caller-owned; h
+ * must not overlap an input (GLA_ERR_ALIAS).  channels must be a multiple of 64
+ * (GLA_ERR_UNSUPPORTED).  fp32 arithmetic, fp16 output; a result outside the fp16 range (or
+ * NaN) latches GLA_ERR_RANGE.  Asynchronous on `stream`.
+ */
+int gla_sswiglu(const void *value, const void *gate, const float *conv_w, const float *conv_b, void *out,
+                int batch, int grid_h, int grid_w, int channels, void *stream);
+
+/*
  * gla_scan_layout -- host-only (no device work, no CUDA call): the token each tile row of
  * each chunk holds when `kernel` (GLA_KERNEL_PIPE64 only) runs a scan of a
  * grid_h x grid_w grid in `direction` (0..3) with chunks of at most `chunk` positions

@@ -18,6 +18,7 @@
 #include "gla_chunk.cuh"
 #include "gla_pipe.cuh"
 #include "gla_gate.cuh"
+#include "gla_sswiglu.cuh"
 #include "gla_common.cuh"
 #include "gla_simt.cuh"
 #include "gla_tc.cuh"
@@ -928,6 +929,81 @@ int gla_gate_proj(const void *x, const void *w1, const void *w2, const float *bi
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     if (cudaLaunchKernelEx(&cfg, gla::gp::gla_gate_kernel, xmap, amap, p) != cudaSuccess) {
+        cudaGetLastError();
+        return GLA_ERR_CUDA;
+    }
+    return GLA_OK;
+}
+
+int gla_sswiglu(const void *value, const void *gate, const float *conv_w, const float *conv_b, void *out,
+                int batch, int grid_h, int grid_w, int channels, void *stream) {
+    if (!value || !gate || !conv_w || !conv_b || !out) return GLA_ERR_NULL;
+    if (batch <= 0 || grid_h <= 0 || grid_w <= 0 || channels <= 0) return GLA_ERR_SHAPE;
+    const long long tokens = (long long)batch * grid_h * grid_w;
+    if (tokens * channels > (1LL << 40) || grid_h > (1 << 24) || grid_w > (1 << 24)) return GLA_ERR_SHAPE;
+    if (channels % gla::sw::kSlab != 0) return GLA_ERR_UNSUPPORTED;
+    const void *const io[3] = {value, gate, out};
+    for (const void *ptr : io)
+        if (reinterpret_cast<uintptr_t>(ptr) & 15u) return GLA_ERR_UNSUPPORTED;
+    if ((reinterpret_cast<uintptr_t>(conv_w) | reinterpret_cast<uintptr_t>(conv_b)) & 3u) return GLA_ERR_UNSUPPORTED;
+    const size_t act = (size_t)tokens * channels * 2;
+    const uintptr_t ob = reinterpret_cast<uintptr_t>(out), oe = ob + act;
+    const struct { const void *p; size_t n; } ins[4] = {
+        {value, act}, {gate, act}, {conv_w, (size_t)channels * 9 * 4}, {conv_b, (size_t)channels * 4}};
+    for (const auto &in : ins) {
+        const uintptr_t pb = reinterpret_cast<uintptr_t>(in.p), pe = pb + in.n;
+        if (pb < oe && ob < pe) return GLA_ERR_ALIAS;
+    }
+    DeviceInfo di;
+    int rc = current_device_info(&di);
+    if (rc != GLA_OK) return rc;
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return GLA_ERR_CUDA;
+    // tile extents: the grid split into near-equal blocks of at most 16 rows / columns
+    gla::sw::SwParams p;
+    p.gate = static_cast<const __half *>(gate);
+    p.w = conv_w;
+    p.b = conv_b;
+    p.out = static_cast<__half *>(out);
+    p.B = batch;
+    p.H = grid_h;
+    p.W = grid_w;
+    p.C = channels;
+    p.nyb = (grid_h + gla::sw::kMaxTile - 1) / gla::sw::kMaxTile;
+    p.nxb = (grid_w + gla::sw::kMaxTile - 1) / gla::sw::kMaxTile;
+    p.R = (grid_h + p.nyb - 1) / p.nyb;
+    p.Wt = (grid_w + p.nxb - 1) / p.nxb;
+    p.nslab = channels / gla::sw::kSlab;
+    p.tiles = (long long)batch * p.nyb * p.nxb * p.nslab;
+    p.wait_limit = 1LL << 32;
+    // value as {C, W, H, B}: one box = 64 channels x (Wt + 2) columns x (R + 2) rows of one image
+    CUtensorMap vmap;
+    const cuuint64_t dims[4] = {(cuuint64_t)channels, (cuuint64_t)grid_w, (cuuint64_t)grid_h, (cuuint64_t)batch};
+    const cuuint64_t strides[3] = {(cuuint64_t)channels * 2, (cuuint64_t)grid_w * channels * 2,
+                                   (cuuint64_t)grid_h * grid_w * channels * 2};
+    const cuuint32_t box[4] = {(cuuint32_t)gla::sw::kSlab, (cuuint32_t)p.Wt + 2, (cuuint32_t)p.R + 2, 1};
+    const cuuint32_t estr[4] = {1, 1, 1, 1};
+    if (fn(&vmap, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 4, const_cast<void *>(value), dims, strides, box, estr,
+           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+        return GLA_ERR_CUDA;
+    const size_t smem = 2 * (size_t)gla::sw::sw_buf_bytes(p.R, p.Wt) + 128;
+    if (cudaFuncSetAttribute(gla::sw::gla_sswiglu_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+        cudaSuccess) {
+        cudaGetLastError();
+        return GLA_ERR_CUDA;
+    }
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3((unsigned)std::min<long long>(p.tiles, 2LL * di.sms), 1, 1);
+    cfg.blockDim = dim3(gla::sw::kThreads, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = static_cast<cudaStream_t>(stream);
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, gla::sw::gla_sswiglu_kernel, vmap, p) != cudaSuccess) {
         cudaGetLastError();
         return GLA_ERR_CUDA;
     }

@@ -436,6 +436,16 @@ __device__ __forceinline__ void tma_load_3d(uint32_t dst, const void *tmap, int 
         "l"(tmap), "r"(x), "r"(y), "r"(z), "r"(bar)
         : "memory");
 }
+// Box of a 4-D tensor map at coordinates (x, y, z, w) into shared memory at dst (tile mode),
+// completing its bytes on the mbarrier.  Elements outside the tensor are filled with zeros.
+__device__ __forceinline__ void tma_load_4d(uint32_t dst, const void *tmap, int x, int y, int z, int w,
+                                            uint32_t bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%2, %3, %4, %5}], [%6];" ::"r"(dst),
+        "l"(tmap), "r"(x), "r"(y), "r"(z), "r"(w), "r"(bar)
+        : "memory");
+}
 // Box of shared memory at src into a 3-D tensor map at (x, y, z) (tile mode), tracked in this
 // thread's bulk async-group; rows outside the tensor are not written.
 __device__ __forceinline__ void tma_store_3d(const void *tmap, uint32_t src, int x, int y, int z) {

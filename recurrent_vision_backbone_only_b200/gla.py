@@ -73,6 +73,8 @@ def load() -> ctypes.CDLL:
         lib.gla_scan_layout.restype = ctypes.c_int
         lib.gla_gate_proj.argtypes = [vp] * 5 + [i] * 4 + [vp]
         lib.gla_gate_proj.restype = ctypes.c_int
+        lib.gla_sswiglu.argtypes = [vp] * 5 + [i] * 4 + [vp]
+        lib.gla_sswiglu.restype = ctypes.c_int
         lib.gla_selftest_fault.argtypes = [vp] * 7 + [i] * 7 + [ll, i, i, vp]
         lib.gla_selftest_rcp.argtypes = [vp, vp, i, vp]
         lib.gla_selftest_rcp.restype = ctypes.c_int
@@ -239,6 +241,27 @@ def gate_proj(x, w1, w2, bias, a, stream=None):
     _check(load().gla_gate_proj(*[ctypes.c_void_p(t.data_ptr()) for t in (x, w1, w2, bias, a)],
                                 tokens, d_model, rank, n_out, _stream_ptr(stream)), "gla_gate_proj")
     return a
+
+
+def sswiglu(value, gate, conv_w, conv_b, out, grid_h: int, grid_w: int, stream=None):
+    """h = SiLU(gate) * (DWConv3x3(value) + conv_b): Spatial SwiGLU's mixing step.
+
+    value, gate, out [B, grid_h * grid_w, C] fp16; conv_w [C, 3, 3] and conv_b [C] fp32; CUDA
+    tensors, contiguous."""
+    import torch
+    if value.dim() != 3 or value.shape[1] != grid_h * grid_w:
+        raise ValueError("sswiglu: value must be [B, grid_h * grid_w, C]")
+    B, _, C = value.shape
+    for t, dt, shape in ((value, torch.float16, None), (gate, torch.float16, tuple(value.shape)),
+                         (out, torch.float16, tuple(value.shape)), (conv_w, torch.float32, (C, 3, 3)),
+                         (conv_b, torch.float32, (C,))):
+        if not (t.is_cuda and t.is_contiguous() and t.dtype == dt):
+            raise ValueError("sswiglu: contiguous CUDA tensors of the documented dtypes expected")
+        if shape is not None and tuple(t.shape) != shape:
+            raise ValueError("sswiglu: shape %s expected, got %s" % (shape, tuple(t.shape)))
+    _check(load().gla_sswiglu(*[ctypes.c_void_p(t.data_ptr()) for t in (value, gate, conv_w, conv_b, out)],
+                              B, grid_h, grid_w, C, _stream_ptr(stream)), "gla_sswiglu")
+    return out
 
 
 def empty_launch(B: int, H: int, grid_h: int, grid_w: int, stream=None):

@@ -131,3 +131,22 @@ def make_gate_inputs(tokens: int, d_model: int, n_out: int, rank: int = 16, seed
     w2 = normal((rank, n_out), 0.0, rank ** -0.5, np.float16)
     b = normal((n_out,), b_mean, b_std, np.float32)
     return {"x": x, "w1": w1, "w2": w2, "b": b}
+
+
+def make_sswiglu_inputs(B: int, grid_h: int, grid_w: int, channels: int, seed: int = 0,
+                        w_std: float = 1.0 / 3.0, b_std: float = 0.1) -> Dict[str, np.ndarray]:
+    """Draw Spatial SwiGLU's mixing-step inputs: value and gate [B][grid_h*grid_w][channels]
+    (fp16, the two branches' projections, N(0, 1)), conv_w [channels][3][3] (fp32,
+    N(0, w_std): fan-in 9) and conv_b [channels] (fp32, N(0, b_std)).  Draw order: value,
+    gate, conv_w, conv_b."""
+    rng = np.random.Generator(np.random.PCG64(seed))
+    L = grid_h * grid_w
+
+    def normal(shape, std, dt):
+        return (rng.standard_normal(size=shape, dtype=np.float32) * np.float32(std)).astype(dt)
+
+    value = normal((B, L, channels), 1.0, np.float16)
+    gate = normal((B, L, channels), 1.0, np.float16)
+    conv_w = normal((channels, 3, 3), w_std, np.float32)
+    conv_b = normal((channels,), b_std, np.float32)
+    return {"value": value, "gate": gate, "conv_w": conv_w, "conv_b": conv_b}

@@ -187,3 +187,26 @@ def test_gate_projection_argument_errors(lib):
     import torch
     if not torch.cuda.is_available():
         assert gate() == 9                                 # GLA_ERR_NO_DEVICE, nothing faked
+
+
+def test_sswiglu_argument_errors(lib):
+    def sw(ptrs=ALIGNED[:5], B=1, gh=4, gw=5, C=64):
+        args = [ctypes.c_void_p(p) if p is not None else None for p in ptrs]
+        return gla.raw_call("gla_sswiglu", *args, B, gh, gw, C, None)
+    for i in range(5):
+        ptrs = list(ALIGNED[:5])
+        ptrs[i] = None
+        assert sw(ptrs) == 1                               # GLA_ERR_NULL
+    for kw in (dict(B=0), dict(gh=-1), dict(gw=0), dict(C=0), dict(B=1 << 20, gh=1 << 10, gw=1 << 10, C=1024)):
+        assert sw(**kw) == 2                               # GLA_ERR_SHAPE
+    for kw in (dict(C=32), dict(C=96)):
+        assert sw(**kw) == 3                               # GLA_ERR_UNSUPPORTED
+    mis = list(ALIGNED[:5])
+    mis[1] += 8
+    assert sw(mis) == 3                                    # gate not 16-byte aligned
+    alias = list(ALIGNED[:5])
+    alias[4] = alias[1] + 16                               # out overlaps gate
+    assert sw(alias) == 5                                  # GLA_ERR_ALIAS
+    import torch
+    if not torch.cuda.is_available():
+        assert sw() == 9                                   # GLA_ERR_NO_DEVICE

@@ -112,3 +112,11 @@ def test_gate_bytes_and_traffic_entry(tmp_path, capsys):
     # one launch per call: the mean over launches
     assert e["dram_bytes_per_launch"] == pytest.approx((2 * 235.09e6 + 60e6) / 3)
     assert e["algorithmic_bytes_per_launch"] == bench.gate_bytes(wl, 384)
+
+
+def test_sswiglu_bytes():
+    from recurrent_vision_backbone_only_b200 import synth
+    wl = synth.WORKLOADS["gtr640"]
+    C = 4 * 384
+    # value and gate read, h written (fp16); 9 taps and a bias (fp32) per channel
+    assert bench.sswiglu_bytes(wl, 384) == 3 * 2 * 1600 * C + 4 * 10 * C

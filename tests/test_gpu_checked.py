@@ -5,7 +5,7 @@ coordinates, remote exchange rows, chunk geometry -- is checked before use in th
 a violation latches GLA_ERR_CHECK instead of touching memory.  These cases run every kernel
 over the shapes whose index arithmetic differs (ragged and packed grids, reversed and cycling
 directions, 1 to 16 segments, a partial-wave split, d = 32 / 64 / 128, fp16 and fp32, and the
-gate projection's ragged tiles and split unit ranges) and
+gate projection's ragged tiles and split unit ranges, Spatial SwiGLU's ragged tiles and padding) and
 require that no check fires and that the results still match the oracle.  This stands in for
 a device memory checker, which cannot run on this hardware.
 """
@@ -107,4 +107,18 @@ def test_gate_projection(T, d, n):
     assert status == 0, gla.status_string(status)
     ref = oracle.gate_projection(*(inp[k].astype(np.float64) for k in ("x", "w1", "w2", "b")))
     d_ = a.cpu().numpy().astype(np.float64) - ref
+    assert np.max(np.abs(d_)) <= 1e-2 and np.linalg.norm(d_) <= 2e-3 * np.linalg.norm(ref)
+
+
+@pytest.mark.parametrize("B,gh,gw,C", [(2, 33, 17, 128), (1, 40, 40, 256), (1, 1, 1, 64), (1, 3, 256, 64)])
+def test_sswiglu(B, gh, gw, C):
+    import torch
+    inp = synth.make_sswiglu_inputs(B, gh, gw, C, seed=gh)
+    t = {k: torch.from_numpy(np.ascontiguousarray(v)).cuda() for k, v in inp.items()}
+    out = torch.empty_like(t["value"])
+    gla.sswiglu(t["value"], t["gate"], t["conv_w"], t["conv_b"], out, gh, gw)
+    status = gla.get_status()
+    assert status == 0, gla.status_string(status)
+    ref = oracle.spatial_swiglu_mix(*(inp[k].astype(np.float64) for k in ("value", "gate", "conv_w", "conv_b")), gh, gw)
+    d_ = out.cpu().numpy().astype(np.float64) - ref
     assert np.max(np.abs(d_)) <= 1e-2 and np.linalg.norm(d_) <= 2e-3 * np.linalg.norm(ref)
