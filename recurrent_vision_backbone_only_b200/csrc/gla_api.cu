@@ -961,7 +961,6 @@ int gla_sswiglu(const void *value, const void *gate, const float *conv_w, const 
     if (!fn) return GLA_ERR_CUDA;
     // tile extents: the grid split into near-equal blocks of at most 16 rows / columns
     gla::sw::SwParams p;
-    p.gate = static_cast<const __half *>(gate);
     p.w = conv_w;
     p.b = conv_b;
     p.out = static_cast<__half *>(out);
@@ -969,21 +968,26 @@ int gla_sswiglu(const void *value, const void *gate, const float *conv_w, const 
     p.H = grid_h;
     p.W = grid_w;
     p.C = channels;
-    p.nyb = (grid_h + gla::sw::kMaxTile - 1) / gla::sw::kMaxTile;
-    p.nxb = (grid_w + gla::sw::kMaxTile - 1) / gla::sw::kMaxTile;
+    p.nyb = (grid_h + gla::sw::kMaxR - 1) / gla::sw::kMaxR;
+    p.nxb = (grid_w + gla::sw::kMaxWt - 1) / gla::sw::kMaxWt;
     p.R = (grid_h + p.nyb - 1) / p.nyb;
     p.Wt = (grid_w + p.nxb - 1) / p.nxb;
     p.nslab = channels / gla::sw::kSlab;
     p.tiles = (long long)batch * p.nyb * p.nxb * p.nslab;
     p.wait_limit = 1LL << 32;
-    // value as {C, W, H, B}: one box = 64 channels x (Wt + 2) columns x (R + 2) rows of one image
-    CUtensorMap vmap;
+    // value and gate as {C, W, H, B}: boxes of 64 channels x (Wt + 2) columns x (R + 2) rows (the
+    // value, with its halo) and 64 x Wt x R (the gate) of one image
+    CUtensorMap vmap, gmap;
     const cuuint64_t dims[4] = {(cuuint64_t)channels, (cuuint64_t)grid_w, (cuuint64_t)grid_h, (cuuint64_t)batch};
     const cuuint64_t strides[3] = {(cuuint64_t)channels * 2, (cuuint64_t)grid_w * channels * 2,
                                    (cuuint64_t)grid_h * grid_w * channels * 2};
-    const cuuint32_t box[4] = {(cuuint32_t)gla::sw::kSlab, (cuuint32_t)p.Wt + 2, (cuuint32_t)p.R + 2, 1};
+    const cuuint32_t vbox[4] = {(cuuint32_t)gla::sw::kSlab, (cuuint32_t)p.Wt + 2, (cuuint32_t)p.R + 2, 1};
+    const cuuint32_t gbox[4] = {(cuuint32_t)gla::sw::kSlab, (cuuint32_t)p.Wt, (cuuint32_t)p.R, 1};
     const cuuint32_t estr[4] = {1, 1, 1, 1};
-    if (fn(&vmap, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 4, const_cast<void *>(value), dims, strides, box, estr,
+    if (fn(&vmap, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 4, const_cast<void *>(value), dims, strides, vbox, estr,
+           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS ||
+        fn(&gmap, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 4, const_cast<void *>(gate), dims, strides, gbox, estr,
            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
         return GLA_ERR_CUDA;
@@ -994,7 +998,11 @@ int gla_sswiglu(const void *value, const void *gate, const float *conv_w, const 
         return GLA_ERR_CUDA;
     }
     cudaLaunchConfig_t cfg{};
-    cfg.gridDim = dim3((unsigned)std::min<long long>(p.tiles, 2LL * di.sms), 1, 1);
+    // two CTAs per SM; when tiles outnumber them, a multiple of the slab count, so every CTA
+    // keeps one channel slab (tiles are numbered slab fastest)
+    long long grid = std::min<long long>(p.tiles, 2LL * di.sms);
+    if (p.tiles > grid && p.nslab <= grid) grid -= grid % p.nslab;
+    cfg.gridDim = dim3((unsigned)grid, 1, 1);
     cfg.blockDim = dim3(gla::sw::kThreads, 1, 1);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = static_cast<cudaStream_t>(stream);
@@ -1003,7 +1011,7 @@ int gla_sswiglu(const void *value, const void *gate, const float *conv_w, const 
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    if (cudaLaunchKernelEx(&cfg, gla::sw::gla_sswiglu_kernel, vmap, p) != cudaSuccess) {
+    if (cudaLaunchKernelEx(&cfg, gla::sw::gla_sswiglu_kernel, vmap, gmap, p) != cudaSuccess) {
         cudaGetLastError();
         return GLA_ERR_CUDA;
     }

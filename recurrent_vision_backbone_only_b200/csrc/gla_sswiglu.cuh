@@ -9,14 +9,18 @@
 //     h[b][y][x][c] = SiLU(gate[b][y][x][c]) * (bias[c] + sum_{i,j in 0..2} w[c][i][j] value[b][y+i-1][x+j-1][c])
 // value, gate, h are token-major [B][grid_h * grid_w][C] (C contiguous); w [C][3][3], bias [C].
 //
-// Tiling: a CTA tile is R grid rows x Wt grid columns x 64 channels.  One TMA box of a 4-D view
-// {C, W, H, B} brings the tile's values with a one-token halo, (R + 2) x (Wt + 2) x 128 B, into
-// shared memory; halo positions outside the grid (the zero padding) come back as zeros from the
-// TMA bounds check, so no thread special-cases the border.  Two buffers: the next tile's box
-// loads while this tile computes.  Thread (xl, q) owns grid column x0 + xl and channels
-// 4q .. 4q+3 of the slab and walks down the R rows with a 3 x 3 window of fp32 values in
-// registers: each output reads one new smem row segment (3 x 8 B), loads its gate directly from
-// global memory two rows ahead, and stores 8 B of h.  A warp's 32 threads cover two grid
+// Tiling: a CTA tile is R <= 8 grid rows x Wt <= 16 grid columns x 64 channels.  Two TMA boxes
+// of 4-D views {C, W, H, B} bring the tile's values with a one-token halo ((R + 2) x (Wt + 2) x
+// 128 B) and its gates (R x Wt x 128 B) into shared memory; halo positions outside the grid
+// (the zero padding) come back as zeros from the TMA bounds check, so no thread special-cases
+// the border.  Two stages: the next tile's boxes load while this tile computes (with two CTAs
+// per SM, about 80 KB of loads in flight per SM).  The grid is a multiple of the channel-slab
+// count, so a CTA keeps one slab and loads its taps once.  Thread (xl, q) owns grid column
+// x0 + xl and channels 4q .. 4q+3 of the slab and walks down the R rows with a 3 x 3 window of
+// fp32 values in registers (rows taken three at a time, so the window is renamed rather than
+// copied): each output reads one new value row segment (3 x 8 B) and its gate (8 B) from shared
+// memory and stores 8 B of h.  The taps, the window and the SiLU arithmetic use packed
+// fp32 pairs (f32x2 FMA / multiply / add), two channels per instruction.  A warp's 32 threads cover two grid
 // columns x 128 B, so shared loads, gate loads and stores are all contiguous 256-byte runs.
 #pragma once
 
@@ -31,12 +35,11 @@ namespace sw {
 
 constexpr int kSlab = 64;                       // channels per tile: one 128-byte row per token
 constexpr int kQ = kSlab / 4;                   // 4-channel groups per slab (threads per column)
-constexpr int kMaxTile = 16;                    // R, Wt <= 16
-constexpr int kThreads = kQ * kMaxTile;         // 256
+constexpr int kMaxR = 8, kMaxWt = 16;           // tile extent limits
+constexpr int kThreads = kQ * kMaxWt;           // 256
 
 struct SwParams {
-    const __half *gate;
-    const float *w, *b;
+    const float *w, *b;                         // value and gate come through their tensor maps
     __half *out;
     int B, H, W, C;
     int R, Wt;                                  // tile extent: grid rows, grid columns
@@ -45,19 +48,56 @@ struct SwParams {
     long long wait_limit;
 };
 
-__host__ __device__ constexpr uint32_t sw_buf_bytes(int R, int Wt) {
+// Packed fp32 pairs (Blackwell's f32x2 arithmetic): two channels per instruction.
+__device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+__device__ __forceinline__ float2 f2_unpack(uint64_t v) {
+    float2 r;
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(r.x), "=f"(r.y) : "l"(v));
+    return r;
+}
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+    uint64_t r;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+    return r;
+}
+__device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
+    uint64_t r;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
+}
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
+    uint64_t r;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
+}
+// two fp16 (low half first) -> a packed fp32 pair
+__device__ __forceinline__ uint64_t f2_from_h2(uint32_t h2) {
+    const float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&h2));
+    return f2_pack(f.x, f.y);
+}
+
+// one stage: the value box with its halo, then the gate box
+__host__ __device__ constexpr uint32_t sw_val_bytes(int R, int Wt) {
     return (uint32_t)(R + 2) * (uint32_t)(Wt + 2) * 128u;
+}
+__host__ __device__ constexpr uint32_t sw_buf_bytes(int R, int Wt) {
+    return sw_val_bytes(R, Wt) + (uint32_t)R * (uint32_t)Wt * 128u;
 }
 
 __global__ void __launch_bounds__(kThreads, 2)
-    gla_sswiglu_kernel(const __grid_constant__ CUtensorMap vmap, const SwParams p) {
+    gla_sswiglu_kernel(const __grid_constant__ CUtensorMap vmap, const __grid_constant__ CUtensorMap gmap,
+                       const SwParams p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
     __shared__ uint64_t full[2];
     __shared__ int abort_sh;
     volatile int &abort_flag = abort_sh;
     const uint32_t sbase = ptx::smem_u32(sm);
-    const uint32_t buf_bytes = sw_buf_bytes(p.R, p.Wt);
+    const uint32_t buf_bytes = sw_buf_bytes(p.R, p.Wt), val_bytes = sw_val_bytes(p.R, p.Wt);
     const int tid = threadIdx.x;
     const int xl = tid / kQ, q = tid % kQ;
     const bool active = xl < p.Wt;
@@ -68,6 +108,7 @@ __global__ void __launch_bounds__(kThreads, 2)
         ptx::fence_mbarrier_init();
         abort_sh = 0;
         ptx::prefetch_tmap(&vmap);
+        ptx::prefetch_tmap(&gmap);
     }
     __syncthreads();
     ptx::pdl_launch_dependents();
@@ -91,12 +132,16 @@ __global__ void __launch_bounds__(kThreads, 2)
             ptx::mbar_arrive_expect_tx(&full[buf], buf_bytes);
             ptx::tma_load_4d(sbase + buf * buf_bytes, &vmap, slab * kSlab, xb * p.Wt - 1, yb * p.R - 1, b,
                              ptx::smem_u32(&full[buf]));
+            ptx::tma_load_4d(sbase + buf * buf_bytes + val_bytes, &gmap, slab * kSlab, xb * p.Wt, yb * p.R, b,
+                             ptx::smem_u32(&full[buf]));
         } else {
             ptx::mbar_arrive(&full[buf]);
         }
     };
 
     float amax = 0.0f;
+    uint64_t wt[9][2], bias[2];
+    int cur_slab = -1;
     if (tid == 0 && (long long)blockIdx.x < p.tiles) issue(blockIdx.x, 0);
     int it = 0;
     for (long long t = blockIdx.x; t < p.tiles; t += gridDim.x, ++it) {
@@ -110,21 +155,21 @@ __global__ void __launch_bounds__(kThreads, 2)
         const int y0 = yb * p.R;
         const int rows = min(p.R, p.H - y0);
         const bool live = active && x < p.W;
-        // this thread's taps and bias (4 channels)
-        float wt[9][4], bias[4];
+        // this thread's taps and bias (4 channels as two packed fp32 pairs), reloaded only
+        // when the slab changes
+        if (slab != cur_slab) {
+            cur_slab = slab;
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            bias[i] = live ? p.b[c + i] : 0.0f;
+            for (int pr = 0; pr < 2; ++pr) {
+                const int ca = c + 2 * pr;
+                bias[pr] = active ? f2_pack(p.b[ca], p.b[ca + 1]) : 0ull;
 #pragma unroll
-            for (int k = 0; k < 9; ++k) wt[k][i] = live ? p.w[(size_t)(c + i) * 9 + k] : 0.0f;
+                for (int k = 0; k < 9; ++k)
+                    wt[k][pr] = active ? f2_pack(p.w[(size_t)ca * 9 + k], p.w[(size_t)(ca + 1) * 9 + k]) : 0ull;
+            }
         }
-        // gate of output rows 0 and 1, two rows ahead of use
         const size_t row_stride = (size_t)p.W * p.C;
-        const __half *gbase = p.gate + ((size_t)b * p.H + y0) * row_stride + (size_t)x * p.C + c;
         __half *obase = p.out + ((size_t)b * p.H + y0) * row_stride + (size_t)x * p.C + c;
-        uint2 g0 = make_uint2(0, 0), g1 = make_uint2(0, 0);
-        if (live) g0 = __ldcs(reinterpret_cast<const uint2 *>(gbase));
-        if (live && rows > 1) g1 = __ldcs(reinterpret_cast<const uint2 *>(gbase + row_stride));
 
         // wait for the tile's values (bounded)
         if (!abort_flag) {
@@ -137,68 +182,69 @@ __global__ void __launch_bounds__(kThreads, 2)
                 }
             }
         }
+        const bool go = active && !abort_flag;
         const uint8_t *tb = sm + buf * buf_bytes + 8 * q;
+        const uint8_t *gtb = tb + val_bytes;
         const uint32_t row_bytes = (uint32_t)(p.Wt + 2) * 128u;
-        auto load3 = [&](int tr, float (&dst)[3][4]) {          // tile row tr, columns xl .. xl+2
+        // tile row tr, columns xl .. xl+2 -> [column][channel pair]
+        auto load3 = [&](int tr, uint64_t (&dst)[3][2]) {
 #pragma unroll
             for (int j = 0; j < 3; ++j) {
                 const uint32_t off = (uint32_t)tr * row_bytes + (uint32_t)(xl + j) * 128u;
                 uint2 u = make_uint2(0, 0);
                 if (GLA_CHECK(off + 8 * q + 8 <= buf_bytes)) u = *reinterpret_cast<const uint2 *>(tb + off);
-                const float2 lo = __half22float2(*reinterpret_cast<const __half2 *>(&u.x));
-                const float2 hi = __half22float2(*reinterpret_cast<const __half2 *>(&u.y));
-                dst[j][0] = lo.x;
-                dst[j][1] = lo.y;
-                dst[j][2] = hi.x;
-                dst[j][3] = hi.y;
+                dst[j][0] = f2_from_h2(u.x);
+                dst[j][1] = f2_from_h2(u.y);
             }
         };
-        float win[3][3][4];                                     // [window row][column][channel]
-        if (active && !abort_flag) {
-            load3(0, win[0]);
-            load3(1, win[1]);
-        }
-#pragma unroll 1
-        for (int r = 0; r < rows; ++r) {
-            uint2 g2 = make_uint2(0, 0);
-            if (live && r + 2 < rows) g2 = __ldcs(reinterpret_cast<const uint2 *>(gbase + (size_t)(r + 2) * row_stride));
-            if (active && !abort_flag) {
-                load3(r + 2, win[2]);
-                float acc[4];
+        // one output row: window rows (A, B, C) = tile rows (r, r+1, r+2), C loaded here
+        auto step = [&](int r, uint64_t (&A)[3][2], uint64_t (&Bw)[3][2], uint64_t (&Cw)[3][2]) {
+            load3(r + 2, Cw);
+            const uint32_t goff = ((uint32_t)r * (uint32_t)p.Wt + (uint32_t)xl) * 128u;
+            uint2 GA = make_uint2(0, 0);
+            if (GLA_CHECK(val_bytes + goff + 8 * q + 8 <= buf_bytes)) GA = *reinterpret_cast<const uint2 *>(gtb + goff);
+            uint64_t acc[2];
 #pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    float s = bias[i];
+            for (int pr = 0; pr < 2; ++pr) {
+                uint64_t s2 = bias[pr];
 #pragma unroll
-                    for (int a = 0; a < 3; ++a)
-#pragma unroll
-                        for (int j = 0; j < 3; ++j) s = fmaf(wt[3 * a + j][i], win[a][j][i], s);
-                    acc[i] = s;
+                for (int j = 0; j < 3; ++j) {
+                    s2 = f2_fma(wt[j][pr], A[j][pr], s2);
+                    s2 = f2_fma(wt[3 + j][pr], Bw[j][pr], s2);
+                    s2 = f2_fma(wt[6 + j][pr], Cw[j][pr], s2);
                 }
-                const float2 ga = __half22float2(*reinterpret_cast<const __half2 *>(&g0.x));
-                const float2 gb = __half22float2(*reinterpret_cast<const __half2 *>(&g0.y));
-                const float gv[4] = {ga.x, ga.y, gb.x, gb.y};
-                float h[4];
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    h[i] = __fdividef(gv[i], 1.0f + __expf(-gv[i])) * acc[i];
-                    amax = fmaxf(amax, fabsf(h[i]));
-                }
-                if (live) {
-                    const __half2 o0 = __floats2half2_rn(h[0], h[1]);
-                    const __half2 o1 = __floats2half2_rn(h[2], h[3]);
-                    __stcs(reinterpret_cast<uint2 *>(obase + (size_t)r * row_stride),
-                           make_uint2(*reinterpret_cast<const uint32_t *>(&o0), *reinterpret_cast<const uint32_t *>(&o1)));
-                }
-#pragma unroll
-                for (int j = 0; j < 3; ++j)
-#pragma unroll
-                    for (int i = 0; i < 4; ++i) {
-                        win[0][j][i] = win[1][j][i];
-                        win[1][j][i] = win[2][j][i];
-                    }
+                acc[pr] = s2;
             }
-            g0 = g1;
-            g1 = g2;
+            // SiLU(g) = g / (1 + 2^(-g log2 e)), times the convolution
+            const uint64_t g2[2] = {f2_from_h2(GA.x), f2_from_h2(GA.y)};
+            uint32_t packed[2];
+#pragma unroll
+            for (int pr = 0; pr < 2; ++pr) {
+                const float2 t = f2_unpack(f2_mul(g2[pr], f2_pack(-1.4426950408889634f, -1.4426950408889634f)));
+                const uint64_t den = f2_add(f2_pack(ptx::ex2(t.x), ptx::ex2(t.y)), f2_pack(1.0f, 1.0f));
+                const float2 dv = f2_unpack(den);
+                const uint64_t sg = f2_mul(g2[pr], f2_pack(ptx::rcp(dv.x), ptx::rcp(dv.y)));
+                const float2 h = f2_unpack(f2_mul(sg, acc[pr]));
+                amax = fmaxf(amax, fmaxf(fabsf(h.x), fabsf(h.y)));
+                const __half2 o = __floats2half2_rn(h.x, h.y);
+                packed[pr] = *reinterpret_cast<const uint32_t *>(&o);
+            }
+            if (live) __stcs(reinterpret_cast<uint2 *>(obase + (size_t)r * row_stride), make_uint2(packed[0], packed[1]));
+        };
+        uint64_t W0[3][2], W1[3][2], W2[3][2];
+        if (go) {
+            load3(0, W0);
+            load3(1, W1);
+            // rows in threes with the window and gate registers renamed, not copied
+            int r = 0;
+#pragma unroll 1
+            for (; r + 3 <= rows; r += 3) {
+                step(r, W0, W1, W2);
+                step(r + 1, W1, W2, W0);
+                step(r + 2, W2, W0, W1);
+            }
+            if (r < rows) step(r, W0, W1, W2);
+            if (r + 1 < rows) step(r + 1, W1, W2, W0);
         }
         __syncthreads();                                        // buffer `buf` free for reuse
     }

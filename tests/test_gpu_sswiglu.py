@@ -42,8 +42,9 @@ def check(h, inp, gh, gw):
     assert np.linalg.norm(d) <= 2e-3 * np.linalg.norm(ref)
 
 
-# Tiles are near-equal blocks of at most 16 rows x 16 columns x 64 channels with a one-token
-# halo: 40 -> 3 blocks of 14 (ragged last block), 33 -> 3 of 11, 17 -> 2 of 9, 256 -> 16 of 16.
+# Tiles are near-equal blocks of at most 8 rows x 16 columns x 64 channels, values with a
+# one-token halo: 40 columns -> 3 blocks of 14 (ragged last block), 33 rows -> 5 of 7, 17
+# columns -> 2 of 9, 256 columns -> 16 of 16.
 @pytest.mark.parametrize("B,gh,gw,C", [
     (1, 40, 40, 1536),       # GTR-L at 640 px: width 384, expansion 4
     (2, 7, 5, 64),
@@ -62,8 +63,8 @@ def test_sswiglu_matches_oracle(B, gh, gw, C):
 
 
 def test_more_tiles_than_ctas():
-    # 16 x 40x40 x 512 channels = 9 x 16 x 8 = 1152 tiles on at most 296 CTAs: both smem
-    # buffers reused many times
+    # 16 x 40x40 x 512 channels = 16 x 15 x 8 = 1920 tiles on 296 CTAs (a multiple of the 8
+    # slabs): both stages reused many times, one slab per CTA
     inp = synth.make_sswiglu_inputs(16, 40, 40, 512, seed=3)
     h, status = run(inp, 40, 40)
     assert status == 0
