@@ -173,3 +173,45 @@ def spatial_swiglu_mix(value, gate, conv_w, conv_b, grid_h, grid_w):
             conv += w[:, dy + 1, dx + 1] * padded[:, 1 + dy:1 + dy + grid_h, 1 + dx:1 + dx + grid_w, :]
     silu = g / (1.0 + np.exp(-g))
     return silu * conv.reshape(B, L, C)
+
+
+def linear(x, w, bias=None):
+    """y = x W (+ bias), fp64: one library matmul.
+
+    The block's dense projections (GTR paper, arXiv 2609.26590, method section): the input
+    projections Q = X W_Q, K = X W_K, V = X W_V and the output gate's x_t W_r (GLA recurrence
+    and output-gate paragraphs, no bias written), and the output projection that maps the
+    concatenated heads back to the model dimension (output-gate paragraph).  x [T][K],
+    w [K][N], bias [N] or None  ->  y [T][N].
+    """
+    x64 = np.asarray(x, dtype=np.float64)
+    w64 = np.asarray(w, dtype=np.float64)
+    if x64.ndim != 2 or w64.ndim != 2 or x64.shape[1] != w64.shape[0]:
+        raise ValueError("linear: x [T][K], w [K][N] expected")
+    y = x64 @ w64
+    if bias is not None:
+        b64 = np.asarray(bias, dtype=np.float64)
+        if b64.shape != (w64.shape[1],):
+            raise ValueError("linear: bias [N] expected")
+        y = y + b64
+    return y
+
+
+def input_projections(x, w_q, w_k, w_v, w_r):
+    """The block's input side, fp64: q = x W_Q, k = x W_K, v = x W_V and the output gate's
+    pre-activation x W_r, all heads at once.
+
+    GTR paper, method section, GLA recurrence paragraph (Q = X W_Q, K = X W_K, V = X W_V per
+    head, W_Q, W_K in R^{d x d_k}, W_V in R^{d x d_v}) and output-gate paragraph
+    (r_t = SiLU(x_t W_r)).  Each weight holds every head's columns head-major, [d][H d], so
+    each result is [T][H d] = the operator's [B][L][H][d] layout.  Returns (q, k, v, g).
+    """
+    return tuple(linear(x, w) for w in (w_q, w_k, w_v, w_r))
+
+
+def output_projection(u, w_o):
+    """Heads concatenated and projected back to the model dimension, fp64: y = concat_h(u_h) W_O.
+
+    GTR paper, method section, output-gate paragraph.  u [T][H d_v] is the operator's output
+    [B][L][H][d_v] viewed per token (the concatenation is that layout), w_o [H d_v][d]."""
+    return linear(u, w_o)
