@@ -40,12 +40,27 @@ PROFILE_TRAFFIC = os.path.join(ROOT, "profiles", "traffic.json")
 GATE_KERNEL = "gate projection (tcgen05)"
 GATE_RANK = 16
 SSWIGLU_KERNEL = "spatial swiglu mix"
+LINEAR_KERNEL = "dense projection (tcgen05)"
+FALLBACK_TENSOR_TFLOPS = 1590.0
 SSWIGLU_EXPANSION = 4
 
 
 def gate_shape(wl, d_model: int):
     """(tokens, d_model, n_out) of the gate projection feeding the workload's operator."""
     return wl.B * wl.L, d_model, wl.H * wl.d_k
+
+
+def linear_bytes(rows: int, k_dim: int, n_dim: int) -> int:
+    """Algorithmic HBM bytes of one projection: x read, y written and W read once (fp16)."""
+    return 2 * (rows * k_dim + rows * n_dim + k_dim * n_dim)
+
+
+def measured_tensor_peak():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return float(json.load(f)["bf16_tflops"]), "measured"
+    except Exception:
+        return FALLBACK_TENSOR_TFLOPS, "fallback"
 
 
 def sswiglu_bytes(wl, d_model: int) -> int:
@@ -77,11 +92,13 @@ def parse():
     ap.add_argument("--workload", default=WORKLOAD,
                     help="synthetic workload to time (default: the 40x40 headline); the others "
                          "are reported with their own metric name")
-    ap.add_argument("--op", choices=["gla", "gate", "sswiglu"], default="gla",
+    ap.add_argument("--op", choices=["gla", "gate", "sswiglu", "proj_in", "proj_out"], default="gla",
                     help="gla: the operator (default); gate: the retention gate's low-rank "
                          "projection a = x W1 W2 + b over the workload's tokens (B*L), its output "
                          "width H*d_k, model width --d-model; sswiglu: Spatial SwiGLU's "
-                         "dwconv + gating step on the workload's grid, 4 x d_model channels")
+                         "dwconv + gating step on the workload's grid, 4 x d_model channels; "
+                         "proj_in / proj_out: the block's input projections (x -> q, k, v, W_r) "
+                         "and output projection (heads -> d_model)")
     ap.add_argument("--d-model", type=int, default=384,
                     help="with --op gate / sswiglu: the model width d (GTR-L: 384)")
     ap.add_argument("--record-traffic", metavar="NCU_CSV",
@@ -191,9 +208,15 @@ def record_traffic(args):
     from recurrent_vision_backbone_only_b200 import build as _b, gla, synth
     wl = synth.WORKLOADS[args.workload]
     op = getattr(args, "op", "gla")
-    if op in ("gate", "sswiglu"):
-        symbol, kname, alg = {"gate": ("gla_gate_kernel", GATE_KERNEL, gate_bytes),
-                              "sswiglu": ("gla_sswiglu_kernel", SSWIGLU_KERNEL, sswiglu_bytes)}[op]
+    if op in ("gate", "sswiglu", "proj_in", "proj_out"):
+        T, n = wl.B * wl.L, wl.H * wl.d_k
+        symbol, kname, alg = {
+            "gate": ("gla_gate_kernel", GATE_KERNEL, gate_bytes),
+            "sswiglu": ("gla_sswiglu_kernel", SSWIGLU_KERNEL, sswiglu_bytes),
+            "proj_in": ("gla_linear_kernel", LINEAR_KERNEL + ", input side", lambda w_, d: linear_bytes(T, d, 4 * n)),
+            "proj_out": ("gla_linear_kernel", LINEAR_KERNEL + ", output side",
+                         lambda w_, d: linear_bytes(T, w_.H * w_.d_v, d)),
+        }[op]
         got = [v for k, v in read_ncu_csv(args.record_traffic) if re.search(symbol, k)]
         got = [v for v in got if "dram__bytes_read.sum" in v and "dram__bytes_write.sum" in v]
         if not got:
@@ -682,6 +705,45 @@ def sswiglu_op(args, wl, dev):
         cpu=lambda budget: cpu_sswiglu_sample(inp, gh, gw, budget))
 
 
+def linear_op(args, wl, dev, side):
+    """gla_linear as the block's input side (x -> q, k, v and the output gate's pre-activation,
+    four [B][L][H][d] parts) or output side (the concatenated heads -> the model width)."""
+    import torch
+    from recurrent_vision_backbone_only_b200 import gla, synth
+    T, d, n = wl.B * wl.L, args.d_model, wl.H * wl.d_k
+    rows, K, N, n_part = (T, d, 4 * n, n) if side == "in" else (T, wl.H * wl.d_v, d, d)
+    inp = synth.make_linear_inputs(rows, K, N, seed=wl.seed)
+    w = torch.from_numpy(inp["w"]).to(dev)
+    set_bytes = 2 * rows * (K + N)
+    n_sets = max(2 if set_bytes > L2_BYTES else 8, math.ceil(2 * L2_BYTES / set_bytes))
+    x0 = torch.from_numpy(inp["x"]).to(dev)
+    sets = [(x0.clone(), torch.empty((N // n_part, rows, n_part), dtype=torch.float16, device=dev))
+            for _ in range(n_sets)]
+    hx = torch.from_numpy(inp["x"]).pin_memory()
+    hy = torch.empty((N // n_part, rows, n_part), dtype=torch.float16).pin_memory()
+
+    def step(i):
+        xs, y = sets[i % n_sets]
+        gla.linear(xs, w, y, n_part=n_part)
+
+    def e2e_step():
+        xs, y = sets[0]
+        xs.copy_(hx, non_blocking=True)
+        gla.linear(xs, w, y, n_part=n_part)
+        hy.copy_(y, non_blocking=True)
+
+    what = ("x -> q, k, v, W_r pre-activation (4 parts of H*d_k=%d)" % n if side == "in"
+            else "concatenated heads (H*d_v=%d) -> d_model" % K)
+    return AuxOp(
+        name="proj_" + side, kernel="%s, %s side" % (LINEAR_KERNEL, "input" if side == "in" else "output"), tokens=rows, bytes_per_launch=linear_bytes(rows, K, N),
+        flops_per_launch=2 * rows * K * N, step=step, e2e_step=e2e_step, h2d=hx.numel() * 2,
+        d2h=hy.numel() * 2, n_sets=n_sets, set_bytes=set_bytes,
+        metric="%s projection Mtokens/s (B·L), %s workload" % ("input" if side == "in" else "output", wl.name),
+        workload="%s tokens: %s, rows=%d (B=%d x %dx%d), K=%d, N=%d, fp16 I/O, fp32 accumulation; "
+                 "one step = 1 launch" % (wl.name, what, rows, wl.B, wl.grid_h, wl.grid_w, K, N),
+        cpu=lambda budget: cpu_linear_sample(inp, budget))
+
+
 def run_aux(args, ws, rank, local):
     """Time one of the steps next to the operator (--op gate / sswiglu) like the operator."""
     import torch
@@ -692,7 +754,9 @@ def run_aux(args, ws, rank, local):
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
     wl = synth.WORKLOADS[args.workload]
-    op = {"gate": gate_op, "sswiglu": sswiglu_op}[args.op](args, wl, dev)
+    op = {"gate": gate_op, "sswiglu": sswiglu_op,
+          "proj_in": lambda a, w_, d_: linear_op(a, w_, d_, "in"),
+          "proj_out": lambda a, w_, d_: linear_op(a, w_, d_, "out")}[args.op](args, wl, dev)
 
     stream = torch.cuda.Stream(device=dev)
     torch.cuda.synchronize()
@@ -739,6 +803,20 @@ def run_aux(args, ws, rank, local):
     launch_s = max_ms / 1e3 / K
     peak, peak_kind = measured_peaks()
     achieved = op.bytes_per_launch / launch_s / 1e9
+    roof = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+            "peak_source": "%s (MEASURED_PEAKS.json hbm_gbs)" % peak_kind
+            if peak_kind == "measured" else "fallback 6.65 TB/s"}
+    flops = getattr(op, "flops_per_launch", 0)
+    if flops:
+        tpeak, tkind = measured_tensor_peak()
+        # the bound is whichever roof the launch's work needs more time on
+        if flops / (tpeak * 1e12) > op.bytes_per_launch / (peak * 1e9):
+            ta = flops / launch_s / 1e12
+            roof = {"bound": "tensor", "achieved": ta, "peak": tpeak, "unit": "TFLOP/s", "frac": ta / tpeak,
+                    "peak_source": "%s (MEASURED_PEAKS.json bf16_tflops; fp16 runs at the same nominal "
+                                   "dense rate)" % tkind if tkind == "measured" else "fallback 1.59 PFLOP/s",
+                    "hbm_achieved_gbs": achieved, "hbm_frac": achieved / peak}
+        roof["flops_per_launch"] = flops
 
     # e2e: inputs from pinned host memory, the launch, the result back to pinned host memory
     e2e_steps = max(1, min(args.e2e_steps, K))
@@ -771,11 +849,8 @@ def run_aux(args, ws, rank, local):
                       % G,
             "parallelism": "replicas" if ws > 1 else "single GPU",
         },
-        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-                     "frac": achieved / peak, "traffic": profile_traffic(wl.name, op.kernel),
-                     "peak_source": "%s (MEASURED_PEAKS.json hbm_gbs)" % peak_kind
-                     if peak_kind == "measured" else "fallback 6.65 TB/s",
-                     "bytes_per_launch": op.bytes_per_launch, "launch_us": launch_s * 1e6},
+        "roofline": dict(roof, traffic=profile_traffic(wl.name, op.kernel),
+                         bytes_per_launch=op.bytes_per_launch, launch_us=launch_s * 1e6),
         "e2e": {"value": job_throughput(op.tokens, e2e_steps, ws, e2e_ms), "unit": "Mtokens/s",
                 "h2d_bytes_per_step": op.h2d, "d2h_bytes_per_step": op.d2h,
                 "steps": e2e_steps, "ms_per_step": e2e_ms / e2e_steps},
@@ -804,6 +879,24 @@ def cpu_gate_sample(inp, budget_s: float):
             "cores": os.cpu_count(), "kind": "oracle",
             "sample": "%d whole-input calls of the fp64 oracle (numpy matmuls, %d tokens each)"
                       % (calls, x.shape[0])}
+
+
+def cpu_linear_sample(inp, budget_s: float):
+    """The oracle's dense projection (fp64 numpy matmul) over the whole input, repeated until
+    about a tenth of the budget has passed."""
+    import oracle
+    x, w = inp["x"].astype("float64"), inp["w"].astype("float64")
+    t0 = time.perf_counter()
+    calls = 0
+    while True:
+        oracle.linear(x, w)
+        calls += 1
+        el = time.perf_counter() - t0
+        if el >= budget_s / 10:
+            break
+    return {"value": calls * x.shape[0] / el / 1e6, "unit": "Mtokens/s", "cores": os.cpu_count(),
+            "kind": "oracle", "sample": "%d whole-input calls of the fp64 oracle (numpy matmul, %d x %d x %d)"
+                                        % (calls, x.shape[0], x.shape[1], w.shape[1])}
 
 
 def cpu_sswiglu_sample(inp, gh: int, gw: int, budget_s: float):

@@ -278,6 +278,24 @@ int gla_gate_proj(const void *x, const void *w1, const void *w2, const float *bi
                   int tokens, int d_model, int rank, int n_out, void *stream);
 
 /*
+ * gla_linear -- the block's dense projections, y = x W (+ bias):
+ *     y[part][t][c] = sum_k x[t][k] W[k][part * n_part + c] (+ bias[part * n_part + c])
+ * GTR paper's method section: the input projections Q = X W_Q, K = X W_K, V = X W_V (GLA
+ * recurrence paragraph) and the output gate's x W_r, and the output projection of the
+ * concatenated heads back to the model dimension (output-gate paragraph).  x: [rows][k_dim]
+ * fp16, W: [k_dim][n_dim] fp16 (row-major), bias: [n_dim] float32 or NULL, y: fp16 written as
+ * n_dim / n_part parts of [rows][n_part] each, one after another (n_part = n_dim: a plain
+ * [rows][n_dim] matrix; W = [W_Q | W_K | W_V | W_r] with n_part = H * d: q, k, v and the output
+ * gate's pre-activation as four [B][L][H][d] tensors).  DEVICE pointers, 16-byte aligned,
+ * caller-owned; y must not overlap an input (GLA_ERR_ALIAS).  k_dim and n_part must be
+ * multiples of 64 and n_dim a multiple of 128 or 192 divisible by n_part, else
+ * GLA_ERR_UNSUPPORTED.  tcgen05 tensor cores, fp32 accumulation, fp16 output.  Asynchronous
+ * on `stream`.
+ */
+int gla_linear(const void *x, const void *w, const float *bias, void *y, int rows, int k_dim, int n_dim,
+               int n_part, void *stream);
+
+/*
  * gla_sswiglu -- Spatial SwiGLU's token mixing step, fused:
  *     h[b][y][x][c] = SiLU(gate[b][y][x][c]) *
  *                     (conv_b[c] + sum_{i,j=0..2} conv_w[c][i][j] value[b][y+i-1][x+j-1][c])

@@ -19,6 +19,7 @@
 #include "gla_pipe.cuh"
 #include "gla_gate.cuh"
 #include "gla_sswiglu.cuh"
+#include "gla_linear.cuh"
 #include "gla_common.cuh"
 #include "gla_simt.cuh"
 #include "gla_tc.cuh"
@@ -929,6 +930,85 @@ int gla_gate_proj(const void *x, const void *w1, const void *w2, const float *bi
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     if (cudaLaunchKernelEx(&cfg, gla::gp::gla_gate_kernel, xmap, amap, p) != cudaSuccess) {
+        cudaGetLastError();
+        return GLA_ERR_CUDA;
+    }
+    return GLA_OK;
+}
+
+int gla_linear(const void *x, const void *w, const float *bias, void *y, int rows, int k_dim, int n_dim,
+               int n_part, void *stream) {
+    if (!x || !w || !y) return GLA_ERR_NULL;
+    if (rows <= 0 || k_dim <= 0 || n_dim <= 0 || n_part <= 0) return GLA_ERR_SHAPE;
+    if ((long long)rows * std::max(k_dim, n_dim) > (1LL << 40)) return GLA_ERR_SHAPE;
+    if (k_dim % gla::ln::kBK != 0 || n_part % 64 != 0 || n_dim % n_part != 0) return GLA_ERR_UNSUPPORTED;
+    const int nt = n_dim % 256 == 0 ? 256 : n_dim % 192 == 0 ? 192 : n_dim % 128 == 0 ? 128 : 0;
+    if (nt == 0) return GLA_ERR_UNSUPPORTED;
+    const void *const ptrs[4] = {x, w, y, bias};
+    for (const void *ptr : ptrs)
+        if (reinterpret_cast<uintptr_t>(ptr) & 15u) return GLA_ERR_UNSUPPORTED;
+    const uintptr_t yb = reinterpret_cast<uintptr_t>(y), ye = yb + (size_t)rows * n_dim * 2;
+    const struct { const void *p; size_t n; } ins[3] = {
+        {x, (size_t)rows * k_dim * 2}, {w, (size_t)k_dim * n_dim * 2}, {bias, bias ? (size_t)n_dim * 4 : 0}};
+    for (const auto &in : ins) {
+        const uintptr_t pb = reinterpret_cast<uintptr_t>(in.p), pe = pb + in.n;
+        if (in.n && pb < ye && yb < pe) return GLA_ERR_ALIAS;
+    }
+    DeviceInfo di;
+    int rc = current_device_info(&di);
+    if (rc != GLA_OK) return rc;
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return GLA_ERR_CUDA;
+    // x {K, 1, M} in boxes of 64 x 128 rows; W {N, 1, K} in boxes of 64 columns x 64 K rows;
+    // y {n_part, M, parts} in boxes of 64 columns x 128 rows; all 128-byte swizzled
+    CUtensorMap xmap, wmap, ymap;
+    const struct {
+        CUtensorMap *map; void *base; cuuint64_t d0, d1, d2, s1, s2; cuuint32_t b0, b1, b2;
+    } maps[3] = {
+        {&xmap, const_cast<void *>(x), (cuuint64_t)k_dim, 1, (cuuint64_t)rows, (cuuint64_t)k_dim * 2,
+         (cuuint64_t)k_dim * 2, 64, 1, (cuuint32_t)gla::ln::kTileM},
+        {&wmap, const_cast<void *>(w), (cuuint64_t)n_dim, 1, (cuuint64_t)k_dim, (cuuint64_t)n_dim * 2,
+         (cuuint64_t)n_dim * 2, 64, 1, (cuuint32_t)gla::ln::kBK},
+        {&ymap, y, (cuuint64_t)n_part, (cuuint64_t)rows, (cuuint64_t)(n_dim / n_part), (cuuint64_t)n_part * 2,
+         (cuuint64_t)rows * n_part * 2, 64, (cuuint32_t)gla::ln::kTileM, 1}};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    for (const auto &mp : maps) {
+        const cuuint64_t dims[3] = {mp.d0, mp.d1, mp.d2};
+        const cuuint64_t strides[2] = {mp.s1, mp.s2};
+        const cuuint32_t box[3] = {mp.b0, mp.b1, mp.b2};
+        if (fn(mp.map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3, mp.base, dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return GLA_ERR_CUDA;
+    }
+    const gla::ln::LinLayout lay = gla::ln::lin_layout(nt, (size_t)di.max_smem_optin);
+    if (lay.stages < 2) return GLA_ERR_UNSUPPORTED;
+    if (cudaFuncSetAttribute(gla::ln::gla_linear_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)lay.bytes) != cudaSuccess) {
+        cudaGetLastError();
+        return GLA_ERR_CUDA;
+    }
+    gla::ln::LinParams p;
+    p.bias = bias;
+    p.M = rows;
+    p.K = k_dim;
+    p.N = n_dim;
+    p.n_part = n_part;
+    p.nt = nt;
+    p.lay = lay;
+    p.wait_limit = 1LL << 32;
+    const long long tiles = (long long)((rows + gla::ln::kTileM - 1) / gla::ln::kTileM) * (n_dim / nt);
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3((unsigned)std::min<long long>(tiles, di.sms), 1, 1);
+    cfg.blockDim = dim3(gla::ln::kThreads, 1, 1);
+    cfg.dynamicSmemBytes = lay.bytes;
+    cfg.stream = static_cast<cudaStream_t>(stream);
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, gla::ln::gla_linear_kernel, xmap, wmap, ymap, p) != cudaSuccess) {
         cudaGetLastError();
         return GLA_ERR_CUDA;
     }

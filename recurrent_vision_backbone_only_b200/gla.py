@@ -75,6 +75,8 @@ def load() -> ctypes.CDLL:
         lib.gla_gate_proj.restype = ctypes.c_int
         lib.gla_sswiglu.argtypes = [vp] * 5 + [i] * 4 + [vp]
         lib.gla_sswiglu.restype = ctypes.c_int
+        lib.gla_linear.argtypes = [vp] * 4 + [i] * 4 + [vp]
+        lib.gla_linear.restype = ctypes.c_int
         lib.gla_selftest_fault.argtypes = [vp] * 7 + [i] * 7 + [ll, i, i, vp]
         lib.gla_selftest_rcp.argtypes = [vp, vp, i, vp]
         lib.gla_selftest_rcp.restype = ctypes.c_int
@@ -241,6 +243,31 @@ def gate_proj(x, w1, w2, bias, a, stream=None):
     _check(load().gla_gate_proj(*[ctypes.c_void_p(t.data_ptr()) for t in (x, w1, w2, bias, a)],
                                 tokens, d_model, rank, n_out, _stream_ptr(stream)), "gla_gate_proj")
     return a
+
+
+def linear(x, w, y, bias=None, n_part: int = 0, stream=None):
+    """y = x W (+ bias): the block's dense projections on tensor cores.
+
+    x [rows, K] fp16, w [K, N] fp16, bias [N] fp32 or None; y holds N / n_part parts of
+    [rows, n_part] one after another (default n_part = N: y is [rows, N]).  Leading dims of x
+    are rows.  CUDA tensors, contiguous."""
+    import torch
+    K, N = w.shape
+    rows = x.numel() // K if x.dim() else 0
+    n_part = n_part or N
+    for t, dt in ((x, torch.float16), (w, torch.float16), (y, torch.float16)):
+        if not (t.is_cuda and t.is_contiguous() and t.dtype == dt):
+            raise ValueError("linear: contiguous fp16 CUDA tensors expected")
+    if x.shape[-1] != K or y.numel() != rows * N:
+        raise ValueError("linear: x [rows, K] and y holding rows x N expected")
+    if bias is not None and not (bias.is_cuda and bias.is_contiguous() and bias.dtype == torch.float32
+                                 and tuple(bias.shape) == (N,)):
+        raise ValueError("linear: bias must be a contiguous fp32 CUDA tensor [N]")
+    _check(load().gla_linear(ctypes.c_void_p(x.data_ptr()), ctypes.c_void_p(w.data_ptr()),
+                             ctypes.c_void_p(bias.data_ptr()) if bias is not None else None,
+                             ctypes.c_void_p(y.data_ptr()), rows, K, N, n_part, _stream_ptr(stream)),
+           "gla_linear")
+    return y
 
 
 def sswiglu(value, gate, conv_w, conv_b, out, grid_h: int, grid_w: int, stream=None):

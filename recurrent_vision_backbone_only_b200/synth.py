@@ -150,3 +150,18 @@ def make_sswiglu_inputs(B: int, grid_h: int, grid_w: int, channels: int, seed: i
     conv_w = normal((channels, 3, 3), w_std, np.float32)
     conv_b = normal((channels,), b_std, np.float32)
     return {"value": value, "gate": gate, "conv_w": conv_w, "conv_b": conv_b}
+
+
+def make_linear_inputs(rows: int, k_dim: int, n_dim: int, seed: int = 0, bias: bool = False) -> Dict[str, np.ndarray]:
+    """Draw a dense projection's inputs: x [rows][k_dim] fp16 ~ N(0, 1), w [k_dim][n_dim] fp16
+    ~ N(0, 1/k_dim) (unit-scale outputs) and, if asked, bias [n_dim] fp32 ~ N(0, 0.1).  Draw
+    order: x, w, bias."""
+    rng = np.random.Generator(np.random.PCG64(seed))
+
+    def normal(shape, std, dt):
+        return (rng.standard_normal(size=shape, dtype=np.float32) * np.float32(std)).astype(dt)
+
+    out = {"x": normal((rows, k_dim), 1.0, np.float16), "w": normal((k_dim, n_dim), k_dim ** -0.5, np.float16)}
+    if bias:
+        out["b"] = normal((n_dim,), 0.1, np.float32)
+    return out

@@ -210,3 +210,29 @@ def test_sswiglu_argument_errors(lib):
     import torch
     if not torch.cuda.is_available():
         assert sw() == 9                                   # GLA_ERR_NO_DEVICE
+
+
+def test_linear_argument_errors(lib):
+    def ln(ptrs=ALIGNED[:4], rows=128, K=64, N=256, n_part=256):
+        args = [ctypes.c_void_p(p) if p is not None else None for p in ptrs]
+        return gla.raw_call("gla_linear", *args, rows, K, N, n_part, None)
+    for i in (0, 1, 3):
+        ptrs = list(ALIGNED[:4])
+        ptrs[i] = None
+        assert ln(ptrs) == 1                               # GLA_ERR_NULL (x, w or y)
+    for kw in (dict(rows=0), dict(K=-64), dict(N=0), dict(n_part=0), dict(rows=1 << 30, K=2048)):
+        assert ln(**kw) == 2                               # GLA_ERR_SHAPE
+    for kw in (dict(K=96), dict(N=320, n_part=320), dict(N=256, n_part=96), dict(N=512, n_part=384)):
+        assert ln(**kw) == 3                               # GLA_ERR_UNSUPPORTED
+    mis = list(ALIGNED[:4])
+    mis[2] += 8
+    assert ln(mis) == 3                                    # bias not 16-byte aligned
+    alias = list(ALIGNED[:4])
+    alias[3] = alias[0] + 32                               # y overlaps x
+    assert ln(alias) == 5                                  # GLA_ERR_ALIAS
+    import torch
+    if not torch.cuda.is_available():
+        assert ln() == 9                                   # GLA_ERR_NO_DEVICE
+        nb = list(ALIGNED[:4])
+        nb[2] = None                                       # no bias is allowed
+        assert ln(nb) == 9

@@ -120,3 +120,10 @@ def test_sswiglu_bytes():
     C = 4 * 384
     # value and gate read, h written (fp16); 9 taps and a bias (fp32) per channel
     assert bench.sswiglu_bytes(wl, 384) == 3 * 2 * 1600 * C + 4 * 10 * C
+
+
+def test_linear_bytes_and_bound_inputs():
+    # x read, y written, W read once (fp16)
+    assert bench.linear_bytes(1600, 384, 1536) == 2 * (1600 * 384 + 1600 * 1536 + 384 * 1536)
+    tpeak, kind = bench.measured_tensor_peak()
+    assert tpeak > 100 and kind in ("measured", "fallback")

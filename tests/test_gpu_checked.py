@@ -5,7 +5,7 @@ coordinates, remote exchange rows, chunk geometry -- is checked before use in th
 a violation latches GLA_ERR_CHECK instead of touching memory.  These cases run every kernel
 over the shapes whose index arithmetic differs (ragged and packed grids, reversed and cycling
 directions, 1 to 16 segments, a partial-wave split, d = 32 / 64 / 128, fp16 and fp32, and the
-gate projection's ragged tiles and split unit ranges, Spatial SwiGLU's ragged tiles and padding) and
+gate projection's ragged tiles and split unit ranges, Spatial SwiGLU's ragged tiles and padding, the projections' row and column tiles and parts) and
 require that no check fires and that the results still match the oracle.  This stands in for
 a device memory checker, which cannot run on this hardware.
 """
@@ -122,3 +122,17 @@ def test_sswiglu(B, gh, gw, C):
     ref = oracle.spatial_swiglu_mix(*(inp[k].astype(np.float64) for k in ("value", "gate", "conv_w", "conv_b")), gh, gw)
     d_ = out.cpu().numpy().astype(np.float64) - ref
     assert np.max(np.abs(d_)) <= 1e-2 and np.linalg.norm(d_) <= 2e-3 * np.linalg.norm(ref)
+
+
+@pytest.mark.parametrize("rows,K,N,n_part", [(300, 64, 128, 128), (1600, 384, 1536, 384), (129, 192, 576, 192)])
+def test_linear(rows, K, N, n_part):
+    import torch
+    inp = synth.make_linear_inputs(rows, K, N, seed=rows, bias=True)
+    x, w, b = (torch.from_numpy(inp[k]).cuda() for k in ("x", "w", "b"))
+    y = torch.empty((N // n_part, rows, n_part), dtype=torch.float16, device="cuda")
+    gla.linear(x, w, y, bias=b, n_part=n_part)
+    status = gla.get_status()
+    assert status == 0, gla.status_string(status)
+    ref = oracle.linear(inp["x"].astype(np.float64), inp["w"].astype(np.float64), inp["b"].astype(np.float64))
+    got = np.concatenate(list(y.cpu().numpy()), axis=1).astype(np.float64)
+    assert np.max(np.abs(got - ref)) <= 1e-2
