@@ -15,14 +15,15 @@
 //   swizzle) and nt / 64 boxes of W [64 K rows][64 columns] (MN-major, 128-byte swizzle);
 //   4 tcgen05.mma of K = 16 per block into a TMEM accumulator (two accumulators, so one
 //   tile's epilogue overlaps the next tile's products);
-//   epilogue: TMEM -> registers (+ bias) -> fp16 -> 128-byte swizzled staging boxes of
-//   [128 rows][64 columns] -> TMA stores (rows past M are clipped by TMA).
+//   epilogue: TMEM -> registers (+ bias) -> fp16 -> two 128-byte swizzled staging boxes of
+//   [128 rows][64 columns], two boxes per round -> TMA stores (rows past M are clipped by TMA).
+//   Staging two boxes rather than the whole tile leaves room for one more ring stage.
 // Tiles are numbered column tile fastest, and CTAs stride over them, so the CTAs working at the
 // same time share x tiles through L2.
 //
 // Roles (320 threads, one CTA per SM): warps 0-7 epilogue (warp w reads TMEM lanes
-// 32 (w % 4) .. +31 = tile rows, and the staging boxes j with j % 2 == w / 4), warp 8 TMA
-// producer, warp 9 MMA issuer.
+// 32 (w % 4) .. +31 = tile rows), warp 8 TMA
+// producer, warp 9 MMA issuer.  In round r the warps with w / 4 = h convert box 2 r + h.
 #pragma once
 
 #include <cuda.h>
@@ -51,7 +52,7 @@ struct LinMisc {
 };
 
 // Shared-memory layout for an nt-column tile: the ring (stages of one x block and nt / 64 W
-// boxes), the nt / 64 staging boxes, then the barriers.  Offsets are from the 1024-aligned
+// boxes), two staging boxes, then the barriers.  Offsets are from the 1024-aligned
 // base; `bytes` includes the alignment slack.
 struct LinLayout {
     uint32_t stage_bytes, ring, o, misc, bytes;
@@ -62,7 +63,7 @@ __host__ __device__ inline LinLayout lin_layout(int nt, size_t smem_cap) {
     LinLayout L;
     L.stage_bytes = kABytes + (uint32_t)(nt / 64) * kBBox;
     L.ring = 0;
-    const uint32_t staging = (uint32_t)(nt / 64) * kOBox;
+    const uint32_t staging = 2 * kOBox;
     const size_t fixed = (size_t)staging + sizeof(LinMisc) + 1024;
     const long long fit = smem_cap > fixed ? (long long)((smem_cap - fixed) / L.stage_bytes) : 0;
     L.stages = (int)(fit < kMaxStages ? fit : kMaxStages);
@@ -156,49 +157,53 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int mt = (int)(t / ntiles), n0 = (int)(t % ntiles) * p.nt;
             const int ab = tc & 1;
             wait(&m.accfull[ab], tc >> 1);
-            // the previous tile's TMA stores have read the staging boxes
-            if (tid == 0) ptx::bulk_wait_group_read<0>();
-            ptx::named_bar_sync(1, kEpi);
             ptx::tc_fence_after_sync();
-            for (int j = half; j < nbox; j += 2) {
-                float v0[32], v1[32];
-                const uint32_t taddr = tmem + lanes + (uint32_t)(ab * 256 + 64 * j);
-                ptx::tmem_ld32(taddr, v0);
-                ptx::tmem_ld32(taddr + 32, v1);
-                ptx::tmem_ld_wait();
-                const int cb = n0 + 64 * j;                     // first output column of box j
+            for (int r0 = 0; r0 < nbox; r0 += 2) {
+                const int j = r0 + half;
+                // the previous round's TMA stores have read the two staging boxes
+                if (tid == 0) ptx::bulk_wait_group_read<0>();
+                ptx::named_bar_sync(1, kEpi);
+                if (j < nbox) {
+                    float v0[32], v1[32];
+                    const uint32_t taddr = tmem + lanes + (uint32_t)(ab * 256 + 64 * j);
+                    ptx::tmem_ld32(taddr, v0);
+                    ptx::tmem_ld32(taddr + 32, v1);
+                    ptx::tmem_ld_wait();
+                    const int cb = n0 + 64 * j;                     // first output column of box j
 #pragma unroll
-                for (int u = 0; u < 8; ++u) {
-                    const float *v = u < 4 ? &v0[8 * u] : &v1[8 * (u - 4)];
-                    float4 ba = make_float4(0.f, 0.f, 0.f, 0.f), bb = ba;
-                    if (p.bias) {
-                        ba = __ldg(reinterpret_cast<const float4 *>(p.bias + cb + 8 * u));
-                        bb = __ldg(reinterpret_cast<const float4 *>(p.bias + cb + 8 * u + 4));
-                    }
-                    const __half2 o0 = __floats2half2_rn(v[0] + ba.x, v[1] + ba.y);
-                    const __half2 o1 = __floats2half2_rn(v[2] + ba.z, v[3] + ba.w);
-                    const __half2 o2 = __floats2half2_rn(v[4] + bb.x, v[5] + bb.y);
-                    const __half2 o3 = __floats2half2_rn(v[6] + bb.z, v[7] + bb.w);
-                    const uint32_t off = L.o + (uint32_t)j * kOBox + ptx::sw128(row, u);
-                    if (GLA_CHECK(off + 16 <= L.misc))
-                        *reinterpret_cast<uint4 *>(sm + off) =
-                            make_uint4(*reinterpret_cast<const uint32_t *>(&o0), *reinterpret_cast<const uint32_t *>(&o1),
-                                       *reinterpret_cast<const uint32_t *>(&o2), *reinterpret_cast<const uint32_t *>(&o3));
-                }
-            }
-            ptx::tc_fence_before_sync();
-            ptx::fence_proxy_async_smem();
-            ptx::named_bar_sync(1, kEpi);
-            if (tid == 0) {
-                ptx::mbar_arrive(&m.accempty[ab]);              // accumulator ab read
-                if (!*abort_flag) {
-                    for (int j = 0; j < nbox; ++j) {
-                        const int c = n0 + 64 * j, part = c / p.n_part, col = c % p.n_part;
-                        if (GLA_CHECK(c < p.N && mt < mtiles))
-                            ptx::tma_store_3d(&ymap, sbase + L.o + (uint32_t)j * kOBox, col, mt * kTileM, part);
+                    for (int u = 0; u < 8; ++u) {
+                        const float *v = u < 4 ? &v0[8 * u] : &v1[8 * (u - 4)];
+                        float4 ba = make_float4(0.f, 0.f, 0.f, 0.f), bb = ba;
+                        if (p.bias) {
+                            ba = __ldg(reinterpret_cast<const float4 *>(p.bias + cb + 8 * u));
+                            bb = __ldg(reinterpret_cast<const float4 *>(p.bias + cb + 8 * u + 4));
+                        }
+                        const __half2 o0 = __floats2half2_rn(v[0] + ba.x, v[1] + ba.y);
+                        const __half2 o1 = __floats2half2_rn(v[2] + ba.z, v[3] + ba.w);
+                        const __half2 o2 = __floats2half2_rn(v[4] + bb.x, v[5] + bb.y);
+                        const __half2 o3 = __floats2half2_rn(v[6] + bb.z, v[7] + bb.w);
+                        const uint32_t off = L.o + (uint32_t)half * kOBox + ptx::sw128(row, u);
+                        if (GLA_CHECK(off + 16 <= L.misc))
+                            *reinterpret_cast<uint4 *>(sm + off) =
+                                make_uint4(*reinterpret_cast<const uint32_t *>(&o0), *reinterpret_cast<const uint32_t *>(&o1),
+                                           *reinterpret_cast<const uint32_t *>(&o2), *reinterpret_cast<const uint32_t *>(&o3));
                     }
                 }
-                ptx::bulk_commit_group();
+                ptx::tc_fence_before_sync();
+                ptx::fence_proxy_async_smem();
+                ptx::named_bar_sync(1, kEpi);
+                if (tid == 0) {
+                    if (r0 + 2 >= nbox) ptx::mbar_arrive(&m.accempty[ab]);   // accumulator ab read
+                    if (!*abort_flag) {
+                        for (int jj = r0; jj < r0 + 2 && jj < nbox; ++jj) {
+                            const int c = n0 + 64 * jj, part = c / p.n_part, col = c % p.n_part;
+                            if (GLA_CHECK(c < p.N && mt < mtiles))
+                                ptx::tma_store_3d(&ymap, sbase + L.o + (uint32_t)(jj - r0) * kOBox, col, mt * kTileM,
+                                                  part);
+                        }
+                    }
+                    ptx::bulk_commit_group();
+                }
             }
         }
         if (tid == 0) ptx::bulk_wait_group_all();               // stores done before smem is freed
