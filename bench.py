@@ -744,8 +744,29 @@ def linear_op(args, wl, dev, side):
         cpu=lambda budget: cpu_linear_sample(inp, budget))
 
 
+def aux_roofline(bytes_per_launch: int, flops_per_launch: int, launch_s: float, hbm, tensor):
+    """Roofline entry for one launch: HBM-bound unless its FLOPs need more time on the tensor
+    roof than its bytes need on the HBM roof.  hbm = (GB/s, kind), tensor = (TFLOP/s, kind)."""
+    peak, peak_kind = hbm
+    achieved = bytes_per_launch / launch_s / 1e9
+    roof = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+            "peak_source": "%s (MEASURED_PEAKS.json hbm_gbs)" % peak_kind
+            if peak_kind == "measured" else "fallback 6.65 TB/s"}
+    if flops_per_launch:
+        tpeak, tkind = tensor
+        if flops_per_launch / (tpeak * 1e12) > bytes_per_launch / (peak * 1e9):
+            ta = flops_per_launch / launch_s / 1e12
+            roof = {"bound": "tensor", "achieved": ta, "peak": tpeak, "unit": "TFLOP/s", "frac": ta / tpeak,
+                    "peak_source": "%s (MEASURED_PEAKS.json bf16_tflops; fp16 runs at the same nominal "
+                                   "dense rate)" % tkind if tkind == "measured" else "fallback 1.59 PFLOP/s",
+                    "hbm_achieved_gbs": achieved, "hbm_frac": achieved / peak}
+        roof["flops_per_launch"] = flops_per_launch
+    return roof
+
+
 def run_aux(args, ws, rank, local):
-    """Time one of the steps next to the operator (--op gate / sswiglu) like the operator."""
+    """Time one of the steps next to the operator (--op gate / sswiglu / proj_in / proj_out) like
+    the operator."""
     import torch
     import torch.distributed as dist
     from recurrent_vision_backbone_only_b200 import build as _b, gla, synth
@@ -801,22 +822,8 @@ def run_aux(args, ws, rank, local):
     max_ms = max_over_ranks(ev0.elapsed_time(ev1), dev)
     value = job_throughput(op.tokens, K, ws, max_ms)
     launch_s = max_ms / 1e3 / K
-    peak, peak_kind = measured_peaks()
-    achieved = op.bytes_per_launch / launch_s / 1e9
-    roof = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
-            "peak_source": "%s (MEASURED_PEAKS.json hbm_gbs)" % peak_kind
-            if peak_kind == "measured" else "fallback 6.65 TB/s"}
-    flops = getattr(op, "flops_per_launch", 0)
-    if flops:
-        tpeak, tkind = measured_tensor_peak()
-        # the bound is whichever roof the launch's work needs more time on
-        if flops / (tpeak * 1e12) > op.bytes_per_launch / (peak * 1e9):
-            ta = flops / launch_s / 1e12
-            roof = {"bound": "tensor", "achieved": ta, "peak": tpeak, "unit": "TFLOP/s", "frac": ta / tpeak,
-                    "peak_source": "%s (MEASURED_PEAKS.json bf16_tflops; fp16 runs at the same nominal "
-                                   "dense rate)" % tkind if tkind == "measured" else "fallback 1.59 PFLOP/s",
-                    "hbm_achieved_gbs": achieved, "hbm_frac": achieved / peak}
-        roof["flops_per_launch"] = flops
+    roof = aux_roofline(op.bytes_per_launch, getattr(op, "flops_per_launch", 0), launch_s,
+                        measured_peaks(), measured_tensor_peak())
 
     # e2e: inputs from pinned host memory, the launch, the result back to pinned host memory
     e2e_steps = max(1, min(args.e2e_steps, K))

@@ -236,3 +236,19 @@ def test_linear_argument_errors(lib):
         nb = list(ALIGNED[:4])
         nb[2] = None                                       # no bias is allowed
         assert ln(nb) == 9
+
+
+def test_new_bindings_check_tensors_before_any_call():
+    # host (CPU) tensors and wrong dtypes are rejected in Python, before the library is called
+    import torch
+    x = torch.zeros(128, 64, dtype=torch.float16)
+    with pytest.raises(ValueError):
+        gla.gate_proj(x, torch.zeros(64, 16, dtype=torch.float16), torch.zeros(16, 128, dtype=torch.float16),
+                      torch.zeros(128), torch.zeros(128, 128, dtype=torch.float16))
+    with pytest.raises(ValueError):
+        gla.linear(x, torch.zeros(64, 128, dtype=torch.float16), torch.zeros(128, 128, dtype=torch.float16))
+    v = torch.zeros(1, 20, 64, dtype=torch.float16)
+    with pytest.raises(ValueError):
+        gla.sswiglu(v, v, torch.zeros(64, 3, 3), torch.zeros(64), torch.zeros_like(v), 4, 5)
+    with pytest.raises(ValueError):
+        gla.sswiglu(v, v, torch.zeros(64, 3, 3), torch.zeros(64), torch.zeros_like(v), 5, 5)   # L != 25

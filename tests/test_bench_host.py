@@ -127,3 +127,21 @@ def test_linear_bytes_and_bound_inputs():
     assert bench.linear_bytes(1600, 384, 1536) == 2 * (1600 * 384 + 1600 * 1536 + 384 * 1536)
     tpeak, kind = bench.measured_tensor_peak()
     assert tpeak > 100 and kind in ("measured", "fallback")
+
+
+def test_aux_roofline_picks_the_binding_roof():
+    hbm, tensor = (6545.9, "measured"), (1609.7, "measured")
+    # the batched input projections: 60.4 GFLOP need 37.5 us on the tensor roof, 179 MB need
+    # 27.4 us on the HBM roof -> tensor-bound
+    r = bench.aux_roofline(179_306_496, 60_397_977_600, 74.8e-6, hbm, tensor)
+    assert r["bound"] == "tensor" and r["unit"] == "TFLOP/s"
+    assert r["achieved"] == pytest.approx(60_397_977_600 / 74.8e-6 / 1e12)
+    assert r["frac"] == pytest.approx(r["achieved"] / 1609.7)
+    assert r["hbm_frac"] == pytest.approx(179_306_496 / 74.8e-6 / 1e9 / 6545.9)
+    # the 40x40 B=1 output projection: 0.47 GFLOP vs 2.5 MB -> HBM-bound
+    r = bench.aux_roofline(2_752_512, 471_859_200, 7.28e-6, hbm, tensor)
+    assert r["bound"] == "hbm" and r["unit"] == "GB/s" and r["flops_per_launch"] == 471_859_200
+    # no FLOPs given (gate, Spatial SwiGLU): HBM, no tensor keys
+    r = bench.aux_roofline(59_022_336, 0, 17.42e-6, hbm, tensor)
+    assert r["bound"] == "hbm" and "flops_per_launch" not in r
+    assert r["frac"] == pytest.approx(59_022_336 / 17.42e-6 / 1e9 / 6545.9)
