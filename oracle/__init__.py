@@ -120,7 +120,7 @@ def gate_projection(x, w1, w2, b):
 
     GTR paper (arXiv 2609.26590), method section, GLA recurrence paragraph: the gate is
     gamma_t = sigma(x_t W_alpha^(1) W_alpha^(2) + b_alpha)^(1/tau), a low-rank projection of
-    rank r = 16 "following GLA".  Reading taken here (the paragraph writes one head, d_k key
+    rank r = 16 built the way GLA builds its gate.  Reading taken here (the paragraph writes one head, d_k key
     channels): as in GLA, one first factor W1 [d][r] is shared by the heads and the second factor
     W2 [r][H d_k] maps to every head's key channels, with one bias per key channel.
 
