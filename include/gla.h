@@ -263,8 +263,8 @@ int gla_selftest_load(const void *q, const void *k, const void *gate_preact, con
  * gla_gate_proj -- the retention gate's pre-activation, the input gate_preact of gla_fwd:
  *     a[t][c] = sum_j (sum_i x[t][i] w1[i][j]) w2[j][c] + bias[c]
  * GTR paper's method section, GLA recurrence paragraph: gamma_t = sigma(x_t W_alpha^(1)
- * W_alpha^(2) + b_alpha)^(1/tau), a low-rank projection of rank r = 16 "following GLA" -- read
- * as GLA builds it: one first factor shared by the heads, a second factor onto every head's
+ * W_alpha^(2) + b_alpha)^(1/tau), a low-rank projection of rank r = 16, read as GLA builds
+ * it: one first factor shared by the heads, a second factor onto every head's
  * key channels.  x: [tokens][d_model] fp16 (token-major, tokens = B * L), w1: [d_model][rank]
  * fp16, w2: [rank][n_out] fp16 (n_out = H * d_k, head-major), bias: [n_out] float32, a:
  * [tokens][n_out] fp16 -- the [B][L][H][d_k] layout gla_fwd reads.  DEVICE pointers, 16-byte

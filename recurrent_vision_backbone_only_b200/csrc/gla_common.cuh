@@ -13,7 +13,7 @@
 
 namespace gla {
 
-// Retention-gate temperature tau (method section: "rank r=16, temperature tau=16").
+// Retention-gate temperature tau = 16 (method section, GLA recurrence paragraph).
 constexpr float kTau = 16.0f;
 constexpr float kInvTau = 1.0f / kTau;
 

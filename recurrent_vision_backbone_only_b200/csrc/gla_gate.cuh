@@ -3,7 +3,7 @@
 //
 // Operation (GTR paper, arXiv 2609.26590, method section, GLA recurrence paragraph): the key-wise
 // retention gate is gamma_t = sigma(x_t W_alpha^(1) W_alpha^(2) + b_alpha)^(1/tau), a low-rank
-// projection of rank r = 16 "following GLA": one first factor W1 [d][16] shared by the heads, a
+// projection of rank r = 16 built as GLA builds it: one first factor W1 [d][16] shared by the heads, a
 // second factor W2 [16][n] onto every head's key channels (n = H d_k), a bias per key channel.
 // The output a [T][n] is the operator's gate_preact input, [B][L][H][d_k].
 //
