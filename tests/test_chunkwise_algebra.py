@@ -100,6 +100,50 @@ def chunkwise_o(q, k, v, a, gh, gw, direction, chunk, segs, chunk_fn, exchange_r
     return o
 
 
+def lookback_scan(q, k, v, lg, chunk, segs, chunk_fn):
+    """The segment scan with every segment combining all earlier aggregates itself instead of
+    receiving a running state: S_in(s) = sum_{j<s} Diag(2^{G_{j+1} + ... + G_{s-1}}) S_agg(j)
+    -- the form a grid-wide exchange through a workspace would take, where all aggregates are
+    published at once and no segment waits for its predecessor's combine."""
+    L, dk = q.shape
+    dv = v.shape[1]
+    seg_len = -(-L // segs)
+    bounds = [(s0, min(L, s0 + seg_len)) for s0 in range(0, L, seg_len)]
+
+    def run(s0, s1, S):
+        outs, G = [], np.zeros(dk)
+        for c0 in range(s0, s1, chunk):
+            c1 = min(s1, c0 + chunk)
+            O, S, B = chunk_fn(q[c0:c1], k[c0:c1], v[c0:c1], lg[c0:c1], S)
+            outs.append(O)
+            G = G + B
+        return np.concatenate(outs), S, G
+
+    aggs = [run(s0, s1, np.zeros((dk, dv)))[1:] for s0, s1 in bounds]     # (S_agg, G) each
+    outs = []
+    for s, (s0, s1) in enumerate(bounds):
+        S_in = np.zeros((dk, dv))
+        for j in range(s):
+            decay = np.sum([aggs[i][1] for i in range(j + 1, s)], axis=0) if j + 1 < s else np.zeros(dk)
+            S_in = S_in + np.exp2(decay)[:, None] * aggs[j][0]
+        outs.append(run(s0, s1, S_in)[0])
+    return np.concatenate(outs)
+
+
+@pytest.mark.parametrize("direction", [0, 3])
+def test_lookback_combine_with_eighteen_segments_is_exact(direction):
+    rng = np.random.default_rng(11)
+    gh, gw = 24, 30                                  # 720 tokens: 18 segments of 40
+    q, k, v, a, g, w = rand_inputs(rng, 1, gh, gw, 1, 32, 24, a_mean=0.0, a_std=3.0)
+    _, o_ref = oracle.gla_forward(q, k, v, a, g, w, gh, gw, direction, return_o=True)
+    lg = log2_gate(a)
+    perm = scan_perm(direction, gh, gw)
+    fn = lambda *t: chunk_exact(*t, where="middle")   # noqa: E731
+    o = np.zeros(v.shape)
+    o[0, perm, 0] = lookback_scan(q[0, perm, 0], k[0, perm, 0], v[0, perm, 0], lg[0, perm, 0], 16, 18, fn)
+    assert np.max(np.abs(o - o_ref)) <= 1e-12 * max(1.0, np.max(np.abs(o_ref)))
+
+
 @pytest.mark.parametrize("direction", [0, 1, 2, 3])
 @pytest.mark.parametrize("chunk,segs,where", [(16, 1, "middle"), (32, 3, "first"),
                                               (64, 16, "middle"), (100, 5, "last"),
